@@ -1,0 +1,228 @@
+"""VSA-H3 forward -- plain CPU oracle (ctypes wrapper around ``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference arm may import this package.  The
+CUDA library never links or calls it, and it shares no code with that library.
+
+The C file states the method and every reading of the pages it takes.  This
+wrapper only marshals numpy arrays and runs whole-forward compositions in the
+order the method states them:
+
+    geometry -> pool(q, k, v) -> scores -> top-k -> compression, fine -> output
+
+Parity unpinned: the compression key scope (all tiles, reading R9) and the
+compression on prefix query rows (reading R10) follow a reading, not a printed
+value; nothing on the pages fixes them.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+import time
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f32, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+        lib.vsa_oracle_geometry.argtypes = [i32, P, i32, i32, i32, P, P, P]
+        lib.vsa_oracle_tiles.argtypes = [i32, P, i32, i32, i32, P, P]
+        lib.vsa_oracle_topk_count.argtypes = [f64, i32]
+        lib.vsa_oracle_topk_count.restype = i32
+        lib.vsa_oracle_pool.argtypes = [P, i32, i64, i32, i32, i32, P, P, P]
+        lib.vsa_oracle_scores.argtypes = [P, P, i32, i32, i32, f32, P]
+        lib.vsa_oracle_select.argtypes = [P, i32, i32, i32, i32, P]
+        lib.vsa_oracle_compress.argtypes = [P, P, i32, i32, i32, P]
+        lib.vsa_oracle_fine.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
+        lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P]
+        lib.vsa_oracle_output.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P, P, P]
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+@dataclass
+class Geometry:
+    """The oracle's own tiling of one packed sequence."""
+
+    segments: tuple
+    grid: tuple
+    n_tiles: int
+    n_prefix: int
+    n_video: int
+    tile_token: np.ndarray  # [n_tiles, 64] int32, -1 = pad
+    tile_valid: np.ndarray  # [n_tiles] int32
+
+    @property
+    def seq_len(self) -> int:
+        return int(sum(self.segments)) + int(np.prod(self.grid))
+
+
+def geometry(segments, grid) -> Geometry:
+    lib = _load()
+    seg = np.asarray(segments, dtype=np.int32)
+    T, H, W = (int(x) for x in grid)
+    nt, npf, nv = (ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32())
+    rc = lib.vsa_oracle_geometry(len(seg), _p(seg), T, H, W, ctypes.byref(nt), ctypes.byref(npf), ctypes.byref(nv))
+    if rc:
+        raise ValueError("bad geometry")
+    tok = np.empty((nt.value, 64), np.int32)
+    val = np.empty((nt.value,), np.int32)
+    lib.vsa_oracle_tiles(len(seg), _p(seg), T, H, W, _p(tok), _p(val))
+    return Geometry(tuple(int(s) for s in segments), (T, H, W), nt.value, npf.value, nv.value, tok, val)
+
+
+def topk_count(sparsity: float, n_video: int) -> int:
+    return int(_load().vsa_oracle_topk_count(float(sparsity), int(n_video)))
+
+
+def default_scale(head_dim: int) -> float:
+    """1/sqrt(D) rounded once to binary32."""
+    return float(np.float32(1.0 / math.sqrt(float(head_dim))))
+
+
+def pool(x_bf16: np.ndarray, geo: Geometry) -> np.ndarray:
+    """x_bf16: [B, L, H, D] uint16 (bf16 bits) -> pooled [B, H, n_t, D] float32."""
+    x = _c(x_bf16, np.uint16)
+    B, L, H, D = x.shape
+    out = np.empty((B, H, geo.n_tiles, D), np.float32)
+    _load().vsa_oracle_pool(_p(x), B, L, H, D, geo.n_tiles, _p(geo.tile_token), _p(geo.tile_valid), _p(out))
+    return out
+
+
+def scores(pq: np.ndarray, pk: np.ndarray, scale: float) -> np.ndarray:
+    """pq, pk: [B, H, n_t, D] float32 -> S [B, H, n_t, n_t] float32."""
+    pq = _c(pq, np.float32)
+    pk = _c(pk, np.float32)
+    B, H, n_t, D = pq.shape
+    S = np.empty((B, H, n_t, n_t), np.float32)
+    _load().vsa_oracle_scores(_p(pq), _p(pk), B * H, n_t, D, ctypes.c_float(scale), _p(S))
+    return S
+
+
+def select(S: np.ndarray, n_prefix: int, k: int) -> np.ndarray:
+    """S: [B, H, n_t, n_t] -> idx [B, H, V, k] int32 (global tile indices, ascending)."""
+    S = _c(S, np.float32)
+    B, H, n_t, _ = S.shape
+    V = n_t - n_prefix
+    idx = np.empty((B, H, V, k), np.int32)
+    if _load().vsa_oracle_select(_p(S), B * H, n_t, n_prefix, k, _p(idx)):
+        raise ValueError("NaN pooled score")
+    return idx
+
+
+def compress(S: np.ndarray, pv: np.ndarray) -> np.ndarray:
+    """-> o_c [B, H, n_t, D] float64."""
+    S = _c(S, np.float32)
+    pv = _c(pv, np.float32)
+    B, H, n_t, D = pv.shape
+    out = np.empty((B, H, n_t, D), np.float64)
+    _load().vsa_oracle_compress(_p(S), _p(pv), B * H, n_t, D, _p(out))
+    return out
+
+
+def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None) -> np.ndarray:
+    """List formulation of the fine branch -> o_f [B, L, H, D] float64 (NaN where not computed)."""
+    q, k, v = (_c(t, np.uint16) for t in (q, k, v))
+    B, L, H, D = q.shape
+    idx = _c(idx, np.int32)
+    if todo is not None:
+        todo = _c(todo.astype(np.uint8), np.uint8)
+    out = np.full((B, L, H, D), np.nan, np.float64)
+    _load().vsa_oracle_fine(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+                            _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(todo), _p(out))
+    return out
+
+
+def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndarray:
+    """Mask formulation (dense L x L masked softmax attention) -> [B, L, H, D] float64."""
+    q, k, v = (_c(t, np.uint16) for t in (q, k, v))
+    B, L, H, D = q.shape
+    idx = _c(idx, np.int32)
+    out = np.full((B, L, H, D), np.nan, np.float64)
+    _load().vsa_oracle_fine_masked(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+                                   _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(out))
+    return out
+
+
+def output(o_f, o_c, gate, geo: Geometry, todo=None) -> np.ndarray:
+    o_f = _c(o_f, np.float64)
+    o_c = _c(o_c, np.float64)
+    gate = _c(gate, np.uint16)
+    B, L, H, D = o_f.shape
+    if todo is not None:
+        todo = _c(todo.astype(np.uint8), np.uint8)
+    out = np.full((B, L, H, D), np.nan, np.float64)
+    _load().vsa_oracle_output(_p(o_f), _p(o_c), _p(gate), B, L, H, D, geo.n_tiles,
+                              _p(geo.tile_token), _p(geo.tile_valid), _p(todo), _p(out))
+    return out
+
+
+@dataclass
+class ForwardResult:
+    geo: Geometry
+    topk: int
+    scale: float
+    pq: np.ndarray
+    pk: np.ndarray
+    pv: np.ndarray
+    S: np.ndarray
+    idx: np.ndarray
+    o_c: np.ndarray
+    o_f: np.ndarray
+    out: np.ndarray
+    seconds: float
+
+
+def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None) -> ForwardResult:
+    """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H].
+
+    Selection (pool, scores, top-k) always runs in full; the fine branch and
+    the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
+    None = all)."""
+    t0 = time.perf_counter()
+    geo = geometry(segments, grid)
+    D = q.shape[-1]
+    if scale is None:
+        scale = default_scale(D)
+    kc = topk_count(sparsity, geo.n_video)
+    pq, pk, pv = pool(q, geo), pool(k, geo), pool(v, geo)
+    S = scores(pq, pk, scale)
+    idx = select(S, geo.n_prefix, kc)
+    o_c = compress(S, pv)
+    o_f = fine(q, k, v, geo, idx, kc, scale, todo)
+    out = output(o_f, o_c, gate, geo, todo)
+    return ForwardResult(geo, kc, scale, pq, pk, pv, S, idx, o_c, o_f, out, time.perf_counter() - t0)

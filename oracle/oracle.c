@@ -1,0 +1,427 @@
+/*
+ * VSA-H3 forward -- plain CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the bench's
+ * CPU-baseline / reference arm use it.  It shares no code, header, table or
+ * constant with the CUDA library; it is written straight from the method's
+ * statement and is meant to be read against it line by line.
+ *
+ * Source of the method (the only place the pages state what VSA-H3 computes):
+ *   "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse Attention is
+ *   not optional here": 64-token (4,4,4) tiles over the post-patchify video
+ *   grid, segment-pure prefix tiles, per-head fp32 pooled tile scores,
+ *   topk = max(1, min(ceil((1 - sparsity) * n_video_tiles), n_video_tiles)),
+ *   prefix keys always selected, prefix queries dense, and a compression
+ *   branch softmax(scores) @ pool(v) broadcast over each tile row and scaled
+ *   by the gate with no activation.
+ * Supporting passages:
+ *   "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse FP4
+ *   attention for VSA tiles": per-query-block lists of key blocks, partially
+ *   filled tiles carry valid counts, exempt mode gives every query the first
+ *   prefix tile; section "Model integration": pad rows are zero.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   R1 video tokens follow the prefix in raster (t, h, w) order, w fastest;
+ *   R2 a grid side that is not a multiple of 4 gives partial edge cubes
+ *      (ceil-divided cube grid);
+ *   R3 inside a tile the valid tokens come first, pads last;
+ *   R4 a pooled tile is the mean over its valid tokens (divisor = count);
+ *   R5 pooled scores use the same softmax scale as the fine branch;
+ *   R6 the fp32 arithmetic order is pinned: pooling adds rows in tile order
+ *      starting from +0.0f, then one IEEE division; a score is a chain of
+ *      fmaf over d = 0..D-1 starting from +0.0f, then one multiply by scale;
+ *   R7 ties in the top-k order go to the lower video tile index; the chosen
+ *      tiles are listed in ascending index;
+ *   R8 topk uses binary64 arithmetic for (1 - sparsity) * V and its ceiling,
+ *      and is 0 when there are no video tiles;
+ *   R9 the compression softmax runs over ALL tiles (prefix and video)
+ *      -- parity unpinned;
+ *   R10 the compression branch is added to every tile row, prefix tiles
+ *      included -- parity unpinned;
+ *   R11 the gate is one scalar per (batch, token, head).
+ *
+ * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
+ * order above; fine attention, compression and the output in binary64.
+ *
+ * Build: gcc -O2 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define TILE 64
+#define CUBE 4
+
+/* ------------------------------------------------------------------ */
+/* helpers                                                             */
+/* ------------------------------------------------------------------ */
+
+static float bf16_to_float(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+/* ------------------------------------------------------------------ */
+/* O1 geometry                                                         */
+/* ------------------------------------------------------------------ */
+
+/* Tile counts of a packed sequence: each prefix segment of n tokens gives
+ * ceil(n/64) segment-pure tiles; the T x H x W video grid gives
+ * ceil(T/4) * ceil(H/4) * ceil(W/4) cubes (reading R2).
+ * Returns 0, or -1 on a bad argument. */
+int vsa_oracle_geometry(int n_seg, const int32_t *seg_len, int T, int Hg, int W,
+                        int32_t *n_tiles, int32_t *n_prefix, int32_t *n_video) {
+    if (n_seg < 0 || T < 0 || Hg < 0 || W < 0) return -1;
+    int64_t p = 0;
+    for (int s = 0; s < n_seg; ++s) {
+        if (seg_len[s] < 0) return -1;
+        p += ceil_div(seg_len[s], TILE);
+    }
+    int64_t v = (T > 0 && Hg > 0 && W > 0)
+                    ? ceil_div(T, CUBE) * ceil_div(Hg, CUBE) * ceil_div(W, CUBE)
+                    : 0;
+    *n_prefix = (int32_t)p;
+    *n_video = (int32_t)v;
+    *n_tiles = (int32_t)(p + v);
+    return 0;
+}
+
+/* Token table: tile_token[tile*64 + r] is the packed-sequence index of row r
+ * of the tile, or -1 for a pad row; tile_valid[tile] counts the valid rows.
+ * Prefix tiles first, in sequence order; then the cubes in raster (a,b,c)
+ * order; inside a cube, raster (t,h,w) (readings R1, R3). */
+int vsa_oracle_tiles(int n_seg, const int32_t *seg_len, int T, int Hg, int W,
+                     int32_t *tile_token, int32_t *tile_valid) {
+    int32_t nt, np, nv;
+    if (vsa_oracle_geometry(n_seg, seg_len, T, Hg, W, &nt, &np, &nv)) return -1;
+    for (int64_t i = 0; i < (int64_t)nt * TILE; ++i) tile_token[i] = -1;
+
+    int tile = 0;
+    int64_t offset = 0; /* first token of the current segment */
+    for (int s = 0; s < n_seg; ++s) {
+        int64_t n = seg_len[s];
+        for (int64_t first = 0; first < n; first += TILE) {
+            int cnt = 0;
+            for (int64_t t = first; t < n && t < first + TILE; ++t)
+                tile_token[(int64_t)tile * TILE + cnt++] = (int32_t)(offset + t);
+            tile_valid[tile++] = cnt;
+        }
+        offset += n;
+    }
+    if (nv > 0) {
+        int64_t video_base = offset;
+        for (int a = 0; a < ceil_div(T, CUBE); ++a)
+            for (int b = 0; b < ceil_div(Hg, CUBE); ++b)
+                for (int c = 0; c < ceil_div(W, CUBE); ++c) {
+                    int cnt = 0;
+                    for (int t = CUBE * a; t < CUBE * a + CUBE && t < T; ++t)
+                        for (int h = CUBE * b; h < CUBE * b + CUBE && h < Hg; ++h)
+                            for (int w = CUBE * c; w < CUBE * c + CUBE && w < W; ++w)
+                                tile_token[(int64_t)tile * TILE + cnt++] =
+                                    (int32_t)(video_base + ((int64_t)t * Hg + h) * W + w);
+                    tile_valid[tile++] = cnt;
+                }
+    }
+    return 0;
+}
+
+/* O4 count: topk = max(1, min(ceil((1 - s) * V), V)) in binary64 (R8). */
+int vsa_oracle_topk_count(double sparsity, int n_video) {
+    if (n_video <= 0) return 0;
+    double k = ceil((1.0 - sparsity) * (double)n_video);
+    if (k > (double)n_video) k = (double)n_video;
+    if (k < 1.0) k = 1.0;
+    return (int)k;
+}
+
+/* ------------------------------------------------------------------ */
+/* O2 pooling (binary32, pinned order)                                 */
+/* ------------------------------------------------------------------ */
+
+/* x: [B, L, H, D] bf16 bits.  pooled: [B, H, n_t, D] float.
+ * pooled = (((0 + x_0) + x_1) + ... + x_{n-1}) / n  over the valid rows in
+ * tile order, every step one IEEE binary32 rounding (R4, R6). */
+void vsa_oracle_pool(const uint16_t *x, int B, int64_t L, int H, int D, int n_t,
+                     const int32_t *tile_token, const int32_t *tile_valid, float *pooled) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int tile = 0; tile < n_t; ++tile)
+                for (int d = 0; d < D; ++d) {
+                    float sum = 0.0f;
+                    for (int r = 0; r < tile_valid[tile]; ++r) {
+                        int64_t tok = tile_token[(int64_t)tile * TILE + r];
+                        sum = sum + bf16_to_float(x[(((int64_t)b * L + tok) * H + h) * D + d]);
+                    }
+                    pooled[(((int64_t)b * H + h) * n_t + tile) * D + d] =
+                        sum / (float)tile_valid[tile];
+                }
+}
+
+/* ------------------------------------------------------------------ */
+/* O3 pooled tile scores (binary32, pinned order)                      */
+/* ------------------------------------------------------------------ */
+
+/* S[bh, i, j] = fl(fmaf-chain_{d=0..D-1}(pq[bh,i,d] * pk[bh,j,d]) * scale). */
+void vsa_oracle_scores(const float *pq, const float *pk, int BH, int n_t, int D,
+                       float scale, float *S) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < n_t; ++i)
+            for (int j = 0; j < n_t; ++j) {
+                const float *a = pq + ((int64_t)bh * n_t + i) * D;
+                const float *b = pk + ((int64_t)bh * n_t + j) * D;
+                float acc = 0.0f;
+                for (int d = 0; d < D; ++d) acc = fmaf(a[d], b[d], acc);
+                S[((int64_t)bh * n_t + i) * n_t + j] = acc * scale;
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* O4 top-k selection                                                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    float s;
+    int32_t j;
+} scored_tile;
+
+/* order: higher score first; equal scores -> lower tile index first (R7) */
+static int by_score_then_index(const void *pa, const void *pb) {
+    const scored_tile *a = (const scored_tile *)pa, *b = (const scored_tile *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int by_index(const void *pa, const void *pb) {
+    int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+    return (a > b) - (a < b);
+}
+
+/* For each (bh, video query tile iv) pick the k video key tiles with the
+ * highest S[bh, P+iv, P+j]; write their GLOBAL tile indices (P + j) in
+ * ascending order to idx[bh, iv, 0..k-1].  Returns -1 if any compared score
+ * is NaN (inputs with NaN are rejected), else 0. */
+int vsa_oracle_select(const float *S, int BH, int n_t, int P, int k, int32_t *idx) {
+    int V = n_t - P;
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(static) reduction(| : bad)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int iv = 0; iv < V; ++iv) {
+            scored_tile *row = (scored_tile *)malloc(sizeof(scored_tile) * (size_t)(V > 0 ? V : 1));
+            const float *srow = S + ((int64_t)bh * n_t + (P + iv)) * n_t;
+            for (int j = 0; j < V; ++j) {
+                row[j].s = srow[P + j];
+                row[j].j = j;
+                if (isnan(row[j].s)) bad = 1;
+            }
+            qsort(row, (size_t)V, sizeof(scored_tile), by_score_then_index);
+            int32_t *out = idx + ((int64_t)bh * V + iv) * k;
+            for (int t = 0; t < k; ++t) out[t] = P + row[t].j;
+            qsort(out, (size_t)k, sizeof(int32_t), by_index);
+            free(row);
+        }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* O6 compression branch (binary64)                                    */
+/* ------------------------------------------------------------------ */
+
+/* o_c[bh, i, :] = sum_j softmax_j(S[bh, i, :]) * pv[bh, j, :], j over all
+ * n_t tiles (reading R9). */
+void vsa_oracle_compress(const float *S, const float *pv, int BH, int n_t, int D, double *o_c) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < n_t; ++i) {
+            const float *srow = S + ((int64_t)bh * n_t + i) * n_t;
+            double m = -INFINITY;
+            for (int j = 0; j < n_t; ++j)
+                if ((double)srow[j] > m) m = (double)srow[j];
+            double denom = 0.0;
+            for (int j = 0; j < n_t; ++j) denom += exp((double)srow[j] - m);
+            double *o = o_c + ((int64_t)bh * n_t + i) * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            for (int j = 0; j < n_t; ++j) {
+                double w = exp((double)srow[j] - m) / denom;
+                const float *pvj = pv + ((int64_t)bh * n_t + j) * D;
+                for (int d = 0; d < D; ++d) o[d] += w * (double)pvj[d];
+            }
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* O5 fine branch, list formulation (binary64)                         */
+/* ------------------------------------------------------------------ */
+
+/* The key set of query tile i: every tile for a prefix query tile (dense
+ * prefix queries); the P prefix tiles plus idx[b,h,i-P,:] for a video query
+ * tile (exempt prefix keys).  Writes the set into keys[] and returns its size. */
+static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t *keys) {
+    if (i < P) {
+        for (int j = 0; j < n_t; ++j) keys[j] = j;
+        return n_t;
+    }
+    for (int j = 0; j < P; ++j) keys[j] = j;
+    for (int t = 0; t < k; ++t) keys[P + t] = idx_row[t];
+    return P + k;
+}
+
+/* o_f[b, tok, h, :] for every valid query token tok of every (b, h, i) with
+ * todo[(b*H + h)*n_t + i] != 0 (todo == NULL: all).  For a query row r:
+ *   logit_c = scale * <q_r, k_c> over the valid key rows c of its key set,
+ *   o_f = sum_c softmax(logit)_c * v_c.
+ * q, k, v: [B, L, H, D] bf16 bits; idx: [B, H, V, k] global tile indices. */
+void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B, int64_t L,
+                     int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                     const int32_t *tile_valid, const int32_t *idx, double scale,
+                     const uint8_t *todo, double *o_f) {
+    int V = n_t - P;
+#pragma omp parallel for collapse(3) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < n_t; ++i) {
+                int64_t bhi = ((int64_t)b * H + h) * n_t + i;
+                if (todo && !todo[bhi]) continue;
+                int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
+                const int32_t *idx_row =
+                    (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
+                int nk = key_set(i, n_t, P, k, idx_row, keys);
+                /* every valid key row of the key set, in list order */
+                int64_t max_rows = (int64_t)nk * TILE;
+                int64_t *ktok = (int64_t *)malloc(sizeof(int64_t) * (size_t)max_rows);
+                double *logit = (double *)malloc(sizeof(double) * (size_t)max_rows);
+                int64_t nrows = 0;
+                for (int t = 0; t < nk; ++t)
+                    for (int c = 0; c < tile_valid[keys[t]]; ++c)
+                        ktok[nrows++] = tile_token[(int64_t)keys[t] * TILE + c];
+
+                for (int r = 0; r < tile_valid[i]; ++r) {
+                    int64_t qt = tile_token[(int64_t)i * TILE + r];
+                    const uint16_t *qr = q + (((int64_t)b * L + qt) * H + h) * D;
+                    double m = -INFINITY;
+                    for (int64_t c = 0; c < nrows; ++c) {
+                        const uint16_t *kc = kk + (((int64_t)b * L + ktok[c]) * H + h) * D;
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            dot += (double)bf16_to_float(qr[d]) * (double)bf16_to_float(kc[d]);
+                        logit[c] = scale * dot;
+                        if (logit[c] > m) m = logit[c];
+                    }
+                    double denom = 0.0;
+                    for (int64_t c = 0; c < nrows; ++c) {
+                        logit[c] = exp(logit[c] - m);
+                        denom += logit[c];
+                    }
+                    double *o = o_f + (((int64_t)b * L + qt) * H + h) * D;
+                    for (int d = 0; d < D; ++d) o[d] = 0.0;
+                    for (int64_t c = 0; c < nrows; ++c) {
+                        const uint16_t *vc = v + (((int64_t)b * L + ktok[c]) * H + h) * D;
+                        double w = logit[c] / denom;
+                        for (int d = 0; d < D; ++d) o[d] += w * (double)bf16_to_float(vc[d]);
+                    }
+                }
+                free(logit);
+                free(ktok);
+                free(keys);
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* O5' fine branch, mask formulation (binary64, second definition)     */
+/* ------------------------------------------------------------------ */
+
+/* Dense softmax attention over the packed sequence in token order, where
+ * query token a may attend key token c iff c's tile is in the key set of a's
+ * tile (the "masked reference" the pages compare the block-sparse kernel
+ * against).  Tokens outside every tile do not occur.  Used on small inputs
+ * only: builds an L x L mask per (b, h). */
+void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B,
+                            int64_t L, int H, int D, int n_t, int P, int k,
+                            const int32_t *tile_token, const int32_t *tile_valid,
+                            const int32_t *idx, double scale, double *o_f) {
+    int V = n_t - P;
+    int32_t *tile_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)L);
+    for (int i = 0; i < n_t; ++i)
+        for (int r = 0; r < tile_valid[i]; ++r) tile_of[tile_token[(int64_t)i * TILE + r]] = i;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            /* allowed[i * n_t + j]: key tile j in the key set of query tile i */
+            uint8_t *allowed = (uint8_t *)calloc((size_t)n_t * n_t, 1);
+            int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
+            for (int i = 0; i < n_t; ++i) {
+                const int32_t *idx_row =
+                    (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
+                int nk = key_set(i, n_t, P, k, idx_row, keys);
+                for (int t = 0; t < nk; ++t) allowed[(int64_t)i * n_t + keys[t]] = 1;
+            }
+            double *logit = (double *)malloc(sizeof(double) * (size_t)L);
+            for (int64_t a = 0; a < L; ++a) {
+                int ti = tile_of[a];
+                const uint16_t *qa = q + (((int64_t)b * L + a) * H + h) * D;
+                double m = -INFINITY;
+                for (int64_t c = 0; c < L; ++c) {
+                    if (!allowed[(int64_t)ti * n_t + tile_of[c]]) {
+                        logit[c] = -INFINITY;
+                        continue;
+                    }
+                    const uint16_t *kc = kk + (((int64_t)b * L + c) * H + h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += (double)bf16_to_float(qa[d]) * (double)bf16_to_float(kc[d]);
+                    logit[c] = scale * dot;
+                    if (logit[c] > m) m = logit[c];
+                }
+                double denom = 0.0;
+                for (int64_t c = 0; c < L; ++c) {
+                    logit[c] = (logit[c] == -INFINITY) ? 0.0 : exp(logit[c] - m);
+                    denom += logit[c];
+                }
+                double *o = o_f + (((int64_t)b * L + a) * H + h) * D;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int64_t c = 0; c < L; ++c) {
+                    if (logit[c] == 0.0) continue;
+                    const uint16_t *vc = v + (((int64_t)b * L + c) * H + h) * D;
+                    double w = logit[c] / denom;
+                    for (int d = 0; d < D; ++d) o[d] += w * (double)bf16_to_float(vc[d]);
+                }
+            }
+            free(logit);
+            free(keys);
+            free(allowed);
+        }
+    free(tile_of);
+}
+
+/* ------------------------------------------------------------------ */
+/* O7 output                                                           */
+/* ------------------------------------------------------------------ */
+
+/* out[b, tok, h, :] = o_f[b, tok, h, :] + gate[b, tok, h] * o_c[b, h, tile(tok), :]
+ * for the valid rows of every tile with todo set (NULL: all); gate: [B, L, H]
+ * bf16 bits; one scalar gate per token and head, no activation (R10, R11). */
+void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gate, int B,
+                       int64_t L, int H, int D, int n_t, const int32_t *tile_token,
+                       const int32_t *tile_valid, const uint8_t *todo, double *out) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < n_t; ++i) {
+                if (todo && !todo[((int64_t)b * H + h) * n_t + i]) continue;
+                const double *oc = o_c + (((int64_t)b * H + h) * n_t + i) * D;
+                for (int r = 0; r < tile_valid[i]; ++r) {
+                    int64_t tok = tile_token[(int64_t)i * TILE + r];
+                    int64_t row = (((int64_t)b * L + tok) * H + h);
+                    double g = (double)bf16_to_float(gate[row]);
+                    for (int d = 0; d < D; ++d) out[row * D + d] = o_f[row * D + d] + g * oc[d];
+                }
+            }
+}
