@@ -390,3 +390,36 @@ def test_output_gate(oracle_mod):
         for h in range(w.heads):
             expect = r.o_f[0, toks, h] + g[0, toks, h][:, None] * r.o_c[0, h, i][None, :]
             assert np.abs(r.out[0, toks, h] - expect).max() < 1e-15
+
+
+def test_scores_fused_chain_in_d_order(oracle_mod):
+    """Reading R6 fixes the score arithmetic: one fused multiply-add per d,
+    d ascending, from +0.  Two hand-worked cases pin it:
+      [-1, 1+2^-12] . [1, 1+2^-12]: -1, then fma gives 2^-11 + 2^-24 exactly
+        (an unfused multiply would round a*a first and give 2^-11);
+      [2^-30, 1, -1] . [1, 1, 1]: 2^-30, then 1 + 2^-30 rounds to 1, then 0
+        (the reverse order would give 2^-30)."""
+    a = np.float32(1 + 2.0 ** -12)
+    pq = np.zeros((1, 1, 2, 4), np.float32)
+    pk = np.zeros((1, 1, 2, 4), np.float32)
+    pq[0, 0, 0, :2] = [-1.0, a]
+    pk[0, 0, 0, :2] = [1.0, a]
+    pq[0, 0, 1, :3] = [2.0 ** -30, 1.0, -1.0]
+    pk[0, 0, 1, :3] = [1.0, 1.0, 1.0]
+    S = oracle_mod.scores(pq, pk, 1.0)
+    assert S[0, 0, 0, 0] == np.float32(2.0 ** -11 + 2.0 ** -24)
+    assert S[0, 0, 1, 1] == 0.0
+
+
+def test_pool_adds_rows_in_tile_order(oracle_mod):
+    """Reading R6 for pooling: rows are added in tile order from +0.  Rows
+    (2^-30, 1, -1) give ((0 + 2^-30) + 1) - 1 = 0 in binary32; any other
+    order that adds 2^-30 last would give 2^-30 / 3."""
+    segments, grid = (3,), (0, 0, 0)
+    geo = oracle_mod.geometry(segments, grid)
+    x = np.zeros((1, 3, 1, 8), np.float32)
+    x[0, :, 0, 0] = [2.0 ** -30, 1.0, -1.0]
+    x[0, :, 0, 1] = [1.0, -1.0, 2.0 ** -30]
+    p = oracle_mod.pool(bf16_bits(torch.from_numpy(x)), geo)
+    assert p[0, 0, 0, 0] == 0.0
+    assert p[0, 0, 0, 1] == np.float32(2.0 ** -30) / np.float32(3.0)
