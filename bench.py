@@ -1,0 +1,379 @@
+"""Benchmark of the VSA-H3 forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vsa|reference] [--workload NAME]
+
+One step = one whole VSA-H3 forward (gather + pool, pooled scores, top-k +
+compression, block-sparse attention + gated epilogue) over one synthetic
+input already resident in HBM.  The default workload is the 1344x768-shaped
+one at sparsity 0.9 (56 heads, D=128, 73,728 video + 1,280 prefix tokens).
+
+Metric: effective TFLOP/s counting only the selected (query tile, key tile)
+pairs, 4*64*64*D FLOP each, per whole forward; ms per call is reported too.
+Multi-GPU (torchrun): every rank runs its own forward on its own seeded input
+(the forward shards by (batch, head) with no exchange), value = all ranks'
+FLOPs / the slowest rank's time ("scaling": "weak").
+
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "VSA-H3 fwd ms/call & effective TFLOPS (selected tiles) at 73.7k tok, 56 heads"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def tile_flops(D: int) -> int:
+    return 4 * 64 * 64 * D
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(source="measured", bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), hbm_gbs=d["hbm_gbs"])
+    return dict(source="fallback", bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if (args.impl == "vsa" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+
+
+def oracle_sample(w, every: int, seed: int = 0):
+    """Time the CPU oracle on head 0 of the workload: full selection (pool,
+    scores, top-k, compression) and the fine branch + output of every
+    ``every``-th query tile.  Returns (seconds, selected-tile FLOPs, description)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synth
+
+    x = synth.make_inputs(dataclasses.replace(w, heads=1), seed=seed, device="cpu")
+    xb = {n: synth.as_bits(x[n]) for n in ("q", "k", "v", "gate")}
+    t0 = time.perf_counter()
+    sel = oracle.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity)
+    geo = sel["geo"]
+    items = np.arange(0, geo.n_tiles, every, dtype=np.int64)
+    of = oracle.fine_tiles(xb["q"], xb["k"], xb["v"], geo, sel["idx"], sel["topk"], sel["scale"], items)
+    oracle.output_tiles(of, sel["o_c"], xb["gate"], geo, items, 1)
+    dt = time.perf_counter() - t0
+    pairs = sum((geo.n_tiles if i < geo.n_prefix else geo.n_prefix + sel["topk"]) for i in items)
+    flops = pairs * tile_flops(w.head_dim)
+    desc = (f"head 0 of 56: full selection (pool, fp32 scores, top-k, compression over {geo.n_tiles} tiles) "
+            f"+ fine branch and output of every {every}th query tile ({len(items)} of {geo.n_tiles} tiles, "
+            f"{pairs} selected tile pairs)")
+    del torch
+    return dt, flops, desc
+
+
+def omp_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def run_reference(args, w, world, rank):
+    """CPU oracle arm: rank 0 only."""
+    if rank != 0:
+        return
+    every = args.ref_every
+    for _ in range(args.warmup):
+        oracle_sample(w, every)
+    times, flops, desc = [], 0, ""
+    for _ in range(args.steps):
+        dt, flops, desc = oracle_sample(w, every)
+        times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    value = flops / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based normal)",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+
+def config_dict(w, dims=None):
+    import oracle
+
+    geo = oracle.geometry(w.segments, w.grid) if dims is None else None
+    n_t = dims["n_tiles"] if dims else geo.n_tiles
+    P = dims["n_prefix_tiles"] if dims else geo.n_prefix
+    V = n_t - P
+    k = dims["topk"] if dims else oracle.topk_count(w.sparsity, V)
+    pairs = V * (P + k) + P * n_t
+    return {
+        "workload": w.name, "description": w.description, "batch": w.batch, "heads": w.heads,
+        "head_dim": w.head_dim, "seq_len": w.seq_len, "prefix_segments": list(w.segments), "grid": list(w.grid),
+        "n_tiles": n_t, "n_prefix_tiles": P, "n_video_tiles": V, "sparsity": w.sparsity, "topk": k,
+        "selected_tile_pairs": pairs * w.batch * w.heads,
+        "selected_tflop_per_call": pairs * w.batch * w.heads * tile_flops(w.head_dim) / 1e12,
+        "l2": "no flush: Q/K/V/out are %.1f GB per step, > 126 MB L2" % (4 * w.batch * w.seq_len * w.heads * w.head_dim * 2 / 1e9),
+    }
+
+
+def run_vsa(args, w, world, rank, local):
+    import torch
+
+    import block_sparse_tiled_b200 as vsa
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x = synth.make_inputs(w, seed=rank, device=dev)
+    torch.cuda.synchronize()
+    plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
+                              sparsity=w.sparsity)
+    dims = plan.dims
+    ws = vsa.alloc_workspace(plan, dev)
+    v = vsa.workspace_views(plan, ws)
+    out = torch.empty_like(x["q"])
+    stream = torch.cuda.current_stream(dev)
+    flops_call = dims["selected_pairs"] * w.batch * w.heads * tile_flops(w.head_dim)
+
+    ev = {n: [] for n in ("t0", "t1", "t2", "t3", "t4")}
+
+    def step(record):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
+        if record:
+            e[0].record(stream)
+        vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], v["q_t"], v["k_t"], v["v_t"], v["pq"], v["pk"], v["pv"],
+                             stream=stream)
+        if record:
+            e[1].record(stream)
+        vsa.vsa_pool_and_score(plan, None, None, None, v["pq"], v["pk"], v["pv"], v["scores"], stream=stream)
+        if record:
+            e[2].record(stream)
+        vsa.vsa_topk_select(plan, v["scores"], v["pv"], v["idx"], v["o_c"], stream=stream)
+        if record:
+            e[3].record(stream)
+        vsa.vsa_sparse_attn_fwd(plan, v["q_t"], v["k_t"], v["v_t"], v["idx"], v["o_c"], x["gate"], out,
+                                stream=stream)
+        if record:
+            e[4].record(stream)
+            for n, evt in zip(("t0", "t1", "t2", "t3", "t4"), e):
+                ev[n].append(evt)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    code, where = vsa.device_status(plan)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at site {where} during warm-up")
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = start.elapsed_time(stop)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    code, where = vsa.device_status(plan)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at site {where} in the timed region")
+
+    def avg(a, b):
+        return statistics.mean(x.elapsed_time(y) for x, y in zip(ev[a], ev[b]))
+
+    stage_ms = {"gather_pool": avg("t0", "t1"), "scores": avg("t1", "t2"), "topk_compress": avg("t2", "t3"),
+                "attention": avg("t3", "t4")}
+    ms_step = elapsed_ms / args.steps
+    value = world * flops_call / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "gate")}
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    vsa.vsa_forward(plan, hx["q"], hx["k"], hx["v"], hx["gate"], out=hout, workspace=ws)
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier(world)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        vsa.vsa_forward(plan, hx["q"], hx["k"], hx["v"], hx["gate"], out=hout, workspace=ws)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps, world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hout.numel() * hout.element_size()
+
+    peaks = load_peaks()
+    attn_tflops = flops_call / (stage_ms["attention"] * 1e-3) / 1e12
+    roofline = {
+        "kernel": "vsa_attn_kernel<128>", "bound": "tensor", "achieved": attn_tflops,
+        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+        "frac": attn_tflops / peaks["bf16_tflops_sustained"],
+        "peak_kind": f"{peaks['source']} sustained dense bf16 (kernel timed inside a seconds-long loop)",
+        "frac_of_burst_peak": attn_tflops / peaks["bf16_tflops"],
+        "algorithmic_flop_per_launch": flops_call,
+        "traffic": None,
+    }
+    launches = 5 * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based normal, structured tile offsets)",
+        "config": dict(config_dict(w, dims), parallelism=f"independent forward per GPU x{world}"),
+        "stage_ms": stage_ms, "roofline": roofline,
+        "e2e": {"value": world * flops_call / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc = oracle_sample(w, args.cpu_every)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    plan.destroy()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["vsa", "reference"], default="vsa")
+    ap.add_argument("--workload", default="768p_s0.9")
+    ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-every", type=int, default=4)
+    ap.add_argument("--ref-every", type=int, default=16)
+    args = ap.parse_args()
+    import synth
+
+    w = synth.workload(args.workload)
+    if args.sparsity is not None:
+        w = dataclasses.replace(w, sparsity=args.sparsity, name=f"{w.name}@s{args.sparsity}")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, world, rank)
+        else:
+            run_vsa(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,326 @@
+"""Python binding of libvsa, the VSA-H3 block-sparse attention forward for B200.
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels
+of ``libvsa.so`` (built from ``csrc/`` for sm_100a).  PyTorch supplies device
+memory and streams.  There is no fallback: if the library is missing or the
+device is not sm_100, the calls raise.
+
+The functions mirror the C ABI in ``include/vsa.h``:
+
+    vsa_plan_tiles      S1  tile plan (host) + upload of the tile tables
+    vsa_gather_tiles    S2  sequence order -> tile order (optionally pooled)
+    vsa_pool_and_score  S3  pooled tiles and fp32 pooled tile scores
+    vsa_topk_select     S4  top-k key tiles per video query tile + compression
+    vsa_sparse_attn_fwd S5  block-sparse attention + gated epilogue
+    vsa_forward             S2..S5 in one call
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvsa.so")
+
+VSA_OK = 0
+STATUS_NAMES = {
+    0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR_UNSUPPORTED",
+    4: "VSA_ERR_WORKSPACE", 5: "VSA_ERR_CUDA", 6: "VSA_ERR_TIMEOUT", 7: "VSA_ERR_DEVICE",
+}
+
+# every symbol include/vsa.h declares
+EXPORTED = (
+    "vsa_plan_tiles", "vsa_plan_info", "vsa_plan_tables", "vsa_plan_query", "vsa_plan_tables_host",
+    "vsa_plan_destroy",
+    "vsa_gather_tiles", "vsa_pool_and_score", "vsa_topk_select", "vsa_sparse_attn_fwd", "vsa_forward",
+    "vsa_plan_workspace", "vsa_device_status", "vsa_last_error", "vsa_version",
+)
+
+
+class VsaError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {message}")
+
+
+class Geometry(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("n_segments", ctypes.c_int32), ("segment_len", ctypes.POINTER(ctypes.c_int32)),
+        ("token_tags", ctypes.POINTER(ctypes.c_int32)), ("seq_len", ctypes.c_int64),
+        ("video_tag", ctypes.c_int32),
+        ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+        ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+    ]
+
+
+class PlanDims(ctypes.Structure):
+    _fields_ = [
+        ("n_tiles", ctypes.c_int32), ("n_prefix_tiles", ctypes.c_int32), ("n_video_tiles", ctypes.c_int32),
+        ("topk", ctypes.c_int32), ("seq_len", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
+        ("workspace_bytes", ctypes.c_size_t), ("selected_pairs", ctypes.c_int64),
+    ]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("q_t", "k_t", "v_t", "pq", "pk", "pv", "scores", "idx", "o_c", "total")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libvsa.so; raise if it is missing (no fallback path exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libvsa.so not found at {path}; build it with `python -m block_sparse_tiled_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, st = ctypes.c_void_p, ctypes.c_int
+    lib.vsa_last_error.restype = ctypes.c_char_p
+    lib.vsa_version.restype = ctypes.c_char_p
+    lib.vsa_plan_query.argtypes = [ctypes.POINTER(Geometry), ctypes.POINTER(PlanDims)]
+    lib.vsa_plan_tables_host.argtypes = [ctypes.POINTER(Geometry), P, P]
+    lib.vsa_plan_tiles.argtypes = [ctypes.POINTER(Geometry), P, ctypes.POINTER(P)]
+    lib.vsa_plan_info.argtypes = [P, ctypes.POINTER(PlanDims)]
+    lib.vsa_plan_tables.argtypes = [P, P, P]
+    lib.vsa_plan_workspace.argtypes = [P, ctypes.POINTER(WorkspaceLayout)]
+    lib.vsa_plan_destroy.argtypes = [P]
+    lib.vsa_gather_tiles.argtypes = [P] * 11
+    lib.vsa_pool_and_score.argtypes = [P] * 9
+    lib.vsa_topk_select.argtypes = [P] * 6
+    lib.vsa_sparse_attn_fwd.argtypes = [P] * 9
+    lib.vsa_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.vsa_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
+    for name in EXPORTED:
+        if name not in ("vsa_last_error", "vsa_version"):
+            getattr(lib, name).restype = st
+    _lib = lib
+    return lib
+
+
+def _check(rc: int, where: str):
+    if rc != VSA_OK:
+        raise VsaError(rc, where, load_library().vsa_last_error().decode())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
+                  token_tags=None, video_tag=0, tile_size=64):
+    """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers)."""
+    g = Geometry()
+    g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
+    keep = []
+    if token_tags is not None:
+        tags = (ctypes.c_int32 * len(token_tags))(*[int(t) for t in token_tags])
+        keep.append(tags)
+        g.token_tags = ctypes.cast(tags, ctypes.POINTER(ctypes.c_int32))
+        g.seq_len = len(token_tags)
+        g.video_tag = int(video_tag)
+        g.n_segments = 0
+    else:
+        seg = (ctypes.c_int32 * max(1, len(segments)))(*[int(s) for s in segments])
+        keep.append(seg)
+        g.segment_len = ctypes.cast(seg, ctypes.POINTER(ctypes.c_int32))
+        g.n_segments = len(segments)
+        g.seq_len = 0
+    g.grid_t, g.grid_h, g.grid_w = (int(x) for x in grid)
+    g.tile_size = int(tile_size)
+    g.sparsity = float(sparsity)
+    g.softmax_scale = float(softmax_scale)
+    return g, keep
+
+
+def vsa_plan_query(**kw) -> dict:
+    """Resolve sizes without touching a device."""
+    g, keep = make_geometry(**kw)
+    d = PlanDims()
+    _check(load_library().vsa_plan_query(ctypes.byref(g), ctypes.byref(d)), "vsa_plan_query")
+    return d.as_dict()
+
+
+def vsa_plan_tables_host(**kw):
+    """Host-only token table of a geometry: (tile_token [n_tiles, 64], tile_valid [n_tiles])."""
+    import numpy as np
+
+    d = vsa_plan_query(**kw)
+    g, keep = make_geometry(**kw)
+    n = d["n_tiles"]
+    tok = np.empty((max(n, 1), 64), np.int32)
+    val = np.empty((max(n, 1),), np.int32)
+    _check(load_library().vsa_plan_tables_host(ctypes.byref(g), tok.ctypes.data_as(ctypes.c_void_p),
+                                               val.ctypes.data_as(ctypes.c_void_p)), "vsa_plan_tables_host")
+    return tok[:n], val[:n]
+
+
+class Plan:
+    """Owns a ``vsa_plan`` handle (the device tile tables of one geometry)."""
+
+    def __init__(self, handle, geometry_kwargs):
+        self._h = handle
+        self.geometry = dict(geometry_kwargs)
+        d = PlanDims()
+        _check(load_library().vsa_plan_info(self._h, ctypes.byref(d)), "vsa_plan_info")
+        self.dims = d.as_dict()
+        ws = WorkspaceLayout()
+        _check(load_library().vsa_plan_workspace(self._h, ctypes.byref(ws)), "vsa_plan_workspace")
+        self.workspace_layout = {f: getattr(ws, f) for f, _ in WorkspaceLayout._fields_}
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise ValueError("plan destroyed")
+        return self._h
+
+    def tables(self):
+        import numpy as np
+
+        n = self.dims["n_tiles"]
+        tok = np.empty((max(n, 1), 64), np.int32)
+        val = np.empty((max(n, 1),), np.int32)
+        _check(load_library().vsa_plan_tables(self.handle, tok.ctypes.data_as(ctypes.c_void_p),
+                                              val.ctypes.data_as(ctypes.c_void_p)), "vsa_plan_tables")
+        return tok[:n], val[:n]
+
+    def destroy(self):
+        if self._h is not None:
+            load_library().vsa_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
+                   token_tags=None, video_tag=0, tile_size=64, stream=None) -> Plan:
+    kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
+              sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
+              tile_size=tile_size)
+    g, keep = make_geometry(**kw)
+    h = ctypes.c_void_p()
+    _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")
+    return Plan(h, kw)
+
+
+def vsa_gather_tiles(plan, q, k, v, q_t, k_t, v_t, pq=None, pk=None, pv=None, stream=None):
+    bf, f32 = torch.bfloat16, torch.float32
+    _check(load_library().vsa_gather_tiles(
+        plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(q_t, bf, "q_t"),
+        _ptr(k_t, bf, "k_t"), _ptr(v_t, bf, "v_t"), _ptr(pq, f32, "pq"), _ptr(pk, f32, "pk"), _ptr(pv, f32, "pv"),
+        _stream(stream)), "vsa_gather_tiles")
+
+
+def vsa_pool_and_score(plan, q_t, k_t, v_t, pq, pk, pv, scores, stream=None):
+    bf, f32 = torch.bfloat16, torch.float32
+    _check(load_library().vsa_pool_and_score(
+        plan.handle, _ptr(q_t, bf, "q_t"), _ptr(k_t, bf, "k_t"), _ptr(v_t, bf, "v_t"), _ptr(pq, f32, "pq"),
+        _ptr(pk, f32, "pk"), _ptr(pv, f32, "pv"), _ptr(scores, f32, "scores"), _stream(stream)),
+        "vsa_pool_and_score")
+
+
+def vsa_topk_select(plan, scores, pv, idx, o_c, stream=None):
+    f32 = torch.float32
+    _check(load_library().vsa_topk_select(
+        plan.handle, _ptr(scores, f32, "scores"), _ptr(pv, f32, "pv"), _ptr(idx, torch.int32, "idx"),
+        _ptr(o_c, f32, "o_c"), _stream(stream)), "vsa_topk_select")
+
+
+def vsa_sparse_attn_fwd(plan, q_t, k_t, v_t, idx, o_c, gate, out, stream=None):
+    bf = torch.bfloat16
+    _check(load_library().vsa_sparse_attn_fwd(
+        plan.handle, _ptr(q_t, bf, "q_t"), _ptr(k_t, bf, "k_t"), _ptr(v_t, bf, "v_t"),
+        _ptr(idx, torch.int32, "idx"), _ptr(o_c, torch.float32, "o_c"), _ptr(gate, bf, "gate"),
+        _ptr(out, bf, "out"), _stream(stream)), "vsa_sparse_attn_fwd")
+
+
+def alloc_workspace(plan, device=None) -> torch.Tensor:
+    """A uint8 device buffer of ``workspace_bytes`` (torch's allocator aligns to >= 256 bytes)."""
+    n = max(256, plan.dims["workspace_bytes"])
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda", torch.cuda.current_device()))
+
+
+def vsa_forward(plan, q, k, v, gate, out=None, workspace=None, stream=None):
+    """The whole forward.  CUDA inputs: runs in place on the stream.  CPU
+    inputs (ideally pinned): copied to the device, run, and the result copied
+    back into a CPU tensor, all on the stream."""
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, gate = (t.to(dev, non_blocking=True) for t in (q, k, v, gate))
+        host_out = out
+        out = torch.empty_like(q)
+    elif out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(plan, q.device)
+    bf = torch.bfloat16
+    _check(load_library().vsa_forward(
+        plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(gate, bf, "gate"),
+        _ptr(out, bf, "out"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "vsa_forward")
+    if host:
+        if host_out is None:
+            host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        host_out.copy_(out, non_blocking=True)
+        return host_out
+    return out
+
+
+def device_status(plan, stream=None):
+    code, where = ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().vsa_device_status(plan.handle, _stream(stream), ctypes.byref(code), ctypes.byref(where)),
+           "vsa_device_status")
+    return code.value, where.value
+
+
+def workspace_views(plan, workspace):
+    """Typed views of vsa_forward's intermediates inside ``workspace``."""
+    d, g = plan.dims, plan.geometry
+    B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
+    lay = plan.workspace_layout
+
+    def view(off, n, dtype, shape):
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return workspace[off:off + nbytes].view(dtype).view(*shape)
+
+    return {
+        "q_t": view(lay["q_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
+        "k_t": view(lay["k_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
+        "v_t": view(lay["v_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
+        "pq": view(lay["pq"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
+        "pk": view(lay["pk"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
+        "pv": view(lay["pv"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
+        "scores": view(lay["scores"], B * H * n_t * n_t, torch.float32, (B, H, n_t, n_t)),
+        "idx": view(lay["idx"], B * H * V * k, torch.int32, (B, H, V, k)),
+        "o_c": view(lay["o_c"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
+    }

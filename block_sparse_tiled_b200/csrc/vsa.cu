@@ -1,0 +1,583 @@
+// libvsa: C ABI of the VSA-H3 forward (declared in include/vsa.h).
+// Host side: tile plan, argument checks, workspace layout, TMA descriptors
+// and the launch sequence.  No allocation happens per call; a plan owns its
+// small device tables, the caller owns every tensor and workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attn_sm100.cuh"
+#include "prep_kernels.cuh"
+#include "vsa.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+vsa_status fail(vsa_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+#define VSA_CUDA_TRY(call)                                                                  \
+  do {                                                                                      \
+    cudaError_t e_ = (call);                                                                \
+    if (e_ != cudaSuccess) return fail(VSA_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+#define VSA_TRY(expr)                 \
+  do {                                \
+    vsa_status s_ = (expr);           \
+    if (s_ != VSA_OK) return s_;      \
+  } while (0)
+
+constexpr int kTile = VSA_TILE_SIZE;
+constexpr int kCube = 4;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The resolved problem: prefix segments, video grid and derived counts.
+struct Resolved {
+  std::vector<int64_t> segments;
+  int64_t T = 0, Hg = 0, W = 0;
+  int64_t L = 0;
+  int64_t n_prefix = 0, n_video = 0;
+  int32_t topk = 0;
+  float scale = 0.0f;
+};
+
+// topk = max(1, min(ceil((1 - sparsity) * V), V)), evaluated in binary64; 0 without video tiles.
+int32_t topk_for(double sparsity, int64_t V) {
+  if (V <= 0) return 0;
+  double k = std::ceil((1.0 - sparsity) * static_cast<double>(V));
+  if (k > static_cast<double>(V)) k = static_cast<double>(V);
+  if (k < 1.0) k = 1.0;
+  return static_cast<int32_t>(k);
+}
+
+vsa_status resolve(const vsa_geometry* g, Resolved* r) {
+  if (g == nullptr) return fail(VSA_ERR_INVALID_ARG, "geometry is NULL");
+  if (g->batch < 1 || g->heads < 1) return fail(VSA_ERR_INVALID_ARG, "batch and heads must be >= 1");
+  if (g->head_dim != 64 && g->head_dim != 128)
+    return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128, got " + std::to_string(g->head_dim));
+  if (g->tile_size != kTile)
+    return fail(VSA_ERR_UNSUPPORTED, "tile_size must be 64, got " + std::to_string(g->tile_size));
+  if (!(g->sparsity >= 0.0 && g->sparsity <= 1.0)) return fail(VSA_ERR_INVALID_ARG, "sparsity must lie in [0, 1]");
+  if (g->grid_t < 0 || g->grid_h < 0 || g->grid_w < 0) return fail(VSA_ERR_INVALID_ARG, "negative grid size");
+  const bool any_zero = g->grid_t == 0 || g->grid_h == 0 || g->grid_w == 0;
+  const bool all_zero = g->grid_t == 0 && g->grid_h == 0 && g->grid_w == 0;
+  if (any_zero && !all_zero) return fail(VSA_ERR_SHAPE, "grid sides must be all positive or all zero");
+  r->T = g->grid_t;
+  r->Hg = g->grid_h;
+  r->W = g->grid_w;
+  const int64_t n_video_tokens = r->T * r->Hg * r->W;
+
+  r->segments.clear();
+  if (g->token_tags != nullptr) {
+    if (g->seq_len <= 0) return fail(VSA_ERR_INVALID_ARG, "token_tags needs seq_len > 0");
+    // every maximal run of equal tags is one segment
+    std::vector<std::pair<int32_t, int64_t>> runs;
+    for (int64_t t = 0; t < g->seq_len; ++t) {
+      if (runs.empty() || runs.back().first != g->token_tags[t]) runs.push_back({g->token_tags[t], 0});
+      runs.back().second += 1;
+    }
+    size_t n_pre = runs.size();
+    if (n_video_tokens > 0) {
+      if (runs.back().first != g->video_tag || runs.back().second != n_video_tokens)
+        return fail(VSA_ERR_SHAPE, "the last tag run must be the video tokens (T*H*W of video_tag)");
+      n_pre -= 1;
+    }
+    for (size_t s = 0; s < n_pre; ++s) {
+      if (runs[s].first == g->video_tag) return fail(VSA_ERR_SHAPE, "video_tag appears before the last run");
+      r->segments.push_back(runs[s].second);
+    }
+  } else {
+    if (g->n_segments < 0) return fail(VSA_ERR_INVALID_ARG, "n_segments < 0");
+    if (g->n_segments > 0 && g->segment_len == nullptr) return fail(VSA_ERR_INVALID_ARG, "segment_len is NULL");
+    for (int s = 0; s < g->n_segments; ++s) {
+      if (g->segment_len[s] < 0) return fail(VSA_ERR_INVALID_ARG, "negative segment length");
+      r->segments.push_back(g->segment_len[s]);
+    }
+  }
+  int64_t prefix_tokens = 0;
+  r->n_prefix = 0;
+  for (int64_t n : r->segments) {
+    prefix_tokens += n;
+    r->n_prefix += (n + kTile - 1) / kTile;
+  }
+  r->L = prefix_tokens + n_video_tokens;
+  if (g->token_tags == nullptr && g->seq_len != 0 && g->seq_len != r->L)
+    return fail(VSA_ERR_SHAPE, "seq_len " + std::to_string(g->seq_len) + " != prefix + T*H*W = " +
+                                   std::to_string(r->L));
+  r->n_video = all_zero ? 0 : ((r->T + kCube - 1) / kCube) * ((r->Hg + kCube - 1) / kCube) *
+                                  ((r->W + kCube - 1) / kCube);
+  const int64_t n_t = r->n_prefix + r->n_video;
+  if (n_t > (1 << 24)) return fail(VSA_ERR_UNSUPPORTED, "too many tiles");
+  r->topk = topk_for(g->sparsity, r->n_video);
+  r->scale = (g->softmax_scale != 0.0f) ? g->softmax_scale
+                                        : static_cast<float>(1.0 / std::sqrt(static_cast<double>(g->head_dim)));
+  if (!(std::isfinite(r->scale)) || r->scale <= 0.0f) return fail(VSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  const int64_t rows = static_cast<int64_t>(g->batch) * g->heads * n_t * kTile;
+  if (rows >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "B*H*n_tiles*64 must stay below 2^31");
+  if (static_cast<int64_t>(g->batch) * g->heads > 65535 || g->heads > 65535)
+    return fail(VSA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
+  return VSA_OK;
+}
+
+// Token table of every tile (-1 = pad), valid rows first.
+void build_tables(const Resolved& r, std::vector<int32_t>* tok, std::vector<int32_t>* valid) {
+  const int64_t n_t = r.n_prefix + r.n_video;
+  tok->assign(static_cast<size_t>(n_t * kTile), -1);
+  valid->assign(static_cast<size_t>(n_t), 0);
+  int64_t tile = 0, base = 0;
+  for (int64_t n : r.segments) {
+    for (int64_t s = 0; s < n; s += kTile) {
+      const int64_t cnt = std::min<int64_t>(kTile, n - s);
+      for (int64_t j = 0; j < cnt; ++j) (*tok)[tile * kTile + j] = static_cast<int32_t>(base + s + j);
+      (*valid)[tile++] = static_cast<int32_t>(cnt);
+    }
+    base += n;
+  }
+  const int64_t ct = (r.T + 3) / 4, ch = (r.Hg + 3) / 4, cw = (r.W + 3) / 4;
+  for (int64_t a = 0; a < ct && r.n_video > 0; ++a)
+    for (int64_t bb = 0; bb < ch; ++bb)
+      for (int64_t c = 0; c < cw; ++c) {
+        int cnt = 0;
+        const int64_t t1 = std::min(r.T, 4 * a + 4), h1 = std::min(r.Hg, 4 * bb + 4), w1 = std::min(r.W, 4 * c + 4);
+        for (int64_t t = 4 * a; t < t1; ++t)
+          for (int64_t h = 4 * bb; h < h1; ++h)
+            for (int64_t w = 4 * c; w < w1; ++w)
+              (*tok)[tile * kTile + cnt++] = static_cast<int32_t>(base + (t * r.Hg + h) * r.W + w);
+        (*valid)[tile++] = cnt;
+      }
+}
+
+vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk) {
+  vsa_workspace_layout w{};
+  size_t off = 0;
+  const size_t tiles = static_cast<size_t>(B * H * n_t * kTile * D * 2);
+  const size_t pooled = static_cast<size_t>(B * H * n_t * D * 4);
+  w.q_t = off; off += align256(tiles);
+  w.k_t = off; off += align256(tiles);
+  w.v_t = off; off += align256(tiles);
+  w.pq = off; off += align256(pooled);
+  w.pk = off; off += align256(pooled);
+  w.pv = off; off += align256(pooled);
+  w.scores = off; off += align256(static_cast<size_t>(B * H * n_t * n_t * 4));
+  w.idx = off; off += align256(static_cast<size_t>(B * H * V * topk * 4));
+  w.o_c = off; off += align256(pooled);
+  w.total = off;
+  return w;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+vsa_status get_encoder(EncodeTiledFn* out) {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  static std::string err;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || p == nullptr)
+      err = "cuTensorMapEncodeTiled is not available from the driver";
+    else
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (fn == nullptr) return fail(VSA_ERR_CUDA, err);
+  *out = fn;
+  return VSA_OK;
+}
+
+// Tile-order tensor [rows, D] bf16 as a 2-D map with 64 x 64 boxes, 128-byte swizzle.
+vsa_status make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int D) {
+  EncodeTiledFn enc;
+  VSA_TRY(get_encoder(&enc));
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
+  return VSA_OK;
+}
+
+}  // namespace
+
+struct vsa_plan_s {
+  int device = 0;
+  int num_sms = 0;
+  size_t max_smem = 0;
+  int32_t B = 0, H = 0, D = 0;
+  Resolved r;
+  int32_t n_t = 0, P = 0, V = 0, topk = 0;
+  std::vector<int32_t> tile_token, tile_valid;
+  int32_t* d_tile_token = nullptr;
+  int32_t* d_tile_valid = nullptr;
+  int* d_status = nullptr;
+  vsa_workspace_layout ws{};
+};
+
+namespace {
+
+vsa_status check_plan(vsa_plan p) {
+  if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
+  int dev = -1;
+  VSA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != p->device) return fail(VSA_ERR_INVALID_ARG, "the current device is not the plan's device");
+  return VSA_OK;
+}
+
+vsa_status check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs) {
+    if (q == nullptr) return fail(VSA_ERR_INVALID_ARG, "a required device pointer is NULL");
+    if (!aligned16(q)) return fail(VSA_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  }
+  return VSA_OK;
+}
+
+vsa_status launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(VSA_ERR_CUDA, std::string(what) + " launch: " + cudaGetErrorString(e));
+  return VSA_OK;
+}
+
+template <typename K>
+vsa_status allow_smem(K kernel, size_t bytes) {
+  if (bytes > 48 * 1024)
+    VSA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+  return VSA_OK;
+}
+
+vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
+                      float* pk, float* pv, cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  const bool pool = pq != nullptr;
+  const size_t smem = pool ? static_cast<size_t>(3) * kTile * p->D * 2 : 0;
+  dim3 grid(p->n_t, p->H, p->B);
+  const auto* qq = static_cast<const uint16_t*>(q);
+  const auto* kk = static_cast<const uint16_t*>(k);
+  const auto* vv = static_cast<const uint16_t*>(v);
+  auto* qo = static_cast<uint16_t*>(qt);
+  auto* ko = static_cast<uint16_t*>(kt);
+  auto* vo = static_cast<uint16_t*>(vt);
+  if (p->D == 128) {
+    VSA_TRY(allow_smem(vsa::gather_pool_kernel<128>, smem));
+    vsa::gather_pool_kernel<128><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
+                                                         p->d_tile_valid, p->r.L, p->H, p->n_t);
+  } else {
+    VSA_TRY(allow_smem(vsa::gather_pool_kernel<64>, smem));
+    vsa::gather_pool_kernel<64><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
+                                                        p->d_tile_valid, p->r.L, p->H, p->n_t);
+  }
+  return launch_check("gather_pool");
+}
+
+vsa_status run_pool(vsa_plan p, const void* qt, const void* kt, const void* vt, float* pq, float* pk, float* pv,
+                    cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  dim3 grid(p->n_t, p->H, p->B);
+  const auto* a = static_cast<const uint16_t*>(qt);
+  const auto* b = static_cast<const uint16_t*>(kt);
+  const auto* c = static_cast<const uint16_t*>(vt);
+  if (p->D == 128)
+    vsa::pool_tiles_kernel<128><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
+  else
+    vsa::pool_tiles_kernel<64><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
+  return launch_check("pool_tiles");
+}
+
+vsa_status run_scores(vsa_plan p, const float* pq, const float* pk, float* S, cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  const int nb = (p->n_t + vsa::kScoreBlk - 1) / vsa::kScoreBlk;
+  dim3 grid(nb, nb, p->B * p->H);
+  vsa::scores_kernel<<<grid, 256, 0, s>>>(pq, pk, S, p->n_t, p->D, p->r.scale);
+  return launch_check("scores");
+}
+
+vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, float* o_c, cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  const int64_t BH = static_cast<int64_t>(p->B) * p->H;
+  if (p->V > 0 && p->topk > 0) {
+    const size_t row_bytes = static_cast<size_t>(p->V) * 4;
+    int rows = static_cast<int>(std::min<size_t>(8, std::max<size_t>(1, (200 * 1024) / row_bytes)));
+    const size_t smem = row_bytes * rows;
+    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "too many video tiles for the top-k kernel");
+    VSA_TRY(allow_smem(vsa::topk_kernel, smem));
+    const int64_t nrows = BH * p->V;
+    const int64_t blocks = (nrows + rows - 1) / rows;
+    if (blocks > 0x7fffffff) return fail(VSA_ERR_UNSUPPORTED, "top-k grid too large");
+    vsa::topk_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(S, idx, static_cast<int>(BH), p->n_t, p->P,
+                                                                     p->topk, rows);
+    VSA_TRY(launch_check("topk"));
+  }
+  dim3 grid((p->n_t + vsa::kCompRows - 1) / vsa::kCompRows, static_cast<unsigned>(BH));
+  if (p->D == 128)
+    vsa::compress_kernel<128><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
+  else
+    vsa::compress_kernel<64><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
+  return launch_check("compress");
+}
+
+vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
+                    const void* gate, void* out, cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
+  CUtensorMap mq, mk, mv;
+  VSA_TRY(make_tile_map(&mq, qt, rows, p->D));
+  VSA_TRY(make_tile_map(&mk, kt, rows, p->D));
+  VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
+  vsa::AttnArgs a{};
+  a.idx = idx;
+  a.tile_token = p->d_tile_token;
+  a.tile_valid = p->d_tile_valid;
+  a.o_c = o_c;
+  a.gate = static_cast<const uint16_t*>(gate);
+  a.out = static_cast<uint16_t*>(out);
+  a.status = p->d_status;
+  a.L = p->r.L;
+  a.H = p->H;
+  a.n_t = p->n_t;
+  a.P = p->P;
+  a.topk = p->topk;
+  a.scale_log2 = static_cast<float>(static_cast<double>(p->r.scale) * 1.4426950408889634);
+  a.n_items = static_cast<int64_t>(p->B) * p->H * p->n_t;
+  const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
+  if (p->D == 128) {
+    const size_t smem = vsa::AttnLayout<128>::bytes(p->n_t);
+    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
+    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<128>, smem));
+    vsa::vsa_attn_kernel<128><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
+  } else {
+    const size_t smem = vsa::AttnLayout<64>::bytes(p->n_t);
+    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
+    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<64>, smem));
+    vsa::vsa_attn_kernel<64><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
+  }
+  return launch_check("attention");
+}
+
+void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
+  d->n_tiles = static_cast<int32_t>(r.n_prefix + r.n_video);
+  d->n_prefix_tiles = static_cast<int32_t>(r.n_prefix);
+  d->n_video_tiles = static_cast<int32_t>(r.n_video);
+  d->topk = r.topk;
+  d->seq_len = r.L;
+  d->softmax_scale = r.scale;
+  d->workspace_bytes = make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk).total;
+  d->selected_pairs = r.n_video * (r.n_prefix + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vsa_last_error(void) { return g_last_error.c_str(); }
+
+const char* vsa_version(void) { return "vsa-b200 0.1 (sm_100a)"; }
+
+vsa_status vsa_plan_query(const vsa_geometry* g, vsa_plan_dims* out) {
+  if (out == nullptr) return fail(VSA_ERR_INVALID_ARG, "out is NULL");
+  Resolved r;
+  VSA_TRY(resolve(g, &r));
+  fill_dims(g, r, out);
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_tables_host(const vsa_geometry* g, int32_t* tile_token, int32_t* tile_valid) {
+  Resolved r;
+  VSA_TRY(resolve(g, &r));
+  std::vector<int32_t> tok, val;
+  build_tables(r, &tok, &val);
+  if (tile_token) std::memcpy(tile_token, tok.data(), tok.size() * 4);
+  if (tile_valid) std::memcpy(tile_valid, val.data(), val.size() * 4);
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
+  if (out == nullptr) return fail(VSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  Resolved r;
+  VSA_TRY(resolve(g, &r));
+  int dev = 0;
+  VSA_CUDA_TRY(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  VSA_CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(VSA_ERR_DEVICE, "libvsa is built for sm_100a; device " + std::to_string(dev) + " is sm_" +
+                                    std::to_string(prop.major) + std::to_string(prop.minor));
+  auto* p = new vsa_plan_s();
+  p->device = dev;
+  p->num_sms = prop.multiProcessorCount;
+  p->max_smem = prop.sharedMemPerBlockOptin;
+  p->B = g->batch;
+  p->H = g->heads;
+  p->D = g->head_dim;
+  p->r = r;
+  p->n_t = static_cast<int32_t>(r.n_prefix + r.n_video);
+  p->P = static_cast<int32_t>(r.n_prefix);
+  p->V = static_cast<int32_t>(r.n_video);
+  p->topk = r.topk;
+  build_tables(r, &p->tile_token, &p->tile_valid);
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk);
+  auto cleanup = [p] {
+    cudaFree(p->d_tile_token);
+    cudaFree(p->d_tile_valid);
+    cudaFree(p->d_status);
+    delete p;
+  };
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tok_bytes = std::max<size_t>(4, p->tile_token.size() * 4);
+  const size_t val_bytes = std::max<size_t>(4, p->tile_valid.size() * 4);
+  if (cudaMalloc(&p->d_tile_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_tile_valid, val_bytes) != cudaSuccess ||
+      cudaMalloc(&p->d_status, 2 * sizeof(int)) != cudaSuccess) {
+    cleanup();
+    return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
+  }
+  cudaError_t e = cudaSuccess;
+  if (!p->tile_token.empty())
+    e = cudaMemcpyAsync(p->d_tile_token, p->tile_token.data(), p->tile_token.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->tile_valid.empty())
+    e = cudaMemcpyAsync(p->d_tile_valid, p->tile_valid.data(), p->tile_valid.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 2 * sizeof(int), s);
+  if (e != cudaSuccess) {
+    cleanup();
+    return fail(VSA_ERR_CUDA, std::string("plan upload: ") + cudaGetErrorString(e));
+  }
+  *out = p;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_info(vsa_plan p, vsa_plan_dims* out) {
+  if (p == nullptr || out == nullptr) return fail(VSA_ERR_INVALID_ARG, "NULL argument");
+  out->n_tiles = p->n_t;
+  out->n_prefix_tiles = p->P;
+  out->n_video_tiles = p->V;
+  out->topk = p->topk;
+  out->seq_len = p->r.L;
+  out->softmax_scale = p->r.scale;
+  out->workspace_bytes = p->ws.total;
+  out->selected_pairs = static_cast<int64_t>(p->V) * (p->P + p->topk) + static_cast<int64_t>(p->P) * p->n_t;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_tables(vsa_plan p, int32_t* tile_token, int32_t* tile_valid) {
+  if (p == nullptr) return fail(VSA_ERR_INVALID_ARG, "plan is NULL");
+  if (tile_token) std::memcpy(tile_token, p->tile_token.data(), p->tile_token.size() * 4);
+  if (tile_valid) std::memcpy(tile_valid, p->tile_valid.data(), p->tile_valid.size() * 4);
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out) {
+  if (p == nullptr || out == nullptr) return fail(VSA_ERR_INVALID_ARG, "NULL argument");
+  *out = p->ws;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_destroy(vsa_plan p) {
+  if (p == nullptr) return VSA_OK;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->device);
+  cudaDeviceSynchronize();
+  cudaFree(p->d_tile_token);
+  cudaFree(p->d_tile_valid);
+  cudaFree(p->d_status);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete p;
+  return VSA_OK;
+}
+
+vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, vsa_bf16* q_t,
+                            vsa_bf16* k_t, vsa_bf16* v_t, float* pq, float* pk, float* pv, void* stream) {
+  VSA_TRY(check_plan(p));
+  VSA_TRY(check_ptrs({q, k, v, q_t, k_t, v_t}));
+  const int npool = (pq != nullptr) + (pk != nullptr) + (pv != nullptr);
+  if (npool != 0 && npool != 3) return fail(VSA_ERR_INVALID_ARG, "pq, pk, pv must be all NULL or all set");
+  if (npool == 3) VSA_TRY(check_ptrs({pq, pk, pv}));
+  return run_gather(p, q, k, v, q_t, k_t, v_t, pq, pk, pv, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k_t, const vsa_bf16* v_t, float* pq,
+                              float* pk, float* pv, float* scores, void* stream) {
+  VSA_TRY(check_plan(p));
+  VSA_TRY(check_ptrs({pq, pk, pv, scores}));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q_t != nullptr) {
+    VSA_TRY(check_ptrs({q_t, k_t, v_t}));
+    VSA_TRY(run_pool(p, q_t, k_t, v_t, pq, pk, pv, s));
+  }
+  return run_scores(p, pq, pk, scores, s);
+}
+
+vsa_status vsa_topk_select(vsa_plan p, const float* scores, const float* pv, int32_t* idx, float* o_c,
+                           void* stream) {
+  VSA_TRY(check_plan(p));
+  VSA_TRY(check_ptrs({scores, pv, o_c}));
+  if (p->V > 0) VSA_TRY(check_ptrs({idx}));
+  return run_topk(p, scores, pv, idx, o_c, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k_t, const vsa_bf16* v_t,
+                               const int32_t* idx, const float* o_c, const vsa_bf16* gate, vsa_bf16* out,
+                               void* stream) {
+  VSA_TRY(check_plan(p));
+  VSA_TRY(check_ptrs({q_t, k_t, v_t, o_c, gate, out}));
+  if (p->V > 0) VSA_TRY(check_ptrs({idx}));
+  return run_attn(p, q_t, k_t, v_t, idx, o_c, gate, out, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const vsa_bf16* gate,
+                       vsa_bf16* out, void* workspace, size_t workspace_bytes, void* stream) {
+  VSA_TRY(check_plan(p));
+  VSA_TRY(check_ptrs({q, k, v, gate, out, workspace}));
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < p->ws.total)
+    return fail(VSA_ERR_WORKSPACE, "workspace holds " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                       std::to_string(p->ws.total));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* w = static_cast<uint8_t*>(workspace);
+  auto* qt = w + p->ws.q_t;
+  auto* kt = w + p->ws.k_t;
+  auto* vt = w + p->ws.v_t;
+  auto* pq = reinterpret_cast<float*>(w + p->ws.pq);
+  auto* pk = reinterpret_cast<float*>(w + p->ws.pk);
+  auto* pv = reinterpret_cast<float*>(w + p->ws.pv);
+  auto* S = reinterpret_cast<float*>(w + p->ws.scores);
+  auto* idx = reinterpret_cast<int32_t*>(w + p->ws.idx);
+  auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
+  VSA_TRY(run_gather(p, q, k, v, qt, kt, vt, pq, pk, pv, s));
+  VSA_TRY(run_scores(p, pq, pk, S, s));
+  VSA_TRY(run_topk(p, S, pv, idx, oc, s));
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s);
+}
+
+vsa_status vsa_device_status(vsa_plan p, void* stream, int32_t* code, int32_t* where) {
+  VSA_TRY(check_plan(p));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  VSA_CUDA_TRY(cudaMemcpyAsync(h, p->d_status, sizeof h, cudaMemcpyDeviceToHost, s));
+  VSA_CUDA_TRY(cudaStreamSynchronize(s));
+  VSA_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof h, s));
+  VSA_CUDA_TRY(cudaStreamSynchronize(s));
+  if (code) *code = h[0];
+  if (where) *where = h[1];
+  return VSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+/*
+ * vsa.h -- C ABI of libvsa, the VSA-H3 Video Sparse Attention forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (the method as "Mike0021/FastH3-4step-Preview-VSA"
+ * states it in its section "Video Sparse Attention is not optional here"):
+ * the packed [text | cond | audio | video] sequence is cut into 64-token
+ * tiles -- segment-pure prefix tiles and (4,4,4) cubes of the post-patchify
+ * video grid; Q, K and V are pooled per tile; per-head fp32 pooled tile
+ * scores pick, for every video query tile, the top-k video key tiles with
+ *     topk = max(1, min(ceil((1 - sparsity) * n_video_tiles), n_video_tiles));
+ * prefix key tiles are always kept and prefix query tiles attend densely;
+ * block-sparse softmax attention runs over the kept tiles; and the
+ * compression branch softmax(scores) @ pool(V), broadcast over each tile's
+ * rows and scaled by the per-token gate (no activation), is added.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are CUDA device pointers; the caller owns every
+ *    tensor and every workspace and must keep them alive until the work on
+ *    `stream` has finished.  The library never frees caller memory and never
+ *    allocates device memory per call; a plan allocates its own small tables
+ *    once, in vsa_plan_tiles, and frees them in vsa_plan_destroy.
+ *  - bf16 tensors are raw IEEE bfloat16 bit patterns (vsa_bf16).  Every
+ *    device pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  All device work is asynchronous on it; no entry point but
+ *    vsa_device_status synchronises.
+ *  - Layouts (row-major, last index fastest):
+ *      sequence order : q, k, v, out  [B, L, H, D];  gate [B, L, H]
+ *      tile order     : q_t, k_t, v_t [B, H, n_tiles, 64, D]  (pad rows zero)
+ *      pooled         : pq, pk, pv    [B, H, n_tiles, D] float
+ *      scores         : [B, H, n_tiles, n_tiles] float
+ *      selection      : idx [B, H, n_video_tiles, topk] int32, global tile
+ *                       indices (prefix tiles are 0..P-1, video tiles P..),
+ *                       ascending in each row
+ *      compression    : o_c [B, H, n_tiles, D] float
+ *  - Tile geometry: prefix tiles in sequence order (a segment of n tokens
+ *    gives ceil(n/64) tiles, the last one partial); then the video cubes in
+ *    raster (t/4, h/4, w/4) order, edge cubes partial when a grid side is not
+ *    a multiple of 4.  Video tokens follow the prefix in raster (t, h, w)
+ *    order, w fastest.  Inside a tile the valid tokens come first, in
+ *    sequence (prefix) or raster (cube) order, then zero pads.
+ *  - Errors: argument and shape errors are detected on the host and returned
+ *    synchronously with nothing launched; a failed launch returns
+ *    VSA_ERR_CUDA; device-side failures (a bounded wait that ran out) are
+ *    recorded in the plan's device status word, read with vsa_device_status.
+ *    vsa_last_error() returns a message for the calling thread's last error.
+ *    There is no fallback path: an unsupported case is an error.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VSA_TILE_SIZE 64 /* tokens per tile; video tiles are 4x4x4 cubes */
+
+typedef uint16_t vsa_bf16; /* raw bfloat16 bits */
+
+typedef enum vsa_status {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1, /* NULL or misaligned pointer, value out of range */
+  VSA_ERR_SHAPE = 2,       /* inconsistent sizes */
+  VSA_ERR_UNSUPPORTED = 3, /* valid but not implemented (tile size, head_dim) */
+  VSA_ERR_WORKSPACE = 4,   /* workspace smaller than vsa_plan_dims.workspace_bytes */
+  VSA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  VSA_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out */
+  VSA_ERR_DEVICE = 7       /* no usable sm_100 device */
+} vsa_status;
+
+/* Problem statement.  Either `segment_len` (n_segments prefix segments in
+ * order, e.g. {text, cond, audio}; zero lengths allowed) or `token_tags`
+ * (seq_len tags, one per token; every maximal run of equal tags is one
+ * segment; the video run must be last and tagged `video_tag`) describes the
+ * prefix.  Host pointers; read only during vsa_plan_tiles. */
+typedef struct vsa_geometry {
+  int32_t batch;            /* B >= 1 */
+  int32_t heads;            /* H >= 1 */
+  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t n_segments;       /* number of prefix segments (ignored with tags) */
+  const int32_t* segment_len;
+  const int32_t* token_tags; /* NULL to use segment_len */
+  int64_t seq_len;           /* L: required with tags; checked otherwise */
+  int32_t video_tag;         /* tag value of the video tokens (tags only) */
+  int32_t grid_t, grid_h, grid_w; /* post-patchify video grid; 0 = no video */
+  int32_t tile_size;         /* must be 64 */
+  double sparsity;           /* in [0, 1] */
+  float softmax_scale;       /* 0 => (float)(1 / sqrt((double)head_dim)) */
+} vsa_geometry;
+
+typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
+
+/* Sizes a plan resolved. */
+typedef struct vsa_plan_dims {
+  int32_t n_tiles;        /* P + V */
+  int32_t n_prefix_tiles; /* P */
+  int32_t n_video_tiles;  /* V */
+  int32_t topk;           /* kept video key tiles per video query tile */
+  int64_t seq_len;        /* L */
+  float softmax_scale;    /* the scale actually used */
+  size_t workspace_bytes; /* device scratch vsa_forward needs */
+  int64_t selected_pairs; /* (query tile, key tile) pairs per (b, h):
+                             V * (P + topk) + P * n_tiles */
+} vsa_plan_dims;
+
+/* ---- S1: tile plan (host) ------------------------------------------------
+ * vsa_plan_tiles: resolve the tile geometry (segments -> segment-pure prefix
+ * tiles, grid -> (4,4,4) cubes, the topk count), build the token table of
+ * every tile and upload it to the current device, asynchronously on
+ * `stream`.  Allocates the plan's device tables (a few hundred KB at most)
+ * and its device status word.  On success *out owns them.
+ * Passage: "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
+ * Attention is not optional here" (tile geometry, topk formula); "FastH3
+ * NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse FP4 attention for
+ * VSA tiles" (partially filled tiles carry valid counts). */
+vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out);
+
+/* Resolved sizes.  Host only; never blocks. */
+vsa_status vsa_plan_info(vsa_plan p, vsa_plan_dims* out);
+
+/* Host copies of the plan's tables: tile_token[n_tiles * 64] (sequence index
+ * of each tile row, -1 for a pad) and tile_valid[n_tiles] (valid rows).
+ * Either pointer may be NULL.  Host only. */
+vsa_status vsa_plan_tables(vsa_plan p, int32_t* tile_token, int32_t* tile_valid);
+
+/* Resolve sizes without a device (no plan, no allocation). */
+vsa_status vsa_plan_query(const vsa_geometry* g, vsa_plan_dims* out);
+
+/* The token table a plan would upload, computed on the host without a device:
+ * tile_token[n_tiles * 64] and tile_valid[n_tiles] (caller-allocated host
+ * arrays, sized from vsa_plan_query).  Either pointer may be NULL. */
+vsa_status vsa_plan_tables_host(const vsa_geometry* g, int32_t* tile_token, int32_t* tile_valid);
+
+/* Free the plan's device tables (synchronises with the device first). */
+vsa_status vsa_plan_destroy(vsa_plan p);
+
+/* ---- S2: gather to tile order --------------------------------------------
+ * q_t/k_t/v_t[b,h,tile,r,:] = q/k/v[b, token(tile, r), h, :], pad rows zero.
+ * If pq, pk and pv are all non-NULL the pooled tiles (S3's first half) are
+ * written in the same pass, bit-identical to vsa_pool_and_score's.
+ * Passage: "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Model
+ * integration" (gather to tile order once; pad rows zero). */
+vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
+                            const vsa_bf16* v_dev, vsa_bf16* q_t_dev, vsa_bf16* k_t_dev,
+                            vsa_bf16* v_t_dev, float* pq_dev, float* pk_dev, float* pv_dev,
+                            void* stream);
+
+/* ---- S3: pooling and pooled tile scores ----------------------------------
+ * pooled[b,h,t,d] = (sum over the tile's valid rows r, in tile order, from
+ * +0.0f, one binary32 rounding per add) / n_valid  (IEEE division);
+ * scores[b,h,i,j] = fl(fmaf chain over d = 0..D-1 of pq[i,d]*pk[j,d], from
+ * +0.0f) * softmax_scale.  Every (i, j) pair, prefix tiles included.
+ * Inputs in tile order.  If q_t_dev is NULL the pooling is skipped and pq/pk
+ * must already hold pooled tiles (e.g. from vsa_gather_tiles).
+ * Passage: "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
+ * Attention is not optional here" (per-head fp32 pooled tile scores). */
+vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf16* k_t_dev,
+                              const vsa_bf16* v_t_dev, float* pq_dev, float* pk_dev,
+                              float* pv_dev, float* scores_dev, void* stream);
+
+/* ---- S4: top-k selection and the compression branch ---------------------
+ * idx[b,h,iv,:] = the topk video key tiles with the highest scores[b,h,P+iv,
+ * P+j] (ties: lower index first), as global indices in ascending order;
+ * o_c[b,h,i,:] = sum_j softmax_j(scores[b,h,i,:]) * pv[b,h,j,:] over all
+ * n_tiles tiles, in binary32.
+ * Passage: "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
+ * Attention is not optional here" (top-k; compression softmax(scores) @
+ * pool(v)); "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse
+ * FP4 attention for VSA tiles" (per-query-block index lists). */
+vsa_status vsa_topk_select(vsa_plan p, const float* scores_dev, const float* pv_dev,
+                           int32_t* idx_dev, float* o_c_dev, void* stream);
+
+/* ---- S5: block-sparse attention and the gated epilogue -------------------
+ * For a video query tile: softmax attention over the keys of all prefix
+ * tiles and of its idx row; for a prefix query tile: over every tile.  Pad
+ * keys are masked.  Then out[b,l,h,:] = o_fine + gate[b,l,h] * o_c[b,h,
+ * tile(l),:], rounded to bf16 and written in sequence order (pad rows are not
+ * written).  Q/K/V in tile order; BF16 tensor-core products with fp32
+ * accumulation; P rounded to bf16 before the P.V product.
+ * Passage: "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse FP4
+ * attention for VSA tiles" (block lists, exempt prefix key tile visited
+ * first); "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
+ * Attention is not optional here" (dense prefix queries; gated compression
+ * branch with no activation). */
+vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf16* k_t_dev,
+                               const vsa_bf16* v_t_dev, const int32_t* idx_dev,
+                               const float* o_c_dev, const vsa_bf16* gate_dev,
+                               vsa_bf16* out_dev, void* stream);
+
+/* ---- the whole forward ---------------------------------------------------
+ * S2..S5 in one call, sequence order in and out.  `workspace_dev` must hold
+ * vsa_plan_dims.workspace_bytes bytes (256-byte aligned); its contents on
+ * entry do not matter and on return are the intermediates (tile-order Q/K/V,
+ * pooled tiles, scores, idx, o_c) at offsets vsa_workspace_layout gives. */
+vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
+                       const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
+                       void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Byte offsets of the intermediates inside vsa_forward's workspace. */
+typedef struct vsa_workspace_layout {
+  size_t q_t, k_t, v_t, pq, pk, pv, scores, idx, o_c, total;
+} vsa_workspace_layout;
+vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
+
+/* Read (synchronising `stream`) and clear the plan's device status word.
+ * *code receives VSA_OK or VSA_ERR_TIMEOUT; *where a kernel-specific site
+ * code (0 if none). */
+vsa_status vsa_device_status(vsa_plan p, void* stream, int32_t* code, int32_t* where);
+
+/* Message for the calling thread's most recent error ("" if none). */
+const char* vsa_last_error(void);
+
+/* Library version string. */
+const char* vsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

@@ -58,6 +58,7 @@ def _load():
         lib.vsa_oracle_select.argtypes = [P, i32, i32, i32, i32, P]
         lib.vsa_oracle_compress.argtypes = [P, P, i32, i32, i32, P]
         lib.vsa_oracle_fine.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
+        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, i32, P, P]
         lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P]
         lib.vsa_oracle_output.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P, P, P]
         _lib = lib
@@ -165,6 +166,49 @@ def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None) -> np.
     _load().vsa_oracle_fine(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
                             _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(todo), _p(out))
     return out
+
+
+def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items) -> np.ndarray:
+    """Fine branch of the listed query tiles only.  items: int64 array of
+    (b*H + h)*n_t + i.  Returns [n_items, 64, D] float64 in tile row order
+    (pad rows 0)."""
+    q, k, v = (_c(t, np.uint16) for t in (q, k, v))
+    B, L, H, D = q.shape
+    idx = _c(idx, np.int32)
+    items = _c(np.asarray(items, np.int64), np.int64)
+    out = np.zeros((len(items), 64, D), np.float64)
+    _load().vsa_oracle_fine_tiles(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+                                  _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), len(items),
+                                  _p(items), _p(out))
+    return out
+
+
+def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarray:
+    """out rows of the listed tiles: o_f + gate * o_c[tile] (tile row order; pad rows 0)."""
+    gate = _c(gate, np.uint16)
+    gf = (gate.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    res = np.zeros_like(o_f_tiles)
+    for n, bhi in enumerate(np.asarray(items, np.int64)):
+        i = int(bhi % geo.n_tiles)
+        bh = int(bhi // geo.n_tiles)
+        h, b = bh % H, bh // H
+        nv = int(geo.tile_valid[i])
+        toks = geo.tile_token[i, :nv]
+        res[n, :nv] = o_f_tiles[n, :nv] + gf[b, toks, h][:, None] * o_c[b, h, i][None, :]
+    return res
+
+
+def selection(q, k, v, segments, grid, sparsity, scale=None):
+    """Pool, scores, top-k and compression only (every tile, every head)."""
+    geo = geometry(segments, grid)
+    if scale is None:
+        scale = default_scale(q.shape[-1])
+    kc = topk_count(sparsity, geo.n_video)
+    pq, pk, pv = pool(q, geo), pool(k, geo), pool(v, geo)
+    S = scores(pq, pk, scale)
+    idx = select(S, geo.n_prefix, kc)
+    o_c = compress(S, pv)
+    return dict(geo=geo, topk=kc, scale=scale, pq=pq, pk=pk, pv=pv, S=S, idx=idx, o_c=o_c)
 
 
 def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndarray:

@@ -274,64 +274,98 @@ static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t
     return P + k;
 }
 
-/* o_f[b, tok, h, :] for every valid query token tok of every (b, h, i) with
- * todo[(b*H + h)*n_t + i] != 0 (todo == NULL: all).  For a query row r:
+/* Fine branch of one query tile (b, h, i): for each valid query row r,
  *   logit_c = scale * <q_r, k_c> over the valid key rows c of its key set,
- *   o_f = sum_c softmax(logit)_c * v_c.
+ *   o_f[r] = sum_c softmax(logit)_c * v_c,
+ * written to rows[r * D + d] in tile row order (pad rows left untouched). */
+static void fine_one_tile(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int b, int h, int i,
+                          int64_t L, int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                          const int32_t *tile_valid, const int32_t *idx, double scale, double *rows) {
+    int V = n_t - P;
+    int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
+    const int32_t *idx_row = (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
+    int nk = key_set(i, n_t, P, k, idx_row, keys);
+    /* every valid key row of the key set, in list order */
+    int64_t max_rows = (int64_t)nk * TILE;
+    int64_t *ktok = (int64_t *)malloc(sizeof(int64_t) * (size_t)max_rows);
+    double *logit = (double *)malloc(sizeof(double) * (size_t)max_rows);
+    int64_t nrows = 0;
+    for (int t = 0; t < nk; ++t)
+        for (int c = 0; c < tile_valid[keys[t]]; ++c)
+            ktok[nrows++] = tile_token[(int64_t)keys[t] * TILE + c];
+
+    for (int r = 0; r < tile_valid[i]; ++r) {
+        int64_t qt = tile_token[(int64_t)i * TILE + r];
+        const uint16_t *qr = q + (((int64_t)b * L + qt) * H + h) * D;
+        double m = -INFINITY;
+        for (int64_t c = 0; c < nrows; ++c) {
+            const uint16_t *kc = kk + (((int64_t)b * L + ktok[c]) * H + h) * D;
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d)
+                dot += (double)bf16_to_float(qr[d]) * (double)bf16_to_float(kc[d]);
+            logit[c] = scale * dot;
+            if (logit[c] > m) m = logit[c];
+        }
+        double denom = 0.0;
+        for (int64_t c = 0; c < nrows; ++c) {
+            logit[c] = exp(logit[c] - m);
+            denom += logit[c];
+        }
+        double *o = rows + (int64_t)r * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (int64_t c = 0; c < nrows; ++c) {
+            const uint16_t *vc = v + (((int64_t)b * L + ktok[c]) * H + h) * D;
+            double w = logit[c] / denom;
+            for (int d = 0; d < D; ++d) o[d] += w * (double)bf16_to_float(vc[d]);
+        }
+    }
+    free(logit);
+    free(ktok);
+    free(keys);
+}
+
+/* o_f[b, tok, h, :] for every valid query token tok of every (b, h, i) with
+ * todo[(b*H + h)*n_t + i] != 0 (todo == NULL: all).
  * q, k, v: [B, L, H, D] bf16 bits; idx: [B, H, V, k] global tile indices. */
 void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B, int64_t L,
                      int H, int D, int n_t, int P, int k, const int32_t *tile_token,
                      const int32_t *tile_valid, const int32_t *idx, double scale,
                      const uint8_t *todo, double *o_f) {
-    int V = n_t - P;
 #pragma omp parallel for collapse(3) schedule(dynamic, 1)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h)
             for (int i = 0; i < n_t; ++i) {
                 int64_t bhi = ((int64_t)b * H + h) * n_t + i;
                 if (todo && !todo[bhi]) continue;
-                int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
-                const int32_t *idx_row =
-                    (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
-                int nk = key_set(i, n_t, P, k, idx_row, keys);
-                /* every valid key row of the key set, in list order */
-                int64_t max_rows = (int64_t)nk * TILE;
-                int64_t *ktok = (int64_t *)malloc(sizeof(int64_t) * (size_t)max_rows);
-                double *logit = (double *)malloc(sizeof(double) * (size_t)max_rows);
-                int64_t nrows = 0;
-                for (int t = 0; t < nk; ++t)
-                    for (int c = 0; c < tile_valid[keys[t]]; ++c)
-                        ktok[nrows++] = tile_token[(int64_t)keys[t] * TILE + c];
-
+                double *rows = (double *)malloc(sizeof(double) * (size_t)TILE * (size_t)D);
+                fine_one_tile(q, kk, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale,
+                              rows);
                 for (int r = 0; r < tile_valid[i]; ++r) {
-                    int64_t qt = tile_token[(int64_t)i * TILE + r];
-                    const uint16_t *qr = q + (((int64_t)b * L + qt) * H + h) * D;
-                    double m = -INFINITY;
-                    for (int64_t c = 0; c < nrows; ++c) {
-                        const uint16_t *kc = kk + (((int64_t)b * L + ktok[c]) * H + h) * D;
-                        double dot = 0.0;
-                        for (int d = 0; d < D; ++d)
-                            dot += (double)bf16_to_float(qr[d]) * (double)bf16_to_float(kc[d]);
-                        logit[c] = scale * dot;
-                        if (logit[c] > m) m = logit[c];
-                    }
-                    double denom = 0.0;
-                    for (int64_t c = 0; c < nrows; ++c) {
-                        logit[c] = exp(logit[c] - m);
-                        denom += logit[c];
-                    }
-                    double *o = o_f + (((int64_t)b * L + qt) * H + h) * D;
-                    for (int d = 0; d < D; ++d) o[d] = 0.0;
-                    for (int64_t c = 0; c < nrows; ++c) {
-                        const uint16_t *vc = v + (((int64_t)b * L + ktok[c]) * H + h) * D;
-                        double w = logit[c] / denom;
-                        for (int d = 0; d < D; ++d) o[d] += w * (double)bf16_to_float(vc[d]);
-                    }
+                    int64_t tok = tile_token[(int64_t)i * TILE + r];
+                    memcpy(o_f + (((int64_t)b * L + tok) * H + h) * D, rows + (int64_t)r * D,
+                           sizeof(double) * (size_t)D);
                 }
-                free(logit);
-                free(ktok);
-                free(keys);
+                free(rows);
             }
+}
+
+/* The fine branch of selected query tiles only: items[n] = (b*H + h)*n_t + i;
+ * out[n, r, :] for the tile's rows r in tile order (pad rows set to 0). */
+void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B, int64_t L,
+                           int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                           const int32_t *tile_valid, const int32_t *idx, double scale, int n_items,
+                           const int64_t *items, double *out) {
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < n_items; ++n) {
+        int64_t bhi = items[n];
+        int i = (int)(bhi % n_t);
+        int64_t bh = bhi / n_t;
+        int h = (int)(bh % H), b = (int)(bh / H);
+        double *rows = out + (int64_t)n * TILE * D;
+        for (int64_t e = 0; e < (int64_t)TILE * D; ++e) rows[e] = 0.0;
+        fine_one_tile(q, kk, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale, rows);
+    }
 }
 
 /* ------------------------------------------------------------------ */

@@ -1,0 +1,133 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the
+header declares, and its host-side plan (tile geometry, token tables, topk,
+argument checks) agrees with the oracle's independent tiling."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def vsa():
+    from block_sparse_tiled_b200 import build
+
+    build.build()
+    import block_sparse_tiled_b200 as m
+
+    m.load_library()
+    return m
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "vsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(vsa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(vsa):
+    names = declared_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(vsa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(vsa.EXPORTED)
+    dyn = subprocess.run(["nm", "-D", "--defined-only", vsa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (vsa_\w+)", dyn))
+    assert set(names) <= exported
+    assert vsa.load_library().vsa_version().decode().startswith("vsa-b200")
+
+
+def _kw(w, **over):
+    kw = dict(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
+              sparsity=w.sparsity)
+    kw.update(over)
+    return kw
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_plan_matches_oracle_geometry(vsa, oracle_mod, name):
+    w = synth.workload(name)
+    d = vsa.vsa_plan_query(**_kw(w))
+    geo = oracle_mod.geometry(w.segments, w.grid)
+    assert (d["n_tiles"], d["n_prefix_tiles"], d["n_video_tiles"]) == (geo.n_tiles, geo.n_prefix, geo.n_video)
+    assert d["topk"] == oracle_mod.topk_count(w.sparsity, geo.n_video)
+    assert d["seq_len"] == w.seq_len
+    assert d["softmax_scale"] == np.float32(oracle_mod.default_scale(w.head_dim))
+    P, V, k, n = geo.n_prefix, geo.n_video, d["topk"], geo.n_tiles
+    assert d["selected_pairs"] == V * (P + k) + P * n
+    if name in ("tiny", "small", "480p"):
+        tok, val = vsa.vsa_plan_tables_host(**_kw(w))
+        assert np.array_equal(tok, geo.tile_token)
+        assert np.array_equal(val, geo.tile_valid)
+
+
+@pytest.mark.parametrize("segments,grid", [
+    ((), (4, 4, 4)), ((1,), (1, 1, 1)), ((0, 0, 130), (3, 5, 7)), ((64, 64), (0, 0, 0)),
+    ((17,), (9, 2, 13)), ((0,), (4, 8, 4)),
+])
+def test_plan_edge_geometries(vsa, oracle_mod, segments, grid):
+    kw = dict(batch=2, heads=3, head_dim=64, segments=segments, grid=grid, sparsity=0.7)
+    d = vsa.vsa_plan_query(**kw)
+    geo = oracle_mod.geometry(segments, grid)
+    assert (d["n_tiles"], d["n_prefix_tiles"], d["n_video_tiles"]) == (geo.n_tiles, geo.n_prefix, geo.n_video)
+    tok, val = vsa.vsa_plan_tables_host(**kw)
+    assert np.array_equal(tok, geo.tile_token) and np.array_equal(val, geo.tile_valid)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.8, 0.9, 0.95, 1.0])
+def test_plan_topk_sweep(vsa, oracle_mod, s):
+    w = synth.workload("768p_s0.9")
+    assert vsa.vsa_plan_query(**_kw(w, sparsity=s))["topk"] == oracle_mod.topk_count(s, 1152)
+
+
+def test_token_tags_match_segments(vsa):
+    # text 40, cond 0 (absent), audio 24, then 8x8x8 video tagged 9
+    tags = [1] * 40 + [3] * 24 + [9] * 512
+    a = vsa.vsa_plan_query(batch=1, heads=2, head_dim=64, token_tags=tags, video_tag=9, grid=(8, 8, 8), sparsity=0.5)
+    b = vsa.vsa_plan_query(batch=1, heads=2, head_dim=64, segments=(40, 24), grid=(8, 8, 8), sparsity=0.5)
+    assert a == b
+    # interleaved runs of one tag are separate segments
+    tags2 = [1] * 10 + [2] * 10 + [1] * 10 + [9] * 64
+    t2, _ = vsa.vsa_plan_tables_host(batch=1, heads=1, head_dim=64, token_tags=tags2, video_tag=9, grid=(4, 4, 4))
+    assert t2.shape[0] == 4
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(sparsity=1.5), "VSA_ERR_INVALID_ARG"),
+    (dict(sparsity=-0.1), "VSA_ERR_INVALID_ARG"),
+    (dict(sparsity=float("nan")), "VSA_ERR_INVALID_ARG"),
+    (dict(tile_size=128), "VSA_ERR_UNSUPPORTED"),
+    (dict(head_dim=96), "VSA_ERR_UNSUPPORTED"),
+    (dict(grid=(8, 0, 8)), "VSA_ERR_SHAPE"),
+    (dict(batch=0), "VSA_ERR_INVALID_ARG"),
+    (dict(segments=(-1,)), "VSA_ERR_INVALID_ARG"),
+])
+def test_plan_rejects_bad_arguments(vsa, over, status):
+    w = synth.workload("tiny")
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_plan_query(**_kw(w, **over))
+    assert vsa.STATUS_NAMES[e.value.status] == status
+    assert vsa.load_library().vsa_last_error().decode() != ""
+
+
+def test_token_tags_video_not_last(vsa):
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_plan_query(batch=1, heads=1, head_dim=64, token_tags=[9] * 64 + [1] * 3, video_tag=9,
+                           grid=(4, 4, 4))
+    assert vsa.STATUS_NAMES[e.value.status] == "VSA_ERR_SHAPE"
+
+
+def test_workspace_size(vsa):
+    w = synth.workload("768p_s0.9")
+    d = vsa.vsa_plan_query(**_kw(w))
+    n_t, D, H = 1172, 128, 56
+    tiles = H * n_t * 64 * D * 2
+    assert d["workspace_bytes"] >= 3 * tiles + 4 * H * n_t * D * 4 + H * n_t * n_t * 4 + H * 1152 * 116 * 4
+    assert d["workspace_bytes"] < 3 * tiles * 1.2

@@ -1,0 +1,228 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded bytes.
+
+Bar: tile-order gather, pooled Q/K/V and pooled scores bit-exact; tile
+selection bit-exact; compression within 1e-5 relative; the BF16 output within
+max-abs 2e-2 and mean-abs 2e-3 of the float64 oracle.  Small workloads are
+compared in full; the 480p- and 1344x768-shaped workloads compare the whole
+selection and a fixed sample of query tiles of the attention.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def vsa():
+    from block_sparse_tiled_b200 import build
+
+    build.build()
+    import block_sparse_tiled_b200 as m
+
+    m.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(0)
+    return m
+
+
+def bits(t):
+    return synth.as_bits(t)
+
+
+def plan_for(vsa, w):
+    return vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
+                              sparsity=w.sparsity)
+
+
+def run_forward(vsa, w, x):
+    plan = plan_for(vsa, w)
+    ws = vsa.alloc_workspace(plan)
+    out = vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], workspace=ws)
+    torch.cuda.synchronize()
+    assert vsa.device_status(plan) == (0, 0)
+    return plan, ws, out
+
+
+def run_stepwise(vsa, plan, x):
+    """S2..S5 through the separate entry points, pooling from tile order."""
+    d, g = plan.dims, plan.geometry
+    B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
+    dev = x["q"].device
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    t = {n: torch.empty(B, H, n_t, 64, D, **bf) for n in ("q_t", "k_t", "v_t")}
+    vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], t["q_t"], t["k_t"], t["v_t"])
+    pq, pk, pv = (torch.empty(B, H, n_t, D, **f32) for _ in range(3))
+    S = torch.empty(B, H, n_t, n_t, **f32)
+    vsa.vsa_pool_and_score(plan, t["q_t"], t["k_t"], t["v_t"], pq, pk, pv, S)
+    idx = torch.empty(B, H, max(V, 1), max(k, 1), dtype=torch.int32, device=dev)
+    o_c = torch.empty(B, H, n_t, D, **f32)
+    vsa.vsa_topk_select(plan, S, pv, idx, o_c)
+    out = torch.empty_like(x["q"])
+    vsa.vsa_sparse_attn_fwd(plan, t["q_t"], t["k_t"], t["v_t"], idx, o_c, x["gate"], out)
+    torch.cuda.synchronize()
+    return dict(t, pq=pq, pk=pk, pv=pv, S=S, idx=idx[:, :, :V, :k], o_c=o_c, out=out)
+
+
+def expected_tiles(xbits, geo):
+    """Tile-order copy of a [B, L, H, D] array, built from the oracle's token table."""
+    B, L, H, D = xbits.shape
+    tok = geo.tile_token
+    res = np.zeros((B, H, geo.n_tiles, 64, D), np.uint16)
+    valid = tok >= 0
+    for b in range(B):
+        src = xbits[b].transpose(1, 0, 2)  # [H, L, D]
+        res[b][:, valid] = src[:, tok[valid]]
+    return res
+
+
+def compare_out(gpu_out, ref_out, mask=None):
+    g = gpu_out.float().cpu().numpy().astype(np.float64)
+    if mask is not None:
+        g, ref_out = g[mask], ref_out[mask]
+    err = np.abs(g - ref_out)
+    assert np.isfinite(g).all()
+    assert err.max() <= MAX_ABS, f"max-abs {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"mean-abs {err.mean():.3e}"
+    return err.max(), err.mean()
+
+
+def full_parity(vsa, oracle_mod, w, seed=0):
+    x = synth.make_inputs(w, seed=seed, device="cuda")
+    xb = {n: bits(x[n]) for n in ("q", "k", "v", "gate")}
+    ref = oracle_mod.forward(xb["q"], xb["k"], xb["v"], xb["gate"], w.segments, w.grid, w.sparsity)
+    plan, ws, out = run_forward(vsa, w, x)
+    views = vsa.workspace_views(plan, ws)
+    step = run_stepwise(vsa, plan, x)
+    for n in ("q", "k", "v"):
+        exp = expected_tiles(xb[n], ref.geo)
+        assert np.array_equal(bits(views[n + "_t"]), exp), n
+        assert np.array_equal(bits(step[n + "_t"]), exp), n
+    for n in ("pq", "pk", "pv"):
+        r = getattr(ref, n)
+        assert np.array_equal(views[n].cpu().numpy(), r), n
+        assert np.array_equal(step[n].cpu().numpy(), r), n
+    assert np.array_equal(views["scores"].cpu().numpy(), ref.S)
+    assert np.array_equal(step["S"].cpu().numpy(), ref.S)
+    assert np.array_equal(views["idx"].cpu().numpy(), ref.idx)
+    assert np.array_equal(step["idx"].cpu().numpy(), ref.idx)
+    for oc in (views["o_c"], step["o_c"]):
+        g = oc.cpu().numpy().astype(np.float64)
+        assert np.abs(g - ref.o_c).max() <= 1e-5 * max(1.0, np.abs(ref.o_c).max())
+    compare_out(out, ref.out)
+    # both routes run the same kernels on the same intermediates
+    assert torch.equal(out, step["out"])
+    plan.destroy()
+    return ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_full_parity(vsa, oracle_mod, name):
+    full_parity(vsa, oracle_mod, synth.workload(name))
+
+
+def test_tiny_sparsity0_is_dense_attention(vsa, oracle_mod):
+    """At sparsity 0 the fine branch is dense softmax attention over the packed
+    sequence; check the GPU against torch SDPA (float64) plus the gate term."""
+    w = synth.workload("tiny", sparsity=0.0)
+    ref = full_parity(vsa, oracle_mod, w)
+    x = synth.make_inputs(w, device="cuda")
+    plan, ws, out = run_forward(vsa, w, x)
+    q, k, v = (x[n].double()[0].transpose(0, 1) for n in ("q", "k", "v"))  # [H, L, D]
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=ref.scale).transpose(0, 1)
+    comp = ref.out - ref.o_f  # gate * o_c, per row
+    expect = dense.cpu().numpy()[None] + comp
+    compare_out(out, expect)
+
+
+@pytest.mark.parametrize("segments,grid,sparsity,B,H,D", [
+    ((), (8, 8, 8), 0.5, 1, 2, 64),               # no prefix
+    ((100, 30), (0, 0, 0), 0.9, 1, 2, 128),       # prefix only: every query tile dense
+    ((10,), (3, 2, 5), 0.5, 1, 3, 128),           # grid sides below 4: one partial cube
+    ((40, 0, 24), (8, 8, 8), 1.0, 1, 2, 64),      # topk = 1
+    ((40, 0, 24), (8, 8, 8), 0.0, 2, 2, 128),     # topk = V, batch 2
+    ((70, 0, 5), (5, 6, 7), 0.6, 2, 3, 128),      # ragged everywhere
+    ((1,), (4, 4, 4), 0.0, 1, 1, 64),             # one-token prefix tile, one cube
+    ((64, 64, 64), (4, 8, 12), 0.75, 1, 4, 128),  # even count of key tiles
+    ((33,), (4, 4, 12), 0.5, 1, 2, 128),          # odd count of key tiles: half-masked last block
+])
+def test_edge_cases(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
+    w = synth.Workload("edge", B, H, D, tuple(segments), tuple(grid), sparsity)
+    full_parity(vsa, oracle_mod, w, seed=3)
+
+
+def sampled_parity(vsa, oracle_mod, w, heads, video_every):
+    x = synth.make_inputs(w, seed=0, device="cuda")
+    plan, ws, out = run_forward(vsa, w, x)
+    views = vsa.workspace_views(plan, ws)
+    xb = {n: bits(x[n]) for n in ("q", "k", "v", "gate")}
+    sel = oracle_mod.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity)
+    geo = sel["geo"]
+    assert np.array_equal(views["pq"].cpu().numpy(), sel["pq"])
+    assert np.array_equal(views["pk"].cpu().numpy(), sel["pk"])
+    assert np.array_equal(views["scores"].cpu().numpy(), sel["S"])
+    assert np.array_equal(views["idx"].cpu().numpy(), sel["idx"])
+    g = views["o_c"].cpu().numpy().astype(np.float64)
+    assert np.abs(g - sel["o_c"]).max() <= 1e-5 * max(1.0, np.abs(sel["o_c"]).max())
+    tiles = [0, geo.n_prefix - 1] + list(range(geo.n_prefix, geo.n_tiles, video_every)) + [geo.n_tiles - 1]
+    items = np.array([h * geo.n_tiles + i for h in heads for i in sorted(set(tiles))], np.int64)
+    of = oracle_mod.fine_tiles(xb["q"], xb["k"], xb["v"], geo, sel["idx"], sel["topk"], sel["scale"], items)
+    ref = oracle_mod.output_tiles(of, sel["o_c"], xb["gate"], geo, items, w.heads)
+    got = np.zeros_like(ref)
+    o = out[0]  # [L, H, D]
+    for n, bhi in enumerate(items):
+        i, h = int(bhi % geo.n_tiles), int(bhi // geo.n_tiles)
+        nv = int(geo.tile_valid[i])
+        got[n, :nv] = o[torch.from_numpy(geo.tile_token[i, :nv].astype(np.int64)).cuda(), h].double().cpu().numpy()
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    plan.destroy()
+
+
+def test_480p_selection_full_attention_sampled(vsa, oracle_mod):
+    sampled_parity(vsa, oracle_mod, synth.workload("480p"), heads=[0, 27, 55], video_every=19)
+
+
+def test_768p_s09_selection_full_attention_sampled(vsa, oracle_mod):
+    """The 1344x768-shaped workload at sparsity 0.9, in the launch configuration the bench times."""
+    sampled_parity(vsa, oracle_mod, synth.workload("768p_s0.9"), heads=[0, 31, 55], video_every=131)
+
+
+def test_repeatable_and_status_clean(vsa):
+    w = synth.workload("small")
+    x = synth.make_inputs(w, device="cuda")
+    plan, ws, out1 = run_forward(vsa, w, x)
+    out2 = vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+    assert vsa.device_status(plan) == (0, 0)
+
+
+def test_call_errors(vsa):
+    w = synth.workload("tiny")
+    x = synth.make_inputs(w, device="cuda")
+    plan = plan_for(vsa, w)
+    ws = vsa.alloc_workspace(plan)
+    out = torch.empty_like(x["q"])
+    lib = vsa.load_library()
+    import ctypes
+
+    def call(q_ptr, ws_ptr, ws_bytes):
+        return lib.vsa_forward(plan.handle, q_ptr, ctypes.c_void_p(x["k"].data_ptr()),
+                               ctypes.c_void_p(x["v"].data_ptr()), ctypes.c_void_p(x["gate"].data_ptr()),
+                               ctypes.c_void_p(out.data_ptr()), ws_ptr, ws_bytes, None)
+
+    qp = x["q"].data_ptr()
+    wsp = ctypes.c_void_p(ws.data_ptr())
+    assert call(ctypes.c_void_p(qp + 2), wsp, ws.numel()) == 1  # misaligned -> VSA_ERR_INVALID_ARG
+    assert call(None, wsp, ws.numel()) == 1  # NULL -> VSA_ERR_INVALID_ARG
+    assert call(ctypes.c_void_p(qp), wsp, plan.dims["workspace_bytes"] - 256) == 4  # VSA_ERR_WORKSPACE
+    assert call(ctypes.c_void_p(qp), ctypes.c_void_p(ws.data_ptr() + 16), ws.numel() - 16) == 1  # unaligned ws
+    assert call(ctypes.c_void_p(qp), wsp, ws.numel()) == 0
+    torch.cuda.synchronize()
