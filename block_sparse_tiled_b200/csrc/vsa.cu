@@ -256,9 +256,11 @@ vsa_status launch_check(const char* what) {
   return VSA_OK;
 }
 
+// Opt in to `bytes` of dynamic shared memory (static shared memory counts
+// against the same default 48 KB, so the attribute is always set).
 template <typename K>
 vsa_status allow_smem(K kernel, size_t bytes) {
-  if (bytes > 48 * 1024)
+  if (bytes > 0)
     VSA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
   return VSA_OK;
 }
