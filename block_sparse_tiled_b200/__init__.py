@@ -35,6 +35,7 @@ EXPORTED = (
     "vsa_plan_tiles", "vsa_plan_info", "vsa_plan_tables", "vsa_plan_query", "vsa_plan_tables_host",
     "vsa_plan_destroy",
     "vsa_gather_tiles", "vsa_pool_and_score", "vsa_topk_select", "vsa_sparse_attn_fwd", "vsa_forward",
+    "vsa_forward_noalloc",
     "vsa_plan_workspace", "vsa_device_status", "vsa_last_error", "vsa_version",
 )
 
@@ -97,6 +98,7 @@ def load_library(path: str = LIB_PATH):
     lib.vsa_topk_select.argtypes = [P] * 6
     lib.vsa_sparse_attn_fwd.argtypes = [P] * 9
     lib.vsa_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.vsa_forward_noalloc.argtypes = [P] * 7
     lib.vsa_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED:
         if name not in ("vsa_last_error", "vsa_version"):
@@ -293,6 +295,20 @@ def vsa_forward(plan, q, k, v, gate, out=None, workspace=None, stream=None):
             host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         host_out.copy_(out, non_blocking=True)
         return host_out
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def vsa_forward_noalloc(plan, q, k, v, gate, out, stream=None):
+    """The whole forward with the library's static device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory).  Calls
+    on one device share that scratch: do not let them overlap on the GPU."""
+    bf = torch.bfloat16
+    _check(load_library().vsa_forward_noalloc(
+        plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(gate, bf, "gate"),
+        _ptr(out, bf, "out"), _stream(stream)), "vsa_forward_noalloc")
     return out
 
 

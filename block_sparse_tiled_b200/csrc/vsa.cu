@@ -218,6 +218,34 @@ vsa_status make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int D) 
 
 }  // namespace
 
+// Scratch of vsa_forward_noalloc: one array per device, alive until the
+// process exits, shared by every call on that device.  Host code never uses
+// its name as an address; the device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[VSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on `device` (the current device).
+vsa_status noalloc_scratch_address(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return fail(VSA_ERR_DEVICE, "device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[device] == nullptr) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess || addr == nullptr)
+      return fail(VSA_ERR_CUDA, std::string("cudaGetSymbolAddress of the no-alloc scratch: ") + cudaGetErrorString(e));
+    g_noalloc_addr[device] = addr;
+  }
+  *out = g_noalloc_addr[device];
+  return VSA_OK;
+}
+
+}  // namespace
+
 struct vsa_plan_s {
   int device = 0;
   int num_sms = 0;
@@ -567,6 +595,18 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const v
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s));
   return run_attn(p, qt, kt, vt, idx, oc, gate, out, s);
+}
+
+vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                               const vsa_bf16* gate, vsa_bf16* out, void* stream) {
+  VSA_TRY(check_plan(p));
+  if (p->ws.total > VSA_NOALLOC_SCRATCH_BYTES)
+    return fail(VSA_ERR_WORKSPACE, "vsa_forward_noalloc: this geometry needs " + std::to_string(p->ws.total) +
+                                       " bytes of scratch; the static scratch array holds " +
+                                       std::to_string(VSA_NOALLOC_SCRATCH_BYTES) + " bytes (use vsa_forward)");
+  void* scratch = nullptr;
+  VSA_TRY(noalloc_scratch_address(p->device, &scratch));
+  return vsa_forward(p, q, k, v, gate, out, scratch, VSA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 vsa_status vsa_device_status(vsa_plan p, void* stream, int32_t* code, int32_t* where) {

@@ -200,6 +200,31 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                        const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
                        void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* ---- the whole forward without a caller workspace -------------------------
+ * No counterpart on the pages: this entry point exists for callers that
+ * cannot allocate device memory on their call path -- for instance a plugin
+ * running inside a host engine that owns all device memory, or a serving loop
+ * whose memory budget is fixed after start-up -- and so cannot hand
+ * vsa_forward a workspace.  It runs exactly vsa_forward's kernels, with the
+ * scratch held in one file-scope device array of VSA_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) that every GPU which loads libvsa keeps until the process exits.
+ * The caller still passes the inputs and the output.  It allocates nothing:
+ * no cudaMalloc, cudaFree or allocating library routine.
+ *  - A plan whose vsa_plan_dims.workspace_bytes exceeds the array is
+ *    rejected with VSA_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture on the device.
+ *  - Every call on a device uses the same array: calls whose work may
+ *    overlap on the GPU (different streams, or several threads) race and
+ *    must be serialised by the caller.  Nothing in the array needs to start
+ *    at zero; each call overwrites what it reads.
+ * On return the array holds the call's intermediates (not exposed). */
+#define VSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
+                               const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
+                               void* stream);
+
 /* Byte offsets of the intermediates inside vsa_forward's workspace. */
 typedef struct vsa_workspace_layout {
   size_t q_t, k_t, v_t, pq, pk, pv, scores, idx, o_c, total;
