@@ -18,9 +18,18 @@
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
 // D = 64 uses the same M = 128 PV product with a zero upper half of V^T.
 //
-// Roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner + MMA
-// issuer (one thread), warps 2..5 = softmax + epilogue (TMEM lane quadrant =
-// warp % 4).  Every mbarrier wait is bounded; after a timeout the kernel
+// Roles (384 threads, 12 warps):
+//   warp 0  K producer: TMA for the query tile of each item and the K tiles
+//           of each block (4 lanes issue the four 8 KB boxes in parallel),
+//           plus the block's key-valid counts for the softmax;
+//   warp 1  V producer: TMA for the V tiles of each block;
+//   warp 2  S^T issuer (one thread) and TMEM owner;
+//   warp 3  P.V issuer (one thread);
+//   warps 4..11  softmax + epilogue, two groups of four warps; group g owns
+//           query columns [32g, 32g + 32), warp w reads TMEM lane quadrant w % 4.
+// Two issuing threads keep two tcgen05 streams in flight (one thread alone is
+// limited by its issue latency), and several issuing lanes keep enough TMA
+// loads in flight.  Every mbarrier wait is bounded; after a timeout the kernel
 // stops issuing work, finishes its loops without waiting, drains what it
 // issued and returns with the status word set.
 #pragma once
@@ -33,7 +42,7 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-max threshold: exponents stay <= 2^8
 constexpr uint32_t kTmemCols = 256;   // S^T double buffer (2 x 64) + O^T (64), rounded to a power of 2
 
@@ -53,35 +62,44 @@ struct AttnArgs {
 
 template <int D>
 struct AttnLayout {
-  static constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along D
-  static constexpr int kQBytes = 64 * D * 2;      // one query tile
-  static constexpr int kKVBytes = 128 * D * 2;    // 128 keys of K (or of V)
-  static constexpr int kHalfBytes = 128 * 128;    // one 64-column half of a 128-row block
-  static constexpr int kPBytes = 128 * 64 * 2;    // P^T of one block
-  static constexpr int kStages = 2;
+  static constexpr int kHalves = D / 64;        // 128-byte swizzle atoms along D
+  static constexpr int kQBytes = 64 * D * 2;    // one query tile
+  static constexpr int kKVBytes = 128 * D * 2;  // 128 keys of K (or of V)
+  static constexpr int kHalfBytes = 128 * 128;  // one 64-column half of a 128-row block
+  static constexpr int kPBytes = 128 * 64 * 2;  // P^T of one block
+  static constexpr int kQBufs = 2;
+  static constexpr int kKStages = 2;
+  static constexpr int kVStages = 2;
+  static constexpr int kMeta = 8;  // per-block key-valid counts in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
   static constexpr int oQ = 0;
-  static constexpr int oK = oQ + 2 * kQBytes;
-  static constexpr int oV = oK + kStages * kKVBytes;
-  static constexpr int oP = oV + kStages * kKVBytes;
+  static constexpr int oK = oQ + kQBufs * kQBytes;
+  static constexpr int oV = oK + kKStages * kKVBytes;
+  static constexpr int oP = oV + kVStages * kKVBytes;
   static constexpr int oZ = oP + 2 * kPBytes;
   static constexpr int oBar = oZ + kZeroBytes;
-  // barriers (8 bytes each)
-  enum {
-    bQFull = 0, bQEmpty = 2, bKFull = 4, bVFull = 6, bKVEmpty = 8, bSFull = 10, bSEmpty = 12,
-    bPFull = 14, bPEmpty = 16, bOFull = 18, bOEmpty = 19, bDone = 20, kNumBars = 21
-  };
-  static constexpr int oMisc = oBar + kNumBars * 8;             // tmem base, abort flag
-  static constexpr int oM = ((oMisc + 8 + 15) / 16) * 16;       // float m[64]
-  static constexpr int oAlpha = oM + 256;                       // float alpha[64]
-  static constexpr int oRed = oAlpha + 256;                     // float red[4][64]
-  static constexpr int oLsum = oRed + 1024;                     // float lsum[64]
-  static constexpr int oGate = oLsum + 256;                     // float gate[64]
-  static constexpr int oQtok = oGate + 256;                     // int qtok[64]
-  static constexpr int oTileValid = oQtok + 256;                // uint8 [n_t]
+  // barrier indices (8 bytes each)
+  static constexpr int bQFull = 0, bQEmpty = bQFull + kQBufs;
+  static constexpr int bKFull = bQEmpty + kQBufs, bKEmpty = bKFull + kKStages;
+  static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
+  static constexpr int bSFull = bVEmpty + kVStages, bSEmpty = bSFull + 2;
+  static constexpr int bPFull = bSEmpty + 2, bPEmpty = bPFull + 2;
+  static constexpr int bMFull = bPEmpty + 2, bMEmpty = bMFull + kMeta;
+  static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 1;
+  static constexpr int bDoneS = bOEmpty + 1, bDonePV = bDoneS + 1;
+  static constexpr int kNumBars = bDonePV + 1;
+  static constexpr int oMisc = oBar + kNumBars * 8;          // tmem base, abort flag
+  static constexpr int oMeta = ((oMisc + 8 + 15) / 16) * 16;  // int2 meta[kMeta]
+  static constexpr int oM = oMeta + kMeta * 8;               // float m[64]
+  static constexpr int oAlpha = oM + 256;                    // float alpha[64]
+  static constexpr int oRed = oAlpha + 256;                  // float red[2 groups][4 quadrants][32]
+  static constexpr int oRl = oRed + 1024;                    // float 1 / l[64]
+  static constexpr int oGate = oRl + 256;                    // float gate[64]
+  static constexpr int oQtok = oGate + 256;                  // int qtok[64]
+  static constexpr int oTileValid = oQtok + 256;             // uint8 [n_t]
   static size_t bytes(int n_t) {
     const size_t tv = ((static_cast<size_t>(n_t) + 15) / 16) * 16;
-    return 1024 /*alignment slack*/ + oTileValid + 2 * tv;
+    return 1024 /*alignment slack*/ + oTileValid + tv;
   }
 };
 
@@ -90,23 +108,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// In-warp reduce-scatter of 64 per-lane columns: afterwards v[0], v[1] hold the
-// reduction over the warp's 32 lanes for columns 2*lane and 2*lane + 1.  The
-// input array is consumed.
-template <bool kMax>
-__device__ __forceinline__ void warp_reduce_scatter64(float* v, int lane) {
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// In-warp reduce-scatter (sum) of 32 per-lane columns: afterwards v[0] holds the
+// sum over the warp's 32 lanes of column `lane`.  The input array is consumed.
+__device__ __forceinline__ void warp_sum_scatter32(float* v, int lane) {
 #pragma unroll
   for (int step = 0; step < 5; ++step) {
-    const int half = 32 >> step;      // 32, 16, 8, 4, 2
-    const int bit = 4 - step;         // lane bit that picks the kept half
+    const int half = 16 >> step;  // 16, 8, 4, 2, 1
+    const int bit = 4 - step;     // lane bit that picks the kept half
     const bool upper = (lane >> bit) & 1;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
       const float lo = v[i], hi = v[i + half];
       const float send = upper ? lo : hi;
       const float keep = upper ? hi : lo;
-      const float recv = __shfl_xor_sync(0xffffffffu, send, 1 << bit);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << bit);
     }
   }
 }
@@ -127,14 +148,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::oBar);
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::oMisc + 4);
+  int2* meta_s = reinterpret_cast<int2*>(sm + Ly::oMeta);
   float* m_s = reinterpret_cast<float*>(sm + Ly::oM);
   float* alpha_s = reinterpret_cast<float*>(sm + Ly::oAlpha);
   float* red_s = reinterpret_cast<float*>(sm + Ly::oRed);
-  float* lsum_s = reinterpret_cast<float*>(sm + Ly::oLsum);
+  float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
   float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
   int32_t* qtok_s = reinterpret_cast<int32_t*>(sm + Ly::oQtok);
   uint8_t* tile_valid_s = sm + Ly::oTileValid;
-  uint8_t* kvalid_s = tile_valid_s + ((a.n_t + 15) / 16) * 16;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = a.n_t, P = a.P, topk = a.topk, V = n_t - P;
@@ -149,20 +170,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Ly::kQBufs; ++s) {
       mbar_init(&bars[Ly::bQFull + s], 1);
       mbar_init(&bars[Ly::bQEmpty + s], 1);
+    }
+    for (int s = 0; s < Ly::kKStages; ++s) {
       mbar_init(&bars[Ly::bKFull + s], 1);
+      mbar_init(&bars[Ly::bKEmpty + s], 1);
+    }
+    for (int s = 0; s < Ly::kVStages; ++s) {
       mbar_init(&bars[Ly::bVFull + s], 1);
-      mbar_init(&bars[Ly::bKVEmpty + s], 1);
+      mbar_init(&bars[Ly::bVEmpty + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[Ly::bSFull + s], 1);
-      mbar_init(&bars[Ly::bSEmpty + s], 4);
-      mbar_init(&bars[Ly::bPFull + s], 4);
+      mbar_init(&bars[Ly::bSEmpty + s], 8);
+      mbar_init(&bars[Ly::bPFull + s], 8);
       mbar_init(&bars[Ly::bPEmpty + s], 1);
     }
+    for (int s = 0; s < Ly::kMeta; ++s) {
+      mbar_init(&bars[Ly::bMFull + s], 1);
+      mbar_init(&bars[Ly::bMEmpty + s], 8);
+    }
     mbar_init(&bars[Ly::bOFull], 1);
-    mbar_init(&bars[Ly::bOEmpty], 4);
-    mbar_init(&bars[Ly::bDone], 1);
+    mbar_init(&bars[Ly::bOEmpty], 8);
+    mbar_init(&bars[Ly::bDoneS], 1);
+    mbar_init(&bars[Ly::bDonePV], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -170,7 +203,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc(tmem_base_s, kTmemCols);
     tmem_relinquish();
   }
@@ -185,8 +218,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return __ldg(a.idx + (bh * V + (i - P)) * topk + (t - P));
   };
 
-  if (warp == 0) {
-    // ============================================================ TMA producer
+  if (warp <= 1) {
+    // ============================================================ TMA producers (warp 0: Q + K, warp 1: V)
+    const bool is_k = (warp == 0);
+    const int nstages = is_k ? Ly::kKStages : Ly::kVStages;
+    const int b_full = is_k ? Ly::bKFull : Ly::bVFull;
+    const int b_empty = is_k ? Ly::bKEmpty : Ly::bVEmpty;
+    uint8_t* ring = sm + (is_k ? Ly::oK : Ly::oV);
+    const void* tmap = is_k ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
@@ -194,133 +233,163 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int nk = list_len(i), nb = (nk + 1) / 2;
-      if (lane == 0) {
-        const int qb = it & 1;
-        ok = mbar_wait(&bars[Ly::bQEmpty + qb], ((it >> 1) & 1) ^ 1, ctl, 1);
-        if (ok) {
-          mbar_arrive_expect_tx(&bars[Ly::bQFull + qb], Ly::kQBytes);
+      if (is_k) {
+        // the query tile of this item (loaded by the K warp, which runs ahead with the S^T issuer)
+        const int qb = it % Ly::kQBufs;
+        const uint32_t qu = it / Ly::kQBufs;
+        if (lane == 0) {
+          ok = mbar_wait(&bars[Ly::bQEmpty + qb], (qu & 1) ^ 1, ctl, 1);
+          if (ok) mbar_arrive_expect_tx(&bars[Ly::bQFull + qb], Ly::kQBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok && lane < Ly::kHalves) {
           const int row = static_cast<int>((bh * n_t + i) * 64);
-          for (int hh = 0; hh < Ly::kHalves; ++hh)
-            tma_load_2d(sm + Ly::oQ + qb * Ly::kQBytes + hh * 8192, &tm_q, &bars[Ly::bQFull + qb], hh * 64, row);
+          tma_load_2d(sm + Ly::oQ + qb * Ly::kQBytes + lane * 8192, &tm_q, &bars[Ly::bQFull + qb], lane * 64, row);
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       for (int n0 = 0; n0 < nb && ok; n0 += 32) {
         const int n = n0 + lane;
-        int ta = 0, tb = 0;
+        int ta = 0, tb = -1;
         if (n < nb) {
           ta = key_tile(bh, i, 2 * n);
-          tb = (2 * n + 1 < nk) ? key_tile(bh, i, 2 * n + 1) : ta;
+          tb = (2 * n + 1 < nk) ? key_tile(bh, i, 2 * n + 1) : -1;
         }
         const int cnt = min(32, nb - n0);
-        for (int j = 0; j < cnt; ++j) {
+        for (int j = 0; j < cnt; ++j, ++g) {
           const int ka = __shfl_sync(0xffffffffu, ta, j);
-          const int kb = __shfl_sync(0xffffffffu, tb, j);
-          if (lane == 0 && ok) {
-            const int st = g & 1;
-            const uint32_t u = g >> 1;
-            ok = mbar_wait(&bars[Ly::bKVEmpty + st], (u & 1) ^ 1, ctl, 2);
-            if (ok) {
-              const int ra = static_cast<int>((bh * n_t + ka) * 64);
-              const int rb = static_cast<int>((bh * n_t + kb) * 64);
-              uint8_t* kdst = sm + Ly::oK + st * Ly::kKVBytes;
-              uint8_t* vdst = sm + Ly::oV + st * Ly::kKVBytes;
-              mbar_arrive_expect_tx(&bars[Ly::bKFull + st], Ly::kKVBytes);
-              for (int hh = 0; hh < Ly::kHalves; ++hh) {
-                tma_load_2d(kdst + hh * Ly::kHalfBytes, &tm_k, &bars[Ly::bKFull + st], hh * 64, ra);
-                tma_load_2d(kdst + hh * Ly::kHalfBytes + 8192, &tm_k, &bars[Ly::bKFull + st], hh * 64, rb);
-              }
-              mbar_arrive_expect_tx(&bars[Ly::bVFull + st], Ly::kKVBytes);
-              for (int hh = 0; hh < Ly::kHalves; ++hh) {
-                tma_load_2d(vdst + hh * Ly::kHalfBytes, &tm_v, &bars[Ly::bVFull + st], hh * 64, ra);
-                tma_load_2d(vdst + hh * Ly::kHalfBytes + 8192, &tm_v, &bars[Ly::bVFull + st], hh * 64, rb);
+          const int kb_raw = __shfl_sync(0xffffffffu, tb, j);
+          const int kb = kb_raw < 0 ? ka : kb_raw;  // an odd list repeats its last tile; the softmax masks it
+          const int st = g % nstages;
+          const uint32_t u = g / nstages;
+          if (lane == 0) {
+            ok = mbar_wait(&bars[b_empty + st], (u & 1) ^ 1, ctl, is_k ? 2 : 3);
+            if (ok) mbar_arrive_expect_tx(&bars[b_full + st], Ly::kKVBytes);
+            if (ok && is_k) {
+              // the block's key-valid counts, for the softmax
+              const int ms = g % Ly::kMeta;
+              ok = mbar_wait(&bars[Ly::bMEmpty + ms], ((g / Ly::kMeta) & 1) ^ 1, ctl, 4);
+              if (ok) {
+                meta_s[ms] = make_int2(tile_valid_s[ka], kb_raw < 0 ? 0 : tile_valid_s[kb_raw]);
+                mbar_arrive(&bars[Ly::bMFull + ms]);
               }
             }
           }
-          ++g;
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
+          // lanes [0, 2*kHalves) issue one 8 KB box each: (half, tile a|b)
+          if (lane < 2 * Ly::kHalves) {
+            const int hh = lane >> 1, second = lane & 1;
+            const int row = static_cast<int>((bh * n_t + (second ? kb : ka)) * 64);
+            tma_load_2d(ring + st * Ly::kKVBytes + hh * Ly::kHalfBytes + second * 8192, tmap, &bars[b_full + st],
+                        hh * 64, row);
+          }
+          __syncwarp();
         }
       }
     }
-    // drain: every load issued must have landed before the CTA may exit
+    // drain: every load this warp issued must land before the CTA exits
     if (lane == 0) {
-      for (int s = 0; s < 2; ++s) {
-        if (g > static_cast<uint32_t>(s)) {
-          const uint32_t last = (g - 1 - s) >> 1;  // last use of stage ((g - 1 - s) & 1)
-          const int st = (g - 1 - s) & 1;
-          wait_slow(&bars[Ly::bKFull + st], last & 1, WaitCtl{abort_flag, a.status}, 3);
-          wait_slow(&bars[Ly::bVFull + st], last & 1, WaitCtl{abort_flag, a.status}, 3);
+      const WaitCtl drain{abort_flag, a.status};
+      for (int s = 0; s < nstages && static_cast<uint32_t>(s) < g; ++s) {
+        const uint32_t last = g - 1 - s;
+        wait_slow(&bars[b_full + (last % nstages)], (last / nstages) & 1, drain, 20);
+      }
+      if (is_k && it > 0) {
+        for (int s = 0; s < Ly::kQBufs && s < it; ++s) {
+          const int lastq = it - 1 - s;
+          wait_slow(&bars[Ly::bQFull + (lastq % Ly::kQBufs)], (lastq / Ly::kQBufs) & 1, drain, 21);
         }
       }
     }
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
+    __syncwarp();
+  } else if (warp == 2) {
+    // ============================================================ S^T issuer
     if (lane == 0) {
       uint32_t g = 0;
       int it = 0;
       bool ok = true;
-      auto issue_pv = [&](uint32_t gp, bool first) -> bool {
-        const int st = gp & 1;
-        const uint32_t u = gp >> 1;
-        if (!mbar_wait(&bars[Ly::bVFull + st], u & 1, ctl, 4)) return false;
-        if (!mbar_wait(&bars[Ly::bPFull + st], u & 1, ctl, 5)) return false;
-        if (first && !mbar_wait(&bars[Ly::bOEmpty], (it & 1) ^ 1, ctl, 6)) return false;
-        tc_fence_after();
-        const uint32_t vbase = smem_u32(sm + Ly::oV + st * Ly::kKVBytes);
-        const uint32_t pbase = smem_u32(sm + Ly::oP + st * Ly::kPBytes);
-        // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
-        const uint32_t lbo_v = (D == 128) ? Ly::kHalfBytes
-                                          : static_cast<uint32_t>(Ly::oZ - (Ly::oV + st * Ly::kKVBytes));
-#pragma unroll
-        for (int kk = 0; kk < kPVSteps; ++kk) {
-          const uint64_t ad = umma_desc_sw128(vbase + kk * 2048, lbo_v, 1024);
-          const uint64_t bd = umma_desc_sw128(pbase + kk * 2048, 8192, 1024);
-          umma_ss(tmem + 128, ad, bd, kIdescPV, (!first || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars[Ly::bKVEmpty + st]);
-        umma_commit(&bars[Ly::bPEmpty + st]);
-        return true;
-      };
       for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
         const int nb = (list_len(i) + 1) / 2;
-        const int qb = it & 1;
-        ok = mbar_wait(&bars[Ly::bQFull + qb], (it >> 1) & 1, ctl, 7);
+        const int qb = it % Ly::kQBufs;
+        ok = mbar_wait(&bars[Ly::bQFull + qb], (it / Ly::kQBufs) & 1, ctl, 5);
         const uint32_t qbase = smem_u32(sm + Ly::oQ + qb * Ly::kQBytes);
         for (int n = 0; n < nb && ok; ++n, ++g) {
-          const int st = g & 1;
-          const uint32_t u = g >> 1;
-          ok = mbar_wait(&bars[Ly::bKFull + st], u & 1, ctl, 8) &&
-               mbar_wait(&bars[Ly::bSEmpty + st], (u & 1) ^ 1, ctl, 9);
+          const int kst = g % Ly::kKStages;
+          const int sb = g & 1;
+          ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6) &&
+               mbar_wait(&bars[Ly::bSEmpty + sb], ((g >> 1) & 1) ^ 1, ctl, 7);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sm + Ly::oK + st * Ly::kKVBytes);
+          const uint32_t kbase = smem_u32(sm + Ly::oK + kst * Ly::kKVBytes);
 #pragma unroll
           for (int kk = 0; kk < kQKSteps; ++kk) {
             const uint64_t ad = umma_desc_sw128(kbase + (kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = umma_desc_sw128(qbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-            umma_ss(tmem + st * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&bars[Ly::bSFull + st]);
+          umma_commit(&bars[Ly::bKEmpty + kst]);
+          umma_commit(&bars[Ly::bSFull + sb]);
           if (n == nb - 1) umma_commit(&bars[Ly::bQEmpty + qb]);
-          if (n > 0) ok = issue_pv(g - 1, n == 1);
         }
-        if (ok) ok = issue_pv(g - 1, nb == 1);
-        if (ok) umma_commit(&bars[Ly::bOFull]);
       }
-      // drain: all issued tcgen05 work completes before TMEM is released
-      umma_commit(&bars[Ly::bDone]);
-      wait_slow(&bars[Ly::bDone], 0, WaitCtl{abort_flag, a.status}, 10);
+      umma_commit(&bars[Ly::bDoneS]);
+      wait_slow(&bars[Ly::bDoneS], 0, WaitCtl{abort_flag, a.status}, 22);
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ============================================================ P.V issuer
+    if (lane == 0) {
+      uint32_t g = 0;
+      int it = 0;
+      bool ok = true;
+      for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
+        const int64_t bh = w / n_t;
+        const int i = static_cast<int>(w - bh * n_t);
+        const int nb = (list_len(i) + 1) / 2;
+        for (int n = 0; n < nb && ok; ++n, ++g) {
+          const int vst = g % Ly::kVStages;
+          const int pb = g & 1;
+          ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8) &&
+               mbar_wait(&bars[Ly::bPFull + pb], (g >> 1) & 1, ctl, 9) &&
+               (n > 0 || mbar_wait(&bars[Ly::bOEmpty], (it & 1) ^ 1, ctl, 10));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vbase = smem_u32(sm + Ly::oV + vst * Ly::kKVBytes);
+          const uint32_t pbase = smem_u32(sm + Ly::oP + pb * Ly::kPBytes);
+          // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
+          const uint32_t lbo_v = (D == 128) ? Ly::kHalfBytes
+                                            : static_cast<uint32_t>(Ly::oZ - (Ly::oV + vst * Ly::kKVBytes));
+#pragma unroll
+          for (int kk = 0; kk < kPVSteps; ++kk) {
+            const uint64_t ad = umma_desc_sw128(vbase + kk * 2048, lbo_v, 1024);
+            const uint64_t bd = umma_desc_sw128(pbase + kk * 2048, 8192, 1024);
+            umma_ss(tmem + 128, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars[Ly::bVEmpty + vst]);
+          umma_commit(&bars[Ly::bPEmpty + pb]);
+          if (n == nb - 1) umma_commit(&bars[Ly::bOFull]);
+        }
+      }
+      umma_commit(&bars[Ly::bDonePV]);
+      wait_slow(&bars[Ly::bDonePV], 0, WaitCtl{abort_flag, a.status}, 23);
     }
     __syncwarp();
   } else {
     // ============================================================ softmax + epilogue
-    const int tid = threadIdx.x - 64;  // 0..127
-    const int qd = warp & 3;           // TMEM lane quadrant this warp may access
-    const int kl = qd * 32 + lane;     // key lane (S^T) / d lane (O^T)
+    const int grp = (warp - 4) >> 2;           // column group: queries [32 grp, 32 grp + 32)
+    const int tid = threadIdx.x - 128 * (grp + 1);  // 0..127 within the group
+    const int qd = warp & 3;                   // TMEM lane quadrant this warp may access
+    const int kl = qd * 32 + lane;             // key lane (S^T) / d lane (O^T)
+    const int c0 = grp * 32;
+    const int bar_vote = 1 + 2 * grp, bar_sync = 2 + 2 * grp;  // named barriers of this group
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    float* m_g = m_s + c0;
+    float* alpha_g = alpha_s + c0;
+    float* red_g = red_s + grp * 128;
+    float* rl_g = rl_s + c0;
+    const float cl = a.scale_log2;
     uint32_t g = 0;
     int it = 0;
     for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
@@ -328,97 +397,95 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int i = static_cast<int>(w - bh * n_t);
       const int64_t b = bh / a.H;
       const int h = static_cast<int>(bh - b * a.H);
-      const int nk = list_len(i), nb = (nk + 1) / 2;
+      const int nb = (list_len(i) + 1) / 2;
       const int valid_i = tile_valid_s[i];
-      for (int t = tid; t < nk; t += 128) kvalid_s[t] = tile_valid_s[key_tile(bh, i, t)];
-      if (tid < 64) {
-        const int32_t tok = a.tile_token[static_cast<int64_t>(i) * 64 + tid];
-        qtok_s[tid] = tok;
-        gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(a.gate[(b * a.L + tok) * a.H + h]) : 0.0f;
+      // per-item values, loaded now and used in the epilogue
+      int32_t my_tok = -1;
+      float my_gate = 0.0f;
+      if (tid < 32) {
+        my_tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + c0 + tid);
+        if (my_tok >= 0) my_gate = bf16_bits_to_f32(__ldg(a.gate + (b * a.L + my_tok) * a.H + h));
       }
-      named_bar_sync(1, 128);
+      const float my_oc = (kl < D) ? __ldg(a.o_c + (bh * n_t + i) * D + kl) : 0.0f;
 
-      float l[64];
+      float l[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) l[j] = 0.0f;
+      for (int j = 0; j < 32; ++j) l[j] = 0.0f;
 
       for (int n = 0; n < nb; ++n, ++g) {
         const int sb = g & 1;
         const uint32_t su = g >> 1;
-        mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 11);
+        const int ms = g % Ly::kMeta;
+        mbar_wait(&bars[Ly::bMFull + ms], (g / Ly::kMeta) & 1, ctl, 11);
+        const int2 vc = meta_s[ms];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Ly::bMEmpty + ms]);
+        const int vcount = (kl < 64) ? vc.x : vc.y;
+        const bool valid = (kl & 63) < vcount;
+
+        mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
         tc_fence_after();
-        float y[64];
-        tmem_ld32(t_lane + sb * 64, y);
-        tmem_ld32(t_lane + sb * 64 + 32, y + 32);
+        float y[32];
+        tmem_ld32(t_lane + sb * 64 + c0, y);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bSEmpty + sb]);
-
-        const int pos = 2 * n + (kl >> 6);
-        const int vcount = (pos < nk) ? kvalid_s[pos] : 0;
-        const bool valid = (kl & 63) < vcount;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) y[j] = valid ? y[j] * a.scale_log2 : -INFINITY;
+        for (int j = 0; j < 32; ++j) y[j] = valid ? y[j] * cl : -INFINITY;
 
         bool slow = true;
         if (n > 0) {
           float xm = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 64; j += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(m_s + j);
+          for (int j = 0; j < 32; j += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
             xm = fmaxf(xm, fmaxf(fmaxf(y[j] - m4.x, y[j + 1] - m4.y), fmaxf(y[j + 2] - m4.z, y[j + 3] - m4.w)));
           }
-          slow = named_bar_or(2, 128, xm > kRescaleLog2);
+          slow = named_bar_or(bar_vote, 128, xm > kRescaleLog2);
         }
         if (slow) {
-          // exact column maximum of this block: butterfly per column, lane (j % 32) keeps column j
-          float cm0 = -INFINITY, cm1 = -INFINITY;
+          // exact column maximum of this block over the group's 128 lanes
+          float cm = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
+          for (int j = 0; j < 32; ++j) {
             float c = y[j];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
-            if ((j & 31) == lane) {
-              if (j < 32) cm0 = c; else cm1 = c;
-            }
+            if (j == lane) cm = c;
           }
-          red_s[qd * 64 + lane] = cm0;
-          red_s[qd * 64 + 32 + lane] = cm1;
-          named_bar_sync(3, 128);
-          if (tid < 64) {
-            const float cm = fmaxf(fmaxf(red_s[tid], red_s[64 + tid]), fmaxf(red_s[128 + tid], red_s[192 + tid]));
-            const float mo = (n == 0) ? -INFINITY : m_s[tid];
-            float mn = fmaxf(mo, cm);
+          red_g[qd * 32 + lane] = cm;
+          named_bar_sync(bar_sync, 128);
+          if (tid < 32) {
+            const float c = fmaxf(fmaxf(red_g[tid], red_g[32 + tid]), fmaxf(red_g[64 + tid], red_g[96 + tid]));
+            const float mo = (n == 0) ? -INFINITY : m_g[tid];
+            float mn = fmaxf(mo, c);
             if (mn == -INFINITY) mn = 0.0f;
-            alpha_s[tid] = (mo == -INFINITY) ? 0.0f : ex2_approx(mo - mn);
-            m_s[tid] = mn;
+            alpha_g[tid] = (mo == -INFINITY) ? 0.0f : ex2_approx(mo - mn);
+            m_g[tid] = mn;
           }
-          named_bar_sync(3, 128);
+          named_bar_sync(bar_sync, 128);
           if (n > 0) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) l[j] *= alpha_s[j];
-            // O^T holds blocks < n of this item: wait for the last P.V, then rescale its columns
+            for (int j = 0; j < 32; ++j) l[j] *= alpha_g[j];
+            // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
             const uint32_t gp = g - 1;
-            mbar_wait(&bars[Ly::bPEmpty + (gp & 1)], (gp >> 1) & 1, ctl, 12);
+            mbar_wait(&bars[Ly::bPEmpty + (gp & 1)], (gp >> 1) & 1, ctl, 13);
             tc_fence_after();
+            float o[32];
+            tmem_ld32(t_lane + 128 + c0, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int hc = 0; hc < 64; hc += 32) {
-              float o[32];
-              tmem_ld32(t_lane + 128 + hc, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] *= alpha_s[hc + j];
-              tmem_st32(t_lane + 128 + hc, o);
-            }
+            for (int j = 0; j < 32; ++j) o[j] *= alpha_g[j];
+            tmem_st32(t_lane + 128 + c0, o);
             tmem_wait_st();
             tc_fence_before();
           }
         }
-        // probabilities, partial row sums, P^T row of this key lane (bf16, 128-byte swizzle)
+        // probabilities, partial row sums, this group's half of the P^T row (bf16, 128-byte swizzle)
 #pragma unroll
-        for (int j = 0; j < 64; j += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_s + j);
+        for (int j = 0; j < 32; j += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
           y[j] = ex2_approx(y[j] - m4.x);
           y[j + 1] = ex2_approx(y[j + 1] - m4.y);
           y[j + 2] = ex2_approx(y[j + 2] - m4.z);
@@ -428,15 +495,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l[j + 2] += y[j + 2];
           l[j + 3] += y[j + 3];
         }
-        mbar_wait(&bars[Ly::bPEmpty + sb], (su & 1) ^ 1, ctl, 13);
+        mbar_wait(&bars[Ly::bPEmpty + sb], (su & 1) ^ 1, ctl, 14);
         uint8_t* prow = sm + Ly::oP + sb * Ly::kPBytes + kl * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = grp * 4 + cc;  // 16-byte chunk = queries 8c .. 8c+7
           U128 w4;
-          w4.x = pack_bf16x2(y[8 * c + 0], y[8 * c + 1]);
-          w4.y = pack_bf16x2(y[8 * c + 2], y[8 * c + 3]);
-          w4.z = pack_bf16x2(y[8 * c + 4], y[8 * c + 5]);
-          w4.w = pack_bf16x2(y[8 * c + 6], y[8 * c + 7]);
+          w4.x = pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]);
+          w4.y = pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]);
+          w4.z = pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]);
+          w4.w = pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]);
           *reinterpret_cast<U128*>(prow + ((c ^ (kl & 7)) << 4)) = w4;
         }
         fence_proxy_async_smem();
@@ -444,49 +512,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) mbar_arrive(&bars[Ly::bPFull + sb]);
       }
 
-      // ---------------------------------------------------------- epilogue
-      warp_reduce_scatter64<false>(l, lane);
-      red_s[qd * 64 + 2 * lane] = l[0];
-      red_s[qd * 64 + 2 * lane + 1] = l[1];
-      named_bar_sync(3, 128);
-      if (tid < 64) lsum_s[tid] = (red_s[tid] + red_s[64 + tid]) + (red_s[128 + tid] + red_s[192 + tid]);
-      mbar_wait(&bars[Ly::bOFull], it & 1, ctl, 14);
+      // ---------------------------------------------------------- epilogue (this group's 32 queries)
+      warp_sum_scatter32(l, lane);
+      red_g[qd * 32 + lane] = l[0];
+      if (tid < 32) {
+        qtok_s[c0 + tid] = my_tok;
+        gate_s[c0 + tid] = my_gate;
+      }
+      named_bar_sync(bar_sync, 128);
+      if (tid < 32) rl_g[tid] = rcp_approx((red_g[tid] + red_g[32 + tid]) + (red_g[64 + tid] + red_g[96 + tid]));
+      mbar_wait(&bars[Ly::bOFull], it & 1, ctl, 15);
       tc_fence_after();
-      float o[64];
-      tmem_ld32(t_lane + 128, o);
-      tmem_ld32(t_lane + 128 + 32, o + 32);
+      float o[32];
+      tmem_ld32(t_lane + 128 + c0, o);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty]);
-      named_bar_sync(3, 128);  // lsum_s ready
-      uint16_t* stage = reinterpret_cast<uint16_t*>(sm + Ly::oP);  // [64 q][D] bf16; P buffers are idle now
+      named_bar_sync(bar_sync, 128);  // rl, gate, qtok of the group ready
       if (kl < D) {
-        const float oc = a.o_c[(bh * n_t + i) * D + kl];
-#pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          const float val = o[q] / lsum_s[q] + gate_s[q] * oc;
-          stage[q * D + kl] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        const int nq = min(32, valid_i - c0);
+        for (int q = 0; q < nq; ++q) {
+          const float val = fmaf(o[q], rl_g[q], gate_s[c0 + q] * my_oc);
+          a.out[((b * a.L + qtok_s[c0 + q]) * a.H + h) * D + kl] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
         }
       }
-      named_bar_sync(3, 128);
-      constexpr int kChunks = D / 8;
-      for (int e = tid; e < 64 * kChunks; e += 128) {
-        const int q = e / kChunks, c = e - q * kChunks;
-        if (q < valid_i) {
-          const int32_t tok = qtok_s[q];
-          uint16_t* dst = a.out + ((b * a.L + tok) * a.H + h) * D + c * 8;
-          *reinterpret_cast<U128*>(dst) = *reinterpret_cast<const U128*>(stage + q * D + c * 8);
-        }
-      }
-      named_bar_sync(3, 128);
+      named_bar_sync(bar_sync, 128);  // smem of this item no longer read
     }
   }
 
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
