@@ -16,17 +16,21 @@
 //     maximum taken across the 128 lanes and O^T, l rescaled.  Any m with no
 //     overflow gives the same softmax, so this is exact up to rounding;
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
+// O^T is double-buffered in TMEM, so one item's epilogue (in its own warps)
+// overlaps the next item's blocks.
 // D = 64 uses the same M = 128 PV product with a zero upper half of V^T.
 //
-// Roles (384 threads, 12 warps):
+// Roles (512 threads, 16 warps):
 //   warp 0  K producer: TMA for the query tile of each item and the K tiles
 //           of each block (4 lanes issue the four 8 KB boxes in parallel),
 //           plus the block's key-valid counts for the softmax;
 //   warp 1  V producer: TMA for the V tiles of each block;
 //   warp 2  S^T issuer (one thread) and TMEM owner;
 //   warp 3  P.V issuer (one thread);
-//   warps 4..11  softmax + epilogue, two groups of four warps; group g owns
-//           query columns [32g, 32g + 32), warp w reads TMEM lane quadrant w % 4.
+//   warps 4..11  softmax, two groups of four warps; group g owns query
+//           columns [32g, 32g + 32), warp w reads TMEM lane quadrant w % 4;
+//   warps 12..15 epilogue: 1/l, O^T from TMEM, the gated compression term
+//           and the bf16 store in sequence order.
 // Two issuing threads keep two tcgen05 streams in flight (one thread alone is
 // limited by its issue latency), and several issuing lanes keep enough TMA
 // loads in flight.  Every mbarrier wait is bounded; after a timeout the kernel
@@ -42,9 +46,12 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 384;
-constexpr float kRescaleLog2 = 8.0f;  // lazy-max threshold: exponents stay <= 2^8
-constexpr uint32_t kTmemCols = 256;   // S^T double buffer (2 x 64) + O^T (64), rounded to a power of 2
+constexpr int kAttnThreads = 512;
+// Lazy-max threshold: probabilities stay <= 2^24 between exact rescales.  With
+// at most 2^23 keys per row, row sums stay below 2^47 and P.V partial sums far
+// below the binary32 range.
+constexpr float kRescaleLog2 = 24.0f;
+constexpr uint32_t kTmemCols = 256;  // S^T double buffer (2 x 64) + O^T double buffer (2 x 64)
 
 struct AttnArgs {
   const int32_t* idx;         // [B, H, V, topk] global key-tile indices (ascending per row)
@@ -85,17 +92,19 @@ struct AttnLayout {
   static constexpr int bSFull = bVEmpty + kVStages, bSEmpty = bSFull + 2;
   static constexpr int bPFull = bSEmpty + 2, bPEmpty = bPFull + 2;
   static constexpr int bMFull = bPEmpty + 2, bMEmpty = bMFull + kMeta;
-  static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 1;
-  static constexpr int bDoneS = bOEmpty + 1, bDonePV = bDoneS + 1;
+  static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 2;
+  static constexpr int bLFull = bOEmpty + 2;
+  static constexpr int bDoneS = bLFull + 2, bDonePV = bDoneS + 1;
   static constexpr int kNumBars = bDonePV + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;          // tmem base, abort flag
   static constexpr int oMeta = ((oMisc + 8 + 15) / 16) * 16;  // int2 meta[kMeta]
-  static constexpr int oM = oMeta + kMeta * 8;               // float m[64]
-  static constexpr int oAlpha = oM + 256;                    // float alpha[64]
-  static constexpr int oRed = oAlpha + 256;                  // float red[2 groups][4 quadrants][32]
-  static constexpr int oRl = oRed + 1024;                    // float 1 / l[64]
-  static constexpr int oGate = oRl + 256;                    // float gate[64]
-  static constexpr int oQtok = oGate + 256;                  // int qtok[64]
+  static constexpr int oM = oMeta + kMeta * 8;               // float m[64] (log2 units)
+  static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
+  static constexpr int oRed = oDelta + 256;                  // float red[2 groups][4 quadrants][32]
+  static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
+  static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
+  static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
+  static constexpr int oQtok = oGate + 256;                  // int qtok[64]     (epilogue)
   static constexpr int oTileValid = oQtok + 256;             // uint8 [n_t]
   static size_t bytes(int n_t) {
     const size_t tv = ((static_cast<size_t>(n_t) + 15) / 16) * 16;
@@ -150,8 +159,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::oMisc + 4);
   int2* meta_s = reinterpret_cast<int2*>(sm + Ly::oMeta);
   float* m_s = reinterpret_cast<float*>(sm + Ly::oM);
-  float* alpha_s = reinterpret_cast<float*>(sm + Ly::oAlpha);
+  float* delta_s = reinterpret_cast<float*>(sm + Ly::oDelta);
   float* red_s = reinterpret_cast<float*>(sm + Ly::oRed);
+  float* lpart_s = reinterpret_cast<float*>(sm + Ly::oLsum);
   float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
   float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
   int32_t* qtok_s = reinterpret_cast<int32_t*>(sm + Ly::oQtok);
@@ -192,8 +202,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars[Ly::bMFull + s], 1);
       mbar_init(&bars[Ly::bMEmpty + s], 8);
     }
-    mbar_init(&bars[Ly::bOFull], 1);
-    mbar_init(&bars[Ly::bOEmpty], 8);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[Ly::bOFull + s], 1);
+      mbar_init(&bars[Ly::bOEmpty + s], 4);
+      mbar_init(&bars[Ly::bLFull + s], 8);
+    }
     mbar_init(&bars[Ly::bDoneS], 1);
     mbar_init(&bars[Ly::bDonePV], 1);
     fence_mbar_init();
@@ -348,12 +361,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
         const int nb = (list_len(i) + 1) / 2;
+        const int ob = it & 1;
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int vst = g % Ly::kVStages;
           const int pb = g & 1;
           ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8) &&
                mbar_wait(&bars[Ly::bPFull + pb], (g >> 1) & 1, ctl, 9) &&
-               (n > 0 || mbar_wait(&bars[Ly::bOEmpty], (it & 1) ^ 1, ctl, 10));
+               (n > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
           if (!ok) break;
           tc_fence_after();
           const uint32_t vbase = smem_u32(sm + Ly::oV + vst * Ly::kKVBytes);
@@ -365,48 +379,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int kk = 0; kk < kPVSteps; ++kk) {
             const uint64_t ad = umma_desc_sw128(vbase + kk * 2048, lbo_v, 1024);
             const uint64_t bd = umma_desc_sw128(pbase + kk * 2048, 8192, 1024);
-            umma_ss(tmem + 128, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+            umma_ss(tmem + 128 + ob * 64, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars[Ly::bVEmpty + vst]);
           umma_commit(&bars[Ly::bPEmpty + pb]);
-          if (n == nb - 1) umma_commit(&bars[Ly::bOFull]);
+          if (n == nb - 1) umma_commit(&bars[Ly::bOFull + ob]);
         }
       }
       umma_commit(&bars[Ly::bDonePV]);
       wait_slow(&bars[Ly::bDonePV], 0, WaitCtl{abort_flag, a.status}, 23);
     }
     __syncwarp();
-  } else {
-    // ============================================================ softmax + epilogue
-    const int grp = (warp - 4) >> 2;           // column group: queries [32 grp, 32 grp + 32)
-    const int tid = threadIdx.x - 128 * (grp + 1);  // 0..127 within the group
-    const int qd = warp & 3;                   // TMEM lane quadrant this warp may access
-    const int kl = qd * 32 + lane;             // key lane (S^T) / d lane (O^T)
+  } else if (warp < 12) {
+    // ============================================================ softmax
+    const int grp = (warp - 4) >> 2;                 // column group: queries [32 grp, 32 grp + 32)
+    const int tid = threadIdx.x - 128 * (grp + 1);   // 0..127 within the group
+    const int qd = warp & 3;                         // TMEM lane quadrant this warp may access
+    const int kl = qd * 32 + lane;                   // key lane (S^T) / d lane (O^T)
     const int c0 = grp * 32;
     const int bar_vote = 1 + 2 * grp, bar_sync = 2 + 2 * grp;  // named barriers of this group
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     float* m_g = m_s + c0;
-    float* alpha_g = alpha_s + c0;
+    float* delta_g = delta_s + c0;
     float* red_g = red_s + grp * 128;
-    float* rl_g = rl_s + c0;
     const float cl = a.scale_log2;
     uint32_t g = 0;
     int it = 0;
     for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
-      const int64_t b = bh / a.H;
-      const int h = static_cast<int>(bh - b * a.H);
       const int nb = (list_len(i) + 1) / 2;
-      const int valid_i = tile_valid_s[i];
-      // per-item values, loaded now and used in the epilogue
-      int32_t my_tok = -1;
-      float my_gate = 0.0f;
-      if (tid < 32) {
-        my_tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + c0 + tid);
-        if (my_tok >= 0) my_gate = bf16_bits_to_f32(__ldg(a.gate + (b * a.L + my_tok) * a.H + h));
-      }
-      const float my_oc = (kl < D) ? __ldg(a.o_c + (bh * n_t + i) * D + kl) : 0.0f;
+      const int ob = it & 1;
 
       float l[32];
 #pragma unroll
@@ -420,80 +423,92 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int2 vc = meta_s[ms];
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bMEmpty + ms]);
-        const int vcount = (kl < 64) ? vc.x : vc.y;
-        const bool valid = (kl & 63) < vcount;
 
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
         tc_fence_after();
-        float y[32];
-        tmem_ld32(t_lane + sb * 64 + c0, y);
+        float x[32];
+        tmem_ld32(t_lane + sb * 64 + c0, x);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bSEmpty + sb]);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = valid ? y[j] * cl : -INFINITY;
 
-        bool slow = true;
-        if (n > 0) {
-          float xm = -INFINITY;
+        // x = logit * log2(e) - m  (m = 0 before the first block of the item)
+        float xm = -INFINITY;
+        if (n == 0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] *= cl;
+        } else {
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
             const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
-            xm = fmaxf(xm, fmaxf(fmaxf(y[j] - m4.x, y[j + 1] - m4.y), fmaxf(y[j + 2] - m4.z, y[j + 3] - m4.w)));
+            x[j] = fmaf(x[j], cl, -m4.x);
+            x[j + 1] = fmaf(x[j + 1], cl, -m4.y);
+            x[j + 2] = fmaf(x[j + 2], cl, -m4.z);
+            x[j + 3] = fmaf(x[j + 3], cl, -m4.w);
           }
+        }
+        if (vc.x < 64 || vc.y < 64) {  // pad keys or a half-empty block: mask this lane's key
+          const int vcount = (kl < 64) ? vc.x : vc.y;
+          if ((kl & 63) >= vcount) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = -INFINITY;
+          }
+        }
+        bool slow = true;
+        if (n > 0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xm = fmaxf(xm, x[j]);
           slow = named_bar_or(bar_vote, 128, xm > kRescaleLog2);
         }
         if (slow) {
-          // exact column maximum of this block over the group's 128 lanes
+          // exact column maximum of this block over the group's 128 lanes; raise m by it
           float cm = -INFINITY;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            float c = y[j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
-            if (j == lane) cm = c;
+            float r;
+            asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x[j]));
+            if (j == lane) cm = r;
           }
           red_g[qd * 32 + lane] = cm;
           named_bar_sync(bar_sync, 128);
           if (tid < 32) {
             const float c = fmaxf(fmaxf(red_g[tid], red_g[32 + tid]), fmaxf(red_g[64 + tid], red_g[96 + tid]));
-            const float mo = (n == 0) ? -INFINITY : m_g[tid];
-            float mn = fmaxf(mo, c);
-            if (mn == -INFINITY) mn = 0.0f;
-            alpha_g[tid] = (mo == -INFINITY) ? 0.0f : ex2_approx(mo - mn);
-            m_g[tid] = mn;
+            float d;
+            if (n == 0) {
+              d = (c == -INFINITY) ? 0.0f : c;
+              m_g[tid] = d;
+            } else {
+              d = fmaxf(c, 0.0f);
+              m_g[tid] += d;
+            }
+            delta_g[tid] = d;
           }
           named_bar_sync(bar_sync, 128);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] -= delta_g[j];
           if (n > 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) l[j] *= alpha_g[j];
+            for (int j = 0; j < 32; ++j) l[j] *= ex2_approx(-delta_g[j]);
             // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
             const uint32_t gp = g - 1;
             mbar_wait(&bars[Ly::bPEmpty + (gp & 1)], (gp >> 1) & 1, ctl, 13);
             tc_fence_after();
             float o[32];
-            tmem_ld32(t_lane + 128 + c0, o);
+            tmem_ld32(t_lane + 128 + ob * 64 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] *= alpha_g[j];
-            tmem_st32(t_lane + 128 + c0, o);
+            for (int j = 0; j < 32; ++j) o[j] *= ex2_approx(-delta_g[j]);
+            tmem_st32(t_lane + 128 + ob * 64 + c0, o);
             tmem_wait_st();
             tc_fence_before();
           }
         }
         // probabilities, partial row sums, this group's half of the P^T row (bf16, 128-byte swizzle)
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
-          y[j] = ex2_approx(y[j] - m4.x);
-          y[j + 1] = ex2_approx(y[j + 1] - m4.y);
-          y[j + 2] = ex2_approx(y[j + 2] - m4.z);
-          y[j + 3] = ex2_approx(y[j + 3] - m4.w);
-          l[j] += y[j];
-          l[j + 1] += y[j + 1];
-          l[j + 2] += y[j + 2];
-          l[j + 3] += y[j + 3];
+        for (int j = 0; j < 32; ++j) {
+          x[j] = ex2_approx(x[j]);
+          l[j] += x[j];
         }
         mbar_wait(&bars[Ly::bPEmpty + sb], (su & 1) ^ 1, ctl, 14);
         uint8_t* prow = sm + Ly::oP + sb * Ly::kPBytes + kl * 128;
@@ -501,10 +516,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int cc = 0; cc < 4; ++cc) {
           const int c = grp * 4 + cc;  // 16-byte chunk = queries 8c .. 8c+7
           U128 w4;
-          w4.x = pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]);
-          w4.y = pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]);
-          w4.z = pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]);
-          w4.w = pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]);
+          w4.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+          w4.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+          w4.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+          w4.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
           *reinterpret_cast<U128*>(prow + ((c ^ (kl & 7)) << 4)) = w4;
         }
         fence_proxy_async_smem();
@@ -512,32 +527,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) mbar_arrive(&bars[Ly::bPFull + sb]);
       }
 
-      // ---------------------------------------------------------- epilogue (this group's 32 queries)
+      // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored)
       warp_sum_scatter32(l, lane);
-      red_g[qd * 32 + lane] = l[0];
-      if (tid < 32) {
-        qtok_s[c0 + tid] = my_tok;
-        gate_s[c0 + tid] = my_gate;
+      if (it >= 2) mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 15);
+      lpart_s[(ob * 4 + qd) * 64 + c0 + lane] = l[0];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[Ly::bLFull + ob]);
+    }
+  } else {
+    // ============================================================ epilogue
+    const int tid = threadIdx.x - 384;  // 0..127
+    const int qd = warp & 3;
+    const int d = qd * 32 + lane;       // O^T lane = d
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    int it = 0;
+    for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
+      const int64_t bh = w / n_t;
+      const int i = static_cast<int>(w - bh * n_t);
+      const int64_t b = bh / a.H;
+      const int h = static_cast<int>(bh - b * a.H);
+      const int ob = it & 1;
+      const int valid_i = tile_valid_s[i];
+      if (tid < 64) {
+        const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
+        qtok_s[tid] = tok;
+        gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.H + h)) : 0.0f;
       }
-      named_bar_sync(bar_sync, 128);
-      if (tid < 32) rl_g[tid] = rcp_approx((red_g[tid] + red_g[32 + tid]) + (red_g[64 + tid] + red_g[96 + tid]));
-      mbar_wait(&bars[Ly::bOFull], it & 1, ctl, 15);
+      const float oc = (d < D) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
+      mbar_wait(&bars[Ly::bLFull + ob], (it >> 1) & 1, ctl, 16);
+      if (tid < 64) {
+        const float* lp = lpart_s + ob * 4 * 64 + tid;
+        rl_s[tid] = rcp_approx((lp[0] + lp[64]) + (lp[128] + lp[192]));
+      }
+      mbar_wait(&bars[Ly::bOFull + ob], (it >> 1) & 1, ctl, 17);
       tc_fence_after();
-      float o[32];
-      tmem_ld32(t_lane + 128 + c0, o);
+      float o[64];
+      tmem_ld32(t_lane + 128 + ob * 64, o);
+      tmem_ld32(t_lane + 128 + ob * 64 + 32, o + 32);
       tmem_wait_ld();
       tc_fence_before();
+      named_bar_sync(5, 128);  // rl, gate, qtok ready; every lane of O^T read
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty]);
-      named_bar_sync(bar_sync, 128);  // rl, gate, qtok of the group ready
-      if (kl < D) {
-        const int nq = min(32, valid_i - c0);
-        for (int q = 0; q < nq; ++q) {
-          const float val = fmaf(o[q], rl_g[q], gate_s[c0 + q] * my_oc);
-          a.out[((b * a.L + qtok_s[c0 + q]) * a.H + h) * D + kl] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+      if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty + ob]);
+      if (d < D) {
+        uint16_t* out_col = a.out + (b * a.L * a.H + h) * D + d;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          if (q < valid_i) {
+            const float val = fmaf(o[q], rl_s[q], gate_s[q] * oc);
+            out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+          }
         }
       }
-      named_bar_sync(bar_sync, 128);  // smem of this item no longer read
+      named_bar_sync(5, 128);  // smem of this item no longer read
     }
   }
 
