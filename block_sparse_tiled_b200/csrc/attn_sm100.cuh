@@ -20,16 +20,17 @@
 // overlaps the next item's blocks.
 // D = 64 uses the same M = 128 PV product with a zero upper half of V^T.
 //
-// Roles (512 threads, 16 warps):
+// Roles (768 threads, 24 warps):
 //   warp 0  K producer: TMA for the query tile of each item and the K tiles
 //           of each block (4 lanes issue the four 8 KB boxes in parallel),
 //           plus the block's key-valid counts for the softmax;
 //   warp 1  V producer: TMA for the V tiles of each block;
 //   warp 2  S^T issuer (one thread) and TMEM owner;
 //   warp 3  P.V issuer (one thread);
-//   warps 4..11  softmax, two groups of four warps; group g owns query
-//           columns [32g, 32g + 32), warp w reads TMEM lane quadrant w % 4;
-//   warps 12..15 epilogue: 1/l, O^T from TMEM, the gated compression term
+//   warps 4..19  softmax, four groups of four warps; group g owns query
+//           columns [16g, 16g + 16), warp w reads TMEM lane quadrant w % 4
+//           (four softmax warps per SM sub-partition hide each other's latency);
+//   warps 20..23 epilogue: 1/l, O^T from TMEM, the gated compression term
 //           and the bf16 store in sequence order.
 // Two issuing threads keep two tcgen05 streams in flight (one thread alone is
 // limited by its issue latency), and several issuing lanes keep enough TMA
@@ -46,7 +47,43 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 512;
+// Optional per-role cycle accounting (build with -DVSA_ROLE_TIMERS): each role
+// of each CTA adds clock64() deltas into up to 8 counters, read back with
+// vsa_role_timers().  Compiled out otherwise.
+#ifdef VSA_ROLE_TIMERS
+constexpr int kRoleTimerCtas = 160;
+__device__ unsigned long long g_role_cycles[kRoleTimerCtas][8][8];
+#define ROLE_TIMER_START() \
+  unsigned long long rt_acc_[8] = {0, 0, 0, 0, 0, 0, 0, 0}; \
+  unsigned long long rt_t_ = clock64()
+#define ROLE_MARK(c)                         \
+  do {                                       \
+    const unsigned long long n_ = clock64(); \
+    rt_acc_[c] += n_ - rt_t_;                \
+    rt_t_ = n_;                              \
+  } while (0)
+#define ROLE_TIMER_SAVE(role)                                                               \
+  do {                                                                                      \
+    if (blockIdx.x < kRoleTimerCtas)                                                        \
+      for (int c_ = 0; c_ < 8; ++c_) g_role_cycles[blockIdx.x][role][c_] = rt_acc_[c_];     \
+  } while (0)
+#else
+#define ROLE_TIMER_START() \
+  do {                     \
+  } while (0)
+#define ROLE_MARK(c) \
+  do {               \
+  } while (0)
+#define ROLE_TIMER_SAVE(role) \
+  do {                        \
+  } while (0)
+#endif
+
+constexpr int kSoftGroups = 4;                    // softmax column groups
+constexpr int kGroupCols = 64 / kSoftGroups;       // query columns per group
+constexpr int kSoftWarps = 4 * kSoftGroups;        // one warp per TMEM lane quadrant per group
+constexpr int kEpiWarp0 = 4 + kSoftWarps;          // first epilogue warp
+constexpr int kAttnThreads = 32 * (kEpiWarp0 + 4);
 // Lazy-max threshold: probabilities stay <= 2^24 between exact rescales.  With
 // at most 2^23 keys per row, row sums stay below 2^47 and P.V partial sums far
 // below the binary32 range.
@@ -74,9 +111,9 @@ struct AttnLayout {
   static constexpr int kKVBytes = 128 * D * 2;  // 128 keys of K (or of V)
   static constexpr int kHalfBytes = 128 * 128;  // one 64-column half of a 128-row block
   static constexpr int kPBytes = 128 * 64 * 2;  // P^T of one block
-  static constexpr int kQBufs = 2;
+  static constexpr int kQBufs = 1;
   static constexpr int kKStages = 2;
-  static constexpr int kVStages = 2;
+  static constexpr int kVStages = 3;
   static constexpr int kMeta = 8;  // per-block key-valid counts in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
   static constexpr int oQ = 0;
@@ -100,7 +137,7 @@ struct AttnLayout {
   static constexpr int oMeta = ((oMisc + 8 + 15) / 16) * 16;  // int2 meta[kMeta]
   static constexpr int oM = oMeta + kMeta * 8;               // float m[64] (log2 units)
   static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
-  static constexpr int oRed = oDelta + 256;                  // float red[2 groups][4 quadrants][32]
+  static constexpr int oRed = oDelta + 256;                  // float red[groups][4 quadrants][group columns]
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
   static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
   static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
@@ -194,18 +231,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[Ly::bSFull + s], 1);
-      mbar_init(&bars[Ly::bSEmpty + s], 8);
-      mbar_init(&bars[Ly::bPFull + s], 8);
+      mbar_init(&bars[Ly::bSEmpty + s], kSoftWarps);
+      mbar_init(&bars[Ly::bPFull + s], kSoftWarps);
       mbar_init(&bars[Ly::bPEmpty + s], 1);
     }
     for (int s = 0; s < Ly::kMeta; ++s) {
       mbar_init(&bars[Ly::bMFull + s], 1);
-      mbar_init(&bars[Ly::bMEmpty + s], 8);
+      mbar_init(&bars[Ly::bMEmpty + s], kSoftWarps);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[Ly::bOFull + s], 1);
       mbar_init(&bars[Ly::bOEmpty + s], 4);
-      mbar_init(&bars[Ly::bLFull + s], 8);
+      mbar_init(&bars[Ly::bLFull + s], kSoftWarps);
     }
     mbar_init(&bars[Ly::bDoneS], 1);
     mbar_init(&bars[Ly::bDonePV], 1);
@@ -242,6 +279,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
+    ROLE_TIMER_START();
     for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
@@ -251,7 +289,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int qb = it % Ly::kQBufs;
         const uint32_t qu = it / Ly::kQBufs;
         if (lane == 0) {
+          ROLE_MARK(3);
           ok = mbar_wait(&bars[Ly::bQEmpty + qb], (qu & 1) ^ 1, ctl, 1);
+          ROLE_MARK(0);
           if (ok) mbar_arrive_expect_tx(&bars[Ly::bQFull + qb], Ly::kQBytes);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -275,12 +315,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int st = g % nstages;
           const uint32_t u = g / nstages;
           if (lane == 0) {
+            ROLE_MARK(3);
             ok = mbar_wait(&bars[b_empty + st], (u & 1) ^ 1, ctl, is_k ? 2 : 3);
+            ROLE_MARK(1);
             if (ok) mbar_arrive_expect_tx(&bars[b_full + st], Ly::kKVBytes);
             if (ok && is_k) {
               // the block's key-valid counts, for the softmax
               const int ms = g % Ly::kMeta;
+              ROLE_MARK(3);
               ok = mbar_wait(&bars[Ly::bMEmpty + ms], ((g / Ly::kMeta) & 1) ^ 1, ctl, 4);
+              ROLE_MARK(2);
               if (ok) {
                 meta_s[ms] = make_int2(tile_valid_s[ka], kb_raw < 0 ? 0 : tile_valid_s[kb_raw]);
                 mbar_arrive(&bars[Ly::bMFull + ms]);
@@ -299,6 +343,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __syncwarp();
         }
       }
+    }
+    if (lane == 0) {
+      ROLE_MARK(3);
+      ROLE_TIMER_SAVE(warp);
     }
     // drain: every load this warp issued must land before the CTA exits
     if (lane == 0) {
@@ -321,18 +369,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t g = 0;
       int it = 0;
       bool ok = true;
+      ROLE_TIMER_START();
       for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
         const int nb = (list_len(i) + 1) / 2;
         const int qb = it % Ly::kQBufs;
+        ROLE_MARK(3);
         ok = mbar_wait(&bars[Ly::bQFull + qb], (it / Ly::kQBufs) & 1, ctl, 5);
+        ROLE_MARK(0);
         const uint32_t qbase = smem_u32(sm + Ly::oQ + qb * Ly::kQBytes);
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int kst = g % Ly::kKStages;
           const int sb = g & 1;
-          ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6) &&
-               mbar_wait(&bars[Ly::bSEmpty + sb], ((g >> 1) & 1) ^ 1, ctl, 7);
+          ROLE_MARK(3);
+          ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6);
+          ROLE_MARK(1);
+          ok = ok && mbar_wait(&bars[Ly::bSEmpty + sb], ((g >> 1) & 1) ^ 1, ctl, 7);
+          ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kbase = smem_u32(sm + Ly::oK + kst * Ly::kKVBytes);
@@ -347,6 +401,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (n == nb - 1) umma_commit(&bars[Ly::bQEmpty + qb]);
         }
       }
+      ROLE_MARK(3);
+      ROLE_TIMER_SAVE(2);
       umma_commit(&bars[Ly::bDoneS]);
       wait_slow(&bars[Ly::bDoneS], 0, WaitCtl{abort_flag, a.status}, 22);
     }
@@ -357,6 +413,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t g = 0;
       int it = 0;
       bool ok = true;
+      ROLE_TIMER_START();
       for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
@@ -365,9 +422,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int vst = g % Ly::kVStages;
           const int pb = g & 1;
-          ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8) &&
-               mbar_wait(&bars[Ly::bPFull + pb], (g >> 1) & 1, ctl, 9) &&
-               (n > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
+          ROLE_MARK(3);
+          ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8);
+          ROLE_MARK(0);
+          ok = ok && mbar_wait(&bars[Ly::bPFull + pb], (g >> 1) & 1, ctl, 9);
+          ROLE_MARK(1);
+          ok = ok && (n > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
+          ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vbase = smem_u32(sm + Ly::oV + vst * Ly::kKVBytes);
@@ -386,61 +447,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (n == nb - 1) umma_commit(&bars[Ly::bOFull + ob]);
         }
       }
+      ROLE_MARK(3);
+      ROLE_TIMER_SAVE(3);
       umma_commit(&bars[Ly::bDonePV]);
       wait_slow(&bars[Ly::bDonePV], 0, WaitCtl{abort_flag, a.status}, 23);
     }
     __syncwarp();
-  } else if (warp < 12) {
+  } else if (warp < kEpiWarp0) {
     // ============================================================ softmax
-    const int grp = (warp - 4) >> 2;                 // column group: queries [32 grp, 32 grp + 32)
-    const int tid = threadIdx.x - 128 * (grp + 1);   // 0..127 within the group
-    const int qd = warp & 3;                         // TMEM lane quadrant this warp may access
-    const int kl = qd * 32 + lane;                   // key lane (S^T) / d lane (O^T)
-    const int c0 = grp * 32;
+    constexpr int CG = kGroupCols;
+    const int grp = (warp - 4) >> 2;                   // column group: queries [CG grp, CG grp + CG)
+    const int tid = threadIdx.x - 128 * (grp + 1);     // 0..127 within the group
+    const int qd = warp & 3;                           // TMEM lane quadrant this warp may access
+    const int kl = qd * 32 + lane;                     // key lane (S^T) / d lane (O^T)
+    const int c0 = grp * CG;
     const int bar_vote = 1 + 2 * grp, bar_sync = 2 + 2 * grp;  // named barriers of this group
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     float* m_g = m_s + c0;
     float* delta_g = delta_s + c0;
-    float* red_g = red_s + grp * 128;
+    float* red_g = red_s + grp * 4 * CG;
     const float cl = a.scale_log2;
     uint32_t g = 0;
     int it = 0;
+    ROLE_TIMER_START();
     for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int nb = (list_len(i) + 1) / 2;
       const int ob = it & 1;
 
-      float l[32];
+      float l[CG];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) l[j] = 0.0f;
+      for (int j = 0; j < CG; ++j) l[j] = 0.0f;
 
       for (int n = 0; n < nb; ++n, ++g) {
         const int sb = g & 1;
         const uint32_t su = g >> 1;
         const int ms = g % Ly::kMeta;
+        ROLE_MARK(7);
         mbar_wait(&bars[Ly::bMFull + ms], (g / Ly::kMeta) & 1, ctl, 11);
+        ROLE_MARK(0);
         const int2 vc = meta_s[ms];
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bMEmpty + ms]);
 
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
+        ROLE_MARK(1);
         tc_fence_after();
-        float x[32];
-        tmem_ld32(t_lane + sb * 64 + c0, x);
+        float x[CG];
+        tmem_ld16(t_lane + sb * 64 + c0, x);
         tmem_wait_ld();
+        ROLE_MARK(2);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bSEmpty + sb]);
 
         // x = logit * log2(e) - m  (m = 0 before the first block of the item)
-        float xm = -INFINITY;
         if (n == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] *= cl;
+          for (int j = 0; j < CG; ++j) x[j] *= cl;
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
+          for (int j = 0; j < CG; j += 4) {
             const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
             x[j] = fmaf(x[j], cl, -m4.x);
             x[j + 1] = fmaf(x[j + 1], cl, -m4.y);
@@ -452,28 +520,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int vcount = (kl < 64) ? vc.x : vc.y;
           if ((kl & 63) >= vcount) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = -INFINITY;
+            for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
           }
         }
         bool slow = true;
         if (n > 0) {
+          float t8[CG / 2];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) xm = fmaxf(xm, x[j]);
-          slow = named_bar_or(bar_vote, 128, xm > kRescaleLog2);
+          for (int j = 0; j < CG / 2; ++j) t8[j] = fmaxf(x[j], x[j + CG / 2]);
+#pragma unroll
+          for (int wdt = CG / 4; wdt > 0; wdt >>= 1)
+#pragma unroll
+            for (int j = 0; j < wdt; ++j) t8[j] = fmaxf(t8[j], t8[j + wdt]);
+          slow = named_bar_or(bar_vote, 128, t8[0] > kRescaleLog2);
         }
+        ROLE_MARK(3);
         if (slow) {
           // exact column maximum of this block over the group's 128 lanes; raise m by it
           float cm = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < CG; ++j) {
             float r;
             asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x[j]));
             if (j == lane) cm = r;
           }
-          red_g[qd * 32 + lane] = cm;
+          if (lane < CG) red_g[qd * CG + lane] = cm;
           named_bar_sync(bar_sync, 128);
-          if (tid < 32) {
-            const float c = fmaxf(fmaxf(red_g[tid], red_g[32 + tid]), fmaxf(red_g[64 + tid], red_g[96 + tid]));
+          if (tid < CG) {
+            const float c = fmaxf(fmaxf(red_g[tid], red_g[CG + tid]), fmaxf(red_g[2 * CG + tid], red_g[3 * CG + tid]));
             float d;
             if (n == 0) {
               d = (c == -INFINITY) ? 0.0f : c;
@@ -486,35 +560,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           named_bar_sync(bar_sync, 128);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] -= delta_g[j];
+          for (int j = 0; j < CG; ++j) x[j] -= delta_g[j];
           if (n > 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) l[j] *= ex2_approx(-delta_g[j]);
+            for (int j = 0; j < CG; ++j) l[j] *= ex2_approx(-delta_g[j]);
             // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
             const uint32_t gp = g - 1;
             mbar_wait(&bars[Ly::bPEmpty + (gp & 1)], (gp >> 1) & 1, ctl, 13);
             tc_fence_after();
-            float o[32];
-            tmem_ld32(t_lane + 128 + ob * 64 + c0, o);
+            float o[CG];
+            tmem_ld16(t_lane + 128 + ob * 64 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] *= ex2_approx(-delta_g[j]);
-            tmem_st32(t_lane + 128 + ob * 64 + c0, o);
+            for (int j = 0; j < CG; ++j) o[j] *= ex2_approx(-delta_g[j]);
+            tmem_st16(t_lane + 128 + ob * 64 + c0, o);
             tmem_wait_st();
             tc_fence_before();
           }
         }
-        // probabilities, partial row sums, this group's half of the P^T row (bf16, 128-byte swizzle)
+        ROLE_MARK(4);
+        // probabilities, partial row sums, this group's part of the P^T row (bf16, 128-byte swizzle)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < CG; ++j) {
           x[j] = ex2_approx(x[j]);
           l[j] += x[j];
         }
+        ROLE_MARK(5);
         mbar_wait(&bars[Ly::bPEmpty + sb], (su & 1) ^ 1, ctl, 14);
+        ROLE_MARK(6);
         uint8_t* prow = sm + Ly::oP + sb * Ly::kPBytes + kl * 128;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = grp * 4 + cc;  // 16-byte chunk = queries 8c .. 8c+7
+        for (int cc = 0; cc < CG / 8; ++cc) {
+          const int c = grp * (CG / 8) + cc;  // 16-byte chunk = queries 8c .. 8c+7
           U128 w4;
           w4.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
           w4.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
@@ -527,20 +604,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) mbar_arrive(&bars[Ly::bPFull + sb]);
       }
 
-      // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored)
-      warp_sum_scatter32(l, lane);
+      // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored):
+      // reduce-scatter over the warp's 32 lanes, lane j (j < CG) then holds column c0 + j
+#pragma unroll
+      for (int step = 0; step < 4; ++step) {
+        const int half = (CG / 2) >> step;
+        const int bit = 3 - step;
+        const bool upper = (lane >> bit) & 1;
+#pragma unroll
+        for (int j = 0; j < half; ++j) {
+          const float lo = l[j], hi = l[j + half];
+          const float send = upper ? lo : hi;
+          const float keep = upper ? hi : lo;
+          l[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << bit);
+        }
+      }
+      l[0] += __shfl_xor_sync(0xffffffffu, l[0], 16);
       if (it >= 2) mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 15);
-      lpart_s[(ob * 4 + qd) * 64 + c0 + lane] = l[0];
+      if (lane < CG) lpart_s[(ob * 4 + qd) * 64 + c0 + lane] = l[0];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[Ly::bLFull + ob]);
     }
+    ROLE_MARK(7);
+    if (tid == 0) ROLE_TIMER_SAVE(4 + (grp & 1));
   } else {
     // ============================================================ epilogue
-    const int tid = threadIdx.x - 384;  // 0..127
+    const int tid = threadIdx.x - 32 * kEpiWarp0;  // 0..127
     const int qd = warp & 3;
-    const int d = qd * 32 + lane;       // O^T lane = d
+    const int d = qd * 32 + lane;                  // O^T lane = d
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     int it = 0;
+    ROLE_TIMER_START();
     for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
@@ -554,33 +648,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.H + h)) : 0.0f;
       }
       const float oc = (d < D) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
+      ROLE_MARK(3);
       mbar_wait(&bars[Ly::bLFull + ob], (it >> 1) & 1, ctl, 16);
+      ROLE_MARK(0);
       if (tid < 64) {
         const float* lp = lpart_s + ob * 4 * 64 + tid;
         rl_s[tid] = rcp_approx((lp[0] + lp[64]) + (lp[128] + lp[192]));
       }
       mbar_wait(&bars[Ly::bOFull + ob], (it >> 1) & 1, ctl, 17);
-      tc_fence_after();
-      float o[64];
-      tmem_ld32(t_lane + 128 + ob * 64, o);
-      tmem_ld32(t_lane + 128 + ob * 64 + 32, o + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      named_bar_sync(5, 128);  // rl, gate, qtok ready; every lane of O^T read
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty + ob]);
-      if (d < D) {
-        uint16_t* out_col = a.out + (b * a.L * a.H + h) * D + d;
+      ROLE_MARK(1);
+      named_bar_sync(9, 128);  // rl, gate, qtok ready
+      uint16_t* out_col = a.out + (b * a.L * a.H + h) * D + d;
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          if (q < valid_i) {
-            const float val = fmaf(o[q], rl_s[q], gate_s[q] * oc);
-            out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+      for (int half = 0; half < 2; ++half) {
+        tc_fence_after();
+        float o[32];
+        tmem_ld32(t_lane + 128 + ob * 64 + 32 * half, o);
+        tmem_wait_ld();
+        if (half == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty + ob]);
+        }
+        if (d < D) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int q = 32 * half + j;
+            if (q < valid_i) {
+              const float val = fmaf(o[j], rl_s[q], gate_s[q] * oc);
+              out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+            }
           }
         }
       }
-      named_bar_sync(5, 128);  // smem of this item no longer read
+      named_bar_sync(9, 128);  // smem of this item no longer read
     }
+    ROLE_MARK(3);
+    if (tid == 0) ROLE_TIMER_SAVE(6);
   }
 
   // ---------------------------------------------------------------- teardown

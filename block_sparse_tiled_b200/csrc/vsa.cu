@@ -420,6 +420,16 @@ const char* vsa_last_error(void) { return g_last_error.c_str(); }
 
 const char* vsa_version(void) { return "vsa-b200 0.1 (sm_100a)"; }
 
+#ifdef VSA_ROLE_TIMERS
+// Per-role cycle counters of the last attention launch (timer builds only):
+// host[cta][role][counter], 160 x 8 x 8 unsigned 64-bit values.
+vsa_status vsa_role_timers(void* host) {
+  VSA_CUDA_TRY(cudaDeviceSynchronize());
+  VSA_CUDA_TRY(cudaMemcpyFromSymbol(host, vsa::g_role_cycles, sizeof(vsa::g_role_cycles)));
+  return VSA_OK;
+}
+#endif
+
 vsa_status vsa_plan_query(const vsa_geometry* g, vsa_plan_dims* out) {
   if (out == nullptr) return fail(VSA_ERR_INVALID_ARG, "out is NULL");
   Resolved r;
