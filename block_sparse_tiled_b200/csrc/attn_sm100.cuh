@@ -1,8 +1,12 @@
 // Block-sparse VSA-H3 attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// Work item = (b, h, query tile i).  Its key list is every tile for a prefix
-// query tile, else the P prefix tiles followed by the tile's selected video
-// tiles (ascending).  The list is walked two key tiles (128 keys) at a time.
+// Work item = (b, h, query tile i), numbered (b*H + h)*n_t + i.  Its key list
+// is every tile for a prefix query tile, else the P prefix tiles followed by
+// the tile's selected video tiles (ascending).  The list is walked two key
+// tiles (128 keys) at a time.  CTAs claim items in order from a global counter
+// (one per SM, persistent), so the items in flight stay within a head or two
+// and that head's K/V stays resident in L2 even though prefix query tiles cost
+// many times a video query tile.
 //
 // A query tile is only 64 rows, so the kernel works in the transposed form,
 // which keeps every row of the 128-row tcgen05 MMA busy:
@@ -98,6 +102,7 @@ struct AttnArgs {
   const uint16_t* gate;       // [B, L, H] bf16
   uint16_t* out;              // [B, L, H, D] bf16
   int* status;                // [2] device status word
+  int* sched;                 // item counter, zero at launch
   int64_t L;
   int H, n_t, P, topk;
   float scale_log2;  // softmax scale * log2(e)
@@ -115,6 +120,7 @@ struct AttnLayout {
   static constexpr int kKStages = 2;
   static constexpr int kVStages = 3;
   static constexpr int kMeta = 8;  // per-block key-valid counts in flight
+  static constexpr int kRing = 8;  // claimed items in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQBufs * kQBytes;
@@ -131,11 +137,13 @@ struct AttnLayout {
   static constexpr int bMFull = bPEmpty + 2, bMEmpty = bMFull + kMeta;
   static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 2;
   static constexpr int bLFull = bOEmpty + 2;
-  static constexpr int bDoneS = bLFull + 2, bDonePV = bDoneS + 1;
+  static constexpr int bRFull = bLFull + 2, bREmpty = bRFull + kRing;
+  static constexpr int bDoneS = bREmpty + kRing, bDonePV = bDoneS + 1;
   static constexpr int kNumBars = bDonePV + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;          // tmem base, abort flag
   static constexpr int oMeta = ((oMisc + 8 + 15) / 16) * 16;  // int2 meta[kMeta]
-  static constexpr int oM = oMeta + kMeta * 8;               // float m[64] (log2 units)
+  static constexpr int oRing = oMeta + kMeta * 8;            // int ring[kRing]: claimed items, -1 = none left
+  static constexpr int oM = oRing + kRing * 4;               // float m[64] (log2 units)
   static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
   static constexpr int oRed = oDelta + 256;                  // float red[groups][4 quadrants][group columns]
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
@@ -195,6 +203,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::oMisc + 4);
   int2* meta_s = reinterpret_cast<int2*>(sm + Ly::oMeta);
+  int* ring_s = reinterpret_cast<int*>(sm + Ly::oRing);
   float* m_s = reinterpret_cast<float*>(sm + Ly::oM);
   float* delta_s = reinterpret_cast<float*>(sm + Ly::oDelta);
   float* red_s = reinterpret_cast<float*>(sm + Ly::oRed);
@@ -239,6 +248,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars[Ly::bMFull + s], 1);
       mbar_init(&bars[Ly::bMEmpty + s], kSoftWarps);
     }
+    for (int s = 0; s < Ly::kRing; ++s) {
+      mbar_init(&bars[Ly::bRFull + s], 1);
+      mbar_init(&bars[Ly::bREmpty + s], 3 + kSoftWarps + 4);  // V producer, two issuers, softmax, epilogue
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[Ly::bOFull + s], 1);
       mbar_init(&bars[Ly::bOEmpty + s], 4);
@@ -267,6 +280,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (i < P || t < P) return t;
     return __ldg(a.idx + (bh * V + (i - P)) * topk + (t - P));
   };
+  // Claimed item number `it` of this CTA (-1: none left), read by one thread of a consumer warp.
+  auto ring_take = [&](int it, int site) -> int {
+    const int slot = it % Ly::kRing;
+    const bool ok = mbar_wait(&bars[Ly::bRFull + slot], (it / Ly::kRing) & 1, ctl, site);
+    const int w = ok ? ring_s[slot] : -1;
+    mbar_arrive(&bars[Ly::bREmpty + slot]);
+    return w;
+  };
 
   if (warp <= 1) {
     // ============================================================ TMA producers (warp 0: Q + K, warp 1: V)
@@ -280,7 +301,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int it = 0;
     bool ok = true;
     ROLE_TIMER_START();
-    for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
+    // Lane 0 of the K producer claims items (global counter) two ahead of its own use and
+    // publishes them in the ring; -1 marks the end.  The other roles read the ring.
+    int pub = 0;       // items published so far
+    bool more = true;  // the counter may still have items
+    auto publish_next = [&]() {
+      if (!more) return;
+      const int slot = pub % Ly::kRing;
+      if (!mbar_wait(&bars[Ly::bREmpty + slot], ((pub / Ly::kRing) & 1) ^ 1, ctl, 24)) {
+        more = false;
+        return;
+      }
+      const int64_t claimed = atomicAdd(a.sched, 1);
+      const int v = (claimed < a.n_items) ? static_cast<int>(claimed) : -1;
+      ring_s[slot] = v;
+      mbar_arrive(&bars[Ly::bRFull + slot]);
+      ++pub;
+      if (v < 0) more = false;
+    };
+    if (is_k && lane == 0) {
+      publish_next();
+      publish_next();
+    }
+    for (;; ++it) {
+      int w = -1;
+      if (lane == 0) {
+        if (is_k) {
+          w = (it < pub) ? ring_s[it % Ly::kRing] : -1;
+          publish_next();
+        } else {
+          w = ring_take(it, 25);
+        }
+      }
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (w < 0 || !ok) break;
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int nk = list_len(i), nb = (nk + 1) / 2;
@@ -370,7 +424,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int it = 0;
       bool ok = true;
       ROLE_TIMER_START();
-      for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
+      for (;; ++it) {
+        const int w = ring_take(it, 26);
+        if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
         const int nb = (list_len(i) + 1) / 2;
@@ -414,7 +470,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int it = 0;
       bool ok = true;
       ROLE_TIMER_START();
-      for (int64_t w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++it) {
+      for (;; ++it) {
+        const int w = ring_take(it, 27);
+        if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t);
         const int nb = (list_len(i) + 1) / 2;
@@ -470,7 +528,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t g = 0;
     int it = 0;
     ROLE_TIMER_START();
-    for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
+    for (;; ++it) {
+      int w = (lane == 0) ? ring_take(it, 28) : 0;
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int nb = (list_len(i) + 1) / 2;
@@ -635,7 +696,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     int it = 0;
     ROLE_TIMER_START();
-    for (int64_t w = blockIdx.x; w < a.n_items; w += gridDim.x, ++it) {
+    for (;; ++it) {
+      int w = (lane == 0) ? ring_take(it, 29) : 0;
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (named_bar_or(9, 128, w < 0)) break;  // the epilogue warps stop together
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int64_t b = bh / a.H;

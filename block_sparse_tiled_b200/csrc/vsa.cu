@@ -256,7 +256,7 @@ struct vsa_plan_s {
   std::vector<int32_t> tile_token, tile_valid;
   int32_t* d_tile_token = nullptr;
   int32_t* d_tile_valid = nullptr;
-  int* d_status = nullptr;
+  int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter
   vsa_workspace_layout ws{};
 };
 
@@ -379,6 +379,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.gate = static_cast<const uint16_t*>(gate);
   a.out = static_cast<uint16_t*>(out);
   a.status = p->d_status;
+  a.sched = p->d_status + 2;
   a.L = p->r.L;
   a.H = p->H;
   a.n_t = p->n_t;
@@ -387,6 +388,8 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.scale_log2 = static_cast<float>(static_cast<double>(p->r.scale) * 1.4426950408889634);
   a.n_items = static_cast<int64_t>(p->B) * p->H * p->n_t;
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
+  // the item counter of the persistent schedule starts at zero for every launch
+  VSA_CUDA_TRY(cudaMemsetAsync(a.sched, 0, sizeof(int), s));
   if (p->D == 128) {
     const size_t smem = vsa::AttnLayout<128>::bytes(p->n_t);
     if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
@@ -484,7 +487,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   const size_t tok_bytes = std::max<size_t>(4, p->tile_token.size() * 4);
   const size_t val_bytes = std::max<size_t>(4, p->tile_valid.size() * 4);
   if (cudaMalloc(&p->d_tile_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_tile_valid, val_bytes) != cudaSuccess ||
-      cudaMalloc(&p->d_status, 2 * sizeof(int)) != cudaSuccess) {
+      cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
   }
@@ -493,7 +496,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     e = cudaMemcpyAsync(p->d_tile_token, p->tile_token.data(), p->tile_token.size() * 4, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !p->tile_valid.empty())
     e = cudaMemcpyAsync(p->d_tile_valid, p->tile_valid.data(), p->tile_valid.size() * 4, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 2 * sizeof(int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 4 * sizeof(int), s);
   if (e != cudaSuccess) {
     cleanup();
     return fail(VSA_ERR_CUDA, std::string("plan upload: ") + cudaGetErrorString(e));

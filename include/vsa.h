@@ -40,6 +40,9 @@
  *    a multiple of 4.  Video tokens follow the prefix in raster (t, h, w)
  *    order, w fastest.  Inside a tile the valid tokens come first, in
  *    sequence (prefix) or raster (cube) order, then zero pads.
+ *  - A plan's device status word and the attention kernel's work counter are
+ *    shared by every call made with that plan: calls with one plan must not
+ *    overlap on the GPU (use one plan per concurrent stream).
  *  - Errors: argument and shape errors are detected on the host and returned
  *    synchronously with nothing launched; a failed launch returns
  *    VSA_ERR_CUDA; device-side failures (a bounded wait that ran out) are
