@@ -33,7 +33,9 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
     int n_t) {
-  constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  constexpr int kChunks = D / 8;                 // 16-byte chunks per row
+  constexpr int kPerTensor = kTile * kChunks;    // chunks per tile of one tensor
+  constexpr int kIters = kPerTensor / 128;       // each of 128 threads per tensor moves kIters chunks
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);  // [3][64][D]
   __shared__ int32_t tok_s[kTile];
@@ -43,33 +45,35 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   if (threadIdx.x < kTile) tok_s[threadIdx.x] = tile_token[static_cast<int64_t>(tile) * kTile + threadIdx.x];
   __syncthreads();
 
+  // threads [128 t, 128 t + 128) move tensor t; all loads are issued before any store
+  const int tsr = threadIdx.x >> 7, tl = threadIdx.x & 127;
+  const uint16_t* src = (tsr == 0) ? q : (tsr == 1) ? k : v;
+  uint16_t* dst = (tsr == 0) ? q_t : (tsr == 1) ? k_t : v_t;
   const int64_t dst_base = ((static_cast<int64_t>(b) * H + h) * n_t + tile) * kTile * D;
-  const uint16_t* srcs[3] = {q, k, v};
-  uint16_t* dsts[3] = {q_t, k_t, v_t};
-  for (int e = threadIdx.x; e < 3 * kTile * kChunks; e += blockDim.x) {
-    const int tsr = e / (kTile * kChunks);
-    const int rem = e - tsr * (kTile * kChunks);
-    const int r = rem / kChunks, c = rem - r * kChunks;
+  uint4 val[kIters];
+#pragma unroll
+  for (int u = 0; u < kIters; ++u) {
+    const int e = tl + 128 * u;
+    const int r = e / kChunks, c = e - r * kChunks;
     const int32_t tok = tok_s[r];
-    U128 val = {0u, 0u, 0u, 0u};
-    if (tok >= 0) {
-      const uint4* src = reinterpret_cast<const uint4*>(srcs[tsr] + ((static_cast<int64_t>(b) * L + tok) * H + h) * D);
-      const uint4 t4 = __ldg(src + c);
-      val = U128{t4.x, t4.y, t4.z, t4.w};
-    }
-    reinterpret_cast<U128*>(dsts[tsr] + dst_base)[r * kChunks + c] = val;
-    if (pool) reinterpret_cast<U128*>(tiles + tsr * kTile * D)[r * kChunks + c] = val;
+    val[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (tok >= 0) val[u] = __ldg(reinterpret_cast<const uint4*>(src + ((static_cast<int64_t>(b) * L + tok) * H + h) * D) + c);
+  }
+#pragma unroll
+  for (int u = 0; u < kIters; ++u) {
+    const int e = tl + 128 * u;
+    reinterpret_cast<uint4*>(dst + dst_base)[e] = val[u];
+    if (pool) reinterpret_cast<uint4*>(tiles + tsr * kTile * D)[e] = val[u];
   }
   if (!pool) return;
   __syncthreads();
   const int n = tile_valid[tile];
-  float* outs[3] = {pq, pk, pv};
-  for (int e = threadIdx.x; e < 3 * D; e += blockDim.x) {
-    const int tsr = e / D, d = e - tsr * D;
+  float* out = (tsr == 0) ? pq : (tsr == 1) ? pk : pv;
+  for (int d = tl; d < D; d += 128) {
     const uint16_t* col = tiles + tsr * kTile * D + d;
     float sum = 0.0f;
     for (int r = 0; r < n; ++r) sum = __fadd_rn(sum, bf16_bits_to_f32(col[r * D]));
-    outs[tsr][((static_cast<int64_t>(b) * H + h) * n_t + tile) * D + d] = __fdiv_rn(sum, static_cast<float>(n));
+    out[((static_cast<int64_t>(b) * H + h) * n_t + tile) * D + d] = __fdiv_rn(sum, static_cast<float>(n));
   }
 }
 
@@ -104,53 +108,76 @@ __global__ void __launch_bounds__(384) pool_tiles_kernel(const uint16_t* __restr
 // A 64 x 64 block of S per CTA, 4 x 4 outputs per thread, d staged through
 // shared memory 32 at a time; every output's chain runs d = 0..D-1 in order.
 // ---------------------------------------------------------------------------
-constexpr int kScoreBlk = 64;
-constexpr int kScoreDk = 32;
+constexpr int kScoreBlk = 128;
+constexpr int kScoreDk = 16;
 
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ pq, const float* __restrict__ pk,
                                                       float* __restrict__ S, int n_t, int D, float scale) {
-  __shared__ __align__(16) float As[kScoreDk][kScoreBlk + 4];
-  __shared__ __align__(16) float Bs[kScoreDk][kScoreBlk + 4];
+  __shared__ __align__(16) float As[2][kScoreDk][kScoreBlk];
+  __shared__ __align__(16) float Bs[2][kScoreDk][kScoreBlk];
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * kScoreBlk, j0 = blockIdx.x * kScoreBlk;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 8 x 8 outputs: rows ty + 16a, cols tx + 16c
   const float* A = pq + static_cast<int64_t>(bh) * n_t * D;
   const float* Bm = pk + static_cast<int64_t>(bh) * n_t * D;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
 
-  for (int d0 = 0; d0 < D; d0 += kScoreDk) {
-    // stage pq[i0..i0+63][d0..d0+31] and pk[j0..][d0..] transposed (d-major)
-    for (int e = threadIdx.x; e < kScoreBlk * kScoreDk; e += 256) {
-      const int r = e / kScoreDk, dd = e - r * kScoreDk;
+  // staging: 128 rows x 16 d of pq and of pk, one float4 per thread each (d-major in shared memory)
+  const int sr = threadIdx.x >> 2, sd = (threadIdx.x & 3) * 4;  // row 0..63 (+64), d offset 0..12
+  auto load = [&](int d0, float4* ra, float4* rb) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = sr + 64 * hh;
       const int i = i0 + r, j = j0 + r;
-      As[dd][r] = (i < n_t) ? A[static_cast<int64_t>(i) * D + d0 + dd] : 0.0f;
-      Bs[dd][r] = (j < n_t) ? Bm[static_cast<int64_t>(j) * D + d0 + dd] : 0.0f;
+      ra[hh] = (i < n_t) ? *reinterpret_cast<const float4*>(A + static_cast<int64_t>(i) * D + d0 + sd)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      rb[hh] = (j < n_t) ? *reinterpret_cast<const float4*>(Bm + static_cast<int64_t>(j) * D + d0 + sd)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
-#pragma unroll 8
+  };
+  auto store = [&](int buf, const float4* ra, const float4* rb) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = sr + 64 * hh;
+      As[buf][sd + 0][r] = ra[hh].x; As[buf][sd + 1][r] = ra[hh].y; As[buf][sd + 2][r] = ra[hh].z; As[buf][sd + 3][r] = ra[hh].w;
+      Bs[buf][sd + 0][r] = rb[hh].x; Bs[buf][sd + 1][r] = rb[hh].y; Bs[buf][sd + 2][r] = rb[hh].z; Bs[buf][sd + 3][r] = rb[hh].w;
+    }
+  };
+  float4 ra[2], rb[2];
+  load(0, ra, rb);
+  store(0, ra, rb);
+  __syncthreads();
+  const int nsteps = D / kScoreDk;
+  for (int st = 0; st < nsteps; ++st) {
+    const int buf = st & 1;
+    if (st + 1 < nsteps) load((st + 1) * kScoreDk, ra, rb);
+    // d runs 0..D-1 in order for every output: chunks in order, and d in order inside a chunk
+#pragma unroll
     for (int dd = 0; dd < kScoreDk; ++dd) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[dd][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[dd][tx * 4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+      float av[8], bv[8];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 8; ++a) av[a] = As[buf][dd][ty + 16 * a];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = __fmaf_rn(av[a], bv[c], acc[a][c]);
+      for (int c = 0; c < 8; ++c) bv[c] = Bs[buf][dd][tx + 16 * c];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(av[a], bv[c], acc[a][c]);
     }
+    if (st + 1 < nsteps) store(buf ^ 1, ra, rb);
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty * 4 + a;
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + ty + 16 * a;
     if (i >= n_t) continue;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = j0 + tx * 4 + c;
+    for (int c = 0; c < 8; ++c) {
+      const int j = j0 + tx + 16 * c;
       if (j < n_t) S[(static_cast<int64_t>(bh) * n_t + i) * n_t + j] = __fmul_rn(acc[a][c], scale);
     }
   }
@@ -218,45 +245,42 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
 
 // ---------------------------------------------------------------------------
 // S4 compression: o_c[bh, i, :] = sum_j softmax_j(S[bh, i, :]) pv[bh, j, :]
-// over all n_t tiles, binary32.  A CTA owns 64 rows of one (b, h): first each
-// row's max and exp-sum (4 threads per row), then the weighted sum of pooled
-// V rows staged 32 tiles at a time.
+// over all n_t tiles, binary32.  A CTA owns 128 rows of one (b, h): a first
+// pass finds each row's maximum; the second stages w = exp(S - max) (each
+// computed once, its row sum accumulated alongside) and pooled V rows 32
+// tiles at a time, and every thread accumulates 8 rows x D/16 columns.
 // ---------------------------------------------------------------------------
-constexpr int kCompRows = 64;
+constexpr int kCompRows = 128;
 constexpr int kCompJ = 32;
 
 template <int D>
 __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
                                                         float* __restrict__ o_c, int n_t) {
-  __shared__ float m_s[kCompRows], inv_s[kCompRows];
-  __shared__ __align__(16) float W_s[kCompRows][kCompJ + 1];
+  constexpr int kCols = D / 16;  // columns per thread: tx + 16 c
+  __shared__ float m_s[kCompRows], l_s[kCompRows];
+  __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
   __shared__ __align__(16) float PV_s[kCompJ][D];
   const int bh = blockIdx.y, i0 = blockIdx.x * kCompRows;
   const float* Sb = S + static_cast<int64_t>(bh) * n_t * n_t;
   const float* PVb = pv + static_cast<int64_t>(bh) * n_t * D;
 
-  {  // row statistics: 4 threads per row
-    const int r = threadIdx.x >> 2, part = threadIdx.x & 3;
+  {  // row maxima: 2 threads per row
+    const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
     const int i = i0 + r;
     float m = -INFINITY;
     if (i < n_t)
-      for (int j = part; j < n_t; j += 4) m = fmaxf(m, Sb[static_cast<int64_t>(i) * n_t + j]);
+      for (int j = part; j < n_t; j += 2) m = fmaxf(m, __ldg(Sb + static_cast<int64_t>(i) * n_t + j));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    float l = 0.0f;
-    if (i < n_t)
-      for (int j = part; j < n_t; j += 4) l += expf(Sb[static_cast<int64_t>(i) * n_t + j] - m);
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if (part == 0) {
-      m_s[r] = m;
-      inv_s[r] = (i < n_t) ? 1.0f / l : 0.0f;
-    }
+    if (part == 0) m_s[r] = m;
   }
   __syncthreads();
 
-  constexpr int kCols = D / 32;  // d values per thread: thread owns rows r0..r0+7 (step 8) and d = lane + 32c
-  const int lane = threadIdx.x & 31, rgrp = threadIdx.x >> 5;  // 8 row groups of 8 rows
+  // staging map for W: thread -> (row r = t >> 1, 16 consecutive j of the chunk)
+  const int wr = threadIdx.x >> 1, wj0 = (threadIdx.x & 1) * 16;
+  const int wi = i0 + wr;
+  const float wm = m_s[wr];
+  float lsum = 0.0f;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // outputs: rows ty + 16a, cols tx + 16c
   float acc[8][kCols];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
@@ -264,38 +288,45 @@ __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__
     for (int c = 0; c < kCols; ++c) acc[a][c] = 0.0f;
 
   for (int j0 = 0; j0 < n_t; j0 += kCompJ) {
-    for (int e = threadIdx.x; e < kCompRows * kCompJ; e += 256) {
-      const int r = e / kCompJ, jj = e - r * kCompJ;
-      const int i = i0 + r, j = j0 + jj;
-      W_s[r][jj] = (i < n_t && j < n_t) ? expf(Sb[static_cast<int64_t>(i) * n_t + j] - m_s[r]) : 0.0f;
+#pragma unroll 4
+    for (int u = 0; u < 16; ++u) {
+      const int jj = wj0 + u, j = j0 + jj;
+      float w = 0.0f;
+      if (wi < n_t && j < n_t) w = expf(__ldg(Sb + static_cast<int64_t>(wi) * n_t + j) - wm);
+      W_s[jj][wr] = w;
+      lsum += w;
     }
     for (int e = threadIdx.x; e < kCompJ * D; e += 256) {
       const int jj = e / D, d = e - jj * D;
       const int j = j0 + jj;
-      PV_s[jj][d] = (j < n_t) ? PVb[static_cast<int64_t>(j) * D + d] : 0.0f;
+      PV_s[jj][d] = (j < n_t) ? __ldg(PVb + static_cast<int64_t>(j) * D + d) : 0.0f;
     }
     __syncthreads();
 #pragma unroll 4
     for (int jj = 0; jj < kCompJ; ++jj) {
-      float pvv[kCols];
+      float wv[8], pvv[kCols];
 #pragma unroll
-      for (int c = 0; c < kCols; ++c) pvv[c] = PV_s[jj][lane + 32 * c];
+      for (int a = 0; a < 8; ++a) wv[a] = W_s[jj][ty + 16 * a];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const float w = W_s[rgrp * 8 + a][jj];
+      for (int c = 0; c < kCols; ++c) pvv[c] = PV_s[jj][tx + 16 * c];
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) acc[a][c] = fmaf(w, pvv[c], acc[a][c]);
-      }
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) acc[a][c] = fmaf(wv[a], pvv[c], acc[a][c]);
     }
     __syncthreads();
   }
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  if ((threadIdx.x & 1) == 0) l_s[wr] = lsum;
+  __syncthreads();
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    const int r = rgrp * 8 + a, i = i0 + r;
+    const int r = ty + 16 * a, i = i0 + r;
     if (i >= n_t) continue;
+    const float inv = 1.0f / l_s[r];
 #pragma unroll
     for (int c = 0; c < kCols; ++c)
-      o_c[(static_cast<int64_t>(bh) * n_t + i) * D + lane + 32 * c] = acc[a][c] * inv_s[r];
+      o_c[(static_cast<int64_t>(bh) * n_t + i) * D + tx + 16 * c] = acc[a][c] * inv;
   }
 }
 
