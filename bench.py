@@ -354,7 +354,7 @@ def main():
     ap.add_argument("--workload", default="768p_s0.9")
     ap.add_argument("--sparsity", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-every", type=int, default=4)
+    ap.add_argument("--cpu-every", type=int, default=1)
     ap.add_argument("--ref-every", type=int, default=16)
     args = ap.parse_args()
     import synth

@@ -35,7 +35,7 @@ EXPORTED = (
     "vsa_plan_tiles", "vsa_plan_info", "vsa_plan_tables", "vsa_plan_query", "vsa_plan_tables_host",
     "vsa_plan_destroy",
     "vsa_gather_tiles", "vsa_pool_and_score", "vsa_topk_select", "vsa_sparse_attn_fwd", "vsa_forward",
-    "vsa_forward_noalloc",
+    "vsa_forward_noalloc", "vsa_wait_selftest",
     "vsa_plan_workspace", "vsa_device_status", "vsa_last_error", "vsa_version",
 )
 
@@ -99,6 +99,7 @@ def load_library(path: str = LIB_PATH):
     lib.vsa_sparse_attn_fwd.argtypes = [P] * 9
     lib.vsa_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.vsa_forward_noalloc.argtypes = [P] * 7
+    lib.vsa_wait_selftest.argtypes = [P, ctypes.c_int64, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     lib.vsa_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED:
         if name not in ("vsa_last_error", "vsa_version"):
@@ -310,6 +311,14 @@ def vsa_forward_noalloc(plan, q, k, v, gate, out, stream=None):
         plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(gate, bf, "gate"),
         _ptr(out, bf, "out"), _stream(stream)), "vsa_forward_noalloc")
     return out
+
+
+def wait_selftest(plan, timeout_ns=50_000_000, stream=None):
+    """Run the bounded-wait self-test; returns the (code, site) it recorded."""
+    code, where = ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().vsa_wait_selftest(plan.handle, int(timeout_ns), _stream(stream), ctypes.byref(code),
+                                            ctypes.byref(where)), "vsa_wait_selftest")
+    return code.value, where.value
 
 
 def device_status(plan, stream=None):

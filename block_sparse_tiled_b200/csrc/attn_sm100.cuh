@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = a.n_t, P = a.P, topk = a.topk, V = n_t - P;
-  const WaitCtl ctl{abort_flag, a.status};
+  const WaitCtl ctl{abort_flag, a.status, kWaitTimeoutNs};
 
   // ---------------------------------------------------------------- setup
   for (int t = threadIdx.x; t < n_t; t += blockDim.x) tile_valid_s[t] = static_cast<uint8_t>(a.tile_valid[t]);
@@ -404,15 +404,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     // drain: every load this warp issued must land before the CTA exits
     if (lane == 0) {
-      const WaitCtl drain{abort_flag, a.status};
+      const WaitCtl drain{abort_flag, a.status, kWaitTimeoutNs};
       for (int s = 0; s < nstages && static_cast<uint32_t>(s) < g; ++s) {
         const uint32_t last = g - 1 - s;
-        wait_slow(&bars[b_full + (last % nstages)], (last / nstages) & 1, drain, 20);
+        mbar_wait_drain(&bars[b_full + (last % nstages)], (last / nstages) & 1, drain, 20);
       }
       if (is_k && it > 0) {
         for (int s = 0; s < Ly::kQBufs && s < it; ++s) {
           const int lastq = it - 1 - s;
-          wait_slow(&bars[Ly::bQFull + (lastq % Ly::kQBufs)], (lastq / Ly::kQBufs) & 1, drain, 21);
+          mbar_wait_drain(&bars[Ly::bQFull + (lastq % Ly::kQBufs)], (lastq / Ly::kQBufs) & 1, drain, 21);
         }
       }
     }
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ROLE_MARK(3);
       ROLE_TIMER_SAVE(2);
       umma_commit(&bars[Ly::bDoneS]);
-      wait_slow(&bars[Ly::bDoneS], 0, WaitCtl{abort_flag, a.status}, 22);
+      mbar_wait_drain(&bars[Ly::bDoneS], 0, ctl, 22);
     }
     __syncwarp();
   } else if (warp == 3) {
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ROLE_MARK(3);
       ROLE_TIMER_SAVE(3);
       umma_commit(&bars[Ly::bDonePV]);
-      wait_slow(&bars[Ly::bDonePV], 0, WaitCtl{abort_flag, a.status}, 23);
+      mbar_wait_drain(&bars[Ly::bDonePV], 0, ctl, 23);
     }
     __syncwarp();
   } else if (warp < kEpiWarp0) {

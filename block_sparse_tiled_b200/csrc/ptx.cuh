@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05
 // (TMEM allocation, MMA, commit, TMEM load/store), named barriers.
-// Every wait here is bounded: it gives up after kWaitTimeoutNs of wall time,
+// Every wait here is bounded: it gives up after a wall-time limit (WaitCtl),
 // records the failure in the kernel's status word and returns false, so a
 // lost arrival ends the kernel with an error instead of hanging the GPU.
 #pragma once
@@ -8,7 +8,7 @@
 
 namespace vsa {
 
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s: the kernels' limit
 constexpr int kStatusTimeout = 6;                    // == VSA_ERR_TIMEOUT
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -65,6 +65,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 struct WaitCtl {
   volatile int* abort_flag;  // shared memory: set once any wait of the CTA gave up
   int* status;               // global: [0] = error code, [1] = site of the first failure
+  uint64_t timeout_ns;       // wall-time limit of one wait
 };
 
 __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int site) {
@@ -73,7 +74,7 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const Wai
     if (*ctl.abort_flag) return false;
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if ((it & 63) == 0) {
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > ctl.timeout_ns) {
         *ctl.abort_flag = 1;
         if (atomicCAS(ctl.status, 0, kStatusTimeout) == 0) atomicExch(ctl.status + 1, site);
         return false;
@@ -86,6 +87,37 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const Wai
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   return wait_slow(bar, parity, ctl, site);
+}
+
+// Wait for work this thread issued itself (TMA copies, tcgen05 operations) to
+// complete before the CTA exits.  That work completes on its own, so the
+// CTA's abort flag is not consulted; the wait is still bounded by the limit.
+__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int site) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((it & 63) == 0 && globaltimer_ns() - t0 > ctl.timeout_ns) {
+      if (atomicCAS(ctl.status, 0, kStatusTimeout) == 0) atomicExch(ctl.status + 1, site);
+      return false;
+    }
+  }
+}
+
+// Failure-detection self-test: every thread waits on an mbarrier that nothing
+// arrives on, with a limit of timeout_ns.  The first wait to run out records
+// the timeout in `status`; the others give up on seeing the CTA's abort flag.
+__global__ void wait_selftest_kernel(int* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl ctl{&abort_flag, status, timeout_ns};
+  mbar_wait(&bar, 0, ctl, 100 + static_cast<int>(threadIdx.x >> 5));  // phase 0 never completes
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------- TMA

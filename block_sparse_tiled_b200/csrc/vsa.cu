@@ -622,6 +622,17 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k,
   return vsa_forward(p, q, k, v, gate, out, scratch, VSA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+vsa_status vsa_wait_selftest(vsa_plan p, int64_t timeout_ns, void* stream, int32_t* code, int32_t* where) {
+  VSA_TRY(check_plan(p));
+  if (timeout_ns < 1000 || timeout_ns > 10000000000ll)
+    return fail(VSA_ERR_INVALID_ARG, "timeout_ns must lie in [1e3, 1e10]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  VSA_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, 2 * sizeof(int), s));
+  vsa::wait_selftest_kernel<<<1, 64, 0, s>>>(p->d_status, static_cast<uint64_t>(timeout_ns));
+  VSA_TRY(launch_check("wait self-test"));
+  return vsa_device_status(p, stream, code, where);
+}
+
 vsa_status vsa_device_status(vsa_plan p, void* stream, int32_t* code, int32_t* where) {
   VSA_TRY(check_plan(p));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -234,6 +234,17 @@ typedef struct vsa_workspace_layout {
 } vsa_workspace_layout;
 vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
 
+/* Failure-detection self-test.  No counterpart on the pages: it checks the
+ * library's own safety net.  It launches one small kernel whose threads wait,
+ * with the same bounded-wait code the attention kernel uses, on a barrier that
+ * nothing ever arrives on, with a limit of timeout_ns (1e3 .. 1e10).  The first
+ * wait to run out writes VSA_ERR_TIMEOUT and a site code to the plan's device
+ * status word; the other threads give up when they see the abort.  The call
+ * synchronises `stream`, returns the status word in *code and *where (NULL
+ * allowed), and clears it.  A working build returns VSA_OK with *code ==
+ * VSA_ERR_TIMEOUT, after about timeout_ns.  The GPU context stays usable. */
+vsa_status vsa_wait_selftest(vsa_plan p, int64_t timeout_ns, void* stream, int32_t* code, int32_t* where);
+
 /* Read (synchronising `stream`) and clear the plan's device status word.
  * *code receives VSA_OK or VSA_ERR_TIMEOUT; *where a kernel-specific site
  * code (0 if none). */

@@ -7,6 +7,8 @@ max-abs 2e-2 and mean-abs 2e-3 of the float64 oracle.  Small workloads are
 compared in full; the 480p- and 1344x768-shaped workloads compare the whole
 selection and a fixed sample of query tiles of the attention.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -226,3 +228,32 @@ def test_call_errors(vsa):
     assert call(ctypes.c_void_p(qp), ctypes.c_void_p(ws.data_ptr() + 16), ws.numel() - 16) == 1  # unaligned ws
     assert call(ctypes.c_void_p(qp), wsp, ws.numel()) == 0
     torch.cuda.synchronize()
+
+
+def test_768p_s08_selection_full_attention_sampled(vsa, oracle_mod):
+    """The 1344x768-shaped workload at sparsity 0.8 (topk 231)."""
+    sampled_parity(vsa, oracle_mod, synth.workload("768p_s0.8"), heads=[0, 55], video_every=157)
+
+
+@pytest.mark.parametrize("sparsity", [0.0, 0.95])
+def test_768p_sweep_endpoints_sampled(vsa, oracle_mod, sparsity):
+    """Ends of the sparsity sweep at 1344x768: dense video keys (topk 1152) and topk 58."""
+    w = dataclasses.replace(synth.workload("768p_s0.9"), sparsity=sparsity, name=f"768p_s{sparsity}")
+    sampled_parity(vsa, oracle_mod, w, heads=[13], video_every=383)
+
+
+def test_wait_selftest_times_out_and_context_stays_usable(vsa):
+    """A bounded wait on a barrier that nothing arrives on ends with
+    VSA_ERR_TIMEOUT in the status word; the next forward runs normally."""
+    w = synth.workload("tiny")
+    plan = plan_for(vsa, w)
+    code, where = vsa.wait_selftest(plan, timeout_ns=50_000_000)
+    assert code == 6 and where in (100, 101)
+    assert vsa.device_status(plan) == (0, 0)
+    x = synth.make_inputs(w, device="cuda")
+    ws = vsa.alloc_workspace(plan)
+    out = vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    assert vsa.device_status(plan) == (0, 0)
+    plan.destroy()
