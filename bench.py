@@ -50,6 +50,30 @@ def load_peaks():
     return dict(source="fallback", bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0)
 
 
+def measured_attn_traffic():
+    """DRAM bytes (read + write) of one attention launch from the committed ncu
+    capture, or None when the kernel sources changed since it was taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "vsa_attn_kernel_768p_s0.9_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    for rel in ("block_sparse_tiled_b200/csrc/attn_sm100.cuh", "block_sparse_tiled_b200/csrc/ptx.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if vals.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    return int(vals["dram_bytes_read"]) + int(vals["dram_bytes_write"])
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
 
@@ -322,7 +346,8 @@ def run_vsa(args, w, world, rank, local):
         "peak_kind": f"{peaks['source']} sustained dense bf16 (kernel timed inside a seconds-long loop)",
         "frac_of_burst_peak": attn_tflops / peaks["bf16_tflops"],
         "algorithmic_flop_per_launch": flops_call,
-        "traffic": None,
+        "traffic": measured_attn_traffic() if w.name == "768p_s0.9" else None,
+        "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
     }
     launches = 5 * args.steps
     line = {
