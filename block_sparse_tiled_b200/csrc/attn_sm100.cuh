@@ -92,7 +92,9 @@ constexpr int kAttnThreads = 32 * (kEpiWarp0 + 4);
 // at most 2^23 keys per row, row sums stay below 2^47 and P.V partial sums far
 // below the binary32 range.
 constexpr float kRescaleLog2 = 24.0f;
-constexpr uint32_t kTmemCols = 256;  // S^T double buffer (2 x 64) + O^T double buffer (2 x 64)
+constexpr int kSBufs = 2;            // S^T buffers in TMEM (64 columns each)
+constexpr int kOCol0 = 64 * kSBufs;  // O^T double buffer follows (2 x 64 columns)
+constexpr uint32_t kTmemCols = (kOCol0 + 128 <= 256) ? 256 : 512;
 
 struct AttnArgs {
   const int32_t* idx;         // [B, H, V, topk] global key-tile indices (ascending per row)
@@ -119,22 +121,23 @@ struct AttnLayout {
   static constexpr int kQBufs = 1;
   static constexpr int kKStages = 2;
   static constexpr int kVStages = 3;
-  static constexpr int kMeta = 8;  // per-block key-valid counts in flight
+  static constexpr int kPBufs = 2;  // P^T buffers in shared memory
+  static constexpr int kMeta = 8;   // per-block key-valid counts in flight
   static constexpr int kRing = 8;  // claimed items in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQBufs * kQBytes;
   static constexpr int oV = oK + kKStages * kKVBytes;
   static constexpr int oP = oV + kVStages * kKVBytes;
-  static constexpr int oZ = oP + 2 * kPBytes;
+  static constexpr int oZ = oP + kPBufs * kPBytes;
   static constexpr int oBar = oZ + kZeroBytes;
   // barrier indices (8 bytes each)
   static constexpr int bQFull = 0, bQEmpty = bQFull + kQBufs;
   static constexpr int bKFull = bQEmpty + kQBufs, bKEmpty = bKFull + kKStages;
   static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
-  static constexpr int bSFull = bVEmpty + kVStages, bSEmpty = bSFull + 2;
-  static constexpr int bPFull = bSEmpty + 2, bPEmpty = bPFull + 2;
-  static constexpr int bMFull = bPEmpty + 2, bMEmpty = bMFull + kMeta;
+  static constexpr int bSFull = bVEmpty + kVStages, bSEmpty = bSFull + kSBufs;
+  static constexpr int bPFull = bSEmpty + kSBufs, bPEmpty = bPFull + kPBufs;
+  static constexpr int bMFull = bPEmpty + kPBufs, bMEmpty = bMFull + kMeta;
   static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 2;
   static constexpr int bLFull = bOEmpty + 2;
   static constexpr int bRFull = bLFull + 2, bREmpty = bRFull + kRing;
@@ -238,11 +241,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars[Ly::bVFull + s], 1);
       mbar_init(&bars[Ly::bVEmpty + s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[Ly::bSFull + s], 1);
-      mbar_init(&bars[Ly::bSEmpty + s], kSoftWarps);
-      mbar_init(&bars[Ly::bPFull + s], kSoftWarps);
-      mbar_init(&bars[Ly::bPEmpty + s], 1);
+    for (int s = 0; s < 4; ++s) {
+      if (s < kSBufs) {
+        mbar_init(&bars[Ly::bSFull + s], 1);
+        mbar_init(&bars[Ly::bSEmpty + s], kSoftWarps);
+      }
+      if (s < Ly::kPBufs) {
+        mbar_init(&bars[Ly::bPFull + s], kSoftWarps);
+        mbar_init(&bars[Ly::bPEmpty + s], 1);
+      }
     }
     for (int s = 0; s < Ly::kMeta; ++s) {
       mbar_init(&bars[Ly::bMFull + s], 1);
@@ -437,11 +444,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t qbase = smem_u32(sm + Ly::oQ + qb * Ly::kQBytes);
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int kst = g % Ly::kKStages;
-          const int sb = g & 1;
+          const int sb = g % kSBufs;
           ROLE_MARK(3);
           ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6);
           ROLE_MARK(1);
-          ok = ok && mbar_wait(&bars[Ly::bSEmpty + sb], ((g >> 1) & 1) ^ 1, ctl, 7);
+          ok = ok && mbar_wait(&bars[Ly::bSEmpty + sb], ((g / kSBufs) & 1) ^ 1, ctl, 7);
           ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
@@ -479,11 +486,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int ob = it & 1;
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int vst = g % Ly::kVStages;
-          const int pb = g & 1;
+          const int pb = g % Ly::kPBufs;
           ROLE_MARK(3);
           ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8);
           ROLE_MARK(0);
-          ok = ok && mbar_wait(&bars[Ly::bPFull + pb], (g >> 1) & 1, ctl, 9);
+          ok = ok && mbar_wait(&bars[Ly::bPFull + pb], (g / Ly::kPBufs) & 1, ctl, 9);
           ROLE_MARK(1);
           ok = ok && (n > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
           ROLE_MARK(2);
@@ -498,7 +505,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int kk = 0; kk < kPVSteps; ++kk) {
             const uint64_t ad = umma_desc_sw128(vbase + kk * 2048, lbo_v, 1024);
             const uint64_t bd = umma_desc_sw128(pbase + kk * 2048, 8192, 1024);
-            umma_ss(tmem + 128 + ob * 64, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+            umma_ss(tmem + kOCol0 + ob * 64, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars[Ly::bVEmpty + vst]);
           umma_commit(&bars[Ly::bPEmpty + pb]);
@@ -542,8 +549,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int j = 0; j < CG; ++j) l[j] = 0.0f;
 
       for (int n = 0; n < nb; ++n, ++g) {
-        const int sb = g & 1;
-        const uint32_t su = g >> 1;
+        const int sb = g % kSBufs;
+        const uint32_t su = g / kSBufs;
+        const int pb = g % Ly::kPBufs;
+        const uint32_t pu = g / Ly::kPBufs;
         const int ms = g % Ly::kMeta;
         ROLE_MARK(7);
         mbar_wait(&bars[Ly::bMFull + ms], (g / Ly::kMeta) & 1, ctl, 11);
@@ -627,14 +636,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int j = 0; j < CG; ++j) l[j] *= ex2_approx(-delta_g[j]);
             // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
             const uint32_t gp = g - 1;
-            mbar_wait(&bars[Ly::bPEmpty + (gp & 1)], (gp >> 1) & 1, ctl, 13);
+            mbar_wait(&bars[Ly::bPEmpty + (gp % Ly::kPBufs)], (gp / Ly::kPBufs) & 1, ctl, 13);
             tc_fence_after();
             float o[CG];
-            tmem_ld16(t_lane + 128 + ob * 64 + c0, o);
+            tmem_ld16(t_lane + kOCol0 + ob * 64 + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < CG; ++j) o[j] *= ex2_approx(-delta_g[j]);
-            tmem_st16(t_lane + 128 + ob * 64 + c0, o);
+            tmem_st16(t_lane + kOCol0 + ob * 64 + c0, o);
             tmem_wait_st();
             tc_fence_before();
           }
@@ -647,9 +656,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l[j] += x[j];
         }
         ROLE_MARK(5);
-        mbar_wait(&bars[Ly::bPEmpty + sb], (su & 1) ^ 1, ctl, 14);
+        mbar_wait(&bars[Ly::bPEmpty + pb], (pu & 1) ^ 1, ctl, 14);
         ROLE_MARK(6);
-        uint8_t* prow = sm + Ly::oP + sb * Ly::kPBytes + kl * 128;
+        uint8_t* prow = sm + Ly::oP + pb * Ly::kPBytes + kl * 128;
 #pragma unroll
         for (int cc = 0; cc < CG / 8; ++cc) {
           const int c = grp * (CG / 8) + cc;  // 16-byte chunk = queries 8c .. 8c+7
@@ -662,7 +671,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[Ly::bPFull + sb]);
+        if (lane == 0) mbar_arrive(&bars[Ly::bPFull + pb]);
       }
 
       // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored):
@@ -727,7 +736,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int half = 0; half < 2; ++half) {
         tc_fence_after();
         float o[32];
-        tmem_ld32(t_lane + 128 + ob * 64 + 32 * half, o);
+        tmem_ld32(t_lane + kOCol0 + ob * 64 + 32 * half, o);
         tmem_wait_ld();
         if (half == 1) {
           tc_fence_before();
