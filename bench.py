@@ -321,7 +321,10 @@ def run_vsa(args, w, world, rank, local):
     value = world * flops_call / (ms_step * 1e-3) / 1e12
 
     # end to end through the public call with host buffers (pinned), copies inside the timed region
-    hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "gate")}
+    hx = {}
+    for n in ("q", "k", "v", "gate"):  # pinned host copies, allocated once (no pageable intermediate)
+        hx[n] = torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True)
+        hx[n].copy_(x[n])
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     vsa.vsa_forward(plan, hx["q"], hx["k"], hx["v"], hx["gate"], out=hout, workspace=ws)
     torch.cuda.synchronize()

@@ -159,7 +159,7 @@ def test_edge_cases(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
     full_parity(vsa, oracle_mod, w, seed=3)
 
 
-def sampled_parity(vsa, oracle_mod, w, heads, video_every):
+def sampled_parity(vsa, oracle_mod, w, heads, video_every, batches=(0,)):
     x = synth.make_inputs(w, seed=0, device="cuda")
     plan, ws, out = run_forward(vsa, w, x)
     views = vsa.workspace_views(plan, ws)
@@ -173,15 +173,16 @@ def sampled_parity(vsa, oracle_mod, w, heads, video_every):
     g = views["o_c"].cpu().numpy().astype(np.float64)
     assert np.abs(g - sel["o_c"]).max() <= 1e-5 * max(1.0, np.abs(sel["o_c"]).max())
     tiles = [0, geo.n_prefix - 1] + list(range(geo.n_prefix, geo.n_tiles, video_every)) + [geo.n_tiles - 1]
-    items = np.array([h * geo.n_tiles + i for h in heads for i in sorted(set(tiles))], np.int64)
+    items = np.array([(b * w.heads + h) * geo.n_tiles + i for b in batches for h in heads for i in sorted(set(tiles))],
+                     np.int64)
     of = oracle_mod.fine_tiles(xb["q"], xb["k"], xb["v"], geo, sel["idx"], sel["topk"], sel["scale"], items)
     ref = oracle_mod.output_tiles(of, sel["o_c"], xb["gate"], geo, items, w.heads)
     got = np.zeros_like(ref)
-    o = out[0]  # [L, H, D]
     for n, bhi in enumerate(items):
-        i, h = int(bhi % geo.n_tiles), int(bhi // geo.n_tiles)
+        i, bh = int(bhi % geo.n_tiles), int(bhi // geo.n_tiles)
+        b, h = bh // w.heads, bh % w.heads
         nv = int(geo.tile_valid[i])
-        got[n, :nv] = o[torch.from_numpy(geo.tile_token[i, :nv].astype(np.int64)).cuda(), h].double().cpu().numpy()
+        got[n, :nv] = out[b][torch.from_numpy(geo.tile_token[i, :nv].astype(np.int64)).cuda(), h].double().cpu().numpy()
     err = np.abs(got - ref)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     plan.destroy()
@@ -240,6 +241,14 @@ def test_768p_sweep_endpoints_sampled(vsa, oracle_mod, sparsity):
     """Ends of the sparsity sweep at 1344x768: dense video keys (topk 1152) and topk 58."""
     w = dataclasses.replace(synth.workload("768p_s0.9"), sparsity=sparsity, name=f"768p_s{sparsity}")
     sampled_parity(vsa, oracle_mod, w, heads=[13], video_every=383)
+
+
+def test_768p_batch4_offsets_past_2_31_sampled(vsa, oracle_mod):
+    """Batch 4 of the 1344x768-shaped workload: q/k/v/gate/out hold
+    4*75008*56*128 = 2,150,629,376 elements each, past 2^31, so the last
+    batch's token offsets only come out right in 64-bit arithmetic."""
+    w = dataclasses.replace(synth.workload("768p_s0.9"), batch=4, name="768p_s0.9_b4")
+    sampled_parity(vsa, oracle_mod, w, heads=[0, 55], video_every=509, batches=(0, 3))
 
 
 def test_wait_selftest_times_out_and_context_stays_usable(vsa):
