@@ -26,14 +26,15 @@
 //
 // Roles (768 threads, 24 warps):
 //   warp 0  K producer: TMA for the query tile of each item and the K tiles
-//           of each block (4 lanes issue the four 8 KB boxes in parallel),
-//           plus the block's key-valid counts for the softmax;
+//           of each block (4 lanes issue the four 8 KB boxes in parallel);
 //   warp 1  V producer: TMA for the V tiles of each block;
 //   warp 2  S^T issuer (one thread) and TMEM owner;
 //   warp 3  P.V issuer (one thread);
 //   warps 4..19  softmax, four groups of four warps; group g owns query
 //           columns [16g, 16g + 16), warp w reads TMEM lane quadrant w % 4
 //           (four softmax warps per SM sub-partition hide each other's latency);
+//           each warp derives its blocks' valid-key counts from the key list,
+//           32 blocks at a time, and shuffles them out per block;
 //   warps 20..23 epilogue: 1/l, O^T from TMEM, the gated compression term
 //           and the bf16 store in sequence order.
 // Two issuing threads keep two tcgen05 streams in flight (one thread alone is
@@ -122,7 +123,6 @@ struct AttnLayout {
   static constexpr int kKStages = 2;
   static constexpr int kVStages = 3;
   static constexpr int kPBufs = 2;  // P^T buffers in shared memory
-  static constexpr int kMeta = 8;   // per-block key-valid counts in flight
   static constexpr int kRing = 8;  // claimed items in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
   static constexpr int oQ = 0;
@@ -137,15 +137,13 @@ struct AttnLayout {
   static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
   static constexpr int bSFull = bVEmpty + kVStages, bSEmpty = bSFull + kSBufs;
   static constexpr int bPFull = bSEmpty + kSBufs, bPEmpty = bPFull + kPBufs;
-  static constexpr int bMFull = bPEmpty + kPBufs, bMEmpty = bMFull + kMeta;
-  static constexpr int bOFull = bMEmpty + kMeta, bOEmpty = bOFull + 2;
+  static constexpr int bOFull = bPEmpty + kPBufs, bOEmpty = bOFull + 2;
   static constexpr int bLFull = bOEmpty + 2;
   static constexpr int bRFull = bLFull + 2, bREmpty = bRFull + kRing;
   static constexpr int bDoneS = bREmpty + kRing, bDonePV = bDoneS + 1;
   static constexpr int kNumBars = bDonePV + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;          // tmem base, abort flag
-  static constexpr int oMeta = ((oMisc + 8 + 15) / 16) * 16;  // int2 meta[kMeta]
-  static constexpr int oRing = oMeta + kMeta * 8;            // int ring[kRing]: claimed items, -1 = none left
+  static constexpr int oRing = ((oMisc + 8 + 15) / 16) * 16;  // int ring[kRing]: claimed items, -1 = none left
   static constexpr int oM = oRing + kRing * 4;               // float m[64] (log2 units)
   static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
   static constexpr int oRed = oDelta + 256;                  // float red[groups][4 quadrants][group columns]
@@ -205,7 +203,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::oBar);
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::oMisc + 4);
-  int2* meta_s = reinterpret_cast<int2*>(sm + Ly::oMeta);
   int* ring_s = reinterpret_cast<int*>(sm + Ly::oRing);
   float* m_s = reinterpret_cast<float*>(sm + Ly::oM);
   float* delta_s = reinterpret_cast<float*>(sm + Ly::oDelta);
@@ -250,10 +247,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&bars[Ly::bPFull + s], kSoftWarps);
         mbar_init(&bars[Ly::bPEmpty + s], 1);
       }
-    }
-    for (int s = 0; s < Ly::kMeta; ++s) {
-      mbar_init(&bars[Ly::bMFull + s], 1);
-      mbar_init(&bars[Ly::bMEmpty + s], kSoftWarps);
     }
     for (int s = 0; s < Ly::kRing; ++s) {
       mbar_init(&bars[Ly::bRFull + s], 1);
@@ -380,17 +373,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = mbar_wait(&bars[b_empty + st], (u & 1) ^ 1, ctl, is_k ? 2 : 3);
             ROLE_MARK(1);
             if (ok) mbar_arrive_expect_tx(&bars[b_full + st], Ly::kKVBytes);
-            if (ok && is_k) {
-              // the block's key-valid counts, for the softmax
-              const int ms = g % Ly::kMeta;
-              ROLE_MARK(3);
-              ok = mbar_wait(&bars[Ly::bMEmpty + ms], ((g / Ly::kMeta) & 1) ^ 1, ctl, 4);
-              ROLE_MARK(2);
-              if (ok) {
-                meta_s[ms] = make_int2(tile_valid_s[ka], kb_raw < 0 ? 0 : tile_valid_s[kb_raw]);
-                mbar_arrive(&bars[Ly::bMFull + ms]);
-              }
-            }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
@@ -541,8 +523,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
-      const int nb = (list_len(i) + 1) / 2;
+      const int nk = list_len(i), nb = (nk + 1) / 2;
       const int ob = it & 1;
+      int vcache = 0;  // lane j: valid keys of block (n & ~31) + j, tile a in bits 0..7, tile b in bits 8..15
 
       float l[CG];
 #pragma unroll
@@ -553,13 +536,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t su = g / kSBufs;
         const int pb = g % Ly::kPBufs;
         const uint32_t pu = g / Ly::kPBufs;
-        const int ms = g % Ly::kMeta;
         ROLE_MARK(7);
-        mbar_wait(&bars[Ly::bMFull + ms], (g / Ly::kMeta) & 1, ctl, 11);
+        if ((n & 31) == 0) {
+          // valid-key counts of the next 32 blocks (an odd list's last block has no second tile)
+          const int nn = n + lane;
+          vcache = 0;
+          if (nn < nb) {
+            const int ka = key_tile(bh, i, 2 * nn);
+            const int kb = (2 * nn + 1 < nk) ? tile_valid_s[key_tile(bh, i, 2 * nn + 1)] : 0;
+            vcache = tile_valid_s[ka] | (kb << 8);
+          }
+        }
+        const int vpk = __shfl_sync(0xffffffffu, vcache, n & 31);
+        const int2 vc = make_int2(vpk & 0xff, vpk >> 8);
         ROLE_MARK(0);
-        const int2 vc = meta_s[ms];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[Ly::bMEmpty + ms]);
 
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
         ROLE_MARK(1);
