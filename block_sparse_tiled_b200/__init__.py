@@ -35,7 +35,7 @@ EXPORTED = (
     "vsa_plan_tiles", "vsa_plan_info", "vsa_plan_tables", "vsa_plan_query", "vsa_plan_tables_host",
     "vsa_plan_destroy",
     "vsa_gather_tiles", "vsa_pool_and_score", "vsa_topk_select", "vsa_sparse_attn_fwd", "vsa_forward",
-    "vsa_forward_noalloc", "vsa_wait_selftest",
+    "vsa_forward_noalloc", "vsa_forward_host", "vsa_forward_host_workspace", "vsa_wait_selftest",
     "vsa_plan_workspace", "vsa_device_status", "vsa_last_error", "vsa_version",
 )
 
@@ -99,6 +99,8 @@ def load_library(path: str = LIB_PATH):
     lib.vsa_sparse_attn_fwd.argtypes = [P] * 9
     lib.vsa_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.vsa_forward_noalloc.argtypes = [P] * 7
+    lib.vsa_forward_host_workspace.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.vsa_forward_host.argtypes = [P, P, P, P, P, P, ctypes.c_int32, P, ctypes.c_size_t, P]
     lib.vsa_wait_selftest.argtypes = [P, ctypes.c_int64, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     lib.vsa_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED:
@@ -272,17 +274,66 @@ def alloc_workspace(plan, device=None) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda", torch.cuda.current_device()))
 
 
+def default_head_chunk(heads: int) -> int:
+    """Heads per chunk of the host pipeline: four chunks (fewer when there are fewer heads)."""
+    return max(1, -(-heads // 4))
+
+
+def host_workspace_bytes(plan, head_chunk=None) -> int:
+    hc = default_head_chunk(plan.geometry["heads"]) if head_chunk is None else int(head_chunk)
+    n = ctypes.c_size_t()
+    _check(load_library().vsa_forward_host_workspace(plan.handle, hc, ctypes.byref(n)), "vsa_forward_host_workspace")
+    return n.value
+
+
+def _host_ptr(t, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a CPU tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def vsa_forward_host(plan, q, k, v, gate, out=None, workspace=None, head_chunk=None, stream=None):
+    """The whole forward for CPU (ideally pinned) q, k, v, gate; returns the CPU
+    output.  The heads run in chunks whose copies overlap the compute of the
+    neighbouring chunks (vsa_forward_host).  Without a workspace, one is
+    allocated on first use and kept on the plan.  Returns once the stream has
+    drained."""
+    hc = default_head_chunk(plan.geometry["heads"]) if head_chunk is None else int(head_chunk)
+    need = host_workspace_bytes(plan, hc)
+    if workspace is None:
+        cached = getattr(plan, "_host_ws", None)
+        if cached is None or cached.numel() < need:
+            cached = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", torch.cuda.current_device()))
+            plan._host_ws = cached
+        workspace = cached
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    _check(load_library().vsa_forward_host(
+        plan.handle, _host_ptr(q, "q"), _host_ptr(k, "k"), _host_ptr(v, "v"), _host_ptr(gate, "gate"),
+        _host_ptr(out, "out"), hc, _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "vsa_forward_host")
+    if stream is None:
+        torch.cuda.current_stream().synchronize()
+    elif isinstance(stream, torch.cuda.Stream):
+        stream.synchronize()
+    else:
+        torch.cuda.synchronize()
+    return out
+
+
 def vsa_forward(plan, q, k, v, gate, out=None, workspace=None, stream=None):
     """The whole forward.  CUDA inputs: runs in place on the stream.  CPU
-    inputs (ideally pinned): copied to the device, run, and the result copied
-    back into a CPU tensor, all on the stream."""
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        q, k, v, gate = (t.to(dev, non_blocking=True) for t in (q, k, v, gate))
-        host_out = out
-        out = torch.empty_like(q)
-    elif out is None:
+    inputs (ideally pinned): the head-chunked host pipeline (vsa_forward_host),
+    with `workspace` sized by host_workspace_bytes when given."""
+    if not q.is_cuda:
+        return vsa_forward_host(plan, q, k, v, gate, out=out, workspace=workspace, stream=stream)
+    if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(plan, q.device)
@@ -291,11 +342,6 @@ def vsa_forward(plan, q, k, v, gate, out=None, workspace=None, stream=None):
         plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(gate, bf, "gate"),
         _ptr(out, bf, "out"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "vsa_forward")
-    if host:
-        if host_out is None:
-            host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        host_out.copy_(out, non_blocking=True)
-        return host_out
     return out
 
 

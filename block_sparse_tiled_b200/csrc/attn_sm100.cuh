@@ -102,12 +102,13 @@ struct AttnArgs {
   const int32_t* tile_token;  // [n_t * 64]
   const int32_t* tile_valid;  // [n_t]
   const float* o_c;           // [B, H, n_t, D]
-  const uint16_t* gate;       // [B, L, H] bf16
+  const uint16_t* gate;       // [B, L, gate_ld] bf16: the gate of head h at gate[(b*L + t)*gate_ld + h]
   uint16_t* out;              // [B, L, H, D] bf16
   int* status;                // [2] device status word
   int* sched;                 // item counter, zero at launch
   int64_t L;
   int H, n_t, P, topk;
+  int gate_ld;  // gate elements between consecutive tokens (H, or more when a head slice is processed)
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
 };
@@ -708,7 +709,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (tid < 64) {
         const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
         qtok_s[tid] = tok;
-        gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.H + h)) : 0.0f;
+        gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.gate_ld + h)) : 0.0f;
       }
       const float oc = (d < D) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
       ROLE_MARK(3);

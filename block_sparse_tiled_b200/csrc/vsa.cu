@@ -258,6 +258,17 @@ struct vsa_plan_s {
   int32_t* d_tile_valid = nullptr;
   int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter
   vsa_workspace_layout ws{};
+  // Head-slice plans share the parent's device tables and status word and own nothing on the device.
+  bool owns_device = true;
+  // vsa_forward_host: head-slice plans for chunks of `hc` heads (and the remainder), and the copy streams
+  // and events of its pipeline.  Created on first use, released with the plan.
+  struct HostPipe {
+    int32_t hc = 0;
+    vsa_plan_s* sub = nullptr;       // hc heads
+    vsa_plan_s* sub_last = nullptr;  // H % hc heads, when H is not a multiple of hc
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {}, ev_gate = nullptr, ev_start = nullptr;
+  } pipe;
 };
 
 namespace {
@@ -364,7 +375,7 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 }
 
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
-                    const void* gate, void* out, cudaStream_t s) {
+                    const void* gate, void* out, cudaStream_t s, int gate_ld = 0) {
   if (p->n_t == 0) return VSA_OK;
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
   CUtensorMap mq, mk, mv;
@@ -382,6 +393,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.sched = p->d_status + 2;
   a.L = p->r.L;
   a.H = p->H;
+  a.gate_ld = gate_ld > 0 ? gate_ld : p->H;
   a.n_t = p->n_t;
   a.P = p->P;
   a.topk = p->topk;
@@ -402,6 +414,85 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     vsa::vsa_attn_kernel<64><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
   }
   return launch_check("attention");
+}
+
+// ---------------------------------------------------------------- host pipeline helpers
+void release_host_pipe(vsa_plan_s* p) {
+  auto& h = p->pipe;
+  delete h.sub;
+  delete h.sub_last;
+  h.sub = h.sub_last = nullptr;
+  if (h.h2d) cudaStreamDestroy(h.h2d);
+  if (h.d2h) cudaStreamDestroy(h.d2h);
+  h.h2d = h.d2h = nullptr;
+  for (cudaEvent_t* e : {&h.ev_in[0], &h.ev_in[1], &h.ev_comp[0], &h.ev_comp[1], &h.ev_out[0], &h.ev_out[1], &h.ev_gate,
+                         &h.ev_start}) {
+    if (*e) cudaEventDestroy(*e);
+    *e = nullptr;
+  }
+  h.hc = 0;
+}
+
+// A plan for heads [h0, h0 + heads) of `p`'s geometry: same tables and status word, its own workspace layout.
+vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
+  auto* q = new vsa_plan_s();
+  q->device = p->device;
+  q->num_sms = p->num_sms;
+  q->max_smem = p->max_smem;
+  q->B = p->B;
+  q->H = heads;
+  q->D = p->D;
+  q->r = p->r;
+  q->n_t = p->n_t;
+  q->P = p->P;
+  q->V = p->V;
+  q->topk = p->topk;
+  q->d_tile_token = p->d_tile_token;
+  q->d_tile_valid = p->d_tile_valid;
+  q->d_status = p->d_status;
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk);
+  q->owns_device = false;
+  return q;
+}
+
+// Workspace of vsa_forward_host with chunks of hc heads: one head-slice forward workspace, two staging
+// slots (q, k, v and out of one chunk each) and the whole gate.
+struct HostLayout {
+  size_t fwd = 0, slot[2] = {0, 0}, gate = 0, total = 0;
+  size_t chunk_bytes = 0;  // one [B, L, hc, D] bf16 tensor, 256-aligned
+};
+HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
+  HostLayout h;
+  const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
+  h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
+  h.fwd = 0;
+  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk).total);
+  for (int s = 0; s < 2; ++s) {
+    h.slot[s] = off;
+    off += 4 * h.chunk_bytes;  // q, k, v, out
+  }
+  h.gate = off;
+  off += align256(tokens * static_cast<size_t>(p->H) * 2);
+  h.total = off;
+  return h;
+}
+
+// The four steps on one stream; `w` holds p->ws.total bytes.  gate_ld: gate elements between tokens.
+vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v, const void* gate, int gate_ld, void* out,
+                        uint8_t* w, cudaStream_t s) {
+  auto* qt = w + p->ws.q_t;
+  auto* kt = w + p->ws.k_t;
+  auto* vt = w + p->ws.v_t;
+  auto* pq = reinterpret_cast<float*>(w + p->ws.pq);
+  auto* pk = reinterpret_cast<float*>(w + p->ws.pk);
+  auto* pv = reinterpret_cast<float*>(w + p->ws.pv);
+  auto* S = reinterpret_cast<float*>(w + p->ws.scores);
+  auto* idx = reinterpret_cast<int32_t*>(w + p->ws.idx);
+  auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
+  VSA_TRY(run_gather(p, q, k, v, qt, kt, vt, pq, pk, pv, s));
+  VSA_TRY(run_scores(p, pq, pk, S, s));
+  VSA_TRY(run_topk(p, S, pv, idx, oc, s));
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld);
 }
 
 void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
@@ -537,9 +628,12 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
   cudaGetDevice(&prev);
   cudaSetDevice(p->device);
   cudaDeviceSynchronize();
-  cudaFree(p->d_tile_token);
-  cudaFree(p->d_tile_valid);
-  cudaFree(p->d_status);
+  release_host_pipe(p);
+  if (p->owns_device) {
+    cudaFree(p->d_tile_token);
+    cudaFree(p->d_tile_valid);
+    cudaFree(p->d_status);
+  }
   if (prev >= 0) cudaSetDevice(prev);
   delete p;
   return VSA_OK;
@@ -593,21 +687,7 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const v
   if (workspace_bytes < p->ws.total)
     return fail(VSA_ERR_WORKSPACE, "workspace holds " + std::to_string(workspace_bytes) + " bytes, needs " +
                                        std::to_string(p->ws.total));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  auto* w = static_cast<uint8_t*>(workspace);
-  auto* qt = w + p->ws.q_t;
-  auto* kt = w + p->ws.k_t;
-  auto* vt = w + p->ws.v_t;
-  auto* pq = reinterpret_cast<float*>(w + p->ws.pq);
-  auto* pk = reinterpret_cast<float*>(w + p->ws.pk);
-  auto* pv = reinterpret_cast<float*>(w + p->ws.pv);
-  auto* S = reinterpret_cast<float*>(w + p->ws.scores);
-  auto* idx = reinterpret_cast<int32_t*>(w + p->ws.idx);
-  auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
-  VSA_TRY(run_gather(p, q, k, v, qt, kt, vt, pq, pk, pv, s));
-  VSA_TRY(run_scores(p, pq, pk, S, s));
-  VSA_TRY(run_topk(p, S, pv, idx, oc, s));
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s);
+  return forward_impl(p, q, k, v, gate, p->H, out, static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
@@ -620,6 +700,95 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k,
   void* scratch = nullptr;
   VSA_TRY(noalloc_scratch_address(p->device, &scratch));
   return vsa_forward(p, q, k, v, gate, out, scratch, VSA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+vsa_status vsa_forward_host_workspace(vsa_plan p, int32_t head_chunk, size_t* bytes) {
+  if (p == nullptr || bytes == nullptr) return fail(VSA_ERR_INVALID_ARG, "NULL argument");
+  if (head_chunk < 1 || head_chunk > p->H) return fail(VSA_ERR_INVALID_ARG, "head_chunk must lie in [1, heads]");
+  *bytes = host_layout(p, head_chunk).total;
+  return VSA_OK;
+}
+
+vsa_status vsa_forward_host(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const vsa_bf16* gate,
+                            vsa_bf16* out, int32_t head_chunk, void* workspace, size_t workspace_bytes, void* stream) {
+  VSA_TRY(check_plan(p));
+  if (!p->owns_device) return fail(VSA_ERR_INVALID_ARG, "not a plan made by vsa_plan_tiles");
+  if (q == nullptr || k == nullptr || v == nullptr || gate == nullptr || out == nullptr)
+    return fail(VSA_ERR_INVALID_ARG, "a required host pointer is NULL");
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VSA_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device pointer");
+  if (head_chunk < 1 || head_chunk > p->H) return fail(VSA_ERR_INVALID_ARG, "head_chunk must lie in [1, heads]");
+  const HostLayout hl = host_layout(p, head_chunk);
+  if (workspace_bytes < hl.total)
+    return fail(VSA_ERR_WORKSPACE, "workspace holds " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                       std::to_string(hl.total));
+  auto& hp = p->pipe;
+  if (hp.hc != head_chunk) {  // (re)build the head-slice plans, copy streams and events
+    release_host_pipe(p);
+    hp.sub = make_head_slice_plan(p, head_chunk);
+    if (p->H % head_chunk != 0) hp.sub_last = make_head_slice_plan(p, p->H % head_chunk);
+    cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+    for (cudaEvent_t* ev : {&hp.ev_in[0], &hp.ev_in[1], &hp.ev_comp[0], &hp.ev_comp[1], &hp.ev_out[0], &hp.ev_out[1],
+                            &hp.ev_gate, &hp.ev_start})
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      release_host_pipe(p);
+      return fail(VSA_ERR_CUDA, std::string("host pipeline setup: ") + cudaGetErrorString(e));
+    }
+    hp.hc = head_chunk;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* w = static_cast<uint8_t*>(workspace);
+  const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
+  const size_t row = static_cast<size_t>(p->H) * p->D * 2;  // bytes of one token's heads on the host
+  const int nchunks = (p->H + head_chunk - 1) / head_chunk;
+  auto* dgate = reinterpret_cast<uint16_t*>(w + hl.gate);
+
+  // everything earlier on the caller's stream (including a previous call's use of the staging slots)
+  // comes before this call's copies
+  VSA_CUDA_TRY(cudaEventRecord(hp.ev_start, s));
+  VSA_CUDA_TRY(cudaStreamWaitEvent(hp.h2d, hp.ev_start, 0));
+  VSA_CUDA_TRY(cudaStreamWaitEvent(hp.d2h, hp.ev_start, 0));
+  VSA_CUDA_TRY(cudaMemcpyAsync(dgate, gate, tokens * p->H * 2, cudaMemcpyHostToDevice, hp.h2d));
+  VSA_CUDA_TRY(cudaEventRecord(hp.ev_gate, hp.h2d));
+  VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_gate, 0));
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int slot = c & 1;
+    const int h0 = c * head_chunk;
+    const int hn = std::min(head_chunk, p->H - h0);
+    vsa_plan_s* sp = (hn == head_chunk) ? hp.sub : hp.sub_last;
+    uint8_t* base = w + hl.slot[slot];
+    uint8_t* dq = base;
+    uint8_t* dk = base + hl.chunk_bytes;
+    uint8_t* dv = base + 2 * hl.chunk_bytes;
+    uint8_t* dout = base + 3 * hl.chunk_bytes;
+    const size_t width = static_cast<size_t>(hn) * p->D * 2;  // bytes of one token's heads in the chunk
+    const size_t hoff = static_cast<size_t>(h0) * p->D * 2;
+    // host -> device: the chunk's heads of q, k, v (slot free once chunk c-2 has been computed)
+    if (c >= 2) VSA_CUDA_TRY(cudaStreamWaitEvent(hp.h2d, hp.ev_comp[slot], 0));
+    VSA_CUDA_TRY(cudaMemcpy2DAsync(dq, width, reinterpret_cast<const uint8_t*>(q) + hoff, row, width, tokens,
+                                   cudaMemcpyHostToDevice, hp.h2d));
+    VSA_CUDA_TRY(cudaMemcpy2DAsync(dk, width, reinterpret_cast<const uint8_t*>(k) + hoff, row, width, tokens,
+                                   cudaMemcpyHostToDevice, hp.h2d));
+    VSA_CUDA_TRY(cudaMemcpy2DAsync(dv, width, reinterpret_cast<const uint8_t*>(v) + hoff, row, width, tokens,
+                                   cudaMemcpyHostToDevice, hp.h2d));
+    VSA_CUDA_TRY(cudaEventRecord(hp.ev_in[slot], hp.h2d));
+    // the forward of the chunk on the caller's stream (output slot free once chunk c-2 is back on the host)
+    VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_in[slot], 0));
+    if (c >= 2) VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_out[slot], 0));
+    VSA_TRY(forward_impl(sp, dq, dk, dv, dgate + h0, p->H, dout, w + hl.fwd, s));
+    VSA_CUDA_TRY(cudaEventRecord(hp.ev_comp[slot], s));
+    // device -> host: the chunk's heads of the output
+    VSA_CUDA_TRY(cudaStreamWaitEvent(hp.d2h, hp.ev_comp[slot], 0));
+    VSA_CUDA_TRY(cudaMemcpy2DAsync(reinterpret_cast<uint8_t*>(out) + hoff, row, dout, width, width, tokens,
+                                   cudaMemcpyDeviceToHost, hp.d2h));
+    VSA_CUDA_TRY(cudaEventRecord(hp.ev_out[slot], hp.d2h));
+  }
+  // the caller's stream ends after the last copy back (the d2h stream runs its copies in order)
+  VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_out[(nchunks - 1) & 1], 0));
+  return VSA_OK;
 }
 
 vsa_status vsa_wait_selftest(vsa_plan p, int64_t timeout_ns, void* stream, int32_t* code, int32_t* where) {

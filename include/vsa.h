@@ -203,6 +203,34 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                        const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
                        void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* ---- the whole forward with inputs and output in host memory ---------------
+ * The forward of vsa_forward for q, k, v [B, L, H, D], gate [B, L, H] and out
+ * [B, L, H, D] that live in HOST memory (bf16, sequence order).  No
+ * counterpart on the pages: the heads of the attention are independent, so
+ * the call processes them in chunks of `head_chunk` heads and overlaps, on
+ * three streams, the host->device copy of one chunk, the forward of the
+ * previous one on `stream` and the device->host copy of the one before.
+ * The result is bit-identical to vsa_forward on the same inputs.
+ *  - Host buffers should be page-locked; pageable memory still gives the
+ *    right result, but the copies then do not overlap.
+ *  - `workspace_dev` (256-byte aligned) must hold the bytes that
+ *    vsa_forward_host_workspace returns for the same head_chunk: a
+ *    forward workspace for one chunk, two staging slots and the gate.
+ *  - The call returns once everything is enqueued; `out` is complete when
+ *    `stream` has drained (cudaStreamSynchronize).  Earlier work on `stream`
+ *    finishes before the call's copies start.
+ *  - The first call with a given head_chunk creates two copy streams, eight
+ *    events and the head-slice plans; they belong to the plan and are
+ *    released by vsa_plan_destroy.  Calls with one plan must not overlap.
+ * Errors: VSA_ERR_INVALID_ARG (NULL pointer, head_chunk outside [1, H],
+ * unaligned workspace), VSA_ERR_WORKSPACE (workspace too small), VSA_ERR_CUDA
+ * (a copy or launch failed). */
+vsa_status vsa_forward_host_workspace(vsa_plan p, int32_t head_chunk, size_t* bytes);
+vsa_status vsa_forward_host(vsa_plan p, const vsa_bf16* q_host, const vsa_bf16* k_host,
+                            const vsa_bf16* v_host, const vsa_bf16* gate_host, vsa_bf16* out_host,
+                            int32_t head_chunk, void* workspace_dev, size_t workspace_bytes,
+                            void* stream);
+
 /* ---- the whole forward without a caller workspace -------------------------
  * No counterpart on the pages: this entry point exists for callers that
  * cannot allocate device memory on their call path -- for instance a plugin
