@@ -22,7 +22,8 @@
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
 // O^T is double-buffered in TMEM, so one item's epilogue (in its own warps)
 // overlaps the next item's blocks.
-// D = 64 uses the same M = 128 PV product with a zero upper half of V^T.
+// D = 64 uses the same M = 128 PV product with a zero upper half of V^T, and
+// D = 96 one whose upper 32 rows TMA fills with zeros.
 //
 // Roles (768 threads, 24 warps):
 //   warp 0  K producer: TMA for the query tile of each item and the K tiles
@@ -115,9 +116,11 @@ struct AttnArgs {
 
 template <int D>
 struct AttnLayout {
-  static constexpr int kHalves = D / 64;        // 128-byte swizzle atoms along D
-  static constexpr int kQBytes = 64 * D * 2;    // one query tile
-  static constexpr int kKVBytes = 128 * D * 2;  // 128 keys of K (or of V)
+  // 128-byte swizzle atoms along D.  D = 96 uses two, the second half-empty: TMA fills columns 96..127
+  // with zeros, the S^T product stops after D/16 K-steps and O^T rows 96..127 are never stored.
+  static constexpr int kHalves = (D + 63) / 64;
+  static constexpr int kQBytes = 64 * 64 * kHalves * 2;    // one query tile
+  static constexpr int kKVBytes = 128 * 64 * kHalves * 2;  // 128 keys of K (or of V)
   static constexpr int kHalfBytes = 128 * 128;  // one 64-column half of a 128-row block
   static constexpr int kPBytes = 128 * 64 * 2;  // P^T of one block
   static constexpr int kQBufs = 1;
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t vbase = smem_u32(sm + Ly::oV + vst * Ly::kKVBytes);
           const uint32_t pbase = smem_u32(sm + Ly::oP + pb * Ly::kPBytes);
           // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
-          const uint32_t lbo_v = (D == 128) ? Ly::kHalfBytes
+          const uint32_t lbo_v = (D > 64) ? Ly::kHalfBytes
                                             : static_cast<uint32_t>(Ly::oZ - (Ly::oV + vst * Ly::kKVBytes));
 #pragma unroll
           for (int kk = 0; kk < kPVSteps; ++kk) {

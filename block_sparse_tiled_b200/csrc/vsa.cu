@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "attn_sm100.cuh"
@@ -66,8 +67,8 @@ int32_t topk_for(double sparsity, int64_t V) {
 vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g == nullptr) return fail(VSA_ERR_INVALID_ARG, "geometry is NULL");
   if (g->batch < 1 || g->heads < 1) return fail(VSA_ERR_INVALID_ARG, "batch and heads must be >= 1");
-  if (g->head_dim != 64 && g->head_dim != 128)
-    return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128, got " + std::to_string(g->head_dim));
+  if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
+    return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128, got " + std::to_string(g->head_dim));
   if (g->tile_size != kTile)
     return fail(VSA_ERR_UNSUPPORTED, "tile_size must be 64, got " + std::to_string(g->tile_size));
   if (!(g->sparsity >= 0.0 && g->sparsity <= 1.0)) return fail(VSA_ERR_INVALID_ARG, "sparsity must lie in [0, 1]");
@@ -304,6 +305,17 @@ vsa_status allow_smem(K kernel, size_t bytes) {
   return VSA_OK;
 }
 
+// Calls f(std::integral_constant<int, D>{}) for the plan's head dimension (64, 96 or 128).
+template <typename F>
+vsa_status with_head_dim(int D, F&& f) {
+  switch (D) {
+    case 64: return f(std::integral_constant<int, 64>{});
+    case 96: return f(std::integral_constant<int, 96>{});
+    case 128: return f(std::integral_constant<int, 128>{});
+    default: return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128");
+  }
+}
+
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
                       float* pk, float* pv, cudaStream_t s) {
   if (p->n_t == 0) return VSA_OK;
@@ -316,15 +328,13 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   auto* qo = static_cast<uint16_t*>(qt);
   auto* ko = static_cast<uint16_t*>(kt);
   auto* vo = static_cast<uint16_t*>(vt);
-  if (p->D == 128) {
-    VSA_TRY(allow_smem(vsa::gather_pool_kernel<128>, smem));
-    vsa::gather_pool_kernel<128><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                         p->d_tile_valid, p->r.L, p->H, p->n_t);
-  } else {
-    VSA_TRY(allow_smem(vsa::gather_pool_kernel<64>, smem));
-    vsa::gather_pool_kernel<64><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                        p->d_tile_valid, p->r.L, p->H, p->n_t);
-  }
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    VSA_TRY(allow_smem(vsa::gather_pool_kernel<D>, smem));
+    vsa::gather_pool_kernel<D><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
+                                                       p->d_tile_valid, p->r.L, p->H, p->n_t);
+    return VSA_OK;
+  }));
   return launch_check("gather_pool");
 }
 
@@ -335,10 +345,11 @@ vsa_status run_pool(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   const auto* a = static_cast<const uint16_t*>(qt);
   const auto* b = static_cast<const uint16_t*>(kt);
   const auto* c = static_cast<const uint16_t*>(vt);
-  if (p->D == 128)
-    vsa::pool_tiles_kernel<128><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
-  else
-    vsa::pool_tiles_kernel<64><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    vsa::pool_tiles_kernel<D><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
+    return VSA_OK;
+  }));
   return launch_check("pool_tiles");
 }
 
@@ -367,10 +378,11 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
     VSA_TRY(launch_check("topk"));
   }
   dim3 grid((p->n_t + vsa::kCompRows - 1) / vsa::kCompRows, static_cast<unsigned>(BH));
-  if (p->D == 128)
-    vsa::compress_kernel<128><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
-  else
-    vsa::compress_kernel<64><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    vsa::compress_kernel<D><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
+    return VSA_OK;
+  }));
   return launch_check("compress");
 }
 
@@ -402,17 +414,14 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
   // the item counter of the persistent schedule starts at zero for every launch
   VSA_CUDA_TRY(cudaMemsetAsync(a.sched, 0, sizeof(int), s));
-  if (p->D == 128) {
-    const size_t smem = vsa::AttnLayout<128>::bytes(p->n_t);
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    const size_t smem = vsa::AttnLayout<D>::bytes(p->n_t);
     if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
-    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<128>, smem));
-    vsa::vsa_attn_kernel<128><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
-  } else {
-    const size_t smem = vsa::AttnLayout<64>::bytes(p->n_t);
-    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
-    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<64>, smem));
-    vsa::vsa_attn_kernel<64><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
-  }
+    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D>, smem));
+    vsa::vsa_attn_kernel<D><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
+    return VSA_OK;
+  }));
   return launch_check("attention");
 }
 

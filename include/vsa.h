@@ -83,7 +83,7 @@ typedef enum vsa_status {
 typedef struct vsa_geometry {
   int32_t batch;            /* B >= 1 */
   int32_t heads;            /* H >= 1 */
-  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t head_dim;         /* D: 64, 96 or 128 */
   int32_t n_segments;       /* number of prefix segments (ignored with tags) */
   const int32_t* segment_len;
   const int32_t* token_tags; /* NULL to use segment_len */

@@ -104,7 +104,7 @@ def test_token_tags_match_segments(vsa):
     (dict(sparsity=-0.1), "VSA_ERR_INVALID_ARG"),
     (dict(sparsity=float("nan")), "VSA_ERR_INVALID_ARG"),
     (dict(tile_size=128), "VSA_ERR_UNSUPPORTED"),
-    (dict(head_dim=96), "VSA_ERR_UNSUPPORTED"),
+    (dict(head_dim=80), "VSA_ERR_UNSUPPORTED"),
     (dict(grid=(8, 0, 8)), "VSA_ERR_SHAPE"),
     (dict(batch=0), "VSA_ERR_INVALID_ARG"),
     (dict(segments=(-1,)), "VSA_ERR_INVALID_ARG"),

@@ -112,3 +112,16 @@ def test_host_pipeline_errors(vsa):
     out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=1)
     assert torch.equal(out, device_reference(vsa, plan, x))
     plan.destroy()
+
+
+def test_host_pipeline_head_dim_96(vsa):
+    import dataclasses
+
+    w = dataclasses.replace(synth.workload("small"), head_dim=96, name="small_d96")
+    x = synth.make_inputs(w, seed=8, device="cuda")
+    plan = plan_for(vsa, w)
+    ref = device_reference(vsa, plan, x)
+    hx = host_copies(x)
+    out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=3)
+    assert torch.equal(out, ref)
+    plan.destroy()

@@ -153,6 +153,7 @@ def test_tiny_sparsity0_is_dense_attention(vsa, oracle_mod):
     ((1,), (4, 4, 4), 0.0, 1, 1, 64),             # one-token prefix tile, one cube
     ((64, 64, 64), (4, 8, 12), 0.75, 1, 4, 128),  # even count of key tiles
     ((33,), (4, 4, 12), 0.5, 1, 2, 128),          # odd count of key tiles: half-masked last block
+    ((70, 0, 5), (5, 6, 7), 0.6, 2, 3, 96),       # head_dim 96, ragged everywhere
 ])
 def test_edge_cases(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
     w = synth.Workload("edge", B, H, D, tuple(segments), tuple(grid), sparsity)
@@ -266,3 +267,18 @@ def test_wait_selftest_times_out_and_context_stays_usable(vsa):
     assert torch.isfinite(out.float()).all()
     assert vsa.device_status(plan) == (0, 0)
     plan.destroy()
+
+
+@pytest.mark.parametrize("name,seed", [("small", 4), ("tiny", 5)])
+def test_head_dim_96_full_parity(vsa, oracle_mod, name, seed):
+    """head_dim 96 (the model's 5376 / 56): tile copies, pooled tiles, scores and indices bit-exact,
+    compression and output within tolerance.  The attention kernel reads the 96-wide tiles as two
+    64-column TMA boxes whose columns 96..127 are zero-filled."""
+    w = dataclasses.replace(synth.workload(name), head_dim=96, name=f"{name}_d96")
+    full_parity(vsa, oracle_mod, w, seed=seed)
+
+
+def test_head_dim_96_480p_sampled(vsa, oracle_mod):
+    """The 480p-shaped workload at head_dim 96, selection in full and sampled output tiles."""
+    w = dataclasses.replace(synth.workload("480p"), head_dim=96, name="480p_d96")
+    sampled_parity(vsa, oracle_mod, w, heads=[0, 29, 55], video_every=23)
