@@ -60,7 +60,7 @@ def _load():
         lib.vsa_oracle_fine.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
         lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, i32, P, P]
         lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P]
-        lib.vsa_oracle_output.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P, P, P]
+        lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -184,9 +184,15 @@ def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items) -> n
 
 
 def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarray:
-    """out rows of the listed tiles: o_f + gate * o_c[tile] (tile row order; pad rows 0)."""
+    """out rows of the listed tiles: o_f + gate * o_c[tile] (tile row order; pad rows 0); the gate
+    is [B, L, H] (one per token and head) or [B, L, H*D] (one per channel, R12)."""
+    D = o_f_tiles.shape[-1]
+    B, L = np.shape(gate)[0], np.shape(gate)[1]
+    per_channel = gate_is_per_channel(gate, B, L, H, D)
     gate = _c(gate, np.uint16)
     gf = (gate.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if per_channel:
+        gf = gf.reshape(B, L, H, D)
     res = np.zeros_like(o_f_tiles)
     for n, bhi in enumerate(np.asarray(items, np.int64)):
         i = int(bhi % geo.n_tiles)
@@ -194,7 +200,8 @@ def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarr
         h, b = bh % H, bh // H
         nv = int(geo.tile_valid[i])
         toks = geo.tile_token[i, :nv]
-        res[n, :nv] = o_f_tiles[n, :nv] + gf[b, toks, h][:, None] * o_c[b, h, i][None, :]
+        g = gf[b, toks, h] if per_channel else gf[b, toks, h][:, None]
+        res[n, :nv] = o_f_tiles[n, :nv] + g * o_c[b, h, i][None, :]
     return res
 
 
@@ -222,15 +229,26 @@ def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndar
     return out
 
 
+def gate_is_per_channel(gate, B, L, H, D) -> bool:
+    """[B, L, H]: one gate per token and head; [B, L, H*D] or [B, L, H, D]: one per channel (R12)."""
+    shape = tuple(np.shape(gate))
+    if shape == (B, L, H):
+        return False
+    if shape in ((B, L, H * D), (B, L, H, D)):
+        return True
+    raise ValueError(f"gate shape {shape} is neither [B, L, H] nor [B, L, H*D]")
+
+
 def output(o_f, o_c, gate, geo: Geometry, todo=None) -> np.ndarray:
     o_f = _c(o_f, np.float64)
     o_c = _c(o_c, np.float64)
-    gate = _c(gate, np.uint16)
     B, L, H, D = o_f.shape
+    per_channel = gate_is_per_channel(gate, B, L, H, D)
+    gate = _c(gate, np.uint16)
     if todo is not None:
         todo = _c(todo.astype(np.uint8), np.uint8)
     out = np.full((B, L, H, D), np.nan, np.float64)
-    _load().vsa_oracle_output(_p(o_f), _p(o_c), _p(gate), B, L, H, D, geo.n_tiles,
+    _load().vsa_oracle_output(_p(o_f), _p(o_c), _p(gate), int(per_channel), B, L, H, D, geo.n_tiles,
                               _p(geo.tile_token), _p(geo.tile_valid), _p(todo), _p(out))
     return out
 
@@ -252,7 +270,8 @@ class ForwardResult:
 
 
 def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None) -> ForwardResult:
-    """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H].
+    """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H] (or
+    [B,L,H*D], one per channel).
 
     Selection (pool, scores, top-k) always runs in full; the fine branch and
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,

@@ -40,6 +40,7 @@
  *   R10 the compression branch is added to every tile row, prefix tiles
  *      included -- parity unpinned;
  *   R11 the gate is one scalar per (batch, token, head).
+ *   R12 the per-channel variant: one gate per (batch, token, channel h*D + d), [B, L, H*D].
  *
  * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
  * order above; fine attention, compression and the output in binary64.
@@ -439,11 +440,12 @@ void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_
 /* O7 output                                                           */
 /* ------------------------------------------------------------------ */
 
-/* out[b, tok, h, :] = o_f[b, tok, h, :] + gate[b, tok, h] * o_c[b, h, tile(tok), :]
- * for the valid rows of every tile with todo set (NULL: all); gate: [B, L, H]
- * bf16 bits; one scalar gate per token and head, no activation (R10, R11). */
-void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gate, int B,
-                       int64_t L, int H, int D, int n_t, const int32_t *tile_token,
+/* out[b, tok, h, d] = o_f[b, tok, h, d] + gate * o_c[b, h, tile(tok), d] for the valid rows of
+ * every tile with todo set (NULL: all), no activation (R10, R11).  gate: bf16 bits, either
+ * [B, L, H], one scalar per token and head (gate_per_channel = 0), or [B, L, H*D], one per
+ * channel h*D + d of the token (gate_per_channel = 1, R12). */
+void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gate, int gate_per_channel,
+                       int B, int64_t L, int H, int D, int n_t, const int32_t *tile_token,
                        const int32_t *tile_valid, const uint8_t *todo, double *out) {
 #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
@@ -454,8 +456,11 @@ void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gat
                 for (int r = 0; r < tile_valid[i]; ++r) {
                     int64_t tok = tile_token[(int64_t)i * TILE + r];
                     int64_t row = (((int64_t)b * L + tok) * H + h);
-                    double g = (double)bf16_to_float(gate[row]);
-                    for (int d = 0; d < D; ++d) out[row * D + d] = o_f[row * D + d] + g * oc[d];
+                    for (int d = 0; d < D; ++d) {
+                        uint16_t gbits = gate_per_channel ? gate[row * D + d] : gate[row];
+                        double g = (double)bf16_to_float(gbits);
+                        out[row * D + d] = o_f[row * D + d] + g * oc[d];
+                    }
                 }
             }
 }

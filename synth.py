@@ -49,6 +49,7 @@ class Workload:
     structured: bool = False
     gate_std: float = 0.1
     description: str = ""
+    gate_per_channel: bool = False  # gate [B, L, H*D] (one per channel) instead of [B, L, H]
 
     @property
     def seq_len(self) -> int:
@@ -174,7 +175,7 @@ def block_ids(w: Workload) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seed: int = 0, device="cpu", keep_fp64: bool = False):
-    """Q, K, V [B, L, H, D] bf16 and gate [B, L, H] bf16 on ``device``.
+    """Q, K, V [B, L, H, D] bf16 and gate [B, L, H] (or [B, L, H*D] with gate_per_channel) bf16 on ``device``.
 
     With ``keep_fp64`` the unrounded float64 draws are returned as well (the
     tiny workload's "fp32 originals")."""
@@ -204,10 +205,11 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", keep_fp64: bool = Fals
             raw[name] = x.view(B, L, H, D).clone()
         out[name] = x.to(torch.bfloat16).view(B, L, H, D)
         del x
-    g = _normal_tensor(seed, _GATE, B * L * H, device, std=w.gate_std)
-    out["gate"] = g.to(torch.bfloat16).view(B, L, H)
+    gw = H * D if w.gate_per_channel else H
+    g = _normal_tensor(seed, _GATE, B * L * gw, device, std=w.gate_std)
+    out["gate"] = g.to(torch.bfloat16).view(B, L, gw)
     if keep_fp64:
-        raw["gate"] = g.view(B, L, H)
+        raw["gate"] = g.view(B, L, gw)
         out["fp64"] = raw
     return out
 

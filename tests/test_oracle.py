@@ -392,6 +392,34 @@ def test_output_gate(oracle_mod):
             assert np.abs(r.out[0, toks, h] - expect).max() < 1e-15
 
 
+def test_output_gate_per_channel(oracle_mod):
+    """Reading R12, the per-channel gate [B, L, H*D]: channel h*D + d of a token scales column d of
+    head h's compression row.  Pins: a gate equal across the D channels of each (token, head)
+    gives exactly the scalar-gate output; a one-hot gate (1 at one channel of every token, 0
+    elsewhere) changes only that head and column, by the compression value; a zero gate gives
+    o_f."""
+    w, x = _tiny_case(0.5)
+    B, L, H, D = 1, w.seq_len, w.heads, w.head_dim
+    r = oracle_mod.forward(x["q"], x["k"], x["v"], x["gate"], w.segments, w.grid, 0.5)
+    wide = np.repeat(x["gate"][..., None], D, axis=-1).reshape(B, L, H * D)
+    rw = oracle_mod.forward(x["q"], x["k"], x["v"], wide, w.segments, w.grid, 0.5)
+    assert np.array_equal(rw.out, r.out)
+    h1, d1 = 1, 37
+    onehot = np.zeros((B, L, H * D), np.uint16)
+    onehot[:, :, h1 * D + d1] = bf16_bits(torch.ones(1))[0]
+    ro = oracle_mod.forward(x["q"], x["k"], x["v"], onehot, w.segments, w.grid, 0.5)
+    diff = ro.out - ro.o_f
+    mask = np.zeros_like(diff, bool)
+    mask[:, :, h1, d1] = True
+    assert (diff[~mask] == 0).all()
+    geo = ro.geo
+    for i in range(geo.n_tiles):
+        toks = geo.tile_token[i, :geo.tile_valid[i]]
+        assert np.abs(diff[0, toks, h1, d1] - ro.o_c[0, h1, i, d1]).max() < 1e-14  # (a + b) - a rounds
+    rz = oracle_mod.forward(x["q"], x["k"], x["v"], np.zeros((B, L, H * D), np.uint16), w.segments, w.grid, 0.5)
+    assert (rz.out == rz.o_f).all()
+
+
 def test_scores_fused_chain_in_d_order(oracle_mod):
     """Reading R6 fixes the score arithmetic: one fused multiply-add per d,
     d ascending, from +0.  Two hand-worked cases pin it:
