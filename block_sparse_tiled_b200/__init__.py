@@ -54,6 +54,7 @@ class Geometry(ctypes.Structure):
         ("video_tag", ctypes.c_int32),
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+        ("gate_per_channel", ctypes.c_int32),
     ]
 
 
@@ -138,7 +139,7 @@ def _ptr(t, dtype=None, name="tensor"):
 
 
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                  token_tags=None, video_tag=0, tile_size=64):
+                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False):
     """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers)."""
     g = Geometry()
     g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
@@ -160,6 +161,7 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.tile_size = int(tile_size)
     g.sparsity = float(sparsity)
     g.softmax_scale = float(softmax_scale)
+    g.gate_per_channel = int(bool(gate_per_channel))
     return g, keep
 
 
@@ -227,10 +229,10 @@ class Plan:
 
 
 def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                   token_tags=None, video_tag=0, tile_size=64, stream=None) -> Plan:
+                   token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, stream=None) -> Plan:
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
-              tile_size=tile_size)
+              tile_size=tile_size, gate_per_channel=bool(gate_per_channel))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
     _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")

@@ -109,7 +109,8 @@ struct AttnArgs {
   int* sched;                 // item counter, zero at launch
   int64_t L;
   int H, n_t, P, topk;
-  int gate_ld;  // gate elements between consecutive tokens (H, or more when a head slice is processed)
+  int gate_ld;  // gate elements between consecutive tokens (H or H*D, or more when a head slice is processed)
+  int gate_pc;  // 0: one gate per (token, head) at h; 1: one per channel, at h*D + d
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
 };
@@ -712,7 +713,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (tid < 64) {
         const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
         qtok_s[tid] = tok;
-        gate_s[tid] = (tok >= 0) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.gate_ld + h)) : 0.0f;
+        gate_s[tid] = (tok >= 0 && !a.gate_pc) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.gate_ld + h)) : 0.0f;
       }
       const float oc = (d < D) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
       ROLE_MARK(3);
@@ -742,7 +743,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const int q = 32 * half + j;
             if (q < valid_i) {
-              const float val = fmaf(o[j], rl_s[q], gate_s[q] * oc);
+              const float gq = a.gate_pc ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + qtok_s[q]) * a.gate_ld + h * D + d))
+                                         : gate_s[q];
+              const float val = fmaf(o[j], rl_s[q], gq * oc);
               out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
             }
           }

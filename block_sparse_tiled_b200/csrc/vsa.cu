@@ -67,6 +67,8 @@ int32_t topk_for(double sparsity, int64_t V) {
 vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g == nullptr) return fail(VSA_ERR_INVALID_ARG, "geometry is NULL");
   if (g->batch < 1 || g->heads < 1) return fail(VSA_ERR_INVALID_ARG, "batch and heads must be >= 1");
+  if (g->gate_per_channel != 0 && g->gate_per_channel != 1)
+    return fail(VSA_ERR_INVALID_ARG, "gate_per_channel must be 0 or 1");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
     return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128, got " + std::to_string(g->head_dim));
   if (g->tile_size != kTile)
@@ -252,6 +254,7 @@ struct vsa_plan_s {
   int num_sms = 0;
   size_t max_smem = 0;
   int32_t B = 0, H = 0, D = 0;
+  int32_t gate_pc = 0;  // gate [B, L, H*D] (1) or [B, L, H] (0)
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
   std::vector<int32_t> tile_token, tile_valid;
@@ -405,7 +408,8 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.sched = p->d_status + 2;
   a.L = p->r.L;
   a.H = p->H;
-  a.gate_ld = gate_ld > 0 ? gate_ld : p->H;
+  a.gate_pc = p->gate_pc;
+  a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
   a.n_t = p->n_t;
   a.P = p->P;
   a.topk = p->topk;
@@ -451,6 +455,7 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->B = p->B;
   q->H = heads;
   q->D = p->D;
+  q->gate_pc = p->gate_pc;
   q->r = p->r;
   q->n_t = p->n_t;
   q->P = p->P;
@@ -481,7 +486,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
     off += 4 * h.chunk_bytes;  // q, k, v, out
   }
   h.gate = off;
-  off += align256(tokens * static_cast<size_t>(p->H) * 2);
+  off += align256(tokens * static_cast<size_t>(p->gate_pc ? p->H * p->D : p->H) * 2);
   h.total = off;
   return h;
 }
@@ -503,6 +508,9 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   VSA_TRY(run_topk(p, S, pv, idx, oc, s));
   return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld);
 }
+
+// Gate elements per token: H, or H*D for a per-channel gate.
+int64_t gate_width(const vsa_plan_s* p) { return p->gate_pc ? static_cast<int64_t>(p->H) * p->D : p->H; }
 
 void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->n_tiles = static_cast<int32_t>(r.n_prefix + r.n_video);
@@ -570,6 +578,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   p->B = g->batch;
   p->H = g->heads;
   p->D = g->head_dim;
+  p->gate_pc = g->gate_per_channel;
   p->r = r;
   p->n_t = static_cast<int32_t>(r.n_prefix + r.n_video);
   p->P = static_cast<int32_t>(r.n_prefix);
@@ -696,7 +705,8 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const v
   if (workspace_bytes < p->ws.total)
     return fail(VSA_ERR_WORKSPACE, "workspace holds " + std::to_string(workspace_bytes) + " bytes, needs " +
                                        std::to_string(p->ws.total));
-  return forward_impl(p, q, k, v, gate, p->H, out, static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+  return forward_impl(p, q, k, v, gate, static_cast<int>(gate_width(p)), out, static_cast<uint8_t*>(workspace),
+                      static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
@@ -759,7 +769,8 @@ vsa_status vsa_forward_host(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, co
   VSA_CUDA_TRY(cudaEventRecord(hp.ev_start, s));
   VSA_CUDA_TRY(cudaStreamWaitEvent(hp.h2d, hp.ev_start, 0));
   VSA_CUDA_TRY(cudaStreamWaitEvent(hp.d2h, hp.ev_start, 0));
-  VSA_CUDA_TRY(cudaMemcpyAsync(dgate, gate, tokens * p->H * 2, cudaMemcpyHostToDevice, hp.h2d));
+  const int64_t gw = gate_width(p);  // gate elements per token
+  VSA_CUDA_TRY(cudaMemcpyAsync(dgate, gate, tokens * static_cast<size_t>(gw) * 2, cudaMemcpyHostToDevice, hp.h2d));
   VSA_CUDA_TRY(cudaEventRecord(hp.ev_gate, hp.h2d));
   VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_gate, 0));
 
@@ -787,7 +798,9 @@ vsa_status vsa_forward_host(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, co
     // the forward of the chunk on the caller's stream (output slot free once chunk c-2 is back on the host)
     VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_in[slot], 0));
     if (c >= 2) VSA_CUDA_TRY(cudaStreamWaitEvent(s, hp.ev_out[slot], 0));
-    VSA_TRY(forward_impl(sp, dq, dk, dv, dgate + h0, p->H, dout, w + hl.fwd, s));
+    // the chunk's first head in the whole gate: element h0 of each token, or channel h0*D
+    VSA_TRY(forward_impl(sp, dq, dk, dv, dgate + (p->gate_pc ? static_cast<int64_t>(h0) * p->D : h0), static_cast<int>(gw),
+                         dout, w + hl.fwd, s));
     VSA_CUDA_TRY(cudaEventRecord(hp.ev_comp[slot], s));
     // device -> host: the chunk's heads of the output
     VSA_CUDA_TRY(cudaStreamWaitEvent(hp.d2h, hp.ev_comp[slot], 0));

@@ -26,7 +26,8 @@
  *    stream.  All device work is asynchronous on it; no entry point but
  *    vsa_device_status synchronises.
  *  - Layouts (row-major, last index fastest):
- *      sequence order : q, k, v, out  [B, L, H, D];  gate [B, L, H]
+ *      sequence order : q, k, v, out  [B, L, H, D];  gate [B, L, H], or [B, L, H*D]
+ *                       with vsa_geometry.gate_per_channel
  *      tile order     : q_t, k_t, v_t [B, H, n_tiles, 64, D]  (pad rows zero)
  *      pooled         : pq, pk, pv    [B, H, n_tiles, D] float
  *      scores         : [B, H, n_tiles, n_tiles] float
@@ -93,6 +94,8 @@ typedef struct vsa_geometry {
   int32_t tile_size;         /* must be 64 */
   double sparsity;           /* in [0, 1] */
   float softmax_scale;       /* 0 => (float)(1 / sqrt((double)head_dim)) */
+  int32_t gate_per_channel;  /* 0: gate [B, L, H], one scalar per token and head;
+                                1: gate [B, L, H*D], one per channel h*D + d */
 } vsa_geometry;
 
 typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
@@ -181,8 +184,8 @@ vsa_status vsa_topk_select(vsa_plan p, const float* scores_dev, const float* pv_
  * For a video query tile: softmax attention over the keys of all prefix
  * tiles and of its idx row; for a prefix query tile: over every tile.  Pad
  * keys are masked.  Then out[b,l,h,:] = o_fine + gate[b,l,h] * o_c[b,h,
- * tile(l),:], rounded to bf16 and written in sequence order (pad rows are not
- * written).  Q/K/V in tile order; BF16 tensor-core products with fp32
+ * tile(l),:] (with a per-channel gate, gate[b,l,h*D+d] scales column d),
+ * rounded to bf16 and written in sequence order (pad rows are not written).  Q/K/V in tile order; BF16 tensor-core products with fp32
  * accumulation; P rounded to bf16 before the P.V product.
  * Passage: "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse FP4
  * attention for VSA tiles" (block lists, exempt prefix key tile visited
@@ -204,7 +207,7 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                        void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /* ---- the whole forward with inputs and output in host memory ---------------
- * The forward of vsa_forward for q, k, v [B, L, H, D], gate [B, L, H] and out
+ * The forward of vsa_forward for q, k, v [B, L, H, D], gate [B, L, H] (or [B, L, H*D]) and out
  * [B, L, H, D] that live in HOST memory (bf16, sequence order).  No
  * counterpart on the pages: the heads of the attention are independent, so
  * the call processes them in chunks of `head_chunk` heads and overlaps, on

@@ -32,7 +32,7 @@ def vsa():
 
 def plan_for(vsa, w):
     return vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-                              sparsity=w.sparsity)
+                              sparsity=w.sparsity, gate_per_channel=w.gate_per_channel)
 
 
 def device_reference(vsa, plan, x):
@@ -119,6 +119,19 @@ def test_host_pipeline_head_dim_96(vsa):
 
     w = dataclasses.replace(synth.workload("small"), head_dim=96, name="small_d96")
     x = synth.make_inputs(w, seed=8, device="cuda")
+    plan = plan_for(vsa, w)
+    ref = device_reference(vsa, plan, x)
+    hx = host_copies(x)
+    out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=3)
+    assert torch.equal(out, ref)
+    plan.destroy()
+
+
+def test_host_pipeline_gate_per_channel(vsa):
+    import dataclasses
+
+    w = dataclasses.replace(synth.workload("small"), gate_per_channel=True, name="small_pc")
+    x = synth.make_inputs(w, seed=9, device="cuda")
     plan = plan_for(vsa, w)
     ref = device_reference(vsa, plan, x)
     hx = host_copies(x)

@@ -39,7 +39,7 @@ def bits(t):
 
 def plan_for(vsa, w):
     return vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-                              sparsity=w.sparsity)
+                              sparsity=w.sparsity, gate_per_channel=w.gate_per_channel)
 
 
 def run_forward(vsa, w, x):
@@ -282,3 +282,15 @@ def test_head_dim_96_480p_sampled(vsa, oracle_mod):
     """The 480p-shaped workload at head_dim 96, selection in full and sampled output tiles."""
     w = dataclasses.replace(synth.workload("480p"), head_dim=96, name="480p_d96")
     sampled_parity(vsa, oracle_mod, w, heads=[0, 29, 55], video_every=23)
+
+
+@pytest.mark.parametrize("name,D", [("tiny", 64), ("small", 128), ("small", 96)])
+def test_gate_per_channel_full_parity(vsa, oracle_mod, name, D):
+    """Per-channel gate [B, L, H*D]: the epilogue scales column d of head h by channel h*D + d."""
+    w = dataclasses.replace(synth.workload(name), head_dim=D, gate_per_channel=True, name=f"{name}_pc")
+    full_parity(vsa, oracle_mod, w, seed=7)
+
+
+def test_gate_per_channel_480p_sampled(vsa, oracle_mod):
+    w = dataclasses.replace(synth.workload("480p"), gate_per_channel=True, name="480p_pc")
+    sampled_parity(vsa, oracle_mod, w, heads=[3, 54], video_every=29)
