@@ -111,6 +111,7 @@ struct AttnArgs {
   int H, n_t, P, topk;
   int gate_ld;  // gate elements between consecutive tokens (H or H*D, or more when a head slice is processed)
   int gate_pc;  // 0: one gate per (token, head) at h; 1: one per channel, at h*D + d
+  const int* gate_nonzero;  // NULL, or a flag that is 0 when every gate is zero (o_c then unread)
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
 };
@@ -698,6 +699,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int qd = warp & 3;
     const int d = qd * 32 + lane;                  // O^T lane = d
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    // with every gate zero the compression term vanishes and o_c was not computed
+    const bool use_oc = (a.gate_nonzero == nullptr) || (*a.gate_nonzero != 0);
     int it = 0;
     ROLE_TIMER_START();
     for (;; ++it) {
@@ -715,7 +718,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         qtok_s[tid] = tok;
         gate_s[tid] = (tok >= 0 && !a.gate_pc) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.gate_ld + h)) : 0.0f;
       }
-      const float oc = (d < D) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
+      const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
       ROLE_MARK(3);
       mbar_wait(&bars[Ly::bLFull + ob], (it >> 1) & 1, ctl, 16);
       ROLE_MARK(0);
@@ -743,8 +746,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const int q = 32 * half + j;
             if (q < valid_i) {
-              const float gq = a.gate_pc ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + qtok_s[q]) * a.gate_ld + h * D + d))
-                                         : gate_s[q];
+              const float gq = !use_oc   ? 0.0f
+                               : a.gate_pc ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + qtok_s[q]) * a.gate_ld + h * D + d))
+                                           : gate_s[q];
               const float val = fmaf(o[j], rl_s[q], gq * oc);
               out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
             }

@@ -253,9 +253,35 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
 constexpr int kCompRows = 128;
 constexpr int kCompJ = 32;
 
+// ---------------------------------------------------------------------------
+// Gate check: *nonzero = 1 if any of the n bf16 gate values has a nonzero
+// magnitude (-0 counts as zero, NaN as nonzero).  When every gate is zero the
+// compression branch adds nothing, so its kernel and the epilogue term are
+// skipped.  Blocks stop as soon as one of them has found a nonzero value.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gate_any_kernel(const uint16_t* __restrict__ g, int64_t n, int* nonzero) {
+  volatile int* flag = nonzero;
+  if (*flag) return;
+  const int64_t n8 = n / 8;
+  const uint4* g8 = reinterpret_cast<const uint4*>(g);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  bool any = false;
+  int64_t it = 0;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n8; e += stride, ++it) {
+    const uint4 v = __ldg(g8 + e);
+    any = any || (((v.x | v.y | v.z | v.w) & 0x7fff7fffu) != 0u);
+    if ((it & 15) == 15 && (any || *flag)) break;
+  }
+  for (int64_t e = n8 * 8 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += stride)
+    any = any || ((g[e] & 0x7fffu) != 0u);
+  if (__syncthreads_or(any) && threadIdx.x == 0) *flag = 1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
-                                                        float* __restrict__ o_c, int n_t) {
+                                                        float* __restrict__ o_c, int n_t,
+                                                        const int* __restrict__ gate_nonzero) {
+  if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
   constexpr int kCols = D / 16;  // columns per thread: tx + 16 c
   __shared__ float m_s[kCompRows], l_s[kCompRows];
   __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];

@@ -260,7 +260,7 @@ struct vsa_plan_s {
   std::vector<int32_t> tile_token, tile_valid;
   int32_t* d_tile_token = nullptr;
   int32_t* d_tile_valid = nullptr;
-  int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter
+  int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter, [3] gate nonzero
   vsa_workspace_layout ws{};
   // Head-slice plans share the parent's device tables and status word and own nothing on the device.
   bool owns_device = true;
@@ -364,7 +364,8 @@ vsa_status run_scores(vsa_plan p, const float* pq, const float* pk, float* S, cu
   return launch_check("scores");
 }
 
-vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, float* o_c, cudaStream_t s) {
+vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, float* o_c, cudaStream_t s,
+                    const int* gate_nonzero = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const int64_t BH = static_cast<int64_t>(p->B) * p->H;
   if (p->V > 0 && p->topk > 0) {
@@ -383,14 +384,14 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
   dim3 grid((p->n_t + vsa::kCompRows - 1) / vsa::kCompRows, static_cast<unsigned>(BH));
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
-    vsa::compress_kernel<D><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t);
+    vsa::compress_kernel<D><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t, gate_nonzero);
     return VSA_OK;
   }));
   return launch_check("compress");
 }
 
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
-                    const void* gate, void* out, cudaStream_t s, int gate_ld = 0) {
+                    const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
   CUtensorMap mq, mk, mv;
@@ -409,6 +410,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.L = p->r.L;
   a.H = p->H;
   a.gate_pc = p->gate_pc;
+  a.gate_nonzero = gate_nonzero;
   a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
   a.n_t = p->n_t;
   a.P = p->P;
@@ -503,10 +505,27 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   auto* S = reinterpret_cast<float*>(w + p->ws.scores);
   auto* idx = reinterpret_cast<int32_t*>(w + p->ws.idx);
   auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
+  // does any gate differ from zero?  (if not, the compression branch is skipped on the device)
+  int* gate_nz = p->d_status + 3;
+  VSA_CUDA_TRY(cudaMemsetAsync(gate_nz, 0, sizeof(int), s));
+  if (p->n_t > 0) {
+    // scan from the 16-byte boundary at or below the gate (a head slice of a wider gate need not be
+    // aligned) to this plan's last gate element; values of other heads in between can only make the
+    // check say "nonzero", which keeps the branch
+    const int64_t width = p->gate_pc ? static_cast<int64_t>(p->H) * p->D : p->H;  // this plan's gate per token
+    const int64_t last = (static_cast<int64_t>(p->B) * p->r.L - 1) * gate_ld + width;  // one past, in elements
+    const uintptr_t g = reinterpret_cast<uintptr_t>(gate);
+    const uintptr_t g16 = g & ~static_cast<uintptr_t>(15);
+    const int64_t ng = last + static_cast<int64_t>((g - g16) / 2);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((ng / 8 + 255) / 256, 8LL * p->num_sms));
+    vsa::gate_any_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(reinterpret_cast<const uint16_t*>(g16), ng,
+                                                                         gate_nz);
+    VSA_TRY(launch_check("gate check"));
+  }
   VSA_TRY(run_gather(p, q, k, v, qt, kt, vt, pq, pk, pv, s));
   VSA_TRY(run_scores(p, pq, pk, S, s));
-  VSA_TRY(run_topk(p, S, pv, idx, oc, s));
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld);
+  VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz);
 }
 
 // Gate elements per token: H, or H*D for a per-channel gate.
