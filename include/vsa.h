@@ -201,7 +201,10 @@ vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf
  * S2..S5 in one call, sequence order in and out.  `workspace_dev` must hold
  * vsa_plan_dims.workspace_bytes bytes (256-byte aligned); its contents on
  * entry do not matter and on return are the intermediates (tile-order Q/K/V,
- * pooled tiles, scores, idx, o_c) at offsets vsa_workspace_layout gives. */
+ * pooled tiles, scores, idx, o_c) at offsets vsa_workspace_layout gives.
+ * When every gate value is zero (+0 or -0) the compression branch adds
+ * nothing: a device-side check then skips its kernel and its epilogue term,
+ * and the o_c region is left as it was. */
 vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                        const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
                        void* workspace_dev, size_t workspace_bytes, void* stream);
