@@ -54,7 +54,7 @@ class Geometry(ctypes.Structure):
         ("video_tag", ctypes.c_int32),
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-        ("gate_per_channel", ctypes.c_int32),
+        ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32),
     ]
 
 
@@ -139,7 +139,7 @@ def _ptr(t, dtype=None, name="tensor"):
 
 
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False):
+                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False):
     """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers)."""
     g = Geometry()
     g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
@@ -162,6 +162,7 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.sparsity = float(sparsity)
     g.softmax_scale = float(softmax_scale)
     g.gate_per_channel = int(bool(gate_per_channel))
+    g.seq_tiles = int(bool(seq_tiles))
     return g, keep
 
 
@@ -229,10 +230,11 @@ class Plan:
 
 
 def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                   token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, stream=None) -> Plan:
+                   token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False,
+                   stream=None) -> Plan:
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
-              tile_size=tile_size, gate_per_channel=bool(gate_per_channel))
+              tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
     _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")
@@ -378,19 +380,24 @@ def device_status(plan, stream=None):
 
 
 def workspace_views(plan, workspace):
-    """Typed views of vsa_forward's intermediates inside ``workspace``."""
+    """Typed views of vsa_forward's intermediates inside ``workspace`` (no tile-order views for a plan
+    with seq_tiles, whose workspace holds none)."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
+    seq = bool(g.get("seq_tiles", False))
 
     def view(off, n, dtype, shape):
         nbytes = n * torch.tensor([], dtype=dtype).element_size()
         return workspace[off:off + nbytes].view(dtype).view(*shape)
 
+    def tiles(name):
+        return None if seq else view(lay[name], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D))
+
     return {
-        "q_t": view(lay["q_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
-        "k_t": view(lay["k_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
-        "v_t": view(lay["v_t"], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D)),
+        "q_t": tiles("q_t"),
+        "k_t": tiles("k_t"),
+        "v_t": tiles("v_t"),
         "pq": view(lay["pq"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pk": view(lay["pk"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pv": view(lay["pv"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),

@@ -112,8 +112,18 @@ struct AttnArgs {
   int gate_ld;  // gate elements between consecutive tokens (H or H*D, or more when a head slice is processed)
   int gate_pc;  // 0: one gate per (token, head) at h; 1: one per channel, at h*D + d
   const int* gate_nonzero;  // NULL, or a flag that is 0 when every gate is zero (o_c then unread)
+  const uint64_t* key_mask;  // [n_t]: bit r set when row r of the tile as loaded is a key (a token)
+  const int32_t* coord;      // [n_t][4] TMA coordinates of a tile read from sequence order
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
+};
+
+// Tensor maps for loading tiles straight from sequence order (q, k, v): a 4-D map over [b, token, head, d]
+// for prefix runs and, per batch, a 5-D map over [t, y, x, head, d] of the video grid.
+constexpr int kSeqMaxBatch = 4;
+struct SeqMaps {
+  CUtensorMap prefix[3];
+  CUtensorMap video[3][kSeqMaxBatch];
 };
 
 template <int D>
@@ -157,11 +167,8 @@ struct AttnLayout {
   static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
   static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
   static constexpr int oQtok = oGate + 256;                  // int qtok[64]     (epilogue)
-  static constexpr int oTileValid = oQtok + 256;             // uint8 [n_t]
-  static size_t bytes(int n_t) {
-    const size_t tv = ((static_cast<size_t>(n_t) + 15) / 16) * 16;
-    return 1024 /*alignment slack*/ + oTileValid + tv;
-  }
+  static constexpr int oEnd = oQtok + 256;
+  static size_t bytes(int /*n_t*/) { return 1024 /*alignment slack*/ + oEnd; }
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -193,10 +200,13 @@ __device__ __forceinline__ void warp_sum_scatter32(float* v, int lane) {
   }
 }
 
-template <int D>
+// kSeq = false: Q/K/V come from tile-order copies through 2-D maps (tm_q/k/v).  kSeq = true: they come
+// straight from the sequence-order tensors through `seq`, one box per tile (a 64-token prefix run or a
+// 4x4x4 video cube); rows outside the tile are masked by key_mask and not stored.
+template <int D, bool kSeq>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     vsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, const __grid_constant__ SeqMaps seq) {
   using Ly = AttnLayout<D>;
   constexpr int kQKSteps = D / 16;
   constexpr int kPVSteps = 128 / 16;
@@ -217,14 +227,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
   float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
   int32_t* qtok_s = reinterpret_cast<int32_t*>(sm + Ly::oQtok);
-  uint8_t* tile_valid_s = sm + Ly::oTileValid;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = a.n_t, P = a.P, topk = a.topk, V = n_t - P;
   const WaitCtl ctl{abort_flag, a.status, kWaitTimeoutNs};
 
   // ---------------------------------------------------------------- setup
-  for (int t = threadIdx.x; t < n_t; t += blockDim.x) tile_valid_s[t] = static_cast<uint8_t>(a.tile_valid[t]);
   if (Ly::kZeroBytes > 0) {
     uint32_t* z = reinterpret_cast<uint32_t*>(sm + Ly::oZ);
     for (int t = threadIdx.x; t < Ly::kZeroBytes / 4; t += blockDim.x) z[t] = 0u;
@@ -356,8 +364,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (ok && lane < Ly::kHalves) {
-          const int row = static_cast<int>((bh * n_t + i) * 64);
-          tma_load_2d(sm + Ly::oQ + qb * Ly::kQBytes + lane * 8192, &tm_q, &bars[Ly::bQFull + qb], lane * 64, row);
+          void* dst = sm + Ly::oQ + qb * Ly::kQBytes + lane * 8192;
+          if constexpr (kSeq) {
+            const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + i);
+            const int bb = static_cast<int>(bh / a.H), hh = static_cast<int>(bh - static_cast<int64_t>(bb) * a.H);
+            if (c.x == 0)
+              tma_load_4d(dst, &seq.prefix[0], &bars[Ly::bQFull + qb], lane * 64, hh, c.y, bb);
+            else
+              tma_load_5d(dst, &seq.video[0][bb], &bars[Ly::bQFull + qb], lane * 64, hh, c.y, c.z, c.w);
+          } else {
+            const int row = static_cast<int>((bh * n_t + i) * 64);
+            tma_load_2d(dst, &tm_q, &bars[Ly::bQFull + qb], lane * 64, row);
+          }
         }
       }
       for (int n0 = 0; n0 < nb && ok; n0 += 32) {
@@ -385,9 +403,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // lanes [0, 2*kHalves) issue one 8 KB box each: (half, tile a|b)
           if (lane < 2 * Ly::kHalves) {
             const int hh = lane >> 1, second = lane & 1;
-            const int row = static_cast<int>((bh * n_t + (second ? kb : ka)) * 64);
-            tma_load_2d(ring + st * Ly::kKVBytes + hh * Ly::kHalfBytes + second * 8192, tmap, &bars[b_full + st],
-                        hh * 64, row);
+            const int t = second ? kb : ka;
+            void* dst = ring + st * Ly::kKVBytes + hh * Ly::kHalfBytes + second * 8192;
+            if constexpr (kSeq) {
+              const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + t);
+              const int bb = static_cast<int>(bh / a.H), head = static_cast<int>(bh - static_cast<int64_t>(bb) * a.H);
+              const int ti = is_k ? 1 : 2;
+              if (c.x == 0)
+                tma_load_4d(dst, &seq.prefix[ti], &bars[b_full + st], hh * 64, head, c.y, bb);
+              else
+                tma_load_5d(dst, &seq.video[ti][bb], &bars[b_full + st], hh * 64, head, c.y, c.z, c.w);
+            } else {
+              const int row = static_cast<int>((bh * n_t + t) * 64);
+              tma_load_2d(dst, tmap, &bars[b_full + st], hh * 64, row);
+            }
           }
           __syncwarp();
         }
@@ -531,7 +560,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int i = static_cast<int>(w - bh * n_t);
       const int nk = list_len(i), nb = (nk + 1) / 2;
       const int ob = it & 1;
-      int vcache = 0;  // lane j: valid keys of block (n & ~31) + j, tile a in bits 0..7, tile b in bits 8..15
+      // lane j: the key-mask word of block (n & ~31) + j for this warp's TMEM lane quadrant (rows
+      // 32*qd .. 32*qd + 31 of the block: tile a for qd < 2, tile b otherwise)
+      uint32_t vcache = 0;
 
       float l[CG];
 #pragma unroll
@@ -544,17 +575,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t pu = g / Ly::kPBufs;
         ROLE_MARK(7);
         if ((n & 31) == 0) {
-          // valid-key counts of the next 32 blocks (an odd list's last block has no second tile)
+          // key masks of the next 32 blocks (an odd list's last block has no second tile)
           const int nn = n + lane;
           vcache = 0;
           if (nn < nb) {
-            const int ka = key_tile(bh, i, 2 * nn);
-            const int kb = (2 * nn + 1 < nk) ? tile_valid_s[key_tile(bh, i, 2 * nn + 1)] : 0;
-            vcache = tile_valid_s[ka] | (kb << 8);
+            const int t = 2 * nn + (qd >> 1);
+            const uint64_t m = (t < nk) ? __ldg(a.key_mask + key_tile(bh, i, t)) : 0ull;
+            vcache = static_cast<uint32_t>(m >> (32 * (qd & 1)));
           }
         }
-        const int vpk = __shfl_sync(0xffffffffu, vcache, n & 31);
-        const int2 vc = make_int2(vpk & 0xff, vpk >> 8);
+        const uint32_t kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
         ROLE_MARK(0);
 
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
@@ -582,12 +612,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             x[j + 3] = fmaf(x[j + 3], cl, -m4.w);
           }
         }
-        if (vc.x < 64 || vc.y < 64) {  // pad keys or a half-empty block: mask this lane's key
-          const int vcount = (kl < 64) ? vc.x : vc.y;
-          if ((kl & 63) >= vcount) {
+        if (kmask != 0xffffffffu && !((kmask >> lane) & 1u)) {  // not a key: a pad or out-of-tile row
 #pragma unroll
-            for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
-          }
+          for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
         }
         bool slow = true;
         if (n > 0) {
@@ -712,7 +739,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int64_t b = bh / a.H;
       const int h = static_cast<int>(bh - b * a.H);
       const int ob = it & 1;
-      const int valid_i = tile_valid_s[i];
       if (tid < 64) {
         const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
         qtok_s[tid] = tok;
@@ -745,7 +771,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int q = 32 * half + j;
-            if (q < valid_i) {
+            if (qtok_s[q] >= 0) {
               const float gq = !use_oc   ? 0.0f
                                : a.gate_pc ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + qtok_s[q]) * a.gate_ld + h * D + d))
                                            : gate_s[q];

@@ -59,10 +59,12 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     val[u] = make_uint4(0u, 0u, 0u, 0u);
     if (tok >= 0) val[u] = __ldg(reinterpret_cast<const uint4*>(src + ((static_cast<int64_t>(b) * L + tok) * H + h) * D) + c);
   }
+  // q_t == NULL: pooling only (the attention then reads sequence order itself)
+  const bool write_tiles = (q_t != nullptr);
 #pragma unroll
   for (int u = 0; u < kIters; ++u) {
     const int e = tl + 128 * u;
-    reinterpret_cast<uint4*>(dst + dst_base)[e] = val[u];
+    if (write_tiles) reinterpret_cast<uint4*>(dst + dst_base)[e] = val[u];
     if (pool) reinterpret_cast<uint4*>(tiles + tsr * kTile * D)[e] = val[u];
   }
   if (!pool) return;

@@ -69,6 +69,9 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g->batch < 1 || g->heads < 1) return fail(VSA_ERR_INVALID_ARG, "batch and heads must be >= 1");
   if (g->gate_per_channel != 0 && g->gate_per_channel != 1)
     return fail(VSA_ERR_INVALID_ARG, "gate_per_channel must be 0 or 1");
+  if (g->seq_tiles != 0 && g->seq_tiles != 1) return fail(VSA_ERR_INVALID_ARG, "seq_tiles must be 0 or 1");
+  if (g->seq_tiles && g->batch > 4)
+    return fail(VSA_ERR_UNSUPPORTED, "seq_tiles needs batch <= 4 (one 5-D tensor map per batch)");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
     return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128, got " + std::to_string(g->head_dim));
   if (g->tile_size != kTile)
@@ -163,10 +166,63 @@ void build_tables(const Resolved& r, std::vector<int32_t>* tok, std::vector<int3
       }
 }
 
-vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk) {
+// Tables for reading tiles straight from sequence order with TMA: a tile is one box, a 64-token run of
+// a prefix segment (4-D map over [b, token, head, d]) or a 4x4x4 cube of the video grid (5-D map over
+// [t, y, x, head, d] per batch).  Box row r is the token at position r of the run, or cube position
+// ((t - t0)*4 + (y - y0))*4 + (x - x0); rows outside the segment or the grid are masked.
+//   row_token[tile*64 + r]: token of box row r, -1 if masked
+//   mask_seq[tile]: bit r set when box row r is a token of the tile
+//   mask_tiled[tile]: the low tile_valid bits (tile-order copies hold the valid rows first)
+//   coord[tile]: {0, first token, 0, 0} for a prefix run, {1, x0, y0, t0} for a cube
+void build_seq_tables(const Resolved& r, const std::vector<int32_t>& valid, std::vector<int32_t>* row_token,
+                      std::vector<uint64_t>* mask_seq, std::vector<uint64_t>* mask_tiled, std::vector<int32_t>* coord) {
+  const int64_t n_t = r.n_prefix + r.n_video;
+  row_token->assign(static_cast<size_t>(n_t * kTile), -1);
+  mask_seq->assign(static_cast<size_t>(n_t), 0);
+  mask_tiled->assign(static_cast<size_t>(n_t), 0);
+  coord->assign(static_cast<size_t>(n_t * 4), 0);
+  for (int64_t i = 0; i < n_t; ++i)
+    (*mask_tiled)[i] = valid[i] >= 64 ? ~0ull : ((1ull << valid[i]) - 1);
+  int64_t tile = 0, base = 0;
+  for (int64_t n : r.segments) {
+    for (int64_t s = 0; s < n; s += kTile) {
+      const int64_t cnt = std::min<int64_t>(kTile, n - s);
+      for (int64_t j = 0; j < cnt; ++j) (*row_token)[tile * kTile + j] = static_cast<int32_t>(base + s + j);
+      (*mask_seq)[tile] = (*mask_tiled)[tile];
+      (*coord)[tile * 4 + 1] = static_cast<int32_t>(base + s);
+      ++tile;
+    }
+    base += n;
+  }
+  const int64_t ct = (r.T + 3) / 4, ch = (r.Hg + 3) / 4, cw = (r.W + 3) / 4;
+  for (int64_t a = 0; a < ct && r.n_video > 0; ++a)
+    for (int64_t bb = 0; bb < ch; ++bb)
+      for (int64_t c = 0; c < cw; ++c) {
+        uint64_t m = 0;
+        for (int64_t t = 0; t < 4; ++t)
+          for (int64_t h = 0; h < 4; ++h)
+            for (int64_t w = 0; w < 4; ++w) {
+              const int64_t tt = 4 * a + t, hh = 4 * bb + h, ww = 4 * c + w;
+              if (tt >= r.T || hh >= r.Hg || ww >= r.W) continue;
+              const int64_t row = (t * 4 + h) * 4 + w;
+              (*row_token)[tile * kTile + row] = static_cast<int32_t>(base + (tt * r.Hg + hh) * r.W + ww);
+              m |= 1ull << row;
+            }
+        (*mask_seq)[tile] = m;
+        int32_t* cd = coord->data() + tile * 4;
+        cd[0] = 1;
+        cd[1] = static_cast<int32_t>(4 * c);
+        cd[2] = static_cast<int32_t>(4 * bb);
+        cd[3] = static_cast<int32_t>(4 * a);
+        ++tile;
+      }
+}
+
+// seq_tiles: no tile-order copies (their regions are empty).
+vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk, bool seq_tiles) {
   vsa_workspace_layout w{};
   size_t off = 0;
-  const size_t tiles = static_cast<size_t>(B * H * n_t * kTile * D * 2);
+  const size_t tiles = seq_tiles ? 0 : static_cast<size_t>(B * H * n_t * kTile * D * 2);
   const size_t pooled = static_cast<size_t>(B * H * n_t * D * 4);
   w.q_t = off; off += align256(tiles);
   w.k_t = off; off += align256(tiles);
@@ -219,6 +275,42 @@ vsa_status make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int D) 
   return VSA_OK;
 }
 
+// Maps for reading q, k or v [B, L, H, D] straight from sequence order (SeqMaps): the prefix as a 4-D
+// tensor [B][L][H][D] with one box per 64-token run (box 64 d x 1 head x 64 tokens x 1 batch), the video
+// of batch b as a 5-D tensor [T][Hg][W][H][D] starting at token b*L + P with one box per 4x4x4 cube.
+// Out-of-range box rows (past the sequence or the grid) are filled with zeros and masked.
+vsa_status make_seq_maps(CUtensorMap* prefix, CUtensorMap* video, const void* base, int64_t B, int64_t L, int64_t H,
+                         int64_t D, int64_t P, int64_t T, int64_t Hg, int64_t W) {
+  EncodeTiledFn enc;
+  VSA_TRY(get_encoder(&enc));
+  const cuuint64_t e = 2;  // bytes per element
+  {
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {D * e, H * D * e, L * H * D * e};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(prefix, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled (prefix map) failed: " + std::to_string(r));
+  }
+  if (T * Hg * W == 0) return VSA_OK;
+  for (int64_t b = 0; b < B; ++b) {
+    const auto* vbase = static_cast<const uint8_t*>(base) + ((b * L + P) * H * D) * e;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(W),
+                          static_cast<cuuint64_t>(Hg), static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[4] = {D * e, H * D * e, W * H * D * e, Hg * W * H * D * e};
+    cuuint32_t box[5] = {64, 1, 4, 4, 4};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(video + b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<uint8_t*>(vbase), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled (video map) failed: " + std::to_string(r));
+  }
+  return VSA_OK;
+}
+
 }  // namespace
 
 // Scratch of vsa_forward_noalloc: one array per device, alive until the
@@ -255,11 +347,19 @@ struct vsa_plan_s {
   size_t max_smem = 0;
   int32_t B = 0, H = 0, D = 0;
   int32_t gate_pc = 0;  // gate [B, L, H*D] (1) or [B, L, H] (0)
+  bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
   std::vector<int32_t> tile_token, tile_valid;
   int32_t* d_tile_token = nullptr;
   int32_t* d_tile_valid = nullptr;
+  // tables for TMA loads straight from sequence order (build_seq_tables)
+  std::vector<int32_t> row_token, coord;
+  std::vector<uint64_t> mask_seq, mask_tiled;
+  int32_t* d_row_token = nullptr;
+  int32_t* d_coord = nullptr;  // [n_t][4]
+  uint64_t* d_mask_seq = nullptr;
+  uint64_t* d_mask_tiled = nullptr;
   int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter, [3] gate nonzero
   vsa_workspace_layout ws{};
   // Head-slice plans share the parent's device tables and status word and own nothing on the device.
@@ -390,18 +490,33 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
   return launch_check("compress");
 }
 
+// qt/kt/vt: tile-order copies; or, with seq_qkv (q, k, v in sequence order), the kernel reads the
+// tiles itself (needs B <= kSeqMaxBatch).
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
-                    const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr) {
+                    const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
+                    const void* const* seq_qkv = nullptr) {
   if (p->n_t == 0) return VSA_OK;
+  const bool seq = (seq_qkv != nullptr);
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
-  CUtensorMap mq, mk, mv;
-  VSA_TRY(make_tile_map(&mq, qt, rows, p->D));
-  VSA_TRY(make_tile_map(&mk, kt, rows, p->D));
-  VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
+  CUtensorMap mq{}, mk{}, mv{};
+  vsa::SeqMaps sm{};
+  if (seq) {
+    if (p->B > vsa::kSeqMaxBatch) return fail(VSA_ERR_UNSUPPORTED, "sequence-order attention needs batch <= 4");
+    const int64_t vid = p->r.T * p->r.Hg * p->r.W;
+    for (int t = 0; t < 3; ++t)
+      VSA_TRY(make_seq_maps(&sm.prefix[t], sm.video[t], seq_qkv[t], p->B, p->r.L, p->H, p->D, p->r.L - vid, p->r.T,
+                            p->r.Hg, p->r.W));
+  } else {
+    VSA_TRY(make_tile_map(&mq, qt, rows, p->D));
+    VSA_TRY(make_tile_map(&mk, kt, rows, p->D));
+    VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
+  }
   vsa::AttnArgs a{};
   a.idx = idx;
-  a.tile_token = p->d_tile_token;
+  a.tile_token = seq ? p->d_row_token : p->d_tile_token;  // query row -> token (-1: not stored)
   a.tile_valid = p->d_tile_valid;
+  a.key_mask = seq ? p->d_mask_seq : p->d_mask_tiled;
+  a.coord = p->d_coord;
   a.o_c = o_c;
   a.gate = static_cast<const uint16_t*>(gate);
   a.out = static_cast<uint16_t*>(out);
@@ -424,8 +539,13 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     constexpr int D = decltype(dc)::value;
     const size_t smem = vsa::AttnLayout<D>::bytes(p->n_t);
     if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
-    VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D>, smem));
-    vsa::vsa_attn_kernel<D><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a);
+    if (seq) {
+      VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D, true>, smem));
+      vsa::vsa_attn_kernel<D, true><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a, sm);
+    } else {
+      VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D, false>, smem));
+      vsa::vsa_attn_kernel<D, false><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a, sm);
+    }
     return VSA_OK;
   }));
   return launch_check("attention");
@@ -465,8 +585,13 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->topk = p->topk;
   q->d_tile_token = p->d_tile_token;
   q->d_tile_valid = p->d_tile_valid;
+  q->d_row_token = p->d_row_token;
+  q->d_coord = p->d_coord;
+  q->d_mask_seq = p->d_mask_seq;
+  q->d_mask_tiled = p->d_mask_tiled;
   q->d_status = p->d_status;
-  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk);
+  q->seq_tiles = p->seq_tiles;
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk, q->seq_tiles);
   q->owns_device = false;
   return q;
 }
@@ -482,7 +607,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
   h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
   h.fwd = 0;
-  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk).total);
+  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk, p->seq_tiles).total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
     off += 4 * h.chunk_bytes;  // q, k, v, out
@@ -522,10 +647,14 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
                                                                          gate_nz);
     VSA_TRY(launch_check("gate check"));
   }
-  VSA_TRY(run_gather(p, q, k, v, qt, kt, vt, pq, pk, pv, s));
+  // With seq_tiles the attention reads Q/K/V straight from sequence order and the gather only pools;
+  // otherwise the gather writes tile-order copies, which the attention reads with better DRAM locality.
+  const bool seq = p->seq_tiles;
+  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s));
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz);
+  const void* qkv[3] = {q, k, v};
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr);
 }
 
 // Gate elements per token: H, or H*D for a per-channel gate.
@@ -538,7 +667,7 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->topk = r.topk;
   d->seq_len = r.L;
   d->softmax_scale = r.scale;
-  d->workspace_bytes = make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk).total;
+  d->workspace_bytes = make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk, g->seq_tiles != 0).total;
   d->selected_pairs = r.n_video * (r.n_prefix + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
 }
 
@@ -604,17 +733,27 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   p->V = static_cast<int32_t>(r.n_video);
   p->topk = r.topk;
   build_tables(r, &p->tile_token, &p->tile_valid);
-  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk);
+  build_seq_tables(r, p->tile_valid, &p->row_token, &p->mask_seq, &p->mask_tiled, &p->coord);
+  p->seq_tiles = g->seq_tiles != 0;
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk, p->seq_tiles);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
+    cudaFree(p->d_row_token);
+    cudaFree(p->d_coord);
+    cudaFree(p->d_mask_seq);
+    cudaFree(p->d_mask_tiled);
     cudaFree(p->d_status);
     delete p;
   };
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t tok_bytes = std::max<size_t>(4, p->tile_token.size() * 4);
   const size_t val_bytes = std::max<size_t>(4, p->tile_valid.size() * 4);
+  const size_t mask_bytes = std::max<size_t>(8, p->mask_seq.size() * 8);
+  const size_t coord_bytes = std::max<size_t>(16, p->coord.size() * 4);
   if (cudaMalloc(&p->d_tile_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_tile_valid, val_bytes) != cudaSuccess ||
+      cudaMalloc(&p->d_row_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_coord, coord_bytes) != cudaSuccess ||
+      cudaMalloc(&p->d_mask_seq, mask_bytes) != cudaSuccess || cudaMalloc(&p->d_mask_tiled, mask_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
@@ -624,6 +763,14 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     e = cudaMemcpyAsync(p->d_tile_token, p->tile_token.data(), p->tile_token.size() * 4, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !p->tile_valid.empty())
     e = cudaMemcpyAsync(p->d_tile_valid, p->tile_valid.data(), p->tile_valid.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->row_token.empty())
+    e = cudaMemcpyAsync(p->d_row_token, p->row_token.data(), p->row_token.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->coord.empty())
+    e = cudaMemcpyAsync(p->d_coord, p->coord.data(), p->coord.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->mask_seq.empty())
+    e = cudaMemcpyAsync(p->d_mask_seq, p->mask_seq.data(), p->mask_seq.size() * 8, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->mask_tiled.empty())
+    e = cudaMemcpyAsync(p->d_mask_tiled, p->mask_tiled.data(), p->mask_tiled.size() * 8, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 4 * sizeof(int), s);
   if (e != cudaSuccess) {
     cleanup();
@@ -669,6 +816,10 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
   if (p->owns_device) {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
+    cudaFree(p->d_row_token);
+    cudaFree(p->d_coord);
+    cudaFree(p->d_mask_seq);
+    cudaFree(p->d_mask_tiled);
     cudaFree(p->d_status);
   }
   if (prev >= 0) cudaSetDevice(prev);

@@ -96,6 +96,10 @@ typedef struct vsa_geometry {
   float softmax_scale;       /* 0 => (float)(1 / sqrt((double)head_dim)) */
   int32_t gate_per_channel;  /* 0: gate [B, L, H], one scalar per token and head;
                                 1: gate [B, L, H*D], one per channel h*D + d */
+  int32_t seq_tiles;         /* 0: vsa_forward copies Q/K/V to tile order first (faster on B200);
+                                1: the attention reads each tile straight from sequence order
+                                with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
+                                by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4 */
 } vsa_geometry;
 
 typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
@@ -201,7 +205,8 @@ vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf
  * S2..S5 in one call, sequence order in and out.  `workspace_dev` must hold
  * vsa_plan_dims.workspace_bytes bytes (256-byte aligned); its contents on
  * entry do not matter and on return are the intermediates (tile-order Q/K/V,
- * pooled tiles, scores, idx, o_c) at offsets vsa_workspace_layout gives.
+ * unless the plan has seq_tiles; pooled tiles, scores, idx, o_c) at offsets
+ * vsa_workspace_layout gives.
  * When every gate value is zero (+0 or -0) the compression branch adds
  * nothing: a device-side check then skips its kernel and its epilogue term,
  * and the o_c region is left as it was. */

@@ -131,3 +131,15 @@ def test_workspace_size(vsa):
     tiles = H * n_t * 64 * D * 2
     assert d["workspace_bytes"] >= 3 * tiles + 4 * H * n_t * D * 4 + H * n_t * n_t * 4 + H * 1152 * 116 * 4
     assert d["workspace_bytes"] < 3 * tiles * 1.2
+
+
+def test_seq_tiles_workspace_and_limits(vsa):
+    """seq_tiles drops the three tile-order copies from the workspace and needs batch <= 4."""
+    kw = dict(batch=1, heads=56, head_dim=128, segments=(512, 0, 768), grid=(24, 48, 64), sparsity=0.9)
+    a = vsa.vsa_plan_query(**kw)["workspace_bytes"]
+    b = vsa.vsa_plan_query(seq_tiles=True, **kw)["workspace_bytes"]
+    tiles = 3 * 56 * 1172 * 64 * 128 * 2
+    assert a - b == tiles
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_plan_query(batch=5, heads=2, head_dim=64, segments=(64,), grid=(4, 4, 4), seq_tiles=True)
+    assert e.value.status == 3  # VSA_ERR_UNSUPPORTED

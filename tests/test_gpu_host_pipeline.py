@@ -30,9 +30,9 @@ def vsa():
     return m
 
 
-def plan_for(vsa, w):
+def plan_for(vsa, w, seq_tiles=False):
     return vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-                              sparsity=w.sparsity, gate_per_channel=w.gate_per_channel)
+                              sparsity=w.sparsity, gate_per_channel=w.gate_per_channel, seq_tiles=seq_tiles)
 
 
 def device_reference(vsa, plan, x):
@@ -136,5 +136,17 @@ def test_host_pipeline_gate_per_channel(vsa):
     ref = device_reference(vsa, plan, x)
     hx = host_copies(x)
     out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=3)
+    assert torch.equal(out, ref)
+    plan.destroy()
+
+
+def test_host_pipeline_seq_tiles(vsa):
+    """A seq_tiles plan through the host pipeline: its head-slice plans read sequence order too."""
+    w = synth.workload("480p")
+    x = synth.make_inputs(w, seed=10, device="cuda")
+    plan = plan_for(vsa, w, seq_tiles=True)
+    ref = device_reference(vsa, plan, x)
+    hx = host_copies(x)
+    out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=13)
     assert torch.equal(out, ref)
     plan.destroy()
