@@ -376,6 +376,43 @@ def run_vsa(args, w, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_ab_seq_tiles(args, w):
+    """Side measurement (not the contract line): the whole vsa_forward with tile-order copies against a
+    seq_tiles plan, alternating the two plans; prints one JSON line with the medians and workspaces."""
+    import torch
+    import synth
+    import block_sparse_tiled_b200 as vsa
+
+    torch.cuda.set_device(0)
+    x = synth.make_inputs(w, seed=0, device="cuda")
+    res = {"workload": w.name, "steps": args.steps, "warmup": args.warmup, "forward_ms": {}, "workspace_bytes": {}}
+    for rnd in range(2):
+        for seq in (False, True):
+            key = "seq_tiles" if seq else "tile_order"
+            plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments,
+                                      grid=w.grid, sparsity=w.sparsity, seq_tiles=seq)
+            ws = vsa.alloc_workspace(plan)
+            out = torch.empty_like(x["q"])
+            for _ in range(args.warmup):
+                vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], out=out, workspace=ws)
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], out=out, workspace=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            ts.sort()
+            res["forward_ms"].setdefault(key, []).append(ts[len(ts) // 2])
+            res["workspace_bytes"][key] = ws.numel()
+            plan.destroy()
+            del ws, out
+            torch.cuda.empty_cache()
+    print(json.dumps(res))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -387,12 +424,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-every", type=int, default=1)
     ap.add_argument("--ref-every", type=int, default=16)
+    ap.add_argument("--ab-seq-tiles", action="store_true",
+                    help="side measurement: vsa_forward with tile-order copies against a seq_tiles plan")
     args = ap.parse_args()
     import synth
 
     w = synth.workload(args.workload)
     if args.sparsity is not None:
         w = dataclasses.replace(w, sparsity=args.sparsity, name=f"{w.name}@s{args.sparsity}")
+    if args.ab_seq_tiles:
+        run_ab_seq_tiles(args, w)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -60,3 +60,21 @@ def test_noalloc_rejects_oversized_geometry(vsa):
     assert vsa.STATUS_NAMES[e.value.status] == "VSA_ERR_WORKSPACE"
     assert "static scratch" in str(e.value)
     plan.destroy()
+
+
+def test_noalloc_480p_with_seq_tiles(vsa):
+    """A seq_tiles plan needs no tile-order copies, so the 480p-shaped problem (0.69 GB of workspace
+    with copies) fits the 64 MiB static scratch; the result is bit-identical to vsa_forward with the
+    same plan."""
+    w = synth.workload("480p")
+    plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
+                              sparsity=w.sparsity, seq_tiles=True)
+    assert plan.dims["workspace_bytes"] <= vsa.NOALLOC_SCRATCH_BYTES
+    x = synth.make_inputs(w, seed=3, device="cuda")
+    ref = vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], workspace=vsa.alloc_workspace(plan))
+    out = torch.full_like(x["q"], float("nan"))
+    vsa.vsa_forward_noalloc(plan, x["q"], x["k"], x["v"], x["gate"], out)
+    torch.cuda.synchronize()
+    assert vsa.device_status(plan) == (0, 0)
+    assert torch.equal(out, ref)
+    plan.destroy()
