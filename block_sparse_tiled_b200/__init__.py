@@ -35,7 +35,7 @@ EXPORTED = (
     "vsa_plan_tiles", "vsa_plan_info", "vsa_plan_tables", "vsa_plan_query", "vsa_plan_tables_host",
     "vsa_plan_destroy",
     "vsa_gather_tiles", "vsa_pool_and_score", "vsa_topk_select", "vsa_sparse_attn_fwd", "vsa_forward",
-    "vsa_forward_noalloc", "vsa_forward_host", "vsa_forward_host_workspace", "vsa_wait_selftest",
+    "vsa_forward_noalloc", "vsa_forward_host", "vsa_forward_host_workspace", "vsa_forward_parts", "vsa_wait_selftest",
     "vsa_plan_workspace", "vsa_device_status", "vsa_last_error", "vsa_version",
 )
 
@@ -55,6 +55,16 @@ class Geometry(ctypes.Structure):
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
         ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32),
+    ]
+
+
+class SeqParts(ctypes.Structure):
+    _fields_ = [
+        ("nparts", ctypes.c_int32), ("tokens_per_part", ctypes.c_int64), ("heads_total", ctypes.c_int32),
+        ("head_offset", ctypes.c_int32),
+        ("q", ctypes.POINTER(ctypes.c_void_p)), ("k", ctypes.POINTER(ctypes.c_void_p)),
+        ("v", ctypes.POINTER(ctypes.c_void_p)), ("gate", ctypes.POINTER(ctypes.c_void_p)),
+        ("out", ctypes.POINTER(ctypes.c_void_p)),
     ]
 
 
@@ -102,6 +112,7 @@ def load_library(path: str = LIB_PATH):
     lib.vsa_forward_noalloc.argtypes = [P] * 7
     lib.vsa_forward_host_workspace.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
     lib.vsa_forward_host.argtypes = [P, P, P, P, P, P, ctypes.c_int32, P, ctypes.c_size_t, P]
+    lib.vsa_forward_parts.argtypes = [P, ctypes.POINTER(SeqParts), P, ctypes.c_size_t, P]
     lib.vsa_wait_selftest.argtypes = [P, ctypes.c_int64, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     lib.vsa_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
     for name in EXPORTED:
@@ -348,6 +359,43 @@ def vsa_forward(plan, q, k, v, gate, out=None, workspace=None, stream=None):
         _ptr(out, bf, "out"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "vsa_forward")
     return out
+
+
+MAX_PARTS = 64
+
+
+def ulysses_partition(seq_len: int, heads: int, world: int, rank: int):
+    """Sequence-parallel layout of one rank: (tokens per part, heads of this rank, first head).  Rank r
+    holds tokens [r*Ls, (r+1)*Ls) of q/k/v/gate/out and runs the forward for heads [r*Hn, (r+1)*Hn)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside a world of {world}")
+    if seq_len % world or heads % world:
+        raise ValueError(f"the world size {world} must divide the sequence length {seq_len} and the heads {heads}")
+    hn = heads // world
+    return seq_len // world, hn, rank * hn
+
+
+def vsa_forward_parts(plan, q_parts, k_parts, v_parts, gate_parts, out_parts, head_offset, workspace=None, stream=None):
+    """The forward for this plan's heads over a sequence split into parts (lists of CUDA tensors
+    [B, Ls, Htot, D], gate [B, Ls, Htot] or [B, Ls, Htot*D]); parts may be peer mappings of other
+    GPUs' buffers.  Writes heads [head_offset, head_offset + H) of every out part."""
+    n = len(q_parts)
+    if not (len(k_parts) == len(v_parts) == len(gate_parts) == len(out_parts) == n) or not 1 <= n <= MAX_PARTS:
+        raise ValueError("q, k, v, gate and out need the same number of parts, at most MAX_PARTS")
+    B, Ls, Htot, D = q_parts[0].shape
+    if workspace is None:
+        workspace = alloc_workspace(plan, q_parts[0].device)
+    bf = torch.bfloat16
+
+    def arr(ts, name):
+        return (ctypes.c_void_p * n)(*[_ptr(t, bf, f"{name}[{i}]") for i, t in enumerate(ts)])
+
+    keep = [arr(q_parts, "q"), arr(k_parts, "k"), arr(v_parts, "v"), arr(gate_parts, "gate"), arr(out_parts, "out")]
+    cast = lambda a: ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))  # noqa: E731
+    sp = SeqParts(n, Ls, Htot, int(head_offset), *[cast(a) for a in keep])
+    _check(load_library().vsa_forward_parts(plan.handle, ctypes.byref(sp), _ptr(workspace, torch.uint8, "workspace"),
+                                            workspace.numel(), _stream(stream)), "vsa_forward_parts")
+    return out_parts
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20

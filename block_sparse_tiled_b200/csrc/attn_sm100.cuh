@@ -114,6 +114,7 @@ struct AttnArgs {
   const int* gate_nonzero;  // NULL, or a flag that is 0 when every gate is zero (o_c then unread)
   const uint64_t* key_mask;  // [n_t]: bit r set when row r of the tile as loaded is a key (a token)
   const int32_t* coord;      // [n_t][4] TMA coordinates of a tile read from sequence order
+  PartIO io;                 // where gate and out live (one tensor, or sequence parts, possibly on peers)
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
 };
@@ -166,8 +167,9 @@ struct AttnLayout {
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
   static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
   static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
-  static constexpr int oQtok = oGate + 256;                  // int qtok[64]     (epilogue)
-  static constexpr int oEnd = oQtok + 256;
+  static constexpr int oQtok = oGate + 256;                  // int qtok[64]: token within its part (epilogue)
+  static constexpr int oQpart = oQtok + 256;                 // int qpart[64]: part holding the token
+  static constexpr int oEnd = oQpart + 256;
   static size_t bytes(int /*n_t*/) { return 1024 /*alignment slack*/ + oEnd; }
 };
 
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
   float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
   int32_t* qtok_s = reinterpret_cast<int32_t*>(sm + Ly::oQtok);
+  int32_t* qpart_s = reinterpret_cast<int32_t*>(sm + Ly::oQpart);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = a.n_t, P = a.P, topk = a.topk, V = n_t - P;
@@ -741,8 +744,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int ob = it & 1;
       if (tid < 64) {
         const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
-        qtok_s[tid] = tok;
-        gate_s[tid] = (tok >= 0 && !a.gate_pc) ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + tok) * a.gate_ld + h)) : 0.0f;
+        int64_t lt = -1;
+        int part = 0;
+        if (tok >= 0 && a.io.table != nullptr) {
+          part = static_cast<int>(tok / a.io.Ls);
+          lt = tok - part * a.io.Ls;
+        } else if (tok >= 0) {
+          lt = tok;
+        }
+        qtok_s[tid] = static_cast<int32_t>(lt);
+        qpart_s[tid] = part;
+        const uint16_t* gb = a.io.table ? static_cast<const uint16_t*>(a.io.table[kPartGate * a.io.nparts + part]) : a.gate;
+        gate_s[tid] = (tok >= 0 && !a.gate_pc && use_oc)
+                          ? bf16_bits_to_f32(__ldg(gb + (b * a.io.Ls + lt) * a.gate_ld + a.io.h0 + h))
+                          : 0.0f;
       }
       const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
       ROLE_MARK(3);
@@ -755,7 +770,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(&bars[Ly::bOFull + ob], (it >> 1) & 1, ctl, 17);
       ROLE_MARK(1);
       named_bar_sync(9, 128);  // rl, gate, qtok ready
-      uint16_t* out_col = a.out + (b * a.L * a.H + h) * D + d;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         tc_fence_after();
@@ -771,12 +785,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int q = 32 * half + j;
-            if (qtok_s[q] >= 0) {
-              const float gq = !use_oc   ? 0.0f
-                               : a.gate_pc ? bf16_bits_to_f32(__ldg(a.gate + (b * a.L + qtok_s[q]) * a.gate_ld + h * D + d))
-                                           : gate_s[q];
+            const int64_t lt = qtok_s[q];
+            if (lt >= 0) {
+              const int part = qpart_s[q];
+              const int64_t row = b * a.io.Ls + lt;  // row of the token in its part (or in the one tensor)
+              float gq = gate_s[q];
+              if (a.gate_pc && use_oc) {
+                const uint16_t* gb =
+                    a.io.table ? static_cast<const uint16_t*>(a.io.table[kPartGate * a.io.nparts + part]) : a.gate;
+                gq = bf16_bits_to_f32(__ldg(gb + row * a.gate_ld + static_cast<int64_t>(a.io.h0 + h) * D + d));
+              }
               const float val = fmaf(o[j], rl_s[q], gq * oc);
-              out_col[static_cast<int64_t>(qtok_s[q]) * a.H * D] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+              uint16_t* ob = a.io.table ? static_cast<uint16_t*>(const_cast<void*>(a.io.table[kPartOut * a.io.nparts + part]))
+                                        : a.out;
+              ob[(row * a.io.Htot + a.io.h0 + h) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
             }
           }
         }

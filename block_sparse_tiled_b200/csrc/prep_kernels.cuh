@@ -21,6 +21,34 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 }
 
 // ---------------------------------------------------------------------------
+// Where the sequence-order tensors live.  With table == NULL: one tensor per operand (the pointer
+// arguments), [B, L, Htot, D], of which heads [h0, h0 + H) are processed (Ls = L).  With a table: the
+// sequence is split into nparts parts of Ls tokens (part p holds tokens [p*Ls, (p+1)*Ls)), each part a
+// [B, Ls, Htot, D] tensor that may live in another GPU's memory (a peer mapping); table holds nparts
+// pointers per operand, in the order q, k, v, gate, out.  This is how a sequence-parallel (Ulysses)
+// layout is read and written without separate all-to-all exchanges.
+// ---------------------------------------------------------------------------
+struct PartIO {
+  const void* const* table;
+  int nparts;
+  int64_t Ls;
+  int Htot, h0;
+};
+enum : int { kPartQ = 0, kPartK = 1, kPartV = 2, kPartGate = 3, kPartOut = 4 };
+
+// Base of operand `op` holding token `tok`, and the token's index inside it.
+template <typename T>
+__device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int64_t tok, int64_t* local) {
+  if (io.table == nullptr) {
+    *local = tok;
+    return single;
+  }
+  const int64_t p = tok / io.Ls;
+  *local = tok - p * io.Ls;
+  return static_cast<T*>(const_cast<void*>(io.table[op * io.nparts + p]));
+}
+
+// ---------------------------------------------------------------------------
 // S2 (+ S3 pooling): sequence order [B, L, H, D] -> tile order [B, H, n_t, 64, D]
 // One CTA per (tile, head, batch) moves the tile of Q, K and V with 16-byte
 // loads/stores (each 256-byte token row is read by 16 consecutive threads),
@@ -32,7 +60,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     uint16_t* __restrict__ q_t, uint16_t* __restrict__ k_t, uint16_t* __restrict__ v_t,
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
-    int n_t) {
+    int n_t, const PartIO io) {
   constexpr int kChunks = D / 8;                 // 16-byte chunks per row
   constexpr int kPerTensor = kTile * kChunks;    // chunks per tile of one tensor
   constexpr int kIters = kPerTensor / 128;       // each of 128 threads per tensor moves kIters chunks
@@ -57,7 +85,11 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     const int r = e / kChunks, c = e - r * kChunks;
     const int32_t tok = tok_s[r];
     val[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (tok >= 0) val[u] = __ldg(reinterpret_cast<const uint4*>(src + ((static_cast<int64_t>(b) * L + tok) * H + h) * D) + c);
+    if (tok >= 0) {
+      int64_t lt;
+      const uint16_t* base = part_base(io, tsr, src, tok, &lt);
+      val[u] = __ldg(reinterpret_cast<const uint4*>(base + ((static_cast<int64_t>(b) * io.Ls + lt) * io.Htot + io.h0 + h) * D) + c);
+    }
   }
   // q_t == NULL: pooling only (the attention then reads sequence order itself)
   const bool write_tiles = (q_t != nullptr);

@@ -347,6 +347,9 @@ struct vsa_plan_s {
   size_t max_smem = 0;
   int32_t B = 0, H = 0, D = 0;
   int32_t gate_pc = 0;  // gate [B, L, H*D] (1) or [B, L, H] (0)
+  // vsa_forward_parts: the part pointer table (host copy and device copy, 5 operands x kMaxParts)
+  std::vector<const void*> part_table;
+  const void** d_part_table = nullptr;
   bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
@@ -419,8 +422,12 @@ vsa_status with_head_dim(int D, F&& f) {
   }
 }
 
+// One sequence-order tensor per operand, all heads of the plan.
+vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H, 0}; }
+
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
-                      float* pk, float* pv, cudaStream_t s) {
+                      float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr) {
+  const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
   const size_t smem = pool ? static_cast<size_t>(3) * kTile * p->D * 2 : 0;
@@ -435,7 +442,7 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
     constexpr int D = decltype(dc)::value;
     VSA_TRY(allow_smem(vsa::gather_pool_kernel<D>, smem));
     vsa::gather_pool_kernel<D><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                       p->d_tile_valid, p->r.L, p->H, p->n_t);
+                                                       p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
     return VSA_OK;
   }));
   return launch_check("gather_pool");
@@ -494,7 +501,7 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 // tiles itself (needs B <= kSeqMaxBatch).
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
                     const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
-                    const void* const* seq_qkv = nullptr) {
+                    const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
@@ -526,6 +533,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.H = p->H;
   a.gate_pc = p->gate_pc;
   a.gate_nonzero = gate_nonzero;
+  a.io = io ? *io : single_io(p);
   a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
   a.n_t = p->n_t;
   a.P = p->P;
@@ -620,7 +628,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
 
 // The four steps on one stream; `w` holds p->ws.total bytes.  gate_ld: gate elements between tokens.
 vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v, const void* gate, int gate_ld, void* out,
-                        uint8_t* w, cudaStream_t s) {
+                        uint8_t* w, cudaStream_t s, const vsa::PartIO* io = nullptr) {
   auto* qt = w + p->ws.q_t;
   auto* kt = w + p->ws.k_t;
   auto* vt = w + p->ws.v_t;
@@ -632,8 +640,10 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
   // does any gate differ from zero?  (if not, the compression branch is skipped on the device)
   int* gate_nz = p->d_status + 3;
-  VSA_CUDA_TRY(cudaMemsetAsync(gate_nz, 0, sizeof(int), s));
-  if (p->n_t > 0) {
+  // sequence parts: the gate is spread over the parts and is not scanned; the branch is kept
+  const bool parts = (io != nullptr && io->table != nullptr);
+  VSA_CUDA_TRY(cudaMemsetAsync(gate_nz, parts ? 1 : 0, sizeof(int), s));
+  if (p->n_t > 0 && !parts) {
     // scan from the 16-byte boundary at or below the gate (a head slice of a wider gate need not be
     // aligned) to this plan's last gate element; values of other heads in between can only make the
     // check say "nonzero", which keeps the branch
@@ -650,11 +660,11 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   // With seq_tiles the attention reads Q/K/V straight from sequence order and the gather only pools;
   // otherwise the gather writes tile-order copies, which the attention reads with better DRAM locality.
   const bool seq = p->seq_tiles;
-  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s));
+  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io));
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr);
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io);
 }
 
 // Gate elements per token: H, or H*D for a per-channel gate.
@@ -813,6 +823,7 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
   cudaSetDevice(p->device);
   cudaDeviceSynchronize();
   release_host_pipe(p);
+  cudaFree(p->d_part_table);
   if (p->owns_device) {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
@@ -889,6 +900,47 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k,
   void* scratch = nullptr;
   VSA_TRY(noalloc_scratch_address(p->device, &scratch));
   return vsa_forward(p, q, k, v, gate, out, scratch, VSA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+vsa_status vsa_forward_parts(vsa_plan p, const vsa_seq_parts* parts, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  VSA_TRY(check_plan(p));
+  if (parts == nullptr) return fail(VSA_ERR_INVALID_ARG, "parts is NULL");
+  const int n = parts->nparts;
+  if (n < 1 || n > VSA_MAX_PARTS) return fail(VSA_ERR_INVALID_ARG, "nparts must lie in [1, VSA_MAX_PARTS]");
+  if (parts->tokens_per_part < 1 || parts->tokens_per_part * n != p->r.L)
+    return fail(VSA_ERR_SHAPE, "nparts * tokens_per_part must equal the sequence length " + std::to_string(p->r.L));
+  if (parts->head_offset < 0 || parts->head_offset + p->H > parts->heads_total)
+    return fail(VSA_ERR_SHAPE, "head_offset + the plan's heads must not exceed heads_total");
+  if (p->seq_tiles) return fail(VSA_ERR_UNSUPPORTED, "sequence parts need a plan without seq_tiles");
+  if (parts->q == nullptr || parts->k == nullptr || parts->v == nullptr || parts->gate == nullptr || parts->out == nullptr)
+    return fail(VSA_ERR_INVALID_ARG, "a pointer array is NULL");
+  for (int i = 0; i < n; ++i)
+    VSA_TRY(check_ptrs({parts->q[i], parts->k[i], parts->v[i], parts->gate[i], parts->out[i]}));
+  VSA_TRY(check_ptrs({workspace}));
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < p->ws.total)
+    return fail(VSA_ERR_WORKSPACE, "workspace holds " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                       std::to_string(p->ws.total));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->d_part_table == nullptr)
+    VSA_CUDA_TRY(cudaMalloc(reinterpret_cast<void**>(&p->d_part_table), 5 * VSA_MAX_PARTS * sizeof(void*)));
+  // table layout: operand-major, nparts entries each (q, k, v, gate, out)
+  p->part_table.assign(5 * static_cast<size_t>(n), nullptr);
+  for (int i = 0; i < n; ++i) {
+    p->part_table[0 * n + i] = parts->q[i];
+    p->part_table[1 * n + i] = parts->k[i];
+    p->part_table[2 * n + i] = parts->v[i];
+    p->part_table[3 * n + i] = parts->gate[i];
+    p->part_table[4 * n + i] = parts->out[i];
+  }
+  VSA_CUDA_TRY(cudaMemcpyAsync(p->d_part_table, p->part_table.data(), p->part_table.size() * sizeof(void*),
+                               cudaMemcpyHostToDevice, s));
+  const vsa::PartIO io{p->d_part_table, n, parts->tokens_per_part, parts->heads_total, parts->head_offset};
+  const int gate_ld = p->gate_pc ? parts->heads_total * p->D : parts->heads_total;
+  return forward_impl(p, parts->q[0], parts->k[0], parts->v[0], parts->gate[0], gate_ld, parts->out[0],
+                      static_cast<uint8_t*>(workspace), s, &io);
 }
 
 vsa_status vsa_forward_host_workspace(vsa_plan p, int32_t head_chunk, size_t* bytes) {

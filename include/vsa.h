@@ -214,6 +214,42 @@ vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                        const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
                        void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* ---- the whole forward over sequence parts (sequence parallelism) ---------
+ * The forward of vsa_forward for this plan's H heads, when the sequence-order
+ * tensors are split by token into `nparts` parts, as a sequence-parallel
+ * (Ulysses) layout has them: part p holds tokens [p*Ls, (p+1)*Ls) of q, k, v
+ * and gate, and receives those tokens of out.  Each part is a [B, Ls, Htot, D]
+ * tensor ([B, Ls, Htot] or [B, Ls, Htot*D] for the gate), and this call reads
+ * and writes heads [head_offset, head_offset + H) of it.  Parts may be peer
+ * mappings of other GPUs' memory (NVLink): then the seq->head exchange happens
+ * inside the gather kernel's loads and the head->seq exchange inside the
+ * attention epilogue's stores, with no separate all-to-all.  Passage: "FastH3
+ * NVFP4 on RTX PRO 6000 (sm_120)", section "What was tried" (Ulysses sequence
+ * parallelism: all-to-all of q/k/v/gate to heads and of the output back).
+ *  - Requires nparts * tokens_per_part == L, head_offset + H <= heads_total,
+ *    a plan without seq_tiles, and 16-byte aligned pointers.
+ *  - The caller orders the call after the parts' producers (on every GPU
+ *    whose memory a part lives in) and consumers of out after the call, e.g.
+ *    with a barrier on each side; nothing inside the call waits on another
+ *    GPU.  Calls with one plan must not overlap.
+ *  - The all-zero-gate check is not run (the compression branch is kept).
+ * Errors: VSA_ERR_INVALID_ARG, VSA_ERR_SHAPE, VSA_ERR_UNSUPPORTED,
+ * VSA_ERR_WORKSPACE, VSA_ERR_CUDA. */
+#define VSA_MAX_PARTS 64
+typedef struct vsa_seq_parts {
+  int32_t nparts;              /* 1..VSA_MAX_PARTS */
+  int64_t tokens_per_part;     /* Ls */
+  int32_t heads_total;         /* Htot of the parts' layout */
+  int32_t head_offset;         /* first of this plan's heads within Htot */
+  const vsa_bf16* const* q;    /* nparts device pointers each (local or peer-mapped) */
+  const vsa_bf16* const* k;
+  const vsa_bf16* const* v;
+  const vsa_bf16* const* gate;
+  vsa_bf16* const* out;
+} vsa_seq_parts;
+vsa_status vsa_forward_parts(vsa_plan p, const vsa_seq_parts* parts, void* workspace_dev,
+                             size_t workspace_bytes, void* stream);
+
 /* ---- the whole forward with inputs and output in host memory ---------------
  * The forward of vsa_forward for q, k, v [B, L, H, D], gate [B, L, H] (or [B, L, H*D]) and out
  * [B, L, H, D] that live in HOST memory (bf16, sequence order).  No
