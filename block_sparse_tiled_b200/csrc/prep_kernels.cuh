@@ -54,7 +54,7 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 // loads/stores (each 256-byte token row is read by 16 consecutive threads),
 // keeps the three tiles in shared memory and, if asked, pools them there.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kParts>
 __global__ void __launch_bounds__(384) gather_pool_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     uint16_t* __restrict__ q_t, uint16_t* __restrict__ k_t, uint16_t* __restrict__ v_t,
@@ -86,9 +86,13 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     const int32_t tok = tok_s[r];
     val[u] = make_uint4(0u, 0u, 0u, 0u);
     if (tok >= 0) {
-      int64_t lt;
-      const uint16_t* base = part_base(io, tsr, src, tok, &lt);
-      val[u] = __ldg(reinterpret_cast<const uint4*>(base + ((static_cast<int64_t>(b) * io.Ls + lt) * io.Htot + io.h0 + h) * D) + c);
+      if constexpr (kParts) {  // the token's part, and heads h0 + h of its Htot
+        int64_t lt;
+        const uint16_t* base = part_base(io, tsr, src, tok, &lt);
+        val[u] = __ldg(reinterpret_cast<const uint4*>(base + ((static_cast<int64_t>(b) * io.Ls + lt) * io.Htot + io.h0 + h) * D) + c);
+      } else {
+        val[u] = __ldg(reinterpret_cast<const uint4*>(src + ((static_cast<int64_t>(b) * L + tok) * H + h) * D) + c);
+      }
     }
   }
   // q_t == NULL: pooling only (the attention then reads sequence order itself)

@@ -440,9 +440,15 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   auto* vo = static_cast<uint16_t*>(vt);
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
-    VSA_TRY(allow_smem(vsa::gather_pool_kernel<D>, smem));
-    vsa::gather_pool_kernel<D><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                       p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
+    if (pio.table != nullptr) {
+      VSA_TRY(allow_smem(vsa::gather_pool_kernel<D, true>, smem));
+      vsa::gather_pool_kernel<D, true><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
+                                                               p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
+    } else {
+      VSA_TRY(allow_smem(vsa::gather_pool_kernel<D, false>, smem));
+      vsa::gather_pool_kernel<D, false><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
+                                                                p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
+    }
     return VSA_OK;
   }));
   return launch_check("gather_pool");
