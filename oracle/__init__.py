@@ -57,8 +57,15 @@ def _load():
         lib.vsa_oracle_scores.argtypes = [P, P, i32, i32, i32, f32, P]
         lib.vsa_oracle_select.argtypes = [P, i32, i32, i32, i32, P]
         lib.vsa_oracle_compress.argtypes = [P, P, i32, i32, i32, P]
-        lib.vsa_oracle_fine.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
-        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, i32, P, P]
+        lib.vsa_oracle_fine.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
+        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64,
+                                              i32, P, P]
+        lib.vsa_oracle_e4m3_value.argtypes = [i32]
+        lib.vsa_oracle_e4m3_value.restype = f64
+        lib.vsa_oracle_e4m3_round.argtypes = [f32]
+        lib.vsa_oracle_e4m3_round.restype = i32
+        lib.vsa_oracle_e4m3_round_array.argtypes = [P, i64, P]
+        lib.vsa_oracle_quant_e4m3.argtypes = [P, i64, i32, P, P]
         lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P]
         lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, P, P, P, P]
         _lib = lib
@@ -155,32 +162,80 @@ def compress(S: np.ndarray, pv: np.ndarray) -> np.ndarray:
     return out
 
 
-def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None) -> np.ndarray:
-    """List formulation of the fine branch -> o_f [B, L, H, D] float64 (NaN where not computed)."""
+def _qk8_args(qk8, shape):
+    """(q codes, q scales, k codes, k scales) for the 8-bit variant (R13), or four NULLs."""
+    if qk8 is None:
+        return (None, None, None, None)
+    qc, qs, kc, ks = qk8
+    B, L, H, D = shape
+    qc, kc = (_c(t, np.uint8) for t in (qc, kc))
+    qs, ks = (_c(t, np.float32) for t in (qs, ks))
+    assert qc.shape == kc.shape == (B, L, H, D) and qs.shape == ks.shape == (B, L, H)
+    return (qc, qs, kc, ks)
+
+
+def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=None) -> np.ndarray:
+    """List formulation of the fine branch -> o_f [B, L, H, D] float64 (NaN where not computed).
+    qk8 = (q codes, q scales, k codes, k scales) from quant_e4m3: the logits use those instead of q, k."""
     q, k, v = (_c(t, np.uint16) for t in (q, k, v))
     B, L, H, D = q.shape
     idx = _c(idx, np.int32)
     if todo is not None:
         todo = _c(todo.astype(np.uint8), np.uint8)
+    q8 = _qk8_args(qk8, q.shape)
     out = np.full((B, L, H, D), np.nan, np.float64)
-    _load().vsa_oracle_fine(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+    _load().vsa_oracle_fine(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
                             _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(todo), _p(out))
     return out
 
 
-def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items) -> np.ndarray:
+def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items, qk8=None) -> np.ndarray:
     """Fine branch of the listed query tiles only.  items: int64 array of
     (b*H + h)*n_t + i.  Returns [n_items, 64, D] float64 in tile row order
-    (pad rows 0)."""
+    (pad rows 0).  qk8: as for fine()."""
     q, k, v = (_c(t, np.uint16) for t in (q, k, v))
     B, L, H, D = q.shape
     idx = _c(idx, np.int32)
     items = _c(np.asarray(items, np.int64), np.int64)
+    q8 = _qk8_args(qk8, q.shape)
     out = np.zeros((len(items), 64, D), np.float64)
-    _load().vsa_oracle_fine_tiles(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+    _load().vsa_oracle_fine_tiles(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles,
+                                  geo.n_prefix, topk,
                                   _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), len(items),
                                   _p(items), _p(out))
     return out
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """float64 values of E4M3 codes (uint8 array), from the format's definition (R13)."""
+    lib = _load()
+    table = np.array([lib.vsa_oracle_e4m3_value(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, np.uint8)]
+
+
+def e4m3_round(y) -> np.ndarray:
+    """E4M3 codes of binary32 values: nearest, ties to the even code, saturating at +-448."""
+    y = _c(np.asarray(y, np.float32), np.float32)
+    out = np.empty(y.shape, np.uint8)
+    _load().vsa_oracle_e4m3_round_array(_p(y), y.size, _p(out))
+    return out
+
+
+def quant_e4m3(x_bf16: np.ndarray):
+    """The 8-bit Q/K quantiser (R13): x [..., D] bf16 bits -> (codes [..., D] uint8, scale [...] float32),
+    one scale per row of D (per batch, token and head)."""
+    x = _c(x_bf16, np.uint16)
+    D = x.shape[-1]
+    n = x.size // D
+    code = np.empty(x.shape, np.uint8)
+    scale = np.empty(x.shape[:-1], np.float32)
+    _load().vsa_oracle_quant_e4m3(_p(x), n, D, _p(code), _p(scale))
+    return code, scale
+
+
+def dequant_e4m3(code, scale) -> np.ndarray:
+    """code * scale in float64 (exact: a 4-bit significand times a binary32 scale)."""
+    return e4m3_value(code) * np.asarray(scale, np.float64)[..., None]
 
 
 def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarray:
@@ -269,13 +324,14 @@ class ForwardResult:
     seconds: float
 
 
-def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None) -> ForwardResult:
+def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=False) -> ForwardResult:
     """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H] (or
     [B,L,H*D], one per channel).
 
     Selection (pool, scores, top-k) always runs in full; the fine branch and
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
-    None = all)."""
+    None = all).  qk8: the fine branch's logits use 8-bit Q/K (R13); the
+    selection still reads the bf16 inputs."""
     t0 = time.perf_counter()
     geo = geometry(segments, grid)
     D = q.shape[-1]
@@ -286,6 +342,7 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None) -> F
     S = scores(pq, pk, scale)
     idx = select(S, geo.n_prefix, kc)
     o_c = compress(S, pv)
-    o_f = fine(q, k, v, geo, idx, kc, scale, todo)
+    q8 = (*quant_e4m3(q), *quant_e4m3(k)) if qk8 else None
+    o_f = fine(q, k, v, geo, idx, kc, scale, todo, qk8=q8)
     out = output(o_f, o_c, gate, geo, todo)
     return ForwardResult(geo, kc, scale, pq, pk, pv, S, idx, o_c, o_f, out, time.perf_counter() - t0)

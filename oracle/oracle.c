@@ -41,6 +41,16 @@
  *      included -- parity unpinned;
  *   R11 the gate is one scalar per (batch, token, head).
  *   R12 the per-channel variant: one gate per (batch, token, channel h*D + d), [B, L, H*D].
+ *   R13 the 8-bit Q/K variant ("FastH3 OmniRef inference", section "The Blackwell stack" and
+ *      "Fallbacks": query/key rounding to 8 bits with bf16 P.V, per-token FP8 Q/K; the
+ *      multi-GPU notes of "FastH3 NVFP4 on RTX PRO 6000": one scale per token and head):
+ *      8 bits = OCP FP8 E4M3 ("E4M3FN": bias 7, no infinities, largest 448); one binary32
+ *      scale per (batch, token, head), s = amax / 448 in binary32 where amax is the largest
+ *      |x_d| of the token's head row; code_d = E4M3 round-to-nearest-even of the binary32
+ *      quotient x_d / s, saturating at +-448; a row with amax = 0 has s = 0 and all codes
+ *      +0.  The dequantised value code * s replaces Q and K in the fine branch's logits
+ *      only: selection, compression and P.V keep the bf16 inputs.  The variant covers
+ *      every query tile.
  *
  * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
  * order above; fine attention, compression and the output in binary64.
@@ -67,6 +77,99 @@ static float bf16_to_float(uint16_t h) {
 }
 
 static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+/* ------------------------------------------------------------------ */
+/* O0 8-bit Q/K: E4M3 codes with one scale per (batch, token, head)   */
+/* (reading R13)                                                       */
+/* ------------------------------------------------------------------ */
+
+/* Value of an E4M3 code: bit 7 sign, bits 6..3 exponent field e (bias 7),
+ * bits 2..0 mantissa m.  e = 0: subnormal, m/8 * 2^-6; otherwise
+ * (1 + m/8) * 2^(e-7).  e = 15 with m = 7 is NaN; there is no infinity. */
+double vsa_oracle_e4m3_value(int code) {
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* E4M3 code nearest to y; a tie goes to the even code (even mantissa); a
+ * magnitude at or above 448 (the largest finite value, code 0x7E) gives
+ * +-448.  The sign bit is the sign of y, so -0 and negative values that
+ * round to zero give 0x80. */
+int vsa_oracle_e4m3_round(float y) {
+    int sign = signbit(y) ? 0x80 : 0;
+    double a = fabs((double)y);
+    int lo = 0, hi = 126; /* codes 0..126 hold the finite magnitudes in increasing order */
+    double dl, dh;
+    if (a >= 448.0) return sign | 126;
+    /* largest code lo with value(lo) <= a (binary search over 0..126) */
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (vsa_oracle_e4m3_value(mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    dl = a - vsa_oracle_e4m3_value(lo);
+    if (dl == 0.0) return sign | lo;
+    dh = vsa_oracle_e4m3_value(lo + 1) - a;
+    if (dl < dh) return sign | lo;
+    if (dh < dl) return sign | (lo + 1);
+    return sign | ((lo & 1) ? lo + 1 : lo);
+}
+
+void vsa_oracle_e4m3_round_array(const float *y, int64_t n, uint8_t *code) {
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n; ++e) code[e] = (uint8_t)vsa_oracle_e4m3_round(y[e]);
+}
+
+/* Per-row quantisation of x [N, D] (bf16 bits), one row = one (batch, token,
+ * head): amax = max_d |x_d|; s = amax / 448 (binary32 division); code_d =
+ * e4m3_round(x_d / s) (binary32 division); amax = 0 gives s = 0 and codes +0. */
+void vsa_oracle_quant_e4m3(const uint16_t *x, int64_t N, int D, uint8_t *code, float *scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < N; ++r) {
+        const uint16_t *xr = x + r * D;
+        float amax = 0.0f, s;
+        for (int d = 0; d < D; ++d) {
+            float a = fabsf(bf16_to_float(xr[d]));
+            if (a > amax) amax = a;
+        }
+        s = amax / 448.0f;
+        scale[r] = s;
+        for (int d = 0; d < D; ++d) {
+            float q = (amax == 0.0f) ? 0.0f : bf16_to_float(xr[d]) / s;
+            code[r * D + d] = (uint8_t)((amax == 0.0f) ? 0 : vsa_oracle_e4m3_round(q));
+        }
+    }
+}
+
+/* One operand of the fine branch's logits (Q or K), [B, L, H, D]: bf16 bits,
+ * or (code != NULL) E4M3 codes with one binary32 scale per row of D. */
+typedef struct {
+    const uint16_t *bf16;
+    const uint8_t *code;
+    const float *scale;
+} qk_operand;
+
+static double e4m3_table[256];
+static int e4m3_table_ready = 0;
+
+static double qk_value(const qk_operand *x, int64_t row, int D, int d) {
+    if (x->code) return e4m3_table[x->code[row * D + d]] * (double)x->scale[row];
+    return (double)bf16_to_float(x->bf16[row * D + d]);
+}
+
+static void qk_tables(void) {
+    if (e4m3_table_ready) return;
+    for (int c = 0; c < 256; ++c) e4m3_table[c] = vsa_oracle_e4m3_value(c);
+    e4m3_table_ready = 1;
+}
 
 /* ------------------------------------------------------------------ */
 /* O1 geometry                                                         */
@@ -279,7 +382,7 @@ static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t
  *   logit_c = scale * <q_r, k_c> over the valid key rows c of its key set,
  *   o_f[r] = sum_c softmax(logit)_c * v_c,
  * written to rows[r * D + d] in tile row order (pad rows left untouched). */
-static void fine_one_tile(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int b, int h, int i,
+static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint16_t *v, int b, int h, int i,
                           int64_t L, int H, int D, int n_t, int P, int k, const int32_t *tile_token,
                           const int32_t *tile_valid, const int32_t *idx, double scale, double *rows) {
     int V = n_t - P;
@@ -297,13 +400,13 @@ static void fine_one_tile(const uint16_t *q, const uint16_t *kk, const uint16_t 
 
     for (int r = 0; r < tile_valid[i]; ++r) {
         int64_t qt = tile_token[(int64_t)i * TILE + r];
-        const uint16_t *qr = q + (((int64_t)b * L + qt) * H + h) * D;
+        int64_t qrow = ((int64_t)b * L + qt) * H + h;
         double m = -INFINITY;
         for (int64_t c = 0; c < nrows; ++c) {
-            const uint16_t *kc = kk + (((int64_t)b * L + ktok[c]) * H + h) * D;
+            int64_t krow = ((int64_t)b * L + ktok[c]) * H + h;
             double dot = 0.0;
             for (int d = 0; d < D; ++d)
-                dot += (double)bf16_to_float(qr[d]) * (double)bf16_to_float(kc[d]);
+                dot += qk_value(q, qrow, D, d) * qk_value(kk, krow, D, d);
             logit[c] = scale * dot;
             if (logit[c] > m) m = logit[c];
         }
@@ -327,11 +430,16 @@ static void fine_one_tile(const uint16_t *q, const uint16_t *kk, const uint16_t 
 
 /* o_f[b, tok, h, :] for every valid query token tok of every (b, h, i) with
  * todo[(b*H + h)*n_t + i] != 0 (todo == NULL: all).
- * q, k, v: [B, L, H, D] bf16 bits; idx: [B, H, V, k] global tile indices. */
-void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B, int64_t L,
+ * q, k, v: [B, L, H, D] bf16 bits; idx: [B, H, V, k] global tile indices.
+ * q8/qs and k8/ks (both NULL, or both set): the 8-bit variant (R13), E4M3
+ * codes [B, L, H, D] and scales [B, L, H] used for the logits instead of q, k. */
+void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
+                     const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
                      int H, int D, int n_t, int P, int k, const int32_t *tile_token,
                      const int32_t *tile_valid, const int32_t *idx, double scale,
                      const uint8_t *todo, double *o_f) {
+    qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
+    qk_tables();
 #pragma omp parallel for collapse(3) schedule(dynamic, 1)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h)
@@ -339,7 +447,7 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, i
                 int64_t bhi = ((int64_t)b * H + h) * n_t + i;
                 if (todo && !todo[bhi]) continue;
                 double *rows = (double *)malloc(sizeof(double) * (size_t)TILE * (size_t)D);
-                fine_one_tile(q, kk, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale,
+                fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale,
                               rows);
                 for (int r = 0; r < tile_valid[i]; ++r) {
                     int64_t tok = tile_token[(int64_t)i * TILE + r];
@@ -352,11 +460,14 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, i
 
 /* The fine branch of selected query tiles only: items[n] = (b*H + h)*n_t + i;
  * out[n, r, :] for the tile's rows r in tile order (pad rows set to 0). */
-void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B, int64_t L,
+void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
+                           const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
                            int H, int D, int n_t, int P, int k, const int32_t *tile_token,
                            const int32_t *tile_valid, const int32_t *idx, double scale, int n_items,
                            const int64_t *items, double *out) {
+    qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
     (void)B;
+    qk_tables();
 #pragma omp parallel for schedule(dynamic, 1)
     for (int n = 0; n < n_items; ++n) {
         int64_t bhi = items[n];
@@ -365,7 +476,7 @@ void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t
         int h = (int)(bh % H), b = (int)(bh / H);
         double *rows = out + (int64_t)n * TILE * D;
         for (int64_t e = 0; e < (int64_t)TILE * D; ++e) rows[e] = 0.0;
-        fine_one_tile(q, kk, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale, rows);
+        fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale, rows);
     }
 }
 
