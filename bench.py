@@ -376,9 +376,10 @@ def run_vsa(args, w, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_ab_seq_tiles(args, w):
-    """Side measurement (not the contract line): the whole vsa_forward with tile-order copies against a
-    seq_tiles plan, alternating the two plans; prints one JSON line with the medians and workspaces."""
+def run_ab(args, w, variants):
+    """Side measurement (not the contract line): the whole vsa_forward under two plan variants of the
+    same workload, alternating them over two rounds; prints one JSON line with the median forward times
+    and the workspace sizes.  variants: name -> extra vsa_plan_tiles arguments."""
     import torch
     import synth
     import block_sparse_tiled_b200 as vsa
@@ -387,10 +388,9 @@ def run_ab_seq_tiles(args, w):
     x = synth.make_inputs(w, seed=0, device="cuda")
     res = {"workload": w.name, "steps": args.steps, "warmup": args.warmup, "forward_ms": {}, "workspace_bytes": {}}
     for rnd in range(2):
-        for seq in (False, True):
-            key = "seq_tiles" if seq else "tile_order"
+        for key, extra in variants.items():
             plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments,
-                                      grid=w.grid, sparsity=w.sparsity, seq_tiles=seq)
+                                      grid=w.grid, sparsity=w.sparsity, **extra)
             ws = vsa.alloc_workspace(plan)
             out = torch.empty_like(x["q"])
             for _ in range(args.warmup):
@@ -426,6 +426,8 @@ def main():
     ap.add_argument("--ref-every", type=int, default=16)
     ap.add_argument("--ab-seq-tiles", action="store_true",
                     help="side measurement: vsa_forward with tile-order copies against a seq_tiles plan")
+    ap.add_argument("--ab-qk-fp8", action="store_true",
+                    help="side measurement: vsa_forward with bf16 Q/K logits against 8-bit (E4M3) Q/K")
     args = ap.parse_args()
     import synth
 
@@ -433,7 +435,10 @@ def main():
     if args.sparsity is not None:
         w = dataclasses.replace(w, sparsity=args.sparsity, name=f"{w.name}@s{args.sparsity}")
     if args.ab_seq_tiles:
-        run_ab_seq_tiles(args, w)
+        run_ab(args, w, {"tile_order": {}, "seq_tiles": {"seq_tiles": True}})
+        return
+    if args.ab_qk_fp8:
+        run_ab(args, w, {"qk_bf16": {}, "qk_fp8": {"qk_fp8": True}})
         return
     world, rank, local = dist_setup(args)
     try:

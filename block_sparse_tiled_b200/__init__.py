@@ -54,7 +54,7 @@ class Geometry(ctypes.Structure):
         ("video_tag", ctypes.c_int32),
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-        ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32),
+        ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32), ("qk_fp8", ctypes.c_int32),
     ]
 
 
@@ -80,7 +80,8 @@ class PlanDims(ctypes.Structure):
 
 
 class WorkspaceLayout(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_size_t) for n in ("q_t", "k_t", "v_t", "pq", "pk", "pv", "scores", "idx", "o_c", "total")]
+    _fields_ = [(n, ctypes.c_size_t)
+                for n in ("q_t", "k_t", "v_t", "q_s", "k_s", "pq", "pk", "pv", "scores", "idx", "o_c", "total")]
 
 
 _lib = None
@@ -150,7 +151,7 @@ def _ptr(t, dtype=None, name="tensor"):
 
 
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False):
+                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False, qk_fp8=False):
     """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers)."""
     g = Geometry()
     g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
@@ -174,6 +175,7 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.softmax_scale = float(softmax_scale)
     g.gate_per_channel = int(bool(gate_per_channel))
     g.seq_tiles = int(bool(seq_tiles))
+    g.qk_fp8 = int(bool(qk_fp8))
     return g, keep
 
 
@@ -242,10 +244,11 @@ class Plan:
 
 def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
                    token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False,
-                   stream=None) -> Plan:
+                   qk_fp8=False, stream=None) -> Plan:
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
-              tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles))
+              tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles),
+              qk_fp8=bool(qk_fp8))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
     _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")
@@ -429,11 +432,13 @@ def device_status(plan, stream=None):
 
 def workspace_views(plan, workspace):
     """Typed views of vsa_forward's intermediates inside ``workspace`` (no tile-order views for a plan
-    with seq_tiles, whose workspace holds none)."""
+    with seq_tiles, whose workspace holds none).  With qk_fp8, q_t and k_t are the E4M3 codes
+    [B, H, n_t, 64, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, 64]."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
     seq = bool(g.get("seq_tiles", False))
+    f8 = bool(g.get("qk_fp8", False))
 
     def view(off, n, dtype, shape):
         nbytes = n * torch.tensor([], dtype=dtype).element_size()
@@ -442,10 +447,18 @@ def workspace_views(plan, workspace):
     def tiles(name):
         return None if seq else view(lay[name], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D))
 
+    def codes(name):
+        return view(lay[name], B * H * n_t * 64 * 128, torch.uint8, (B, H, n_t, 64, 128))
+
+    def row_scales(name):
+        return view(lay[name], B * H * n_t * 64, torch.float32, (B, H, n_t, 64)) if f8 else None
+
     return {
-        "q_t": tiles("q_t"),
-        "k_t": tiles("k_t"),
+        "q_t": codes("q_t") if f8 else tiles("q_t"),
+        "k_t": codes("k_t") if f8 else tiles("k_t"),
         "v_t": tiles("v_t"),
+        "q_s": row_scales("q_s"),
+        "k_s": row_scales("k_s"),
         "pq": view(lay["pq"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pk": view(lay["pk"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pv": view(lay["pv"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),

@@ -115,6 +115,8 @@ struct AttnArgs {
   const uint64_t* key_mask;  // [n_t]: bit r set when row r of the tile as loaded is a key (a token)
   const int32_t* coord;      // [n_t][4] TMA coordinates of a tile read from sequence order
   PartIO io;                 // where gate and out live (one tensor, or sequence parts, possibly on peers)
+  const float* q_scale;      // 8-bit Q/K only: [B, H, n_t, 64] scale of each query row (tile order)
+  const float* k_scale;      // 8-bit Q/K only: [B, H, n_t, 64] scale of each key row
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_t
 };
@@ -127,27 +129,33 @@ struct SeqMaps {
   CUtensorMap video[3][kSeqMaxBatch];
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 struct AttnLayout {
   // 128-byte swizzle atoms along D.  D = 96 uses two, the second half-empty: TMA fills columns 96..127
   // with zeros, the S^T product stops after D/16 K-steps and O^T rows 96..127 are never stored.
+  // kF8: Q and K are 8-bit codes, one 128-byte atom per row for any D (the S^T product runs D/32
+  // K-steps of 32 bytes); V stays bf16.
   static constexpr int kHalves = (D + 63) / 64;
-  static constexpr int kQBytes = 64 * 64 * kHalves * 2;    // one query tile
-  static constexpr int kKVBytes = 128 * 64 * kHalves * 2;  // 128 keys of K (or of V)
+  static constexpr int kQBytes = kF8 ? 64 * 128 : 64 * 64 * kHalves * 2;    // one query tile
+  static constexpr int kKVBytes = 128 * 64 * kHalves * 2;                  // 128 keys of V (bf16)
+  static constexpr int kKBytes = kF8 ? 128 * 128 : kKVBytes;               // 128 keys of K
   static constexpr int kHalfBytes = 128 * 128;  // one 64-column half of a 128-row block
   static constexpr int kPBytes = 128 * 64 * 2;  // P^T of one block
   static constexpr int kQBufs = 1;
-  static constexpr int kKStages = 2;
+  static constexpr int kKStages = kF8 ? 4 : 2;
   static constexpr int kVStages = 3;
   static constexpr int kPBufs = 2;  // P^T buffers in shared memory
   static constexpr int kRing = 8;  // claimed items in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
+  // kF8: the query scales of the two items in flight in the softmax (64 floats each, times the
+  // softmax scale * log2 e)
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQBufs * kQBytes;
-  static constexpr int oV = oK + kKStages * kKVBytes;
+  static constexpr int oV = oK + kKStages * kKBytes;
   static constexpr int oP = oV + kVStages * kKVBytes;
   static constexpr int oZ = oP + kPBufs * kPBytes;
-  static constexpr int oBar = oZ + kZeroBytes;
+  static constexpr int oQS = oZ + kZeroBytes;
+  static constexpr int oBar = oQS + (kF8 ? 512 : 0);
   // barrier indices (8 bytes each)
   static constexpr int bQFull = 0, bQEmpty = bQFull + kQBufs;
   static constexpr int bKFull = bQEmpty + kQBufs, bKEmpty = bKFull + kKStages;
@@ -205,14 +213,19 @@ __device__ __forceinline__ void warp_sum_scatter32(float* v, int lane) {
 // kSeq = false: Q/K/V come from tile-order copies through 2-D maps (tm_q/k/v).  kSeq = true: they come
 // straight from the sequence-order tensors through `seq`, one box per tile (a 64-token prefix run or a
 // 4x4x4 video cube); rows outside the tile are masked by key_mask and not stored.
-template <int D, bool kSeq>
+// kF8 (tile-order copies only): Q and K are E4M3 codes with one scale per row (a.q_scale, a.k_scale).
+// S^T is then an 8-bit product (kind::f8f6f4, K = 32 per instruction: half the instructions of bf16)
+// of the codes; the softmax multiplies each logit by its key row's scale and its query column's scale
+// before the exponent.  P.V is unchanged (bf16).
+template <int D, bool kSeq, bool kF8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     vsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, const __grid_constant__ SeqMaps seq) {
-  using Ly = AttnLayout<D>;
-  constexpr int kQKSteps = D / 16;
+  static_assert(!(kSeq && kF8), "8-bit Q/K reads tile-order copies");
+  using Ly = AttnLayout<D, kF8>;
+  constexpr int kQKSteps = kF8 ? (D + 31) / 32 : D / 16;
   constexpr int kPVSteps = 128 / 16;
-  constexpr uint32_t kIdescS = umma_idesc_bf16(128, 64, 0, 0);
+  constexpr uint32_t kIdescS = kF8 ? umma_idesc_e4m3(128, 64) : umma_idesc_bf16(128, 64, 0, 0);
   constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 64, 1, 1);
 
   extern __shared__ uint8_t smem_raw[];
@@ -366,7 +379,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (ok) mbar_arrive_expect_tx(&bars[Ly::bQFull + qb], Ly::kQBytes);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok && lane < Ly::kHalves) {
+        if (ok && lane < (kF8 ? 1 : Ly::kHalves)) {
           void* dst = sm + Ly::oQ + qb * Ly::kQBytes + lane * 8192;
           if constexpr (kSeq) {
             const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + i);
@@ -395,19 +408,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int kb = kb_raw < 0 ? ka : kb_raw;  // an odd list repeats its last tile; the softmax masks it
           const int st = g % nstages;
           const uint32_t u = g / nstages;
+          // bytes of one stage: K (8-bit: one 8 KB box per tile), or V plus, with 8-bit Q/K, the key scales
+          const int stage_bytes = is_k ? Ly::kKBytes : Ly::kKVBytes;
+          const int halves = (is_k && kF8) ? 1 : Ly::kHalves;
           if (lane == 0) {
             ROLE_MARK(3);
             ok = mbar_wait(&bars[b_empty + st], (u & 1) ^ 1, ctl, is_k ? 2 : 3);
             ROLE_MARK(1);
-            if (ok) mbar_arrive_expect_tx(&bars[b_full + st], Ly::kKVBytes);
+            if (ok) mbar_arrive_expect_tx(&bars[b_full + st], stage_bytes);
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          // lanes [0, 2*kHalves) issue one 8 KB box each: (half, tile a|b)
-          if (lane < 2 * Ly::kHalves) {
+          // lanes [0, 2*halves) issue one 8 KB box each: (half, tile a|b)
+          if (lane < 2 * halves) {
             const int hh = lane >> 1, second = lane & 1;
             const int t = second ? kb : ka;
-            void* dst = ring + st * Ly::kKVBytes + hh * Ly::kHalfBytes + second * 8192;
+            void* dst = ring + st * stage_bytes + hh * Ly::kHalfBytes + second * 8192;
             if constexpr (kSeq) {
               const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + t);
               const int bb = static_cast<int>(bh / a.H), head = static_cast<int>(bh - static_cast<int64_t>(bb) * a.H);
@@ -472,12 +488,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sm + Ly::oK + kst * Ly::kKVBytes);
+          const uint32_t kbase = smem_u32(sm + Ly::oK + kst * Ly::kKBytes);
 #pragma unroll
           for (int kk = 0; kk < kQKSteps; ++kk) {
+            // 32 bytes of every row per step: 16 bf16 or 32 8-bit elements
             const uint64_t ad = umma_desc_sw128(kbase + (kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = umma_desc_sw128(qbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-            umma_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            if constexpr (kF8)
+              umma_ss_f8(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            else
+              umma_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
           }
           umma_commit(&bars[Ly::bKEmpty + kst]);
           umma_commit(&bars[Ly::bSFull + sb]);
@@ -552,20 +572,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float* delta_g = delta_s + c0;
     float* red_g = red_s + grp * 4 * CG;
     const float cl = a.scale_log2;
+    // 8-bit Q/K: query scales (times cl) of the group's columns, one buffer per item parity (at a fixed
+    // offset from m_g); the group's first warp fills the buffer before the item's first barrier
+    constexpr int kQscFromM = (Ly::oQS - Ly::oM) / 4;
     uint32_t g = 0;
     int it = 0;
     ROLE_TIMER_START();
     for (;; ++it) {
       int w = (lane == 0) ? ring_take(it, 28) : 0;
       w = __shfl_sync(0xffffffffu, w, 0);
+      if constexpr (kF8) {
+        if (qd == 0 && lane < CG && w >= 0)
+          m_g[kQscFromM + (it & 1) * 64 + lane] = __ldg(a.q_scale + static_cast<int64_t>(w) * 64 + c0 + lane) * cl;
+      }
       if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t);
       const int nk = list_len(i), nb = (nk + 1) / 2;
       const int ob = it & 1;
-      // lane j: the key-mask word of block (n & ~31) + j for this warp's TMEM lane quadrant (rows
-      // 32*qd .. 32*qd + 31 of the block: tile a for qd < 2, tile b otherwise)
+      const float* qsc_g = m_g + kQscFromM + ob * 64;
+      // lane j: the key-mask word of block n0 + j for this warp's TMEM lane quadrant (rows
+      // 32*qd .. 32*qd + 31 of the block: tile a for qd < 2, tile b otherwise); with 8-bit Q/K also
+      // that tile's row-scale offset (b, h, tile) * 64 (refilled one block ahead).
       uint32_t vcache = 0;
+      int kcache = 0;  // B*H*n_t*64 < 2^31 (checked when the plan is made)
+      auto refill = [&](int n0) {
+        const int nn = n0 + lane;
+        vcache = 0;
+        if (nn < nb) {
+          const int t = 2 * nn + (qd >> 1);
+          const int kt = (t < nk) ? key_tile(bh, i, t) : -1;
+          const uint64_t m = (kt >= 0) ? __ldg(a.key_mask + kt) : 0ull;
+          vcache = static_cast<uint32_t>(m >> (32 * (qd & 1)));
+          if constexpr (kF8) kcache = static_cast<int>((bh * n_t + max(kt, 0)) * 64);
+        }
+      };
+      // 8-bit Q/K: this lane's key row scale of block n (a missing second tile reads tile 0's, masked)
+      auto key_scale = [&](int n) -> float {
+        return __ldg(a.k_scale + __shfl_sync(0xffffffffu, kcache, n & 31) + (kl & 63));
+      };
+      float ks_next = 1.0f;
+      if constexpr (kF8) {
+        refill(0);
+        ks_next = key_scale(0);
+      }
 
       float l[CG];
 #pragma unroll
@@ -577,17 +627,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int pb = g % Ly::kPBufs;
         const uint32_t pu = g / Ly::kPBufs;
         ROLE_MARK(7);
-        if ((n & 31) == 0) {
-          // key masks of the next 32 blocks (an odd list's last block has no second tile)
-          const int nn = n + lane;
-          vcache = 0;
-          if (nn < nb) {
-            const int t = 2 * nn + (qd >> 1);
-            const uint64_t m = (t < nk) ? __ldg(a.key_mask + key_tile(bh, i, t)) : 0ull;
-            vcache = static_cast<uint32_t>(m >> (32 * (qd & 1)));
-          }
+        uint32_t kmask;
+        float ks = 1.0f;
+        if constexpr (kF8) {
+          // the next block's key scale (and, every 32 blocks, mask words) are fetched one block ahead,
+          // while this block waits and works
+          kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
+          ks = ks_next;
+          if (((n + 1) & 31) == 0 && n + 1 < nb) refill(n + 1);
+          if (n + 1 < nb) ks_next = key_scale(n + 1);
+        } else {
+          if ((n & 31) == 0) refill(n);
+          kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
         }
-        const uint32_t kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
         ROLE_MARK(0);
 
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
@@ -601,8 +653,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Ly::bSEmpty + sb]);
 
-        // x = logit * log2(e) - m  (m = 0 before the first block of the item)
-        if (n == 0) {
+        // x = logit * log2(e) - m  (m = 0 before the first block of the item); with 8-bit Q/K the
+        // logit is the code product times the key and query scales
+        if constexpr (kF8) {
+#pragma unroll
+          for (int j = 0; j < CG; ++j) x[j] *= ks;
+          if (n == 0) {
+#pragma unroll
+            for (int j = 0; j < CG; j += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
+              x[j] *= c4.x;
+              x[j + 1] *= c4.y;
+              x[j + 2] *= c4.z;
+              x[j + 3] *= c4.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < CG; j += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
+              const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
+              x[j] = fmaf(x[j], c4.x, -m4.x);
+              x[j + 1] = fmaf(x[j + 1], c4.y, -m4.y);
+              x[j + 2] = fmaf(x[j + 2], c4.z, -m4.z);
+              x[j + 3] = fmaf(x[j + 3], c4.w, -m4.w);
+            }
+          }
+        } else if (n == 0) {
 #pragma unroll
           for (int j = 0; j < CG; ++j) x[j] *= cl;
         } else {

@@ -6,6 +6,7 @@
 //   score  = fl(fma(pq_{D-1}, pk_{D-1}, ... fma(pq_0, pk_0, +0)) * scale)
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 namespace vsa {
@@ -53,17 +54,29 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 // One CTA per (tile, head, batch) moves the tile of Q, K and V with 16-byte
 // loads/stores (each 256-byte token row is read by 16 consecutive threads),
 // keeps the three tiles in shared memory and, if asked, pools them there.
+//
+// kF8: Q and K are written as 8-bit E4M3 codes instead of bf16 copies, each
+// (token, head) row with its own binary32 scale s = amax / 448: code_d =
+// E4M3(x_d / s), round to nearest even, saturating; amax = 0 gives s = 0 and
+// zero codes.  Code rows are 128 bytes apart whatever D (bytes D..127 are
+// zero); scales are [B, H, n_t, 64] (pad rows 0).  Every row is then handled
+// by one half-warp (16 lanes x 8 elements, lanes past D/8 idle), so its amax
+// is a 16-lane shuffle reduction.  Passages: "FastH3 OmniRef inference",
+// sections "The Blackwell stack" and "Fallbacks" (8-bit Q/K per token with
+// bf16 P.V); "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", multi-GPU notes (one
+// FP8 scale per token and head).
 // ---------------------------------------------------------------------------
-template <int D, bool kParts>
+constexpr int kF8RowBytes = 128;
+
+template <int D, bool kParts, bool kF8>
 __global__ void __launch_bounds__(384) gather_pool_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-    uint16_t* __restrict__ q_t, uint16_t* __restrict__ k_t, uint16_t* __restrict__ v_t,
-    float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
+    void* __restrict__ q_t, void* __restrict__ k_t, uint16_t* __restrict__ v_t, float* __restrict__ q_s,
+    float* __restrict__ k_s, float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
     int n_t, const PartIO io) {
-  constexpr int kChunks = D / 8;                 // 16-byte chunks per row
-  constexpr int kPerTensor = kTile * kChunks;    // chunks per tile of one tensor
-  constexpr int kIters = kPerTensor / 128;       // each of 128 threads per tensor moves kIters chunks
+  constexpr int kChunks = D / 8;                                // 16-byte chunks per row
+  constexpr int kIters = kF8 ? kTile / 8 : kTile * kChunks / 128;  // chunks each thread moves per tensor
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);  // [3][64][D]
   __shared__ int32_t tok_s[kTile];
@@ -76,16 +89,28 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   // threads [128 t, 128 t + 128) move tensor t; all loads are issued before any store
   const int tsr = threadIdx.x >> 7, tl = threadIdx.x & 127;
   const uint16_t* src = (tsr == 0) ? q : (tsr == 1) ? k : v;
-  uint16_t* dst = (tsr == 0) ? q_t : (tsr == 1) ? k_t : v_t;
-  const int64_t dst_base = ((static_cast<int64_t>(b) * H + h) * n_t + tile) * kTile * D;
+  const int64_t tile_row0 = ((static_cast<int64_t>(b) * H + h) * n_t + tile) * kTile;
+  // row and chunk of this thread's u-th chunk (false: an idle lane of an 8-bit row)
+  auto chunk_of = [&](int u, int* r, int* c) -> bool {
+    if constexpr (kF8) {
+      *r = (tl >> 4) + 8 * u;
+      *c = tl & 15;
+      return *c < kChunks;
+    } else {
+      const int e = tl + 128 * u;
+      *r = e / kChunks;
+      *c = e - *r * kChunks;
+      return true;
+    }
+  };
   uint4 val[kIters];
 #pragma unroll
   for (int u = 0; u < kIters; ++u) {
-    const int e = tl + 128 * u;
-    const int r = e / kChunks, c = e - r * kChunks;
+    int r, c;
+    const bool active = chunk_of(u, &r, &c);
     const int32_t tok = tok_s[r];
     val[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (tok >= 0) {
+    if (active && tok >= 0) {
       if constexpr (kParts) {  // the token's part, and heads h0 + h of its Htot
         int64_t lt;
         const uint16_t* base = part_base(io, tsr, src, tok, &lt);
@@ -97,11 +122,43 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   }
   // q_t == NULL: pooling only (the attention then reads sequence order itself)
   const bool write_tiles = (q_t != nullptr);
+  const bool codes = kF8 && tsr < 2;
 #pragma unroll
   for (int u = 0; u < kIters; ++u) {
-    const int e = tl + 128 * u;
-    if (write_tiles) reinterpret_cast<uint4*>(dst + dst_base)[e] = val[u];
-    if (pool) reinterpret_cast<uint4*>(tiles + tsr * kTile * D)[e] = val[u];
+    int r, c;
+    const bool active = chunk_of(u, &r, &c);
+    if (active && pool) reinterpret_cast<uint4*>(tiles + tsr * kTile * D)[r * kChunks + c] = val[u];
+    if (!write_tiles) continue;
+    if (codes) {
+      float f[8];
+      const uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float sc = __fdiv_rn(amax, 448.0f);
+      uint32_t packed[2] = {0u, 0u};
+      if (amax > 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t two = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[2 * j], sc), __fdiv_rn(f[2 * j + 1], sc)),
+                                                        __NV_SATFINITE, __NV_E4M3);
+          packed[j >> 1] |= two << (16 * (j & 1));
+        }
+      }
+      uint8_t* crow = static_cast<uint8_t*>(tsr == 0 ? q_t : k_t) + (tile_row0 + r) * kF8RowBytes;
+      *reinterpret_cast<uint2*>(crow + c * 8) = make_uint2(packed[0], packed[1]);  // idle lanes: zero padding
+      if (c == 0) (tsr == 0 ? q_s : k_s)[tile_row0 + r] = sc;
+    } else if (active) {
+      uint16_t* dst = (tsr == 0) ? static_cast<uint16_t*>(q_t) : (tsr == 1) ? static_cast<uint16_t*>(k_t) : v_t;
+      reinterpret_cast<uint4*>(dst + tile_row0 * D)[r * kChunks + c] = val[u];
+    }
   }
   if (!pool) return;
   __syncthreads();

@@ -72,6 +72,9 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g->seq_tiles != 0 && g->seq_tiles != 1) return fail(VSA_ERR_INVALID_ARG, "seq_tiles must be 0 or 1");
   if (g->seq_tiles && g->batch > 4)
     return fail(VSA_ERR_UNSUPPORTED, "seq_tiles needs batch <= 4 (one 5-D tensor map per batch)");
+  if (g->qk_fp8 != 0 && g->qk_fp8 != 1) return fail(VSA_ERR_INVALID_ARG, "qk_fp8 must be 0 or 1");
+  if (g->qk_fp8 && g->seq_tiles)
+    return fail(VSA_ERR_UNSUPPORTED, "qk_fp8 reads 8-bit tile-order copies: it needs seq_tiles = 0");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
     return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128, got " + std::to_string(g->head_dim));
   if (g->tile_size != kTile)
@@ -219,14 +222,20 @@ void build_seq_tables(const Resolved& r, const std::vector<int32_t>& valid, std:
 }
 
 // seq_tiles: no tile-order copies (their regions are empty).
-vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk, bool seq_tiles) {
+// qk_fp8: q_t and k_t hold 8-bit codes, 128 bytes per row whatever D, and q_s, k_s one float per row.
+vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk, bool seq_tiles,
+                                 bool qk_fp8) {
   vsa_workspace_layout w{};
   size_t off = 0;
-  const size_t tiles = seq_tiles ? 0 : static_cast<size_t>(B * H * n_t * kTile * D * 2);
+  const size_t rows = static_cast<size_t>(B * H * n_t * kTile);
+  const size_t tiles = seq_tiles ? 0 : rows * D * 2;
+  const size_t qk_tiles = qk_fp8 ? rows * vsa::kF8RowBytes : tiles;
   const size_t pooled = static_cast<size_t>(B * H * n_t * D * 4);
-  w.q_t = off; off += align256(tiles);
-  w.k_t = off; off += align256(tiles);
+  w.q_t = off; off += align256(qk_tiles);
+  w.k_t = off; off += align256(qk_tiles);
   w.v_t = off; off += align256(tiles);
+  w.q_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
+  w.k_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
   w.pq = off; off += align256(pooled);
   w.pk = off; off += align256(pooled);
   w.pv = off; off += align256(pooled);
@@ -272,6 +281,21 @@ vsa_status make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int D) 
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
+  return VSA_OK;
+}
+
+// 8-bit tile-order codes [rows, 128 bytes] as a 2-D map with 128-byte x 64-row boxes, 128-byte swizzle.
+vsa_status make_code_map(CUtensorMap* m, const void* base, int64_t rows) {
+  EncodeTiledFn enc;
+  VSA_TRY(get_encoder(&enc));
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(vsa::kF8RowBytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(vsa::kF8RowBytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(vsa::kF8RowBytes), 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VSA_ERR_CUDA, "cuTensorMapEncodeTiled (8-bit map) failed with code " + std::to_string(r));
   return VSA_OK;
 }
 
@@ -351,6 +375,7 @@ struct vsa_plan_s {
   std::vector<const void*> part_table;
   const void** d_part_table = nullptr;
   bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
+  bool qk_fp8 = false;     // 8-bit Q/K (E4M3 codes, one scale per token and head) for the fine logits
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
   std::vector<int32_t> tile_token, tile_valid;
@@ -425,8 +450,10 @@ vsa_status with_head_dim(int D, F&& f) {
 // One sequence-order tensor per operand, all heads of the plan.
 vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H, 0}; }
 
+// qs/ks: with an 8-bit plan, the per-row scales (qt/kt then receive codes).
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
-                      float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr) {
+                      float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr, float* qs = nullptr,
+                      float* ks = nullptr) {
   const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
@@ -435,21 +462,19 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   const auto* qq = static_cast<const uint16_t*>(q);
   const auto* kk = static_cast<const uint16_t*>(k);
   const auto* vv = static_cast<const uint16_t*>(v);
-  auto* qo = static_cast<uint16_t*>(qt);
-  auto* ko = static_cast<uint16_t*>(kt);
   auto* vo = static_cast<uint16_t*>(vt);
+  auto launch = [&](auto kernel) -> vsa_status {
+    VSA_TRY(allow_smem(kernel, smem));
+    kernel<<<grid, 384, smem, s>>>(qq, kk, vv, qt, kt, vo, qs, ks, pq, pk, pv, p->d_tile_token, p->d_tile_valid,
+                                   p->r.L, p->H, p->n_t, pio);
+    return VSA_OK;
+  };
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
-    if (pio.table != nullptr) {
-      VSA_TRY(allow_smem(vsa::gather_pool_kernel<D, true>, smem));
-      vsa::gather_pool_kernel<D, true><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                               p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
-    } else {
-      VSA_TRY(allow_smem(vsa::gather_pool_kernel<D, false>, smem));
-      vsa::gather_pool_kernel<D, false><<<grid, 384, smem, s>>>(qq, kk, vv, qo, ko, vo, pq, pk, pv, p->d_tile_token,
-                                                                p->d_tile_valid, p->r.L, p->H, p->n_t, pio);
-    }
-    return VSA_OK;
+    const bool parts = pio.table != nullptr;
+    if (p->qk_fp8)
+      return parts ? launch(vsa::gather_pool_kernel<D, true, true>) : launch(vsa::gather_pool_kernel<D, false, true>);
+    return parts ? launch(vsa::gather_pool_kernel<D, true, false>) : launch(vsa::gather_pool_kernel<D, false, false>);
   }));
   return launch_check("gather_pool");
 }
@@ -507,7 +532,8 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 // tiles itself (needs B <= kSeqMaxBatch).
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
                     const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
-                    const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr) {
+                    const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr, const float* qs = nullptr,
+                    const float* ks = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
@@ -519,11 +545,16 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     for (int t = 0; t < 3; ++t)
       VSA_TRY(make_seq_maps(&sm.prefix[t], sm.video[t], seq_qkv[t], p->B, p->r.L, p->H, p->D, p->r.L - vid, p->r.T,
                             p->r.Hg, p->r.W));
+  } else if (p->qk_fp8) {
+    VSA_TRY(make_code_map(&mq, qt, rows));
+    VSA_TRY(make_code_map(&mk, kt, rows));
+    VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
   } else {
     VSA_TRY(make_tile_map(&mq, qt, rows, p->D));
     VSA_TRY(make_tile_map(&mk, kt, rows, p->D));
     VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
   }
+  if (p->qk_fp8 && (qs == nullptr || ks == nullptr)) return fail(VSA_ERR_INVALID_ARG, "8-bit Q/K needs its scales");
   vsa::AttnArgs a{};
   a.idx = idx;
   a.tile_token = seq ? p->d_row_token : p->d_tile_token;  // query row -> token (-1: not stored)
@@ -540,6 +571,8 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.gate_pc = p->gate_pc;
   a.gate_nonzero = gate_nonzero;
   a.io = io ? *io : single_io(p);
+  a.q_scale = qs;
+  a.k_scale = ks;
   a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
   a.n_t = p->n_t;
   a.P = p->P;
@@ -549,18 +582,17 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
   // the item counter of the persistent schedule starts at zero for every launch
   VSA_CUDA_TRY(cudaMemsetAsync(a.sched, 0, sizeof(int), s));
+  auto launch = [&](auto kernel, size_t smem) -> vsa_status {
+    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
+    VSA_TRY(allow_smem(kernel, smem));
+    kernel<<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a, sm);
+    return VSA_OK;
+  };
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
-    const size_t smem = vsa::AttnLayout<D>::bytes(p->n_t);
-    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
-    if (seq) {
-      VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D, true>, smem));
-      vsa::vsa_attn_kernel<D, true><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a, sm);
-    } else {
-      VSA_TRY(allow_smem(vsa::vsa_attn_kernel<D, false>, smem));
-      vsa::vsa_attn_kernel<D, false><<<static_cast<unsigned>(grid), vsa::kAttnThreads, smem, s>>>(mq, mk, mv, a, sm);
-    }
-    return VSA_OK;
+    if (seq) return launch(vsa::vsa_attn_kernel<D, true, false>, vsa::AttnLayout<D>::bytes(p->n_t));
+    if (p->qk_fp8) return launch(vsa::vsa_attn_kernel<D, false, true>, vsa::AttnLayout<D, true>::bytes(p->n_t));
+    return launch(vsa::vsa_attn_kernel<D, false, false>, vsa::AttnLayout<D>::bytes(p->n_t));
   }));
   return launch_check("attention");
 }
@@ -605,7 +637,8 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->d_mask_tiled = p->d_mask_tiled;
   q->d_status = p->d_status;
   q->seq_tiles = p->seq_tiles;
-  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk, q->seq_tiles);
+  q->qk_fp8 = p->qk_fp8;
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk, q->seq_tiles, q->qk_fp8);
   q->owns_device = false;
   return q;
 }
@@ -621,7 +654,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
   h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
   h.fwd = 0;
-  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk, p->seq_tiles).total);
+  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk, p->seq_tiles, p->qk_fp8).total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
     off += 4 * h.chunk_bytes;  // q, k, v, out
@@ -644,6 +677,8 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   auto* S = reinterpret_cast<float*>(w + p->ws.scores);
   auto* idx = reinterpret_cast<int32_t*>(w + p->ws.idx);
   auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
+  auto* qsc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.q_s) : nullptr;
+  auto* ksc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.k_s) : nullptr;
   // does any gate differ from zero?  (if not, the compression branch is skipped on the device)
   int* gate_nz = p->d_status + 3;
   // sequence parts: the gate is spread over the parts and is not scanned; the branch is kept
@@ -666,11 +701,11 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   // With seq_tiles the attention reads Q/K/V straight from sequence order and the gather only pools;
   // otherwise the gather writes tile-order copies, which the attention reads with better DRAM locality.
   const bool seq = p->seq_tiles;
-  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io));
+  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io, qsc, ksc));
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io);
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io, qsc, ksc);
 }
 
 // Gate elements per token: H, or H*D for a per-channel gate.
@@ -683,7 +718,8 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->topk = r.topk;
   d->seq_len = r.L;
   d->softmax_scale = r.scale;
-  d->workspace_bytes = make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk, g->seq_tiles != 0).total;
+  d->workspace_bytes =
+      make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk, g->seq_tiles != 0, g->qk_fp8 != 0).total;
   d->selected_pairs = r.n_video * (r.n_prefix + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
 }
 
@@ -751,7 +787,8 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   build_tables(r, &p->tile_token, &p->tile_valid);
   build_seq_tables(r, p->tile_valid, &p->row_token, &p->mask_seq, &p->mask_tiled, &p->coord);
   p->seq_tiles = g->seq_tiles != 0;
-  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk, p->seq_tiles);
+  p->qk_fp8 = g->qk_fp8 != 0;
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk, p->seq_tiles, p->qk_fp8);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
@@ -847,6 +884,7 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
 vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, vsa_bf16* q_t,
                             vsa_bf16* k_t, vsa_bf16* v_t, float* pq, float* pk, float* pv, void* stream) {
   VSA_TRY(check_plan(p));
+  if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q, k, v, q_t, k_t, v_t}));
   const int npool = (pq != nullptr) + (pk != nullptr) + (pv != nullptr);
   if (npool != 0 && npool != 3) return fail(VSA_ERR_INVALID_ARG, "pq, pk, pv must be all NULL or all set");
@@ -860,6 +898,7 @@ vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k
   VSA_TRY(check_ptrs({pq, pk, pv, scores}));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q_t != nullptr) {
+    if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
     VSA_TRY(check_ptrs({q_t, k_t, v_t}));
     VSA_TRY(run_pool(p, q_t, k_t, v_t, pq, pk, pv, s));
   }
@@ -878,6 +917,7 @@ vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* 
                                const int32_t* idx, const float* o_c, const vsa_bf16* gate, vsa_bf16* out,
                                void* stream) {
   VSA_TRY(check_plan(p));
+  if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q_t, k_t, v_t, o_c, gate, out}));
   if (p->V > 0) VSA_TRY(check_ptrs({idx}));
   return run_attn(p, q_t, k_t, v_t, idx, o_c, gate, out, static_cast<cudaStream_t>(stream));

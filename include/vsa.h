@@ -100,6 +100,18 @@ typedef struct vsa_geometry {
                                 1: the attention reads each tile straight from sequence order
                                 with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
                                 by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4 */
+  int32_t qk_fp8;            /* 0: the fine branch's logits use the bf16 Q and K;
+                                1: 8-bit Q/K: each (token, head) row of Q and K is quantised to
+                                OCP FP8 E4M3 codes with one binary32 scale s = amax / 448
+                                (code = E4M3(x / s), round to nearest even, saturating; an
+                                all-zero row has s = 0), and the logits are the 8-bit product
+                                times both scales.  Selection, compression and P.V keep bf16.
+                                Every query tile is covered.  Needs seq_tiles = 0; only the
+                                whole-forward entry points accept such a plan.  Passages:
+                                "FastH3 OmniRef inference", sections "The Blackwell stack" and
+                                "Fallbacks" (8-bit per-token Q/K with bf16 P.V); "FastH3 NVFP4
+                                on RTX PRO 6000 (sm_120)", multi-GPU notes (one FP8 scale per
+                                token and head). */
 } vsa_geometry;
 
 typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
@@ -303,9 +315,12 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
                                const vsa_bf16* v_dev, const vsa_bf16* gate_dev, vsa_bf16* out_dev,
                                void* stream);
 
-/* Byte offsets of the intermediates inside vsa_forward's workspace. */
+/* Byte offsets of the intermediates inside vsa_forward's workspace.  With
+ * qk_fp8, q_t and k_t hold E4M3 codes [B, H, n_tiles, 64, 128] (128 bytes per
+ * row whatever D; bytes D..127 zero) and q_s, k_s the row scales [B, H,
+ * n_tiles, 64] float32 (0 for pad rows); otherwise q_s and k_s are empty. */
 typedef struct vsa_workspace_layout {
-  size_t q_t, k_t, v_t, pq, pk, pv, scores, idx, o_c, total;
+  size_t q_t, k_t, v_t, q_s, k_s, pq, pk, pv, scores, idx, o_c, total;
 } vsa_workspace_layout;
 vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
 

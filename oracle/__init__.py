@@ -163,7 +163,7 @@ def compress(S: np.ndarray, pv: np.ndarray) -> np.ndarray:
 
 
 def _qk8_args(qk8, shape):
-    """(q codes, q scales, k codes, k scales) for the 8-bit variant (R13), or four NULLs."""
+    """(q codes, q scales, k codes, k scales) for the 8-bit variant (R16), or four NULLs."""
     if qk8 is None:
         return (None, None, None, None)
     qc, qs, kc, ks = qk8
@@ -207,7 +207,7 @@ def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items, qk8=
 
 
 def e4m3_value(codes) -> np.ndarray:
-    """float64 values of E4M3 codes (uint8 array), from the format's definition (R13)."""
+    """float64 values of E4M3 codes (uint8 array), from the format's definition (R16)."""
     lib = _load()
     table = np.array([lib.vsa_oracle_e4m3_value(c) for c in range(256)], np.float64)
     return table[np.asarray(codes, np.uint8)]
@@ -222,7 +222,7 @@ def e4m3_round(y) -> np.ndarray:
 
 
 def quant_e4m3(x_bf16: np.ndarray):
-    """The 8-bit Q/K quantiser (R13): x [..., D] bf16 bits -> (codes [..., D] uint8, scale [...] float32),
+    """The 8-bit Q/K quantiser (R16): x [..., D] bf16 bits -> (codes [..., D] uint8, scale [...] float32),
     one scale per row of D (per batch, token and head)."""
     x = _c(x_bf16, np.uint16)
     D = x.shape[-1]
@@ -330,7 +330,7 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
 
     Selection (pool, scores, top-k) always runs in full; the fine branch and
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
-    None = all).  qk8: the fine branch's logits use 8-bit Q/K (R13); the
+    None = all).  qk8: the fine branch's logits use 8-bit Q/K (R16); the
     selection still reads the bf16 inputs."""
     t0 = time.perf_counter()
     geo = geometry(segments, grid)

@@ -41,7 +41,7 @@
  *      included -- parity unpinned;
  *   R11 the gate is one scalar per (batch, token, head).
  *   R12 the per-channel variant: one gate per (batch, token, channel h*D + d), [B, L, H*D].
- *   R13 the 8-bit Q/K variant ("FastH3 OmniRef inference", section "The Blackwell stack" and
+ *   R16 the 8-bit Q/K variant ("FastH3 OmniRef inference", section "The Blackwell stack" and
  *      "Fallbacks": query/key rounding to 8 bits with bf16 P.V, per-token FP8 Q/K; the
  *      multi-GPU notes of "FastH3 NVFP4 on RTX PRO 6000": one scale per token and head):
  *      8 bits = OCP FP8 E4M3 ("E4M3FN": bias 7, no infinities, largest 448); one binary32
@@ -80,7 +80,7 @@ static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 /* ------------------------------------------------------------------ */
 /* O0 8-bit Q/K: E4M3 codes with one scale per (batch, token, head)   */
-/* (reading R13)                                                       */
+/* (reading R16)                                                       */
 /* ------------------------------------------------------------------ */
 
 /* Value of an E4M3 code: bit 7 sign, bits 6..3 exponent field e (bias 7),
@@ -431,7 +431,7 @@ static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint1
 /* o_f[b, tok, h, :] for every valid query token tok of every (b, h, i) with
  * todo[(b*H + h)*n_t + i] != 0 (todo == NULL: all).
  * q, k, v: [B, L, H, D] bf16 bits; idx: [B, H, V, k] global tile indices.
- * q8/qs and k8/ks (both NULL, or both set): the 8-bit variant (R13), E4M3
+ * q8/qs and k8/ks (both NULL, or both set): the 8-bit variant (R16), E4M3
  * codes [B, L, H, D] and scales [B, L, H] used for the logits instead of q, k. */
 void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
                      const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,

@@ -1,4 +1,4 @@
-"""Pins for the oracle's 8-bit Q/K variant (reading R13: E4M3 codes, one
+"""Pins for the oracle's 8-bit Q/K variant (reading R16: E4M3 codes, one
 binary32 scale s = amax / 448 per batch, token and head, round to nearest
 even with saturation at 448; the dequantised Q and K replace the bf16 ones in
 the fine branch's logits only).
