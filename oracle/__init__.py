@@ -49,25 +49,26 @@ def _load():
         lib = ctypes.CDLL(build())
         P = ctypes.c_void_p
         i32, i64, f32, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
-        lib.vsa_oracle_geometry.argtypes = [i32, P, i32, i32, i32, P, P, P]
-        lib.vsa_oracle_tiles.argtypes = [i32, P, i32, i32, i32, P, P]
+        lib.vsa_oracle_geometry.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, P, P, P]
+        lib.vsa_oracle_tiles.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, P, P]
         lib.vsa_oracle_topk_count.argtypes = [f64, i32]
         lib.vsa_oracle_topk_count.restype = i32
-        lib.vsa_oracle_pool.argtypes = [P, i32, i64, i32, i32, i32, P, P, P]
+        lib.vsa_oracle_pool.argtypes = [P, i32, i64, i32, i32, i32, i32, P, P, P]
         lib.vsa_oracle_scores.argtypes = [P, P, i32, i32, i32, f32, P]
         lib.vsa_oracle_select.argtypes = [P, i32, i32, i32, i32, P]
         lib.vsa_oracle_compress.argtypes = [P, P, i32, i32, i32, P]
-        lib.vsa_oracle_fine.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P, P]
-        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64,
-                                              i32, P, P]
+        lib.vsa_oracle_fine.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P, f64, P,
+                                        P]
+        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P,
+                                              f64, i32, P, P]
         lib.vsa_oracle_e4m3_value.argtypes = [i32]
         lib.vsa_oracle_e4m3_value.restype = f64
         lib.vsa_oracle_e4m3_round.argtypes = [f32]
         lib.vsa_oracle_e4m3_round.restype = i32
         lib.vsa_oracle_e4m3_round_array.argtypes = [P, i64, P]
         lib.vsa_oracle_quant_e4m3.argtypes = [P, i64, i32, P, P]
-        lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, P, P, f64, P]
-        lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, P, P, P, P]
+        lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P, f64, P]
+        lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -91,26 +92,36 @@ class Geometry:
     n_tiles: int
     n_prefix: int
     n_video: int
-    tile_token: np.ndarray  # [n_tiles, 64] int32, -1 = pad
+    tile_token: np.ndarray  # [n_tiles, tile] int32, -1 = pad
     tile_valid: np.ndarray  # [n_tiles] int32
+    tile: int = 64
+    cube: tuple = (4, 4, 4)
 
     @property
     def seq_len(self) -> int:
         return int(sum(self.segments)) + int(np.prod(self.grid))
 
 
-def geometry(segments, grid) -> Geometry:
+def default_cube(tile: int) -> tuple:
+    """(ct, ch, cw) of a video tile: 4x4x4 for 64 tokens, 4x4x8 for 128 (R17)."""
+    return {64: (4, 4, 4), 128: (4, 4, 8)}[int(tile)]
+
+
+def geometry(segments, grid, tile=64, cube=None) -> Geometry:
     lib = _load()
     seg = np.asarray(segments, dtype=np.int32)
     T, H, W = (int(x) for x in grid)
+    ct, ch, cw = (int(c) for c in (cube or default_cube(tile)))
     nt, npf, nv = (ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32())
-    rc = lib.vsa_oracle_geometry(len(seg), _p(seg), T, H, W, ctypes.byref(nt), ctypes.byref(npf), ctypes.byref(nv))
+    rc = lib.vsa_oracle_geometry(len(seg), _p(seg), T, H, W, int(tile), ct, ch, cw, ctypes.byref(nt),
+                                 ctypes.byref(npf), ctypes.byref(nv))
     if rc:
         raise ValueError("bad geometry")
-    tok = np.empty((nt.value, 64), np.int32)
+    tok = np.empty((nt.value, int(tile)), np.int32)
     val = np.empty((nt.value,), np.int32)
-    lib.vsa_oracle_tiles(len(seg), _p(seg), T, H, W, _p(tok), _p(val))
-    return Geometry(tuple(int(s) for s in segments), (T, H, W), nt.value, npf.value, nv.value, tok, val)
+    lib.vsa_oracle_tiles(len(seg), _p(seg), T, H, W, int(tile), ct, ch, cw, _p(tok), _p(val))
+    return Geometry(tuple(int(s) for s in segments), (T, H, W), nt.value, npf.value, nv.value, tok, val, int(tile),
+                    (ct, ch, cw))
 
 
 def topk_count(sparsity: float, n_video: int) -> int:
@@ -127,7 +138,8 @@ def pool(x_bf16: np.ndarray, geo: Geometry) -> np.ndarray:
     x = _c(x_bf16, np.uint16)
     B, L, H, D = x.shape
     out = np.empty((B, H, geo.n_tiles, D), np.float32)
-    _load().vsa_oracle_pool(_p(x), B, L, H, D, geo.n_tiles, _p(geo.tile_token), _p(geo.tile_valid), _p(out))
+    _load().vsa_oracle_pool(_p(x), B, L, H, D, geo.n_tiles, geo.tile, _p(geo.tile_token), _p(geo.tile_valid),
+                            _p(out))
     return out
 
 
@@ -185,22 +197,23 @@ def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=No
     q8 = _qk8_args(qk8, q.shape)
     out = np.full((B, L, H, D), np.nan, np.float64)
     _load().vsa_oracle_fine(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+                            geo.tile,
                             _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(todo), _p(out))
     return out
 
 
 def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items, qk8=None) -> np.ndarray:
     """Fine branch of the listed query tiles only.  items: int64 array of
-    (b*H + h)*n_t + i.  Returns [n_items, 64, D] float64 in tile row order
+    (b*H + h)*n_t + i.  Returns [n_items, tile, D] float64 in tile row order
     (pad rows 0).  qk8: as for fine()."""
     q, k, v = (_c(t, np.uint16) for t in (q, k, v))
     B, L, H, D = q.shape
     idx = _c(idx, np.int32)
     items = _c(np.asarray(items, np.int64), np.int64)
     q8 = _qk8_args(qk8, q.shape)
-    out = np.zeros((len(items), 64, D), np.float64)
+    out = np.zeros((len(items), geo.tile, D), np.float64)
     _load().vsa_oracle_fine_tiles(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles,
-                                  geo.n_prefix, topk,
+                                  geo.n_prefix, topk, geo.tile,
                                   _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), len(items),
                                   _p(items), _p(out))
     return out
@@ -260,9 +273,9 @@ def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarr
     return res
 
 
-def selection(q, k, v, segments, grid, sparsity, scale=None):
+def selection(q, k, v, segments, grid, sparsity, scale=None, tile=64, cube=None):
     """Pool, scores, top-k and compression only (every tile, every head)."""
-    geo = geometry(segments, grid)
+    geo = geometry(segments, grid, tile, cube)
     if scale is None:
         scale = default_scale(q.shape[-1])
     kc = topk_count(sparsity, geo.n_video)
@@ -279,7 +292,7 @@ def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndar
     B, L, H, D = q.shape
     idx = _c(idx, np.int32)
     out = np.full((B, L, H, D), np.nan, np.float64)
-    _load().vsa_oracle_fine_masked(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
+    _load().vsa_oracle_fine_masked(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk, geo.tile,
                                    _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(out))
     return out
 
@@ -303,7 +316,7 @@ def output(o_f, o_c, gate, geo: Geometry, todo=None) -> np.ndarray:
     if todo is not None:
         todo = _c(todo.astype(np.uint8), np.uint8)
     out = np.full((B, L, H, D), np.nan, np.float64)
-    _load().vsa_oracle_output(_p(o_f), _p(o_c), _p(gate), int(per_channel), B, L, H, D, geo.n_tiles,
+    _load().vsa_oracle_output(_p(o_f), _p(o_c), _p(gate), int(per_channel), B, L, H, D, geo.n_tiles, geo.tile,
                               _p(geo.tile_token), _p(geo.tile_valid), _p(todo), _p(out))
     return out
 
@@ -324,16 +337,18 @@ class ForwardResult:
     seconds: float
 
 
-def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=False) -> ForwardResult:
+def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=False, tile=64,
+            cube=None) -> ForwardResult:
     """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H] (or
     [B,L,H*D], one per channel).
 
     Selection (pool, scores, top-k) always runs in full; the fine branch and
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
     None = all).  qk8: the fine branch's logits use 8-bit Q/K (R16); the
-    selection still reads the bf16 inputs."""
+    selection still reads the bf16 inputs.  tile, cube: the tile size and video
+    cube shape (64 and 4x4x4 as the method states; 128 per R17)."""
     t0 = time.perf_counter()
-    geo = geometry(segments, grid)
+    geo = geometry(segments, grid, tile, cube)
     D = q.shape[-1]
     if scale is None:
         scale = default_scale(D)

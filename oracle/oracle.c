@@ -51,6 +51,12 @@
  *      +0.  The dequantised value code * s replaces Q and K in the fine branch's logits
  *      only: selection, compression and P.V keep the bf16 inputs.  The variant covers
  *      every query tile.
+ *   R17 128-token tiles ("FastH3 OmniRef inference", section "The Blackwell stack": VSA
+ *      with 128-token tiles; the cube shape is not stated): a prefix tile is a
+ *      segment-pure run of up to 128 tokens and a video tile a ct x ch x cw cube with
+ *      ct*ch*cw = 128, by default 4 x 4 x 8 (the 4 x 4 x 4 cube doubled along w, the
+ *      fastest axis); every other step is the 64-token method with "64" read as the
+ *      tile size.
  *
  * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
  * order above; fine attention, compression and the output in binary64.
@@ -62,8 +68,8 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define TILE 64
-#define CUBE 4
+/* Tile size and cube shape are arguments: 64-token (4,4,4) tiles, or the
+ * 128-token tiles of reading R17. */
 
 /* ------------------------------------------------------------------ */
 /* helpers                                                             */
@@ -175,20 +181,22 @@ static void qk_tables(void) {
 /* O1 geometry                                                         */
 /* ------------------------------------------------------------------ */
 
-/* Tile counts of a packed sequence: each prefix segment of n tokens gives
- * ceil(n/64) segment-pure tiles; the T x H x W video grid gives
- * ceil(T/4) * ceil(H/4) * ceil(W/4) cubes (reading R2).
+/* Tile counts of a packed sequence with `tile`-token tiles whose video cubes are
+ * ct x ch x cw (ct*ch*cw == tile; 64 = 4x4x4 as the method states, R17 for 128):
+ * each prefix segment of n tokens gives ceil(n/tile) segment-pure tiles; the
+ * T x H x W video grid gives ceil(T/ct) * ceil(H/ch) * ceil(W/cw) cubes (R2).
  * Returns 0, or -1 on a bad argument. */
-int vsa_oracle_geometry(int n_seg, const int32_t *seg_len, int T, int Hg, int W,
-                        int32_t *n_tiles, int32_t *n_prefix, int32_t *n_video) {
+int vsa_oracle_geometry(int n_seg, const int32_t *seg_len, int T, int Hg, int W, int tile, int ct, int ch,
+                        int cw, int32_t *n_tiles, int32_t *n_prefix, int32_t *n_video) {
     if (n_seg < 0 || T < 0 || Hg < 0 || W < 0) return -1;
+    if (tile < 1 || ct < 1 || ch < 1 || cw < 1 || ct * ch * cw != tile) return -1;
     int64_t p = 0;
     for (int s = 0; s < n_seg; ++s) {
         if (seg_len[s] < 0) return -1;
-        p += ceil_div(seg_len[s], TILE);
+        p += ceil_div(seg_len[s], tile);
     }
     int64_t v = (T > 0 && Hg > 0 && W > 0)
-                    ? ceil_div(T, CUBE) * ceil_div(Hg, CUBE) * ceil_div(W, CUBE)
+                    ? ceil_div(T, ct) * ceil_div(Hg, ch) * ceil_div(W, cw)
                     : 0;
     *n_prefix = (int32_t)p;
     *n_video = (int32_t)v;
@@ -196,40 +204,40 @@ int vsa_oracle_geometry(int n_seg, const int32_t *seg_len, int T, int Hg, int W,
     return 0;
 }
 
-/* Token table: tile_token[tile*64 + r] is the packed-sequence index of row r
- * of the tile, or -1 for a pad row; tile_valid[tile] counts the valid rows.
+/* Token table: tile_token[i*tile + r] is the packed-sequence index of row r
+ * of tile i, or -1 for a pad row; tile_valid[i] counts the valid rows.
  * Prefix tiles first, in sequence order; then the cubes in raster (a,b,c)
  * order; inside a cube, raster (t,h,w) (readings R1, R3). */
-int vsa_oracle_tiles(int n_seg, const int32_t *seg_len, int T, int Hg, int W,
+int vsa_oracle_tiles(int n_seg, const int32_t *seg_len, int T, int Hg, int W, int tile, int ct, int ch, int cw,
                      int32_t *tile_token, int32_t *tile_valid) {
     int32_t nt, np, nv;
-    if (vsa_oracle_geometry(n_seg, seg_len, T, Hg, W, &nt, &np, &nv)) return -1;
-    for (int64_t i = 0; i < (int64_t)nt * TILE; ++i) tile_token[i] = -1;
+    if (vsa_oracle_geometry(n_seg, seg_len, T, Hg, W, tile, ct, ch, cw, &nt, &np, &nv)) return -1;
+    for (int64_t i = 0; i < (int64_t)nt * tile; ++i) tile_token[i] = -1;
 
-    int tile = 0;
+    int i = 0;
     int64_t offset = 0; /* first token of the current segment */
     for (int s = 0; s < n_seg; ++s) {
         int64_t n = seg_len[s];
-        for (int64_t first = 0; first < n; first += TILE) {
+        for (int64_t first = 0; first < n; first += tile) {
             int cnt = 0;
-            for (int64_t t = first; t < n && t < first + TILE; ++t)
-                tile_token[(int64_t)tile * TILE + cnt++] = (int32_t)(offset + t);
-            tile_valid[tile++] = cnt;
+            for (int64_t t = first; t < n && t < first + tile; ++t)
+                tile_token[(int64_t)i * tile + cnt++] = (int32_t)(offset + t);
+            tile_valid[i++] = cnt;
         }
         offset += n;
     }
     if (nv > 0) {
         int64_t video_base = offset;
-        for (int a = 0; a < ceil_div(T, CUBE); ++a)
-            for (int b = 0; b < ceil_div(Hg, CUBE); ++b)
-                for (int c = 0; c < ceil_div(W, CUBE); ++c) {
+        for (int a = 0; a < ceil_div(T, ct); ++a)
+            for (int b = 0; b < ceil_div(Hg, ch); ++b)
+                for (int c = 0; c < ceil_div(W, cw); ++c) {
                     int cnt = 0;
-                    for (int t = CUBE * a; t < CUBE * a + CUBE && t < T; ++t)
-                        for (int h = CUBE * b; h < CUBE * b + CUBE && h < Hg; ++h)
-                            for (int w = CUBE * c; w < CUBE * c + CUBE && w < W; ++w)
-                                tile_token[(int64_t)tile * TILE + cnt++] =
+                    for (int t = ct * a; t < ct * a + ct && t < T; ++t)
+                        for (int h = ch * b; h < ch * b + ch && h < Hg; ++h)
+                            for (int w = cw * c; w < cw * c + cw && w < W; ++w)
+                                tile_token[(int64_t)i * tile + cnt++] =
                                     (int32_t)(video_base + ((int64_t)t * Hg + h) * W + w);
-                    tile_valid[tile++] = cnt;
+                    tile_valid[i++] = cnt;
                 }
     }
     return 0;
@@ -251,20 +259,20 @@ int vsa_oracle_topk_count(double sparsity, int n_video) {
 /* x: [B, L, H, D] bf16 bits.  pooled: [B, H, n_t, D] float.
  * pooled = (((0 + x_0) + x_1) + ... + x_{n-1}) / n  over the valid rows in
  * tile order, every step one IEEE binary32 rounding (R4, R6). */
-void vsa_oracle_pool(const uint16_t *x, int B, int64_t L, int H, int D, int n_t,
+void vsa_oracle_pool(const uint16_t *x, int B, int64_t L, int H, int D, int n_t, int tile,
                      const int32_t *tile_token, const int32_t *tile_valid, float *pooled) {
 #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h)
-            for (int tile = 0; tile < n_t; ++tile)
+            for (int i = 0; i < n_t; ++i)
                 for (int d = 0; d < D; ++d) {
                     float sum = 0.0f;
-                    for (int r = 0; r < tile_valid[tile]; ++r) {
-                        int64_t tok = tile_token[(int64_t)tile * TILE + r];
+                    for (int r = 0; r < tile_valid[i]; ++r) {
+                        int64_t tok = tile_token[(int64_t)i * tile + r];
                         sum = sum + bf16_to_float(x[(((int64_t)b * L + tok) * H + h) * D + d]);
                     }
-                    pooled[(((int64_t)b * H + h) * n_t + tile) * D + d] =
-                        sum / (float)tile_valid[tile];
+                    pooled[(((int64_t)b * H + h) * n_t + i) * D + d] =
+                        sum / (float)tile_valid[i];
                 }
 }
 
@@ -383,23 +391,23 @@ static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t
  *   o_f[r] = sum_c softmax(logit)_c * v_c,
  * written to rows[r * D + d] in tile row order (pad rows left untouched). */
 static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint16_t *v, int b, int h, int i,
-                          int64_t L, int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                          int64_t L, int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
                           const int32_t *tile_valid, const int32_t *idx, double scale, double *rows) {
     int V = n_t - P;
     int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
     const int32_t *idx_row = (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
     int nk = key_set(i, n_t, P, k, idx_row, keys);
     /* every valid key row of the key set, in list order */
-    int64_t max_rows = (int64_t)nk * TILE;
+    int64_t max_rows = (int64_t)nk * tile;
     int64_t *ktok = (int64_t *)malloc(sizeof(int64_t) * (size_t)max_rows);
     double *logit = (double *)malloc(sizeof(double) * (size_t)max_rows);
     int64_t nrows = 0;
     for (int t = 0; t < nk; ++t)
         for (int c = 0; c < tile_valid[keys[t]]; ++c)
-            ktok[nrows++] = tile_token[(int64_t)keys[t] * TILE + c];
+            ktok[nrows++] = tile_token[(int64_t)keys[t] * tile + c];
 
     for (int r = 0; r < tile_valid[i]; ++r) {
-        int64_t qt = tile_token[(int64_t)i * TILE + r];
+        int64_t qt = tile_token[(int64_t)i * tile + r];
         int64_t qrow = ((int64_t)b * L + qt) * H + h;
         double m = -INFINITY;
         for (int64_t c = 0; c < nrows; ++c) {
@@ -435,7 +443,7 @@ static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint1
  * codes [B, L, H, D] and scales [B, L, H] used for the logits instead of q, k. */
 void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
                      const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
-                     int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                     int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
                      const int32_t *tile_valid, const int32_t *idx, double scale,
                      const uint8_t *todo, double *o_f) {
     qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
@@ -446,11 +454,11 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, c
             for (int i = 0; i < n_t; ++i) {
                 int64_t bhi = ((int64_t)b * H + h) * n_t + i;
                 if (todo && !todo[bhi]) continue;
-                double *rows = (double *)malloc(sizeof(double) * (size_t)TILE * (size_t)D);
-                fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale,
+                double *rows = (double *)malloc(sizeof(double) * (size_t)tile * (size_t)D);
+                fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile, tile_token, tile_valid, idx, scale,
                               rows);
                 for (int r = 0; r < tile_valid[i]; ++r) {
-                    int64_t tok = tile_token[(int64_t)i * TILE + r];
+                    int64_t tok = tile_token[(int64_t)i * tile + r];
                     memcpy(o_f + (((int64_t)b * L + tok) * H + h) * D, rows + (int64_t)r * D,
                            sizeof(double) * (size_t)D);
                 }
@@ -462,7 +470,7 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, c
  * out[n, r, :] for the tile's rows r in tile order (pad rows set to 0). */
 void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
                            const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
-                           int H, int D, int n_t, int P, int k, const int32_t *tile_token,
+                           int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
                            const int32_t *tile_valid, const int32_t *idx, double scale, int n_items,
                            const int64_t *items, double *out) {
     qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
@@ -474,9 +482,9 @@ void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t
         int i = (int)(bhi % n_t);
         int64_t bh = bhi / n_t;
         int h = (int)(bh % H), b = (int)(bh / H);
-        double *rows = out + (int64_t)n * TILE * D;
-        for (int64_t e = 0; e < (int64_t)TILE * D; ++e) rows[e] = 0.0;
-        fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile_token, tile_valid, idx, scale, rows);
+        double *rows = out + (int64_t)n * tile * D;
+        for (int64_t e = 0; e < (int64_t)tile * D; ++e) rows[e] = 0.0;
+        fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile, tile_token, tile_valid, idx, scale, rows);
     }
 }
 
@@ -490,13 +498,13 @@ void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t
  * against).  Tokens outside every tile do not occur.  Used on small inputs
  * only: builds an L x L mask per (b, h). */
 void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B,
-                            int64_t L, int H, int D, int n_t, int P, int k,
+                            int64_t L, int H, int D, int n_t, int P, int k, int tile,
                             const int32_t *tile_token, const int32_t *tile_valid,
                             const int32_t *idx, double scale, double *o_f) {
     int V = n_t - P;
     int32_t *tile_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)L);
     for (int i = 0; i < n_t; ++i)
-        for (int r = 0; r < tile_valid[i]; ++r) tile_of[tile_token[(int64_t)i * TILE + r]] = i;
+        for (int r = 0; r < tile_valid[i]; ++r) tile_of[tile_token[(int64_t)i * tile + r]] = i;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h) {
@@ -556,7 +564,7 @@ void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_
  * [B, L, H], one scalar per token and head (gate_per_channel = 0), or [B, L, H*D], one per
  * channel h*D + d of the token (gate_per_channel = 1, R12). */
 void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gate, int gate_per_channel,
-                       int B, int64_t L, int H, int D, int n_t, const int32_t *tile_token,
+                       int B, int64_t L, int H, int D, int n_t, int tile, const int32_t *tile_token,
                        const int32_t *tile_valid, const uint8_t *todo, double *out) {
 #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
@@ -565,7 +573,7 @@ void vsa_oracle_output(const double *o_f, const double *o_c, const uint16_t *gat
                 if (todo && !todo[((int64_t)b * H + h) * n_t + i]) continue;
                 const double *oc = o_c + (((int64_t)b * H + h) * n_t + i) * D;
                 for (int r = 0; r < tile_valid[i]; ++r) {
-                    int64_t tok = tile_token[(int64_t)i * TILE + r];
+                    int64_t tok = tile_token[(int64_t)i * tile + r];
                     int64_t row = (((int64_t)b * L + tok) * H + h);
                     for (int d = 0; d < D; ++d) {
                         uint16_t gbits = gate_per_channel ? gate[row * D + d] : gate[row];
