@@ -8,7 +8,8 @@ input already resident in HBM.  The default workload is the 1344x768-shaped
 one at sparsity 0.9 (56 heads, D=128, 73,728 video + 1,280 prefix tokens).
 
 Metric: effective TFLOP/s counting only the selected (query tile, key tile)
-pairs, 4*64*64*D FLOP each, per whole forward; ms per call is reported too.
+pairs, 4*T*T*D FLOP each for T-token tiles (T = 64, or 128 for the
+128-token-tile workload), per whole forward; ms per call is reported too.
 Multi-GPU (torchrun): every rank runs its own forward on its own seeded input
 (the forward shards by (batch, head) with no exchange), value = all ranks'
 FLOPs / the slowest rank's time ("scaling": "weak").
@@ -36,8 +37,8 @@ UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
 
 
-def tile_flops(D: int) -> int:
-    return 4 * 64 * 64 * D
+def tile_flops(D: int, tile: int = 64) -> int:
+    return 4 * tile * tile * D
 
 
 def load_peaks():
@@ -181,14 +182,14 @@ def oracle_sample(w, every: int, seed: int = 0):
     x = synth.make_inputs(dataclasses.replace(w, heads=1), seed=seed, device="cpu")
     xb = {n: synth.as_bits(x[n]) for n in ("q", "k", "v", "gate")}
     t0 = time.perf_counter()
-    sel = oracle.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity)
+    sel = oracle.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity, tile=w.tile, cube=w.cube)
     geo = sel["geo"]
     items = np.arange(0, geo.n_tiles, every, dtype=np.int64)
     of = oracle.fine_tiles(xb["q"], xb["k"], xb["v"], geo, sel["idx"], sel["topk"], sel["scale"], items)
     oracle.output_tiles(of, sel["o_c"], xb["gate"], geo, items, 1)
     dt = time.perf_counter() - t0
     pairs = sum((geo.n_tiles if i < geo.n_prefix else geo.n_prefix + sel["topk"]) for i in items)
-    flops = pairs * tile_flops(w.head_dim)
+    flops = pairs * tile_flops(w.head_dim, w.tile)
     desc = (f"head 0 of 56: full selection (pool, fp32 scores, top-k, compression over {geo.n_tiles} tiles) "
             f"+ fine branch and output of every {every}th query tile ({len(items)} of {geo.n_tiles} tiles, "
             f"{pairs} selected tile pairs)")
@@ -231,7 +232,7 @@ def run_reference(args, w, world, rank):
 def config_dict(w, dims=None):
     import oracle
 
-    geo = oracle.geometry(w.segments, w.grid) if dims is None else None
+    geo = oracle.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube) if dims is None else None
     n_t = dims["n_tiles"] if dims else geo.n_tiles
     P = dims["n_prefix_tiles"] if dims else geo.n_prefix
     V = n_t - P
@@ -240,9 +241,9 @@ def config_dict(w, dims=None):
     return {
         "workload": w.name, "description": w.description, "batch": w.batch, "heads": w.heads,
         "head_dim": w.head_dim, "seq_len": w.seq_len, "prefix_segments": list(w.segments), "grid": list(w.grid),
-        "n_tiles": n_t, "n_prefix_tiles": P, "n_video_tiles": V, "sparsity": w.sparsity, "topk": k,
-        "selected_tile_pairs": pairs * w.batch * w.heads,
-        "selected_tflop_per_call": pairs * w.batch * w.heads * tile_flops(w.head_dim) / 1e12,
+        "tile_size": w.tile, "n_tiles": n_t, "n_prefix_tiles": P, "n_video_tiles": V, "sparsity": w.sparsity,
+        "topk": k, "selected_tile_pairs": pairs * w.batch * w.heads,
+        "selected_tflop_per_call": pairs * w.batch * w.heads * tile_flops(w.head_dim, w.tile) / 1e12,
         "l2": "no flush: Q/K/V/out are %.1f GB per step, > 126 MB L2" % (4 * w.batch * w.seq_len * w.heads * w.head_dim * 2 / 1e9),
     }
 
@@ -258,13 +259,13 @@ def run_vsa(args, w, world, rank, local):
     x = synth.make_inputs(w, seed=rank, device=dev)
     torch.cuda.synchronize()
     plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-                              sparsity=w.sparsity)
+                              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube)
     dims = plan.dims
     ws = vsa.alloc_workspace(plan, dev)
     v = vsa.workspace_views(plan, ws)
     out = torch.empty_like(x["q"])
     stream = torch.cuda.current_stream(dev)
-    flops_call = dims["selected_pairs"] * w.batch * w.heads * tile_flops(w.head_dim)
+    flops_call = dims["selected_pairs"] * w.batch * w.heads * tile_flops(w.head_dim, w.tile)
 
     ev = {n: [] for n in ("t0", "t1", "t2", "t3", "t4")}
 
@@ -390,7 +391,7 @@ def run_ab(args, w, variants):
     for rnd in range(2):
         for key, extra in variants.items():
             plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments,
-                                      grid=w.grid, sparsity=w.sparsity, **extra)
+                                      grid=w.grid, sparsity=w.sparsity, tile_size=w.tile, cube=w.cube, **extra)
             ws = vsa.alloc_workspace(plan)
             out = torch.empty_like(x["q"])
             for _ in range(args.warmup):

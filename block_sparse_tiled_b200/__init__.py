@@ -55,6 +55,7 @@ class Geometry(ctypes.Structure):
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
         ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32), ("qk_fp8", ctypes.c_int32),
+        ("cube_t", ctypes.c_int32), ("cube_h", ctypes.c_int32), ("cube_w", ctypes.c_int32),
     ]
 
 
@@ -72,7 +73,7 @@ class PlanDims(ctypes.Structure):
     _fields_ = [
         ("n_tiles", ctypes.c_int32), ("n_prefix_tiles", ctypes.c_int32), ("n_video_tiles", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("seq_len", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
-        ("workspace_bytes", ctypes.c_size_t), ("selected_pairs", ctypes.c_int64),
+        ("workspace_bytes", ctypes.c_size_t), ("selected_pairs", ctypes.c_int64), ("tile_size", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -151,8 +152,10 @@ def _ptr(t, dtype=None, name="tensor"):
 
 
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
-                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False, qk_fp8=False):
-    """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers)."""
+                  token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False, qk_fp8=False,
+                  cube=None):
+    """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers).  cube: (t, h, w) of a
+    video tile, None for the default (4x4x4 for 64-token tiles, 4x4x8 for 128)."""
     g = Geometry()
     g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
     keep = []
@@ -176,6 +179,7 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.gate_per_channel = int(bool(gate_per_channel))
     g.seq_tiles = int(bool(seq_tiles))
     g.qk_fp8 = int(bool(qk_fp8))
+    g.cube_t, g.cube_h, g.cube_w = (int(c) for c in (cube or (0, 0, 0)))
     return g, keep
 
 
@@ -188,13 +192,13 @@ def vsa_plan_query(**kw) -> dict:
 
 
 def vsa_plan_tables_host(**kw):
-    """Host-only token table of a geometry: (tile_token [n_tiles, 64], tile_valid [n_tiles])."""
+    """Host-only token table of a geometry: (tile_token [n_tiles, tile_size], tile_valid [n_tiles])."""
     import numpy as np
 
     d = vsa_plan_query(**kw)
     g, keep = make_geometry(**kw)
     n = d["n_tiles"]
-    tok = np.empty((max(n, 1), 64), np.int32)
+    tok = np.empty((max(n, 1), d["tile_size"]), np.int32)
     val = np.empty((max(n, 1),), np.int32)
     _check(load_library().vsa_plan_tables_host(ctypes.byref(g), tok.ctypes.data_as(ctypes.c_void_p),
                                                val.ctypes.data_as(ctypes.c_void_p)), "vsa_plan_tables_host")
@@ -224,7 +228,7 @@ class Plan:
         import numpy as np
 
         n = self.dims["n_tiles"]
-        tok = np.empty((max(n, 1), 64), np.int32)
+        tok = np.empty((max(n, 1), self.dims["tile_size"]), np.int32)
         val = np.empty((max(n, 1),), np.int32)
         _check(load_library().vsa_plan_tables(self.handle, tok.ctypes.data_as(ctypes.c_void_p),
                                               val.ctypes.data_as(ctypes.c_void_p)), "vsa_plan_tables")
@@ -244,11 +248,11 @@ class Plan:
 
 def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
                    token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False,
-                   qk_fp8=False, stream=None) -> Plan:
+                   qk_fp8=False, cube=None, stream=None) -> Plan:
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
               tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles),
-              qk_fp8=bool(qk_fp8))
+              qk_fp8=bool(qk_fp8), cube=None if cube is None else tuple(cube))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
     _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")
@@ -433,25 +437,26 @@ def device_status(plan, stream=None):
 def workspace_views(plan, workspace):
     """Typed views of vsa_forward's intermediates inside ``workspace`` (no tile-order views for a plan
     with seq_tiles, whose workspace holds none).  With qk_fp8, q_t and k_t are the E4M3 codes
-    [B, H, n_t, 64, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, 64]."""
+    [B, H, n_t, tile, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, tile]."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
     seq = bool(g.get("seq_tiles", False))
     f8 = bool(g.get("qk_fp8", False))
+    T = d["tile_size"]  # rows per tile
 
     def view(off, n, dtype, shape):
         nbytes = n * torch.tensor([], dtype=dtype).element_size()
         return workspace[off:off + nbytes].view(dtype).view(*shape)
 
     def tiles(name):
-        return None if seq else view(lay[name], B * H * n_t * 64 * D, torch.bfloat16, (B, H, n_t, 64, D))
+        return None if seq else view(lay[name], B * H * n_t * T * D, torch.bfloat16, (B, H, n_t, T, D))
 
     def codes(name):
-        return view(lay[name], B * H * n_t * 64 * 128, torch.uint8, (B, H, n_t, 64, 128))
+        return view(lay[name], B * H * n_t * T * 128, torch.uint8, (B, H, n_t, T, 128))
 
     def row_scales(name):
-        return view(lay[name], B * H * n_t * 64, torch.float32, (B, H, n_t, 64)) if f8 else None
+        return view(lay[name], B * H * n_t * T, torch.float32, (B, H, n_t, T)) if f8 else None
 
     return {
         "q_t": codes("q_t") if f8 else tiles("q_t"),

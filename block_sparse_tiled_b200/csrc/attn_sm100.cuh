@@ -1,9 +1,11 @@
 // Block-sparse VSA-H3 attention forward for sm_100a (tcgen05 + TMEM + TMA).
 //
-// Work item = (b, h, query tile i), numbered (b*H + h)*n_t + i.  Its key list
-// is every tile for a prefix query tile, else the P prefix tiles followed by
-// the tile's selected video tiles (ascending).  The list is walked two key
-// tiles (128 keys) at a time.  CTAs claim items in order from a global counter
+// Work item = (b, h, 64-row block s of the query tiles), numbered (b*H + h)*n_rb + s.
+// With 64-token tiles a row block is a tile; with 128-token tiles (sub_shift = 1)
+// tile i is row blocks 2i and 2i+1, which share its key list.  The key list of
+// query tile i is every tile for a prefix query tile, else the P prefix tiles
+// followed by the tile's selected video tiles (ascending), taken as row blocks
+// and walked two row blocks (128 keys) at a time.  CTAs claim items in order from a global counter
 // (one per SM, persistent), so the items in flight stay within a head or two
 // and that head's K/V stays resident in L2 even though prefix query tiles cost
 // many times a video query tile.
@@ -100,25 +102,26 @@ constexpr uint32_t kTmemCols = (kOCol0 + 128 <= 256) ? 256 : 512;
 
 struct AttnArgs {
   const int32_t* idx;         // [B, H, V, topk] global key-tile indices (ascending per row)
-  const int32_t* tile_token;  // [n_t * 64]
+  const int32_t* tile_token;  // [n_rb * 64]: token of each row of each 64-row block
   const int32_t* tile_valid;  // [n_t]
-  const float* o_c;           // [B, H, n_t, D]
+  const float* o_c;           // [B, H, n_t, D] (per tile)
   const uint16_t* gate;       // [B, L, gate_ld] bf16: the gate of head h at gate[(b*L + t)*gate_ld + h]
   uint16_t* out;              // [B, L, H, D] bf16
   int* status;                // [2] device status word
   int* sched;                 // item counter, zero at launch
   int64_t L;
-  int H, n_t, P, topk;
+  int H, n_t, P, topk;  // n_t here: 64-row blocks per (b, h) (tiles << sub_shift); P, topk in tiles
+  int sub_shift;         // log2(tile size / 64): 0 for 64-token tiles, 1 for 128
   int gate_ld;  // gate elements between consecutive tokens (H or H*D, or more when a head slice is processed)
   int gate_pc;  // 0: one gate per (token, head) at h; 1: one per channel, at h*D + d
   const int* gate_nonzero;  // NULL, or a flag that is 0 when every gate is zero (o_c then unread)
-  const uint64_t* key_mask;  // [n_t]: bit r set when row r of the tile as loaded is a key (a token)
-  const int32_t* coord;      // [n_t][4] TMA coordinates of a tile read from sequence order
+  const uint64_t* key_mask;  // [n_rb]: bit r set when row r of the block as loaded is a key (a token)
+  const int32_t* coord;      // [n_rb][4] TMA coordinates of a block read from sequence order
   PartIO io;                 // where gate and out live (one tensor, or sequence parts, possibly on peers)
-  const float* q_scale;      // 8-bit Q/K only: [B, H, n_t, 64] scale of each query row (tile order)
-  const float* k_scale;      // 8-bit Q/K only: [B, H, n_t, 64] scale of each key row
+  const float* q_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each query row (tile order)
+  const float* k_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each key row
   float scale_log2;  // softmax scale * log2(e)
-  int64_t n_items;   // B * H * n_t
+  int64_t n_items;   // B * H * n_rb
 };
 
 // Tensor maps for loading tiles straight from sequence order (q, k, v): a 4-D map over [b, token, head, d]
@@ -245,7 +248,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   int32_t* qpart_s = reinterpret_cast<int32_t*>(sm + Ly::oQpart);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_t = a.n_t, P = a.P, topk = a.topk, V = n_t - P;
+  // n_t: 64-row blocks per (b, h); n_sel: tiles (the selection's unit), P and topk count tiles
+  const int n_t = a.n_t, sh = a.sub_shift, n_sel = n_t >> sh, P = a.P, topk = a.topk, V = n_sel - P;
   const WaitCtl ctl{abort_flag, a.status, kWaitTimeoutNs};
 
   // ---------------------------------------------------------------- setup
@@ -305,10 +309,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
 
-  auto list_len = [&](int i) { return (i < P) ? n_t : P + topk; };
+  // key list of query tile i, in 64-row blocks
+  auto list_len = [&](int i) { return ((i < P) ? n_sel : P + topk) << sh; };
+  // row block of list position t (in row blocks) of query tile i
   auto key_tile = [&](int64_t bh, int i, int t) -> int {
-    if (i < P || t < P) return t;
-    return __ldg(a.idx + (bh * V + (i - P)) * topk + (t - P));
+    const int ts = t >> sh;
+    const int sel = (i < P || ts < P) ? ts : __ldg(a.idx + (bh * V + (i - P)) * topk + (ts - P));
+    return (sel << sh) | (t & ((1 << sh) - 1));
   };
   // Claimed item number `it` of this CTA (-1: none left), read by one thread of a consumer warp.
   auto ring_take = [&](int it, int site) -> int {
@@ -366,7 +373,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       w = __shfl_sync(0xffffffffu, w, 0);
       if (w < 0 || !ok) break;
       const int64_t bh = w / n_t;
-      const int i = static_cast<int>(w - bh * n_t);
+      const int s = static_cast<int>(w - bh * n_t);  // query row block
+      const int i = s >> sh;                          // its tile
       const int nk = list_len(i), nb = (nk + 1) / 2;
       if (is_k) {
         // the query tile of this item (loaded by the K warp, which runs ahead with the S^T issuer)
@@ -382,14 +390,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok && lane < (kF8 ? 1 : Ly::kHalves)) {
           void* dst = sm + Ly::oQ + qb * Ly::kQBytes + lane * 8192;
           if constexpr (kSeq) {
-            const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + i);
+            const int4 c = __ldg(reinterpret_cast<const int4*>(a.coord) + s);
             const int bb = static_cast<int>(bh / a.H), hh = static_cast<int>(bh - static_cast<int64_t>(bb) * a.H);
             if (c.x == 0)
               tma_load_4d(dst, &seq.prefix[0], &bars[Ly::bQFull + qb], lane * 64, hh, c.y, bb);
             else
               tma_load_5d(dst, &seq.video[0][bb], &bars[Ly::bQFull + qb], lane * 64, hh, c.y, c.z, c.w);
           } else {
-            const int row = static_cast<int>((bh * n_t + i) * 64);
+            const int row = static_cast<int>((bh * n_t + s) * 64);
             tma_load_2d(dst, &tm_q, &bars[Ly::bQFull + qb], lane * 64, row);
           }
         }
@@ -471,7 +479,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int w = ring_take(it, 26);
         if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
-        const int i = static_cast<int>(w - bh * n_t);
+        const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
         const int nb = (list_len(i) + 1) / 2;
         const int qb = it % Ly::kQBufs;
         ROLE_MARK(3);
@@ -521,7 +529,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int w = ring_take(it, 27);
         if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
-        const int i = static_cast<int>(w - bh * n_t);
+        const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
         const int nb = (list_len(i) + 1) / 2;
         const int ob = it & 1;
         for (int n = 0; n < nb && ok; ++n, ++g) {
@@ -587,7 +595,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
-      const int i = static_cast<int>(w - bh * n_t);
+      const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
       const int nk = list_len(i), nb = (nk + 1) / 2;
       const int ob = it & 1;
       const float* qsc_g = m_g + kQscFromM + ob * 64;
@@ -814,12 +822,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       w = __shfl_sync(0xffffffffu, w, 0);
       if (named_bar_or(9, 128, w < 0)) break;  // the epilogue warps stop together
       const int64_t bh = w / n_t;
-      const int i = static_cast<int>(w - bh * n_t);
+      const int s = static_cast<int>(w - bh * n_t);  // query row block
+      const int i = s >> sh;                          // its tile
       const int64_t b = bh / a.H;
       const int h = static_cast<int>(bh - b * a.H);
       const int ob = it & 1;
       if (tid < 64) {
-        const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(i) * 64 + tid);
+        const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(s) * 64 + tid);
         int64_t lt = -1;
         int part = 0;
         if (tok >= 0 && a.io.table != nullptr) {
@@ -835,7 +844,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                           ? bf16_bits_to_f32(__ldg(gb + (b * a.io.Ls + lt) * a.gate_ld + a.io.h0 + h))
                           : 0.0f;
       }
-      const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_t + i) * D + d) : 0.0f;
+      const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_sel + i) * D + d) : 0.0f;
       ROLE_MARK(3);
       mbar_wait(&bars[Ly::bLFull + ob], (it >> 1) & 1, ctl, 16);
       ROLE_MARK(0);

@@ -50,10 +50,11 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 }
 
 // ---------------------------------------------------------------------------
-// S2 (+ S3 pooling): sequence order [B, L, H, D] -> tile order [B, H, n_t, 64, D]
-// One CTA per (tile, head, batch) moves the tile of Q, K and V with 16-byte
-// loads/stores (each 256-byte token row is read by 16 consecutive threads),
-// keeps the three tiles in shared memory and, if asked, pools them there.
+// S2 (+ S3 pooling): sequence order [B, L, H, D] -> tile order [B, H, n_t, 64*kSub, D]
+// One CTA per (tile, head, batch) moves the tile of Q, K and V (64 rows, or 128
+// for 128-token tiles: kSub = 2) with 16-byte loads/stores (each 256-byte token
+// row is read by 16 consecutive threads), keeps the three tiles in shared memory
+// and, if asked, pools them there.
 //
 // kF8: Q and K are written as 8-bit E4M3 codes instead of bf16 copies, each
 // (token, head) row with its own binary32 scale s = amax / 448: code_d =
@@ -68,28 +69,29 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 // ---------------------------------------------------------------------------
 constexpr int kF8RowBytes = 128;
 
-template <int D, bool kParts, bool kF8>
+template <int D, bool kParts, bool kF8, int kSub>
 __global__ void __launch_bounds__(384) gather_pool_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     void* __restrict__ q_t, void* __restrict__ k_t, uint16_t* __restrict__ v_t, float* __restrict__ q_s,
     float* __restrict__ k_s, float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
     int n_t, const PartIO io) {
-  constexpr int kChunks = D / 8;                                // 16-byte chunks per row
-  constexpr int kIters = kF8 ? kTile / 8 : kTile * kChunks / 128;  // chunks each thread moves per tensor
+  constexpr int kRows = kTile * kSub;                             // rows of one tile
+  constexpr int kChunks = D / 8;                                  // 16-byte chunks per row
+  constexpr int kIters = kF8 ? kRows / 8 : kRows * kChunks / 128;  // chunks each thread moves per tensor
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);  // [3][64][D]
-  __shared__ int32_t tok_s[kTile];
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);  // [3][kRows][D]
+  __shared__ int32_t tok_s[kRows];
 
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool pool = (pq != nullptr);
-  if (threadIdx.x < kTile) tok_s[threadIdx.x] = tile_token[static_cast<int64_t>(tile) * kTile + threadIdx.x];
+  if (threadIdx.x < kRows) tok_s[threadIdx.x] = tile_token[static_cast<int64_t>(tile) * kRows + threadIdx.x];
   __syncthreads();
 
   // threads [128 t, 128 t + 128) move tensor t; all loads are issued before any store
   const int tsr = threadIdx.x >> 7, tl = threadIdx.x & 127;
   const uint16_t* src = (tsr == 0) ? q : (tsr == 1) ? k : v;
-  const int64_t tile_row0 = ((static_cast<int64_t>(b) * H + h) * n_t + tile) * kTile;
+  const int64_t tile_row0 = ((static_cast<int64_t>(b) * H + h) * n_t + tile) * kRows;
   // row and chunk of this thread's u-th chunk (false: an idle lane of an 8-bit row)
   auto chunk_of = [&](int u, int* r, int* c) -> bool {
     if constexpr (kF8) {
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   for (int u = 0; u < kIters; ++u) {
     int r, c;
     const bool active = chunk_of(u, &r, &c);
-    if (active && pool) reinterpret_cast<uint4*>(tiles + tsr * kTile * D)[r * kChunks + c] = val[u];
+    if (active && pool) reinterpret_cast<uint4*>(tiles + tsr * kRows * D)[r * kChunks + c] = val[u];
     if (!write_tiles) continue;
     if (codes) {
       float f[8];
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   const int n = tile_valid[tile];
   float* out = (tsr == 0) ? pq : (tsr == 1) ? pk : pv;
   for (int d = tl; d < D; d += 128) {
-    const uint16_t* col = tiles + tsr * kTile * D + d;
+    const uint16_t* col = tiles + tsr * kRows * D + d;
     float sum = 0.0f;
     for (int r = 0; r < n; ++r) sum = __fadd_rn(sum, bf16_bits_to_f32(col[r * D]));
     out[((static_cast<int64_t>(b) * H + h) * n_t + tile) * D + d] = __fdiv_rn(sum, static_cast<float>(n));
@@ -174,7 +176,8 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
 
 // ---------------------------------------------------------------------------
 // S3 pooling from tile order (the standalone entry point): one CTA per
-// (tile, head, batch), one thread per (tensor, d), rows added in tile order.
+// (tile, head, batch), one thread per (tensor, d), rows added in tile order;
+// `rows` = rows per tile (64 or 128).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(384) pool_tiles_kernel(const uint16_t* __restrict__ q_t,
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(384) pool_tiles_kernel(const uint16_t* __restr
                                                           float* __restrict__ pq, float* __restrict__ pk,
                                                           float* __restrict__ pv,
                                                           const int32_t* __restrict__ tile_valid, int H,
-                                                          int n_t) {
+                                                          int n_t, int rows) {
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t row0 = ((static_cast<int64_t>(b) * H + h) * n_t + tile);
   const int n = tile_valid[tile];
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(384) pool_tiles_kernel(const uint16_t* __restr
   float* outs[3] = {pq, pk, pv};
   for (int e = threadIdx.x; e < 3 * D; e += blockDim.x) {
     const int tsr = e / D, d = e - tsr * D;
-    const uint16_t* col = srcs[tsr] + row0 * kTile * D + d;
+    const uint16_t* col = srcs[tsr] + row0 * rows * D + d;
     float sum = 0.0f;
     for (int r = 0; r < n; ++r) sum = __fadd_rn(sum, bf16_bits_to_f32(__ldg(col + r * D)));
     outs[tsr][row0 * D + d] = __fdiv_rn(sum, static_cast<float>(n));

@@ -38,8 +38,7 @@ vsa_status fail(vsa_status s, const std::string& msg) {
     if (s_ != VSA_OK) return s_;      \
   } while (0)
 
-constexpr int kTile = VSA_TILE_SIZE;
-constexpr int kCube = 4;
+constexpr int kTile = VSA_TILE_SIZE;  // rows of a block in the tile-order copies and the attention kernel
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -53,6 +52,9 @@ struct Resolved {
   int64_t n_prefix = 0, n_video = 0;
   int32_t topk = 0;
   float scale = 0.0f;
+  int32_t tile = 64;             // tokens per tile (64 or 128)
+  int32_t ct = 4, ch = 4, cw = 4;  // video cube shape
+  int32_t sh = 0;                // log2(tile / 64): 64-row blocks per tile = 1 << sh
 };
 
 // topk = max(1, min(ceil((1 - sparsity) * V), V)), evaluated in binary64; 0 without video tiles.
@@ -77,8 +79,23 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
     return fail(VSA_ERR_UNSUPPORTED, "qk_fp8 reads 8-bit tile-order copies: it needs seq_tiles = 0");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
     return fail(VSA_ERR_UNSUPPORTED, "head_dim must be 64, 96 or 128, got " + std::to_string(g->head_dim));
-  if (g->tile_size != kTile)
-    return fail(VSA_ERR_UNSUPPORTED, "tile_size must be 64, got " + std::to_string(g->tile_size));
+  if (g->tile_size != 64 && g->tile_size != 128)
+    return fail(VSA_ERR_UNSUPPORTED, "tile_size must be 64 or 128, got " + std::to_string(g->tile_size));
+  r->tile = g->tile_size;
+  r->sh = (g->tile_size == 128) ? 1 : 0;
+  if (g->cube_t == 0 && g->cube_h == 0 && g->cube_w == 0) {
+    r->ct = 4;
+    r->ch = 4;
+    r->cw = (g->tile_size == 128) ? 8 : 4;
+  } else {
+    if (g->cube_t < 1 || g->cube_h < 1 || g->cube_w < 1 ||
+        static_cast<int64_t>(g->cube_t) * g->cube_h * g->cube_w != g->tile_size)
+      return fail(VSA_ERR_INVALID_ARG, "cube_t * cube_h * cube_w must equal tile_size (or all be 0)");
+    r->ct = g->cube_t;
+    r->ch = g->cube_h;
+    r->cw = g->cube_w;
+  }
+  if (g->seq_tiles && g->tile_size != 64) return fail(VSA_ERR_UNSUPPORTED, "seq_tiles needs 64-token tiles");
   if (!(g->sparsity >= 0.0 && g->sparsity <= 1.0)) return fail(VSA_ERR_INVALID_ARG, "sparsity must lie in [0, 1]");
   if (g->grid_t < 0 || g->grid_h < 0 || g->grid_w < 0) return fail(VSA_ERR_INVALID_ARG, "negative grid size");
   const bool any_zero = g->grid_t == 0 || g->grid_h == 0 || g->grid_w == 0;
@@ -120,53 +137,66 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   r->n_prefix = 0;
   for (int64_t n : r->segments) {
     prefix_tokens += n;
-    r->n_prefix += (n + kTile - 1) / kTile;
+    r->n_prefix += (n + r->tile - 1) / r->tile;
   }
   r->L = prefix_tokens + n_video_tokens;
   if (g->token_tags == nullptr && g->seq_len != 0 && g->seq_len != r->L)
     return fail(VSA_ERR_SHAPE, "seq_len " + std::to_string(g->seq_len) + " != prefix + T*H*W = " +
                                    std::to_string(r->L));
-  r->n_video = all_zero ? 0 : ((r->T + kCube - 1) / kCube) * ((r->Hg + kCube - 1) / kCube) *
-                                  ((r->W + kCube - 1) / kCube);
+  r->n_video = all_zero ? 0 : ((r->T + r->ct - 1) / r->ct) * ((r->Hg + r->ch - 1) / r->ch) *
+                                  ((r->W + r->cw - 1) / r->cw);
   const int64_t n_t = r->n_prefix + r->n_video;
   if (n_t > (1 << 24)) return fail(VSA_ERR_UNSUPPORTED, "too many tiles");
   r->topk = topk_for(g->sparsity, r->n_video);
   r->scale = (g->softmax_scale != 0.0f) ? g->softmax_scale
                                         : static_cast<float>(1.0 / std::sqrt(static_cast<double>(g->head_dim)));
   if (!(std::isfinite(r->scale)) || r->scale <= 0.0f) return fail(VSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
-  const int64_t rows = static_cast<int64_t>(g->batch) * g->heads * n_t * kTile;
-  if (rows >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "B*H*n_tiles*64 must stay below 2^31");
+  const int64_t rows = static_cast<int64_t>(g->batch) * g->heads * n_t * r->tile;
+  if (rows >= (int64_t(1) << 31)) return fail(VSA_ERR_UNSUPPORTED, "B*H*n_tiles*tile_size must stay below 2^31");
   if (static_cast<int64_t>(g->batch) * g->heads > 65535 || g->heads > 65535)
     return fail(VSA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
   return VSA_OK;
 }
 
-// Token table of every tile (-1 = pad), valid rows first.
+// Token table of every tile (-1 = pad), valid rows first: tok[tile * r.tile + row].
 void build_tables(const Resolved& r, std::vector<int32_t>* tok, std::vector<int32_t>* valid) {
-  const int64_t n_t = r.n_prefix + r.n_video;
-  tok->assign(static_cast<size_t>(n_t * kTile), -1);
+  const int64_t n_t = r.n_prefix + r.n_video, T = r.tile;
+  tok->assign(static_cast<size_t>(n_t * T), -1);
   valid->assign(static_cast<size_t>(n_t), 0);
   int64_t tile = 0, base = 0;
   for (int64_t n : r.segments) {
-    for (int64_t s = 0; s < n; s += kTile) {
-      const int64_t cnt = std::min<int64_t>(kTile, n - s);
-      for (int64_t j = 0; j < cnt; ++j) (*tok)[tile * kTile + j] = static_cast<int32_t>(base + s + j);
+    for (int64_t s = 0; s < n; s += T) {
+      const int64_t cnt = std::min<int64_t>(T, n - s);
+      for (int64_t j = 0; j < cnt; ++j) (*tok)[tile * T + j] = static_cast<int32_t>(base + s + j);
       (*valid)[tile++] = static_cast<int32_t>(cnt);
     }
     base += n;
   }
-  const int64_t ct = (r.T + 3) / 4, ch = (r.Hg + 3) / 4, cw = (r.W + 3) / 4;
-  for (int64_t a = 0; a < ct && r.n_video > 0; ++a)
-    for (int64_t bb = 0; bb < ch; ++bb)
-      for (int64_t c = 0; c < cw; ++c) {
+  const int64_t nct = (r.T + r.ct - 1) / r.ct, nch = (r.Hg + r.ch - 1) / r.ch, ncw = (r.W + r.cw - 1) / r.cw;
+  for (int64_t a = 0; a < nct && r.n_video > 0; ++a)
+    for (int64_t bb = 0; bb < nch; ++bb)
+      for (int64_t c = 0; c < ncw; ++c) {
         int cnt = 0;
-        const int64_t t1 = std::min(r.T, 4 * a + 4), h1 = std::min(r.Hg, 4 * bb + 4), w1 = std::min(r.W, 4 * c + 4);
-        for (int64_t t = 4 * a; t < t1; ++t)
-          for (int64_t h = 4 * bb; h < h1; ++h)
-            for (int64_t w = 4 * c; w < w1; ++w)
-              (*tok)[tile * kTile + cnt++] = static_cast<int32_t>(base + (t * r.Hg + h) * r.W + w);
+        const int64_t t1 = std::min(r.T, r.ct * a + r.ct), h1 = std::min(r.Hg, r.ch * bb + r.ch),
+                      w1 = std::min(r.W, r.cw * c + r.cw);
+        for (int64_t t = r.ct * a; t < t1; ++t)
+          for (int64_t h = r.ch * bb; h < h1; ++h)
+            for (int64_t w = r.cw * c; w < w1; ++w)
+              (*tok)[tile * T + cnt++] = static_cast<int32_t>(base + (t * r.Hg + h) * r.W + w);
         (*valid)[tile++] = cnt;
       }
+}
+
+// Key mask of every 64-row block of the tile-order copies: the low `valid rows of the block` bits
+// (a tile holds its valid rows first, so block j of a tile holds min(64, max(0, valid - 64 j))).
+void build_block_masks(const Resolved& r, const std::vector<int32_t>& valid, std::vector<uint64_t>* mask) {
+  const int sub = 1 << r.sh;
+  mask->assign(valid.size() * sub, 0);
+  for (size_t i = 0; i < valid.size(); ++i)
+    for (int j = 0; j < sub; ++j) {
+      const int v = std::min(64, std::max(0, valid[i] - 64 * j));
+      (*mask)[i * sub + j] = v >= 64 ? ~0ull : ((1ull << v) - 1);
+    }
 }
 
 // Tables for reading tiles straight from sequence order with TMA: a tile is one box, a 64-token run of
@@ -175,23 +205,20 @@ void build_tables(const Resolved& r, std::vector<int32_t>* tok, std::vector<int3
 // ((t - t0)*4 + (y - y0))*4 + (x - x0); rows outside the segment or the grid are masked.
 //   row_token[tile*64 + r]: token of box row r, -1 if masked
 //   mask_seq[tile]: bit r set when box row r is a token of the tile
-//   mask_tiled[tile]: the low tile_valid bits (tile-order copies hold the valid rows first)
 //   coord[tile]: {0, first token, 0, 0} for a prefix run, {1, x0, y0, t0} for a cube
-void build_seq_tables(const Resolved& r, const std::vector<int32_t>& valid, std::vector<int32_t>* row_token,
-                      std::vector<uint64_t>* mask_seq, std::vector<uint64_t>* mask_tiled, std::vector<int32_t>* coord) {
+// (64-token tiles only.)
+void build_seq_tables(const Resolved& r, const std::vector<uint64_t>& mask_tiled, std::vector<int32_t>* row_token,
+                      std::vector<uint64_t>* mask_seq, std::vector<int32_t>* coord) {
   const int64_t n_t = r.n_prefix + r.n_video;
   row_token->assign(static_cast<size_t>(n_t * kTile), -1);
   mask_seq->assign(static_cast<size_t>(n_t), 0);
-  mask_tiled->assign(static_cast<size_t>(n_t), 0);
   coord->assign(static_cast<size_t>(n_t * 4), 0);
-  for (int64_t i = 0; i < n_t; ++i)
-    (*mask_tiled)[i] = valid[i] >= 64 ? ~0ull : ((1ull << valid[i]) - 1);
   int64_t tile = 0, base = 0;
   for (int64_t n : r.segments) {
     for (int64_t s = 0; s < n; s += kTile) {
       const int64_t cnt = std::min<int64_t>(kTile, n - s);
       for (int64_t j = 0; j < cnt; ++j) (*row_token)[tile * kTile + j] = static_cast<int32_t>(base + s + j);
-      (*mask_seq)[tile] = (*mask_tiled)[tile];
+      (*mask_seq)[tile] = mask_tiled[tile];
       (*coord)[tile * 4 + 1] = static_cast<int32_t>(base + s);
       ++tile;
     }
@@ -223,11 +250,13 @@ void build_seq_tables(const Resolved& r, const std::vector<int32_t>& valid, std:
 
 // seq_tiles: no tile-order copies (their regions are empty).
 // qk_fp8: q_t and k_t hold 8-bit codes, 128 bytes per row whatever D, and q_s, k_s one float per row.
-vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t V, int64_t topk, bool seq_tiles,
+// tile: tokens per tile (the copies hold n_t * tile rows per (b, h)).
+vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t tile, int64_t V, int64_t topk,
+                                 bool seq_tiles,
                                  bool qk_fp8) {
   vsa_workspace_layout w{};
   size_t off = 0;
-  const size_t rows = static_cast<size_t>(B * H * n_t * kTile);
+  const size_t rows = static_cast<size_t>(B * H * n_t * tile);
   const size_t tiles = seq_tiles ? 0 : rows * D * 2;
   const size_t qk_tiles = qk_fp8 ? rows * vsa::kF8RowBytes : tiles;
   const size_t pooled = static_cast<size_t>(B * H * n_t * D * 4);
@@ -381,7 +410,8 @@ struct vsa_plan_s {
   std::vector<int32_t> tile_token, tile_valid;
   int32_t* d_tile_token = nullptr;
   int32_t* d_tile_valid = nullptr;
-  // tables for TMA loads straight from sequence order (build_seq_tables)
+  // key masks of the 64-row blocks of the tile-order copies (build_block_masks), and the tables for
+  // TMA loads straight from sequence order (build_seq_tables, 64-token tiles)
   std::vector<int32_t> row_token, coord;
   std::vector<uint64_t> mask_seq, mask_tiled;
   int32_t* d_row_token = nullptr;
@@ -457,7 +487,7 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
-  const size_t smem = pool ? static_cast<size_t>(3) * kTile * p->D * 2 : 0;
+  const size_t smem = pool ? static_cast<size_t>(3) * p->r.tile * p->D * 2 : 0;
   dim3 grid(p->n_t, p->H, p->B);
   const auto* qq = static_cast<const uint16_t*>(q);
   const auto* kk = static_cast<const uint16_t*>(k);
@@ -472,9 +502,12 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
     const bool parts = pio.table != nullptr;
+    auto by_tile = [&](auto k64, auto k128) { return p->r.sh ? launch(k128) : launch(k64); };
     if (p->qk_fp8)
-      return parts ? launch(vsa::gather_pool_kernel<D, true, true>) : launch(vsa::gather_pool_kernel<D, false, true>);
-    return parts ? launch(vsa::gather_pool_kernel<D, true, false>) : launch(vsa::gather_pool_kernel<D, false, false>);
+      return parts ? by_tile(vsa::gather_pool_kernel<D, true, true, 1>, vsa::gather_pool_kernel<D, true, true, 2>)
+                   : by_tile(vsa::gather_pool_kernel<D, false, true, 1>, vsa::gather_pool_kernel<D, false, true, 2>);
+    return parts ? by_tile(vsa::gather_pool_kernel<D, true, false, 1>, vsa::gather_pool_kernel<D, true, false, 2>)
+                 : by_tile(vsa::gather_pool_kernel<D, false, false, 1>, vsa::gather_pool_kernel<D, false, false, 2>);
   }));
   return launch_check("gather_pool");
 }
@@ -488,7 +521,7 @@ vsa_status run_pool(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   const auto* c = static_cast<const uint16_t*>(vt);
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
-    vsa::pool_tiles_kernel<D><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t);
+    vsa::pool_tiles_kernel<D><<<grid, 384, 0, s>>>(a, b, c, pq, pk, pv, p->d_tile_valid, p->H, p->n_t, p->r.tile);
     return VSA_OK;
   }));
   return launch_check("pool_tiles");
@@ -536,7 +569,9 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
                     const float* ks = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
-  const int64_t rows = static_cast<int64_t>(p->B) * p->H * p->n_t * kTile;
+  // the kernel works in 64-row blocks: one per tile, or two per 128-token tile
+  const int64_t n_rb = static_cast<int64_t>(p->n_t) << p->r.sh;
+  const int64_t rows = static_cast<int64_t>(p->B) * p->H * n_rb * kTile;
   CUtensorMap mq{}, mk{}, mv{};
   vsa::SeqMaps sm{};
   if (seq) {
@@ -574,11 +609,12 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.q_scale = qs;
   a.k_scale = ks;
   a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
-  a.n_t = p->n_t;
+  a.n_t = static_cast<int>(n_rb);
+  a.sub_shift = p->r.sh;
   a.P = p->P;
   a.topk = p->topk;
   a.scale_log2 = static_cast<float>(static_cast<double>(p->r.scale) * 1.4426950408889634);
-  a.n_items = static_cast<int64_t>(p->B) * p->H * p->n_t;
+  a.n_items = static_cast<int64_t>(p->B) * p->H * n_rb;
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
   // the item counter of the persistent schedule starts at zero for every launch
   VSA_CUDA_TRY(cudaMemsetAsync(a.sched, 0, sizeof(int), s));
@@ -638,7 +674,7 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->d_status = p->d_status;
   q->seq_tiles = p->seq_tiles;
   q->qk_fp8 = p->qk_fp8;
-  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->V, q->topk, q->seq_tiles, q->qk_fp8);
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk, q->seq_tiles, q->qk_fp8);
   q->owns_device = false;
   return q;
 }
@@ -654,7 +690,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
   h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
   h.fwd = 0;
-  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->V, p->topk, p->seq_tiles, p->qk_fp8).total);
+  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk, p->seq_tiles, p->qk_fp8).total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
     off += 4 * h.chunk_bytes;  // q, k, v, out
@@ -719,8 +755,10 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->seq_len = r.L;
   d->softmax_scale = r.scale;
   d->workspace_bytes =
-      make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.n_video, r.topk, g->seq_tiles != 0, g->qk_fp8 != 0).total;
+      make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.tile, r.n_video, r.topk, g->seq_tiles != 0,
+                  g->qk_fp8 != 0).total;
   d->selected_pairs = r.n_video * (r.n_prefix + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
+  d->tile_size = r.tile;
 }
 
 }  // namespace
@@ -785,10 +823,11 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   p->V = static_cast<int32_t>(r.n_video);
   p->topk = r.topk;
   build_tables(r, &p->tile_token, &p->tile_valid);
-  build_seq_tables(r, p->tile_valid, &p->row_token, &p->mask_seq, &p->mask_tiled, &p->coord);
+  build_block_masks(r, p->tile_valid, &p->mask_tiled);
+  if (r.tile == kTile) build_seq_tables(r, p->mask_tiled, &p->row_token, &p->mask_seq, &p->coord);
   p->seq_tiles = g->seq_tiles != 0;
   p->qk_fp8 = g->qk_fp8 != 0;
-  p->ws = make_layout(p->B, p->H, p->D, p->n_t, p->V, p->topk, p->seq_tiles, p->qk_fp8);
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk, p->seq_tiles, p->qk_fp8);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
@@ -803,10 +842,12 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   const size_t tok_bytes = std::max<size_t>(4, p->tile_token.size() * 4);
   const size_t val_bytes = std::max<size_t>(4, p->tile_valid.size() * 4);
   const size_t mask_bytes = std::max<size_t>(8, p->mask_seq.size() * 8);
+  const size_t block_mask_bytes = std::max<size_t>(8, p->mask_tiled.size() * 8);
   const size_t coord_bytes = std::max<size_t>(16, p->coord.size() * 4);
   if (cudaMalloc(&p->d_tile_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_tile_valid, val_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_row_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_coord, coord_bytes) != cudaSuccess ||
-      cudaMalloc(&p->d_mask_seq, mask_bytes) != cudaSuccess || cudaMalloc(&p->d_mask_tiled, mask_bytes) != cudaSuccess ||
+      cudaMalloc(&p->d_mask_seq, mask_bytes) != cudaSuccess ||
+      cudaMalloc(&p->d_mask_tiled, block_mask_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
@@ -843,6 +884,7 @@ vsa_status vsa_plan_info(vsa_plan p, vsa_plan_dims* out) {
   out->softmax_scale = p->r.scale;
   out->workspace_bytes = p->ws.total;
   out->selected_pairs = static_cast<int64_t>(p->V) * (p->P + p->topk) + static_cast<int64_t>(p->P) * p->n_t;
+  out->tile_size = p->r.tile;
   return VSA_OK;
 }
 

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VSA_TILE_SIZE 64 /* tokens per tile; video tiles are 4x4x4 cubes */
+#define VSA_TILE_SIZE 64 /* tokens per tile by default; video tiles are then 4x4x4 cubes */
 
 typedef uint16_t vsa_bf16; /* raw bfloat16 bits */
 
@@ -91,7 +91,10 @@ typedef struct vsa_geometry {
   int64_t seq_len;           /* L: required with tags; checked otherwise */
   int32_t video_tag;         /* tag value of the video tokens (tags only) */
   int32_t grid_t, grid_h, grid_w; /* post-patchify video grid; 0 = no video */
-  int32_t tile_size;         /* must be 64 */
+  int32_t tile_size;         /* tokens per tile: 64, or 128 (the OmniRef variant: "FastH3
+                                OmniRef inference", section "The Blackwell stack").  A prefix
+                                tile is a segment-pure run of up to tile_size tokens, a video
+                                tile a cube_t x cube_h x cube_w block of the grid. */
   double sparsity;           /* in [0, 1] */
   float softmax_scale;       /* 0 => (float)(1 / sqrt((double)head_dim)) */
   int32_t gate_per_channel;  /* 0: gate [B, L, H], one scalar per token and head;
@@ -99,7 +102,7 @@ typedef struct vsa_geometry {
   int32_t seq_tiles;         /* 0: vsa_forward copies Q/K/V to tile order first (faster on B200);
                                 1: the attention reads each tile straight from sequence order
                                 with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
-                                by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4 */
+                                by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4, 64-token tiles */
   int32_t qk_fp8;            /* 0: the fine branch's logits use the bf16 Q and K;
                                 1: 8-bit Q/K: each (token, head) row of Q and K is quantised to
                                 OCP FP8 E4M3 codes with one binary32 scale s = amax / 448
@@ -112,6 +115,9 @@ typedef struct vsa_geometry {
                                 "Fallbacks" (8-bit per-token Q/K with bf16 P.V); "FastH3 NVFP4
                                 on RTX PRO 6000 (sm_120)", multi-GPU notes (one FP8 scale per
                                 token and head). */
+  int32_t cube_t, cube_h, cube_w; /* video cube shape, product = tile_size; all 0 = the default:
+                                     4x4x4 for 64 tokens (the method's), 4x4x8 for 128 (the
+                                     pages do not state it: the 64-token cube doubled along w) */
 } vsa_geometry;
 
 typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
@@ -127,6 +133,7 @@ typedef struct vsa_plan_dims {
   size_t workspace_bytes; /* device scratch vsa_forward needs */
   int64_t selected_pairs; /* (query tile, key tile) pairs per (b, h):
                              V * (P + topk) + P * n_tiles */
+  int32_t tile_size;      /* tokens per tile (64 or 128) */
 } vsa_plan_dims;
 
 /* ---- S1: tile plan (host) ------------------------------------------------
@@ -144,7 +151,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out);
 /* Resolved sizes.  Host only; never blocks. */
 vsa_status vsa_plan_info(vsa_plan p, vsa_plan_dims* out);
 
-/* Host copies of the plan's tables: tile_token[n_tiles * 64] (sequence index
+/* Host copies of the plan's tables: tile_token[n_tiles * tile_size] (sequence index
  * of each tile row, -1 for a pad) and tile_valid[n_tiles] (valid rows).
  * Either pointer may be NULL.  Host only. */
 vsa_status vsa_plan_tables(vsa_plan p, int32_t* tile_token, int32_t* tile_valid);
@@ -153,7 +160,7 @@ vsa_status vsa_plan_tables(vsa_plan p, int32_t* tile_token, int32_t* tile_valid)
 vsa_status vsa_plan_query(const vsa_geometry* g, vsa_plan_dims* out);
 
 /* The token table a plan would upload, computed on the host without a device:
- * tile_token[n_tiles * 64] and tile_valid[n_tiles] (caller-allocated host
+ * tile_token[n_tiles * tile_size] and tile_valid[n_tiles] (caller-allocated host
  * arrays, sized from vsa_plan_query).  Either pointer may be NULL. */
 vsa_status vsa_plan_tables_host(const vsa_geometry* g, int32_t* tile_token, int32_t* tile_valid);
 

@@ -50,6 +50,8 @@ class Workload:
     gate_std: float = 0.1
     description: str = ""
     gate_per_channel: bool = False  # gate [B, L, H*D] (one per channel) instead of [B, L, H]
+    tile: int = 64  # tokens per attention tile (64, or 128 for the OmniRef-style variant)
+    cube: tuple = None  # video cube (t, h, w) of a tile; None = the plan's default for `tile`
 
     @property
     def seq_len(self) -> int:
@@ -69,6 +71,9 @@ WORKLOADS = {
                  description="1344x768-shaped: 56 heads, D=128, text 512 + audio 768, video 24x48x64, sparsity 0.8"),
         Workload("768p_s0.9", 1, 56, 128, (512, 0, 768), (24, 48, 64), 0.9, structured=True,
                  description="1344x768-shaped: 56 heads, D=128, text 512 + audio 768, video 24x48x64, sparsity 0.9"),
+        Workload("768p_t128_s0.9", 1, 56, 128, (512, 0, 768), (24, 48, 64), 0.9, structured=True, tile=128,
+                 description="1344x768-shaped with 128-token tiles (4x4x8 cubes): 56 heads, D=128, text 512 + "
+                             "audio 768, video 24x48x64, sparsity 0.9"),
     ]
 }
 

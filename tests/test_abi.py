@@ -46,7 +46,7 @@ def test_exports_every_declared_symbol(vsa):
 
 def _kw(w, **over):
     kw = dict(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-              sparsity=w.sparsity)
+              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube)
     kw.update(over)
     return kw
 
@@ -55,7 +55,7 @@ def _kw(w, **over):
 def test_plan_matches_oracle_geometry(vsa, oracle_mod, name):
     w = synth.workload(name)
     d = vsa.vsa_plan_query(**_kw(w))
-    geo = oracle_mod.geometry(w.segments, w.grid)
+    geo = oracle_mod.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube)
     assert (d["n_tiles"], d["n_prefix_tiles"], d["n_video_tiles"]) == (geo.n_tiles, geo.n_prefix, geo.n_video)
     assert d["topk"] == oracle_mod.topk_count(w.sparsity, geo.n_video)
     assert d["seq_len"] == w.seq_len
@@ -103,7 +103,9 @@ def test_token_tags_match_segments(vsa):
     (dict(sparsity=1.5), "VSA_ERR_INVALID_ARG"),
     (dict(sparsity=-0.1), "VSA_ERR_INVALID_ARG"),
     (dict(sparsity=float("nan")), "VSA_ERR_INVALID_ARG"),
-    (dict(tile_size=128), "VSA_ERR_UNSUPPORTED"),
+    (dict(tile_size=32), "VSA_ERR_UNSUPPORTED"),
+    (dict(tile_size=128, cube=(4, 4, 4)), "VSA_ERR_INVALID_ARG"),
+    (dict(tile_size=128, seq_tiles=True), "VSA_ERR_UNSUPPORTED"),
     (dict(head_dim=80), "VSA_ERR_UNSUPPORTED"),
     (dict(grid=(8, 0, 8)), "VSA_ERR_SHAPE"),
     (dict(batch=0), "VSA_ERR_INVALID_ARG"),
@@ -162,3 +164,23 @@ def test_qk_fp8_workspace_and_limits(vsa):
 
     d = vsa.PlanDims()
     assert vsa.load_library().vsa_plan_query(ctypes.byref(g), ctypes.byref(d)) == 1  # VSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("segments,grid,cube", [
+    ((512, 0, 768), (24, 48, 64), None),
+    ((384, 0, 384), (8, 30, 56), (8, 4, 4)),
+    ((40, 0, 24), (8, 8, 8), None),
+    ((129, 3), (5, 6, 9), (2, 8, 8)),
+])
+def test_plan_tile128_matches_oracle_geometry(vsa, oracle_mod, segments, grid, cube):
+    """128-token tiles: the host token table equals the oracle's, and the workspace holds 128-row tiles."""
+    kw = dict(batch=1, heads=2, head_dim=128, segments=segments, grid=grid, sparsity=0.9, tile_size=128, cube=cube)
+    d = vsa.vsa_plan_query(**kw)
+    geo = oracle_mod.geometry(segments, grid, tile=128, cube=cube)
+    assert (d["n_tiles"], d["n_prefix_tiles"], d["n_video_tiles"], d["tile_size"]) == (
+        geo.n_tiles, geo.n_prefix, geo.n_video, 128)
+    assert d["topk"] == oracle_mod.topk_count(0.9, geo.n_video)
+    tok, val = vsa.vsa_plan_tables_host(**kw)
+    assert np.array_equal(tok, geo.tile_token) and np.array_equal(val, geo.tile_valid)
+    d64 = vsa.vsa_plan_query(**dict(kw, tile_size=64, cube=None))
+    assert d["workspace_bytes"] > 0 and d64["n_tiles"] >= d["n_tiles"]
