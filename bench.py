@@ -364,7 +364,7 @@ def run_vsa(args, w, world, rank, local):
         "stage_ms": stage_ms, "roofline": roofline,
         "e2e": {"value": world * flops_call / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "head_chunk": vsa.default_head_chunk(w.heads)},
+                "head_chunk": vsa.default_head_chunk(w.heads, w.head_dim)},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }

@@ -296,14 +296,19 @@ def alloc_workspace(plan, device=None) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda", torch.cuda.current_device()))
 
 
-def default_head_chunk(heads: int) -> int:
-    """Heads per chunk of the host pipeline: about 16 chunks, so that the forward and copy-back of
-    the last chunk, which nothing overlaps, are short (56 heads: 14 chunks of 4)."""
-    return max(1, -(-heads // 16))
+def default_head_chunk(heads: int, head_dim: int = 128) -> int:
+    """Heads per chunk of the host pipeline.  Small chunks keep the forward and copy-back of the last
+    chunk, which nothing overlaps, short; but each chunk's copies are strided rows of chunk*head_dim
+    bf16 values, and rows under 512 bytes copy slowly (measured at 1344x768, 56 heads, D = 128:
+    1 head per chunk 104.7 ms, 2: 62.7 ms, 4: 64.2 ms, 8: 67.5 ms, 14: 76.2 ms).  So: the smallest
+    chunk with rows of at least 512 bytes, and at most 32 chunks."""
+    rows = -(-512 // (2 * head_dim))
+    return max(1, min(heads, max(rows, -(-heads // 32))))
 
 
 def host_workspace_bytes(plan, head_chunk=None) -> int:
-    hc = default_head_chunk(plan.geometry["heads"]) if head_chunk is None else int(head_chunk)
+    g = plan.geometry
+    hc = default_head_chunk(g["heads"], g["head_dim"]) if head_chunk is None else int(head_chunk)
     n = ctypes.c_size_t()
     _check(load_library().vsa_forward_host_workspace(plan.handle, hc, ctypes.byref(n)), "vsa_forward_host_workspace")
     return n.value
@@ -327,7 +332,8 @@ def vsa_forward_host(plan, q, k, v, gate, out=None, workspace=None, head_chunk=N
     neighbouring chunks (vsa_forward_host).  Without a workspace, one is
     allocated on first use and kept on the plan.  Returns once the stream has
     drained."""
-    hc = default_head_chunk(plan.geometry["heads"]) if head_chunk is None else int(head_chunk)
+    g = plan.geometry
+    hc = default_head_chunk(g["heads"], g["head_dim"]) if head_chunk is None else int(head_chunk)
     need = host_workspace_bytes(plan, hc)
     if workspace is None:
         cached = getattr(plan, "_host_ws", None)

@@ -209,13 +209,15 @@ __global__ void __launch_bounds__(384) pool_tiles_kernel(const uint16_t* __restr
 constexpr int kScoreBlk = 128;
 constexpr int kScoreDk = 16;
 
-__global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ pq, const float* __restrict__ pk,
+__global__ void __launch_bounds__(256, 2) scores_kernel(const float* __restrict__ pq, const float* __restrict__ pk,
                                                       float* __restrict__ S, int n_t, int D, float scale) {
   __shared__ __align__(16) float As[2][kScoreDk][kScoreBlk];
   __shared__ __align__(16) float Bs[2][kScoreDk][kScoreBlk];
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * kScoreBlk, j0 = blockIdx.x * kScoreBlk;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 8 x 8 outputs: rows ty + 16a, cols tx + 16c
+  // 8 x 8 outputs per thread: rows 8 ty + a; columns 4 tx + c and 64 + 4 tx + c (c < 4), so that the
+  // float4 reads of a quarter-warp hit distinct banks
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const float* A = pq + static_cast<int64_t>(bh) * n_t * D;
   const float* Bm = pk + static_cast<int64_t>(bh) * n_t * D;
   float acc[8][8];
@@ -257,10 +259,10 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ p
 #pragma unroll
     for (int dd = 0; dd < kScoreDk; ++dd) {
       float av[8], bv[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) av[a] = As[buf][dd][ty + 16 * a];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) bv[c] = Bs[buf][dd][tx + 16 * c];
+      *reinterpret_cast<float4*>(av) = *reinterpret_cast<const float4*>(&As[buf][dd][8 * ty]);
+      *reinterpret_cast<float4*>(av + 4) = *reinterpret_cast<const float4*>(&As[buf][dd][8 * ty + 4]);
+      *reinterpret_cast<float4*>(bv) = *reinterpret_cast<const float4*>(&Bs[buf][dd][4 * tx]);
+      *reinterpret_cast<float4*>(bv + 4) = *reinterpret_cast<const float4*>(&Bs[buf][dd][64 + 4 * tx]);
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -271,11 +273,11 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ p
   }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    const int i = i0 + ty + 16 * a;
+    const int i = i0 + 8 * ty + a;
     if (i >= n_t) continue;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const int j = j0 + tx + 16 * c;
+      const int j = j0 + (c < 4 ? 4 * tx + c : 64 + 4 * tx + c - 4);
       if (j < n_t) S[(static_cast<int64_t>(bh) * n_t + i) * n_t + j] = __fmul_rn(acc[a][c], scale);
     }
   }
@@ -376,11 +378,12 @@ __global__ void __launch_bounds__(256) gate_any_kernel(const uint16_t* __restric
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
+__global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
                                                         float* __restrict__ o_c, int n_t,
                                                         const int* __restrict__ gate_nonzero) {
   if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
-  constexpr int kCols = D / 16;  // columns per thread: tx + 16 c
+  constexpr int kCols = D / 16;  // columns per thread (4, 6 or 8)
+  static_assert(kCols == 4 || kCols == 6 || kCols == 8, "head_dim 64, 96 or 128");
   __shared__ float m_s[kCompRows], l_s[kCompRows];
   __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
   __shared__ __align__(16) float PV_s[kCompJ][D];
@@ -404,7 +407,10 @@ __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__
   const int wi = i0 + wr;
   const float wm = m_s[wr];
   float lsum = 0.0f;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // outputs: rows ty + 16a, cols tx + 16c
+  // outputs per thread: rows 8 ty + a; columns 4 tx + c (c < 4) and 64 + (kCols - 4) tx + c - 4 (c >= 4),
+  // so that the vector reads of a quarter-warp hit distinct banks
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  auto out_col = [&](int c) { return c < 4 ? 4 * tx + c : 64 + (kCols - 4) * tx + (c - 4); };
   float acc[8][kCols];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
@@ -429,10 +435,13 @@ __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__
 #pragma unroll 4
     for (int jj = 0; jj < kCompJ; ++jj) {
       float wv[8], pvv[kCols];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) wv[a] = W_s[jj][ty + 16 * a];
-#pragma unroll
-      for (int c = 0; c < kCols; ++c) pvv[c] = PV_s[jj][tx + 16 * c];
+      *reinterpret_cast<float4*>(wv) = *reinterpret_cast<const float4*>(&W_s[jj][8 * ty]);
+      *reinterpret_cast<float4*>(wv + 4) = *reinterpret_cast<const float4*>(&W_s[jj][8 * ty + 4]);
+      *reinterpret_cast<float4*>(pvv) = *reinterpret_cast<const float4*>(&PV_s[jj][4 * tx]);
+      if constexpr (kCols == 8)
+        *reinterpret_cast<float4*>(pvv + 4) = *reinterpret_cast<const float4*>(&PV_s[jj][64 + 4 * tx]);
+      else if constexpr (kCols == 6)
+        *reinterpret_cast<float2*>(pvv + 4) = *reinterpret_cast<const float2*>(&PV_s[jj][64 + 2 * tx]);
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -445,12 +454,12 @@ __global__ void __launch_bounds__(256) compress_kernel(const float* __restrict__
   __syncthreads();
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    const int r = ty + 16 * a, i = i0 + r;
+    const int r = 8 * ty + a, i = i0 + r;
     if (i >= n_t) continue;
     const float inv = 1.0f / l_s[r];
 #pragma unroll
     for (int c = 0; c < kCols; ++c)
-      o_c[(static_cast<int64_t>(bh) * n_t + i) * D + tx + 16 * c] = acc[a][c] * inv;
+      o_c[(static_cast<int64_t>(bh) * n_t + i) * D + out_col(c)] = acc[a][c] * inv;
   }
 }
 

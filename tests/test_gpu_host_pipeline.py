@@ -6,7 +6,7 @@ top-k, compression and the attention items all work per (b, h)), so the
 chunked result must be bit-identical to vsa_forward on the same inputs.
 The cases cover a chunk that divides the heads, one that leaves a remainder
 chunk (a second head-slice plan), one chunk holding every head, the default
-of about 16 chunks, pageable host memory, a second call reusing the pipeline,
+(the smallest chunk with 512-byte copy rows), pageable host memory, a second call reusing the pipeline,
 and the argument errors."""
 import ctypes
 
@@ -69,7 +69,7 @@ def test_host_pipeline_matches_device_forward(vsa, name, chunk):
 
 
 def test_host_pipeline_1344x768_default_chunks(vsa):
-    """The bench workload in the e2e configuration (14 chunks of 4 heads)."""
+    """The bench workload in the e2e configuration (28 chunks of 2 heads)."""
     w = synth.workload("768p_s0.9")
     x = synth.make_inputs(w, seed=0, device="cuda")
     plan = plan_for(vsa, w)
