@@ -57,17 +57,21 @@ def _load():
         lib.vsa_oracle_scores.argtypes = [P, P, i32, i32, i32, f32, P]
         lib.vsa_oracle_select.argtypes = [P, i32, i32, i32, i32, P]
         lib.vsa_oracle_compress.argtypes = [P, P, i32, i32, i32, P]
-        lib.vsa_oracle_fine.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P, f64, P,
-                                        P]
-        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P,
-                                              f64, i32, P, P]
+        lib.vsa_oracle_fine.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, i32, i32, P, P, P,
+                                        f64, P, P]
+        lib.vsa_oracle_fine_tiles.argtypes = [P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, i32, P, i32, i32, P,
+                                              P, P, f64, i32, P, P]
+        lib.vsa_oracle_select_ref.argtypes = [P, i32, i32, i32, P, i32, i32, P]
+        lib.vsa_oracle_ref_count.argtypes = [f64, i32]
+        lib.vsa_oracle_ref_count.restype = i32
         lib.vsa_oracle_e4m3_value.argtypes = [i32]
         lib.vsa_oracle_e4m3_value.restype = f64
         lib.vsa_oracle_e4m3_round.argtypes = [f32]
         lib.vsa_oracle_e4m3_round.restype = i32
         lib.vsa_oracle_e4m3_round_array.argtypes = [P, i64, P]
         lib.vsa_oracle_quant_e4m3.argtypes = [P, i64, i32, P, P]
-        lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, i32, P, P, P, f64, P]
+        lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, f64,
+                                               P]
         lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, P, P, P, P]
         _lib = lib
     return _lib
@@ -96,6 +100,11 @@ class Geometry:
     tile_valid: np.ndarray  # [n_tiles] int32
     tile: int = 64
     cube: tuple = (4, 4, 4)
+    is_ref: np.ndarray = None  # [n_prefix] uint8: 1 for a tile of a reference segment (R18), or None
+
+    @property
+    def n_ref(self) -> int:
+        return 0 if self.is_ref is None else int(self.is_ref.sum())
 
     @property
     def seq_len(self) -> int:
@@ -107,7 +116,8 @@ def default_cube(tile: int) -> tuple:
     return {64: (4, 4, 4), 128: (4, 4, 8)}[int(tile)]
 
 
-def geometry(segments, grid, tile=64, cube=None) -> Geometry:
+def geometry(segments, grid, tile=64, cube=None, ref_segments=None) -> Geometry:
+    """ref_segments: one flag per prefix segment, true for a reference segment (R18), or None."""
     lib = _load()
     seg = np.asarray(segments, dtype=np.int32)
     T, H, W = (int(x) for x in grid)
@@ -120,12 +130,23 @@ def geometry(segments, grid, tile=64, cube=None) -> Geometry:
     tok = np.empty((nt.value, int(tile)), np.int32)
     val = np.empty((nt.value,), np.int32)
     lib.vsa_oracle_tiles(len(seg), _p(seg), T, H, W, int(tile), ct, ch, cw, _p(tok), _p(val))
+    is_ref = None
+    if ref_segments is not None:
+        assert len(ref_segments) == len(seg)
+        is_ref = np.concatenate([np.full(-(-int(n) // int(tile)), int(bool(f)), np.uint8)
+                                 for n, f in zip(seg, ref_segments)] + [np.zeros(0, np.uint8)])
+        assert len(is_ref) == npf.value
     return Geometry(tuple(int(s) for s in segments), (T, H, W), nt.value, npf.value, nv.value, tok, val, int(tile),
-                    (ct, ch, cw))
+                    (ct, ch, cw), is_ref)
 
 
 def topk_count(sparsity: float, n_video: int) -> int:
     return int(_load().vsa_oracle_topk_count(float(sparsity), int(n_video)))
+
+
+def ref_count(keep: float, n_ref: int) -> int:
+    """Reference tiles kept per video query tile (R18)."""
+    return int(_load().vsa_oracle_ref_count(float(keep), int(n_ref)))
 
 
 def default_scale(head_dim: int) -> float:
@@ -153,11 +174,18 @@ def scores(pq: np.ndarray, pk: np.ndarray, scale: float) -> np.ndarray:
     return S
 
 
-def select(S: np.ndarray, n_prefix: int, k: int) -> np.ndarray:
-    """S: [B, H, n_t, n_t] -> idx [B, H, V, k] int32 (global tile indices, ascending)."""
+def select(S: np.ndarray, n_prefix: int, k: int, is_ref=None, kr: int = 0) -> np.ndarray:
+    """S: [B, H, n_t, n_t] -> idx [B, H, V, k] int32 (global tile indices, ascending); with reference
+    tiles (is_ref, R18) [B, H, V, kr + k]: the kr kept reference tiles, then the k video tiles."""
     S = _c(S, np.float32)
     B, H, n_t, _ = S.shape
     V = n_t - n_prefix
+    if is_ref is not None:
+        is_ref = _c(np.asarray(is_ref, np.uint8), np.uint8)
+        idx = np.empty((B, H, V, kr + k), np.int32)
+        if _load().vsa_oracle_select_ref(_p(S), B * H, n_t, n_prefix, _p(is_ref), kr, k, _p(idx)):
+            raise ValueError("NaN pooled score")
+        return idx
     idx = np.empty((B, H, V, k), np.int32)
     if _load().vsa_oracle_select(_p(S), B * H, n_t, n_prefix, k, _p(idx)):
         raise ValueError("NaN pooled score")
@@ -186,6 +214,13 @@ def _qk8_args(qk8, shape):
     return (qc, qs, kc, ks)
 
 
+def _ref_args(geo: Geometry, idx, topk: int):
+    """(reference flags, kr) for the C fine branch: an idx row holds kr reference tiles, then topk (R18)."""
+    if geo.is_ref is None:
+        return None, 0
+    return _c(geo.is_ref, np.uint8), int(np.shape(idx)[-1]) - int(topk)
+
+
 def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=None) -> np.ndarray:
     """List formulation of the fine branch -> o_f [B, L, H, D] float64 (NaN where not computed).
     qk8 = (q codes, q scales, k codes, k scales) from quant_e4m3: the logits use those instead of q, k."""
@@ -196,8 +231,9 @@ def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=No
         todo = _c(todo.astype(np.uint8), np.uint8)
     q8 = _qk8_args(qk8, q.shape)
     out = np.full((B, L, H, D), np.nan, np.float64)
+    ref, kr = _ref_args(geo, idx, topk)
     _load().vsa_oracle_fine(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles, geo.n_prefix, topk,
-                            geo.tile,
+                            _p(ref), kr, geo.tile,
                             _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(todo), _p(out))
     return out
 
@@ -211,9 +247,10 @@ def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items, qk8=
     idx = _c(idx, np.int32)
     items = _c(np.asarray(items, np.int64), np.int64)
     q8 = _qk8_args(qk8, q.shape)
+    ref, kr = _ref_args(geo, idx, topk)
     out = np.zeros((len(items), geo.tile, D), np.float64)
     _load().vsa_oracle_fine_tiles(_p(q), _p(k), _p(v), *(_p(t) for t in q8), B, L, H, D, geo.n_tiles,
-                                  geo.n_prefix, topk, geo.tile,
+                                  geo.n_prefix, topk, _p(ref), kr, geo.tile,
                                   _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), len(items),
                                   _p(items), _p(out))
     return out
@@ -273,17 +310,19 @@ def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarr
     return res
 
 
-def selection(q, k, v, segments, grid, sparsity, scale=None, tile=64, cube=None):
-    """Pool, scores, top-k and compression only (every tile, every head)."""
-    geo = geometry(segments, grid, tile, cube)
+def selection(q, k, v, segments, grid, sparsity, scale=None, tile=64, cube=None, ref_segments=None, ref_keep=None):
+    """Pool, scores, top-k and compression only (every tile, every head).  ref_segments / ref_keep:
+    reference segments and their keep ratio (R18)."""
+    geo = geometry(segments, grid, tile, cube, ref_segments)
     if scale is None:
         scale = default_scale(q.shape[-1])
     kc = topk_count(sparsity, geo.n_video)
+    kr = ref_count(ref_keep, geo.n_ref) if geo.is_ref is not None and geo.n_video > 0 else 0
     pq, pk, pv = pool(q, geo), pool(k, geo), pool(v, geo)
     S = scores(pq, pk, scale)
-    idx = select(S, geo.n_prefix, kc)
+    idx = select(S, geo.n_prefix, kc, geo.is_ref, kr)
     o_c = compress(S, pv)
-    return dict(geo=geo, topk=kc, scale=scale, pq=pq, pk=pk, pv=pv, S=S, idx=idx, o_c=o_c)
+    return dict(geo=geo, topk=kc, kr=kr, scale=scale, pq=pq, pk=pk, pv=pv, S=S, idx=idx, o_c=o_c)
 
 
 def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndarray:
@@ -292,7 +331,9 @@ def fine_masked(q, k, v, geo: Geometry, idx, topk: int, scale: float) -> np.ndar
     B, L, H, D = q.shape
     idx = _c(idx, np.int32)
     out = np.full((B, L, H, D), np.nan, np.float64)
-    _load().vsa_oracle_fine_masked(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk, geo.tile,
+    ref, kr = _ref_args(geo, idx, topk)
+    _load().vsa_oracle_fine_masked(_p(q), _p(k), _p(v), B, L, H, D, geo.n_tiles, geo.n_prefix, topk, _p(ref), kr,
+                                   geo.tile,
                                    _p(geo.tile_token), _p(geo.tile_valid), _p(idx), float(scale), _p(out))
     return out
 
@@ -338,7 +379,7 @@ class ForwardResult:
 
 
 def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=False, tile=64,
-            cube=None) -> ForwardResult:
+            cube=None, ref_segments=None, ref_keep=None) -> ForwardResult:
     """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H] (or
     [B,L,H*D], one per channel).
 
@@ -346,16 +387,18 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
     None = all).  qk8: the fine branch's logits use 8-bit Q/K (R16); the
     selection still reads the bf16 inputs.  tile, cube: the tile size and video
-    cube shape (64 and 4x4x4 as the method states; 128 per R17)."""
+    cube shape (64 and 4x4x4 as the method states; 128 per R17).  ref_segments,
+    ref_keep: reference segments and their keep ratio (R18)."""
     t0 = time.perf_counter()
-    geo = geometry(segments, grid, tile, cube)
+    geo = geometry(segments, grid, tile, cube, ref_segments)
     D = q.shape[-1]
     if scale is None:
         scale = default_scale(D)
     kc = topk_count(sparsity, geo.n_video)
+    kr = ref_count(ref_keep, geo.n_ref) if geo.is_ref is not None and geo.n_video > 0 else 0
     pq, pk, pv = pool(q, geo), pool(k, geo), pool(v, geo)
     S = scores(pq, pk, scale)
-    idx = select(S, geo.n_prefix, kc)
+    idx = select(S, geo.n_prefix, kc, geo.is_ref, kr)
     o_c = compress(S, pv)
     q8 = (*quant_e4m3(q), *quant_e4m3(k)) if qk8 else None
     o_f = fine(q, k, v, geo, idx, kc, scale, todo, qk8=q8)

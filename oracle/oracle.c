@@ -57,6 +57,14 @@
  *      ct*ch*cw = 128, by default 4 x 4 x 8 (the 4 x 4 x 4 cube doubled along w, the
  *      fastest axis); every other step is the 64-token method with "64" read as the
  *      tile size.
+ *   R18 "reference keep" (same passage: "reference keep 0.1"): a prefix segment may be a
+ *      reference segment (the reference vision tokens and reference audio of the
+ *      conditioning prefix).  Its tiles are not always-kept prefix keys: each video query
+ *      tile keeps the kr reference tiles with the highest pooled scores S[i, j] (ties to
+ *      the lower index), kr = max(1, min(ceil(keep * R), R)) in binary64 for R reference
+ *      tiles (0 when R = 0), listed ascending before its topk video tiles.  The other
+ *      prefix tiles stay always kept; prefix query tiles (reference ones included) stay
+ *      dense; the compression still runs over all tiles.
  *
  * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
  * order above; fine attention, compression and the output in binary64.
@@ -343,6 +351,56 @@ int vsa_oracle_select(const float *S, int BH, int n_t, int P, int k, int32_t *id
     return bad ? -1 : 0;
 }
 
+/* Reference keep (R18): kr = max(1, min(ceil(keep * R), R)) in binary64; 0 without reference tiles. */
+int vsa_oracle_ref_count(double keep, int n_ref) {
+    double k;
+    if (n_ref <= 0) return 0;
+    k = ceil(keep * (double)n_ref);
+    if (k > (double)n_ref) k = (double)n_ref;
+    if (k < 1.0) k = 1.0;
+    return (int)k;
+}
+
+/* Selection with reference tiles (R18): for each (bh, video query tile iv), idx[bh, iv, 0..kr)
+ * = the kr reference tiles (prefix tiles j with is_ref[j]) with the highest S[bh, P+iv, j],
+ * ascending; idx[bh, iv, kr..kr+k) = the k video tiles as vsa_oracle_select picks them.  Ties go
+ * to the lower index.  Returns -1 if a compared score is NaN. */
+int vsa_oracle_select_ref(const float *S, int BH, int n_t, int P, const uint8_t *is_ref, int kr, int k,
+                          int32_t *idx) {
+    int V = n_t - P, R = 0, w = kr + k;
+    int bad = 0;
+    for (int j = 0; j < P; ++j) R += is_ref[j] ? 1 : 0;
+#pragma omp parallel for collapse(2) schedule(static) reduction(| : bad)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int iv = 0; iv < V; ++iv) {
+            int n = (V > R ? V : R);
+            scored_tile *row = (scored_tile *)malloc(sizeof(scored_tile) * (size_t)(n > 0 ? n : 1));
+            const float *srow = S + ((int64_t)bh * n_t + (P + iv)) * n_t;
+            int32_t *out = idx + ((int64_t)bh * V + iv) * w;
+            int m = 0;
+            for (int j = 0; j < P; ++j)
+                if (is_ref[j]) {
+                    row[m].s = srow[j];
+                    row[m].j = j;
+                    if (isnan(row[m].s)) bad = 1;
+                    ++m;
+                }
+            qsort(row, (size_t)m, sizeof(scored_tile), by_score_then_index);
+            for (int t = 0; t < kr; ++t) out[t] = row[t].j;
+            qsort(out, (size_t)kr, sizeof(int32_t), by_index);
+            for (int j = 0; j < V; ++j) {
+                row[j].s = srow[P + j];
+                row[j].j = j;
+                if (isnan(row[j].s)) bad = 1;
+            }
+            qsort(row, (size_t)V, sizeof(scored_tile), by_score_then_index);
+            for (int t = 0; t < k; ++t) out[kr + t] = P + row[t].j;
+            qsort(out + kr, (size_t)k, sizeof(int32_t), by_index);
+            free(row);
+        }
+    return bad ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* O6 compression branch (binary64)                                    */
 /* ------------------------------------------------------------------ */
@@ -376,14 +434,20 @@ void vsa_oracle_compress(const float *S, const float *pv, int BH, int n_t, int D
 /* The key set of query tile i: every tile for a prefix query tile (dense
  * prefix queries); the P prefix tiles plus idx[b,h,i-P,:] for a video query
  * tile (exempt prefix keys).  Writes the set into keys[] and returns its size. */
-static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t *keys) {
+/* Key tiles of query tile i: every tile for a prefix query tile; otherwise the always-kept prefix
+ * tiles (all P, or those with is_ref[j] == 0 when is_ref is given, R18) followed by the w = kr + k
+ * entries of its idx row. */
+static int key_set(int i, int n_t, int P, const uint8_t *is_ref, int w, const int32_t *idx_row,
+                   int32_t *keys) {
+    int n = 0;
     if (i < P) {
         for (int j = 0; j < n_t; ++j) keys[j] = j;
         return n_t;
     }
-    for (int j = 0; j < P; ++j) keys[j] = j;
-    for (int t = 0; t < k; ++t) keys[P + t] = idx_row[t];
-    return P + k;
+    for (int j = 0; j < P; ++j)
+        if (!is_ref || !is_ref[j]) keys[n++] = j;
+    for (int t = 0; t < w; ++t) keys[n++] = idx_row[t];
+    return n;
 }
 
 /* Fine branch of one query tile (b, h, i): for each valid query row r,
@@ -391,12 +455,13 @@ static int key_set(int i, int n_t, int P, int k, const int32_t *idx_row, int32_t
  *   o_f[r] = sum_c softmax(logit)_c * v_c,
  * written to rows[r * D + d] in tile row order (pad rows left untouched). */
 static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint16_t *v, int b, int h, int i,
-                          int64_t L, int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
-                          const int32_t *tile_valid, const int32_t *idx, double scale, double *rows) {
-    int V = n_t - P;
+                          int64_t L, int H, int D, int n_t, int P, int k, const uint8_t *is_ref, int kr, int tile,
+                          const int32_t *tile_token, const int32_t *tile_valid, const int32_t *idx, double scale,
+                          double *rows) {
+    int V = n_t - P, w = kr + k;
     int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
-    const int32_t *idx_row = (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
-    int nk = key_set(i, n_t, P, k, idx_row, keys);
+    const int32_t *idx_row = (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * w : NULL;
+    int nk = key_set(i, n_t, P, is_ref, w, idx_row, keys);
     /* every valid key row of the key set, in list order */
     int64_t max_rows = (int64_t)nk * tile;
     int64_t *ktok = (int64_t *)malloc(sizeof(int64_t) * (size_t)max_rows);
@@ -443,8 +508,8 @@ static void fine_one_tile(const qk_operand *q, const qk_operand *kk, const uint1
  * codes [B, L, H, D] and scales [B, L, H] used for the logits instead of q, k. */
 void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
                      const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
-                     int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
-                     const int32_t *tile_valid, const int32_t *idx, double scale,
+                     int H, int D, int n_t, int P, int k, const uint8_t *is_ref, int kr, int tile,
+                     const int32_t *tile_token, const int32_t *tile_valid, const int32_t *idx, double scale,
                      const uint8_t *todo, double *o_f) {
     qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
     qk_tables();
@@ -455,8 +520,8 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, c
                 int64_t bhi = ((int64_t)b * H + h) * n_t + i;
                 if (todo && !todo[bhi]) continue;
                 double *rows = (double *)malloc(sizeof(double) * (size_t)tile * (size_t)D);
-                fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile, tile_token, tile_valid, idx, scale,
-                              rows);
+                fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, is_ref, kr, tile, tile_token, tile_valid,
+                              idx, scale, rows);
                 for (int r = 0; r < tile_valid[i]; ++r) {
                     int64_t tok = tile_token[(int64_t)i * tile + r];
                     memcpy(o_f + (((int64_t)b * L + tok) * H + h) * D, rows + (int64_t)r * D,
@@ -470,7 +535,8 @@ void vsa_oracle_fine(const uint16_t *q, const uint16_t *kk, const uint16_t *v, c
  * out[n, r, :] for the tile's rows r in tile order (pad rows set to 0). */
 void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t *v, const uint8_t *q8,
                            const float *qs, const uint8_t *k8, const float *ks, int B, int64_t L,
-                           int H, int D, int n_t, int P, int k, int tile, const int32_t *tile_token,
+                           int H, int D, int n_t, int P, int k, const uint8_t *is_ref, int kr, int tile,
+                           const int32_t *tile_token,
                            const int32_t *tile_valid, const int32_t *idx, double scale, int n_items,
                            const int64_t *items, double *out) {
     qk_operand qo = {q, q8, qs}, ko = {kk, k8, ks};
@@ -484,7 +550,8 @@ void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t
         int h = (int)(bh % H), b = (int)(bh / H);
         double *rows = out + (int64_t)n * tile * D;
         for (int64_t e = 0; e < (int64_t)tile * D; ++e) rows[e] = 0.0;
-        fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, tile, tile_token, tile_valid, idx, scale, rows);
+        fine_one_tile(&qo, &ko, v, b, h, i, L, H, D, n_t, P, k, is_ref, kr, tile, tile_token, tile_valid, idx, scale,
+                      rows);
     }
 }
 
@@ -498,10 +565,10 @@ void vsa_oracle_fine_tiles(const uint16_t *q, const uint16_t *kk, const uint16_t
  * against).  Tokens outside every tile do not occur.  Used on small inputs
  * only: builds an L x L mask per (b, h). */
 void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_t *v, int B,
-                            int64_t L, int H, int D, int n_t, int P, int k, int tile,
-                            const int32_t *tile_token, const int32_t *tile_valid,
+                            int64_t L, int H, int D, int n_t, int P, int k, const uint8_t *is_ref, int kr,
+                            int tile, const int32_t *tile_token, const int32_t *tile_valid,
                             const int32_t *idx, double scale, double *o_f) {
-    int V = n_t - P;
+    int V = n_t - P, w = kr + k;
     int32_t *tile_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)L);
     for (int i = 0; i < n_t; ++i)
         for (int r = 0; r < tile_valid[i]; ++r) tile_of[tile_token[(int64_t)i * tile + r]] = i;
@@ -513,8 +580,8 @@ void vsa_oracle_fine_masked(const uint16_t *q, const uint16_t *kk, const uint16_
             int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_t);
             for (int i = 0; i < n_t; ++i) {
                 const int32_t *idx_row =
-                    (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * k : NULL;
-                int nk = key_set(i, n_t, P, k, idx_row, keys);
+                    (i >= P) ? idx + (((int64_t)b * H + h) * V + (i - P)) * w : NULL;
+                int nk = key_set(i, n_t, P, is_ref, w, idx_row, keys);
                 for (int t = 0; t < nk; ++t) allowed[(int64_t)i * n_t + keys[t]] = 1;
             }
             double *logit = (double *)malloc(sizeof(double) * (size_t)L);
