@@ -182,13 +182,15 @@ def oracle_sample(w, every: int, seed: int = 0):
     x = synth.make_inputs(dataclasses.replace(w, heads=1), seed=seed, device="cpu")
     xb = {n: synth.as_bits(x[n]) for n in ("q", "k", "v", "gate")}
     t0 = time.perf_counter()
-    sel = oracle.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity, tile=w.tile, cube=w.cube)
+    sel = oracle.selection(xb["q"], xb["k"], xb["v"], w.segments, w.grid, w.sparsity, tile=w.tile, cube=w.cube,
+                           ref_segments=w.ref_segments, ref_keep=w.ref_keep)
     geo = sel["geo"]
     items = np.arange(0, geo.n_tiles, every, dtype=np.int64)
     of = oracle.fine_tiles(xb["q"], xb["k"], xb["v"], geo, sel["idx"], sel["topk"], sel["scale"], items)
     oracle.output_tiles(of, sel["o_c"], xb["gate"], geo, items, 1)
     dt = time.perf_counter() - t0
-    pairs = sum((geo.n_tiles if i < geo.n_prefix else geo.n_prefix + sel["topk"]) for i in items)
+    pairs = sum((geo.n_tiles if i < geo.n_prefix else geo.n_prefix - geo.n_ref + sel["kr"] + sel["topk"])
+                for i in items)
     flops = pairs * tile_flops(w.head_dim, w.tile)
     desc = (f"head 0 of 56: full selection (pool, fp32 scores, top-k, compression over {geo.n_tiles} tiles) "
             f"+ fine branch and output of every {every}th query tile ({len(items)} of {geo.n_tiles} tiles, "
@@ -232,17 +234,21 @@ def run_reference(args, w, world, rank):
 def config_dict(w, dims=None):
     import oracle
 
-    geo = oracle.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube) if dims is None else None
+    geo = oracle.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube, ref_segments=w.ref_segments) \
+        if dims is None else None
     n_t = dims["n_tiles"] if dims else geo.n_tiles
     P = dims["n_prefix_tiles"] if dims else geo.n_prefix
     V = n_t - P
     k = dims["topk"] if dims else oracle.topk_count(w.sparsity, V)
-    pairs = V * (P + k) + P * n_t
+    R = dims["n_ref_tiles"] if dims else geo.n_ref
+    kr = dims["ref_topk"] if dims else (oracle.ref_count(w.ref_keep, R) if R and V else 0)
+    pairs = V * (P - R + kr + k) + P * n_t
     return {
         "workload": w.name, "description": w.description, "batch": w.batch, "heads": w.heads,
         "head_dim": w.head_dim, "seq_len": w.seq_len, "prefix_segments": list(w.segments), "grid": list(w.grid),
         "tile_size": w.tile, "n_tiles": n_t, "n_prefix_tiles": P, "n_video_tiles": V, "sparsity": w.sparsity,
-        "topk": k, "selected_tile_pairs": pairs * w.batch * w.heads,
+        "topk": k, **({"n_ref_tiles": R, "ref_keep": w.ref_keep, "ref_topk": kr} if R else {}),
+        "selected_tile_pairs": pairs * w.batch * w.heads,
         "selected_tflop_per_call": pairs * w.batch * w.heads * tile_flops(w.head_dim, w.tile) / 1e12,
         "l2": "no flush: Q/K/V/out are %.1f GB per step, > 126 MB L2" % (4 * w.batch * w.seq_len * w.heads * w.head_dim * 2 / 1e9),
     }
@@ -259,7 +265,8 @@ def run_vsa(args, w, world, rank, local):
     x = synth.make_inputs(w, seed=rank, device=dev)
     torch.cuda.synchronize()
     plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-                              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube)
+                              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube, ref_segments=w.ref_segments,
+                              ref_keep=w.ref_keep)
     dims = plan.dims
     ws = vsa.alloc_workspace(plan, dev)
     v = vsa.workspace_views(plan, ws)
@@ -391,7 +398,8 @@ def run_ab(args, w, variants):
     for rnd in range(2):
         for key, extra in variants.items():
             plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments,
-                                      grid=w.grid, sparsity=w.sparsity, tile_size=w.tile, cube=w.cube, **extra)
+                                      grid=w.grid, sparsity=w.sparsity, tile_size=w.tile, cube=w.cube,
+                                      ref_segments=w.ref_segments, ref_keep=w.ref_keep, **extra)
             ws = vsa.alloc_workspace(plan)
             out = torch.empty_like(x["q"])
             for _ in range(args.warmup):

@@ -56,6 +56,7 @@ class Geometry(ctypes.Structure):
         ("tile_size", ctypes.c_int32), ("sparsity", ctypes.c_double), ("softmax_scale", ctypes.c_float),
         ("gate_per_channel", ctypes.c_int32), ("seq_tiles", ctypes.c_int32), ("qk_fp8", ctypes.c_int32),
         ("cube_t", ctypes.c_int32), ("cube_h", ctypes.c_int32), ("cube_w", ctypes.c_int32),
+        ("segment_reference", ctypes.POINTER(ctypes.c_int32)), ("reference_keep", ctypes.c_double),
     ]
 
 
@@ -74,6 +75,7 @@ class PlanDims(ctypes.Structure):
         ("n_tiles", ctypes.c_int32), ("n_prefix_tiles", ctypes.c_int32), ("n_video_tiles", ctypes.c_int32),
         ("topk", ctypes.c_int32), ("seq_len", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
         ("workspace_bytes", ctypes.c_size_t), ("selected_pairs", ctypes.c_int64), ("tile_size", ctypes.c_int32),
+        ("n_ref_tiles", ctypes.c_int32), ("ref_topk", ctypes.c_int32),
     ]
 
     def as_dict(self):
@@ -153,9 +155,10 @@ def _ptr(t, dtype=None, name="tensor"):
 
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
                   token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False, qk_fp8=False,
-                  cube=None):
+                  cube=None, ref_segments=None, ref_keep=0.0):
     """Build the ``vsa_geometry`` struct; returns (struct, keep-alive buffers).  cube: (t, h, w) of a
-    video tile, None for the default (4x4x4 for 64-token tiles, 4x4x8 for 128)."""
+    video tile, None for the default (4x4x4 for 64-token tiles, 4x4x8 for 128).  ref_segments: one
+    flag per prefix segment marking reference segments, with their keep ratio ref_keep."""
     g = Geometry()
     g.batch, g.heads, g.head_dim = int(batch), int(heads), int(head_dim)
     keep = []
@@ -180,6 +183,11 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.seq_tiles = int(bool(seq_tiles))
     g.qk_fp8 = int(bool(qk_fp8))
     g.cube_t, g.cube_h, g.cube_w = (int(c) for c in (cube or (0, 0, 0)))
+    if ref_segments is not None:
+        flags = (ctypes.c_int32 * max(1, len(ref_segments)))(*[int(f) for f in ref_segments])
+        keep.append(flags)
+        g.segment_reference = ctypes.cast(flags, ctypes.POINTER(ctypes.c_int32))
+        g.reference_keep = float(ref_keep)
     return g, keep
 
 
@@ -248,11 +256,12 @@ class Plan:
 
 def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
                    token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False,
-                   qk_fp8=False, cube=None, stream=None) -> Plan:
+                   qk_fp8=False, cube=None, ref_segments=None, ref_keep=0.0, stream=None) -> Plan:
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
               tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles),
-              qk_fp8=bool(qk_fp8), cube=None if cube is None else tuple(cube))
+              qk_fp8=bool(qk_fp8), cube=None if cube is None else tuple(cube),
+              ref_segments=None if ref_segments is None else tuple(ref_segments), ref_keep=float(ref_keep))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
     _check(load_library().vsa_plan_tiles(ctypes.byref(g), _stream(stream), ctypes.byref(h)), "vsa_plan_tiles")
@@ -474,6 +483,6 @@ def workspace_views(plan, workspace):
         "pk": view(lay["pk"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pv": view(lay["pv"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "scores": view(lay["scores"], B * H * n_t * n_t, torch.float32, (B, H, n_t, n_t)),
-        "idx": view(lay["idx"], B * H * V * k, torch.int32, (B, H, V, k)),
+        "idx": view(lay["idx"], B * H * V * (k + d["ref_topk"]), torch.int32, (B, H, V, k + d["ref_topk"])),
         "o_c": view(lay["o_c"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
     }

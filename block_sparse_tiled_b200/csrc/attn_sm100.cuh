@@ -5,7 +5,9 @@
 // tile i is row blocks 2i and 2i+1, which share its key list.  The key list of
 // query tile i is every tile for a prefix query tile, else the P prefix tiles
 // followed by the tile's selected video tiles (ascending), taken as row blocks
-// and walked two row blocks (128 keys) at a time.  CTAs claim items in order from a global counter
+// and walked two row blocks (128 keys) at a time.  With reference segments the
+// always-kept prefix tiles are the non-reference ones, and the kept reference
+// tiles come first in the idx row.  CTAs claim items in order from a global counter
 // (one per SM, persistent), so the items in flight stay within a head or two
 // and that head's K/V stays resident in L2 even though prefix query tiles cost
 // many times a video query tile.
@@ -101,7 +103,9 @@ constexpr int kOCol0 = 64 * kSBufs;  // O^T double buffer follows (2 x 64 column
 constexpr uint32_t kTmemCols = (kOCol0 + 128 <= 256) ? 256 : 512;
 
 struct AttnArgs {
-  const int32_t* idx;         // [B, H, V, topk] global key-tile indices (ascending per row)
+  const int32_t* idx;         // [B, H, V, kr + topk]: kept reference tiles, then video tiles (each ascending)
+  const int32_t* exempt;      // NULL: every prefix tile is always kept; else the n_exempt always-kept ones
+  int n_exempt, kr;           // always-kept prefix tiles (P without reference tiles); reference tiles kept
   const int32_t* tile_token;  // [n_rb * 64]: token of each row of each 64-row block
   const int32_t* tile_valid;  // [n_t]
   const float* o_c;           // [B, H, n_t, D] (per tile)
@@ -309,12 +313,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
 
-  // key list of query tile i, in 64-row blocks
-  auto list_len = [&](int i) { return ((i < P) ? n_sel : P + topk) << sh; };
+  // key list of query tile i, in 64-row blocks: all tiles, or the E always-kept prefix tiles and the
+  // kr + topk entries of the tile's idx row
+  const int E = a.n_exempt, W = a.kr + topk;
+  auto list_len = [&](int i) { return ((i < P) ? n_sel : E + W) << sh; };
   // row block of list position t (in row blocks) of query tile i
   auto key_tile = [&](int64_t bh, int i, int t) -> int {
     const int ts = t >> sh;
-    const int sel = (i < P || ts < P) ? ts : __ldg(a.idx + (bh * V + (i - P)) * topk + (ts - P));
+    int sel;
+    if (i < P)
+      sel = ts;
+    else if (ts < E)
+      sel = a.exempt ? __ldg(a.exempt + ts) : ts;
+    else
+      sel = __ldg(a.idx + (bh * V + (i - P)) * W + (ts - E));
     return (sel << sh) | (t & ((1 << sh) - 1));
   };
   // Claimed item number `it` of this CTA (-1: none left), read by one thread of a consumer warp.

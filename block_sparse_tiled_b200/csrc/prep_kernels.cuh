@@ -284,10 +284,13 @@ __global__ void __launch_bounds__(256, 2) scores_kernel(const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// S4 top-k: one warp per (bh, video query tile).  The row's video scores go to
-// shared memory as order-preserving 32-bit keys; a 32-step bitwise search
+// S4 top-k: one warp per (bh, video query tile).  The row's candidate scores go
+// to shared memory as order-preserving 32-bit keys; a 32-step bitwise search
 // finds the k-th largest key T; the tiles with key > T, plus the lowest-index
-// ones with key == T up to k, are emitted in ascending index order.
+// ones with key == T up to k, are emitted in ascending index order.  The
+// candidates are the video tiles (cols == NULL: tiles P..n_t-1) or a listed
+// set of tiles in ascending order (the reference tiles of the reference keep);
+// the picks go to idx[row * out_stride + out_off ...].
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -302,42 +305,45 @@ __device__ __forceinline__ int warp_sum(int x) {
 }
 
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, int32_t* __restrict__ idx,
-                                                    int BH, int n_t, int P, int k, int rows_per_block) {
-  extern __shared__ uint32_t keys_s[];  // [rows_per_block][V]
+                                                    int BH, int n_t, int P, int k, int rows_per_block,
+                                                    const int32_t* __restrict__ cols, int ncols, int out_stride,
+                                                    int out_off) {
+  extern __shared__ uint32_t keys_s[];  // [rows_per_block][ncols]
   const int V = n_t - P;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp;
   if (warp >= rows_per_block || row >= static_cast<int64_t>(BH) * V) return;
   const int bh = static_cast<int>(row / V), iv = static_cast<int>(row - static_cast<int64_t>(bh) * V);
-  uint32_t* keys = keys_s + static_cast<int64_t>(warp) * V;
-  const float* srow = S + (static_cast<int64_t>(bh) * n_t + (P + iv)) * n_t + P;
-  for (int j = lane; j < V; j += 32) keys[j] = order_key(__ldg(srow + j));
+  uint32_t* keys = keys_s + static_cast<int64_t>(warp) * ncols;
+  const float* srow = S + (static_cast<int64_t>(bh) * n_t + (P + iv)) * n_t;
+  auto col = [&](int j) { return cols ? __ldg(cols + j) : P + j; };
+  for (int j = lane; j < ncols; j += 32) keys[j] = order_key(__ldg(srow + col(j)));
   __syncwarp();
 
   uint32_t T = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
     int cnt = 0;
-    for (int j = lane; j < V; j += 32) cnt += (keys[j] >= cand) ? 1 : 0;
+    for (int j = lane; j < ncols; j += 32) cnt += (keys[j] >= cand) ? 1 : 0;
     if (warp_sum(cnt) >= k) T = cand;
   }
   int gt = 0;
-  for (int j = lane; j < V; j += 32) gt += (keys[j] > T) ? 1 : 0;
+  for (int j = lane; j < ncols; j += 32) gt += (keys[j] > T) ? 1 : 0;
   const int need = k - warp_sum(gt);  // how many of the tiles equal to T to take, lowest index first
 
-  int32_t* out = idx + row * k;
+  int32_t* out = idx + row * out_stride + out_off;
   int written = 0, eq_seen = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int j0 = 0; j0 < V; j0 += 32) {
+  for (int j0 = 0; j0 < ncols; j0 += 32) {
     const int j = j0 + lane;
-    const uint32_t key = (j < V) ? keys[j] : 0u;
-    const bool is_gt = (j < V) && key > T;
-    const bool is_eq = (j < V) && key == T;
+    const uint32_t key = (j < ncols) ? keys[j] : 0u;
+    const bool is_gt = (j < ncols) && key > T;
+    const bool is_eq = (j < ncols) && key == T;
     const uint32_t eq_ballot = __ballot_sync(0xffffffffu, is_eq);
     const int eq_before = eq_seen + __popc(eq_ballot & lt_mask);
     const bool take = is_gt || (is_eq && eq_before < need);
     const uint32_t take_ballot = __ballot_sync(0xffffffffu, take);
-    if (take) out[written + __popc(take_ballot & lt_mask)] = P + j;
+    if (take) out[written + __popc(take_ballot & lt_mask)] = col(j);
     written += __popc(take_ballot);
     eq_seen += __popc(eq_ballot);
   }

@@ -55,7 +55,21 @@ struct Resolved {
   int32_t tile = 64;             // tokens per tile (64 or 128)
   int32_t ct = 4, ch = 4, cw = 4;  // video cube shape
   int32_t sh = 0;                // log2(tile / 64): 64-row blocks per tile = 1 << sh
+  // reference keep: per prefix tile, 1 for a tile of a reference segment; R of them; kr kept per video
+  // query tile
+  std::vector<uint8_t> tile_ref;
+  int64_t n_ref = 0;
+  int32_t kr = 0;
 };
+
+// Reference tiles kept per video query tile: max(1, min(ceil(keep * R), R)) in binary64; 0 without any.
+int32_t ref_keep_for(double keep, int64_t R) {
+  if (R <= 0) return 0;
+  double k = std::ceil(keep * static_cast<double>(R));
+  if (k > static_cast<double>(R)) k = static_cast<double>(R);
+  if (k < 1.0) k = 1.0;
+  return static_cast<int32_t>(k);
+}
 
 // topk = max(1, min(ceil((1 - sparsity) * V), V)), evaluated in binary64; 0 without video tiles.
 int32_t topk_for(double sparsity, int64_t V) {
@@ -148,6 +162,22 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   const int64_t n_t = r->n_prefix + r->n_video;
   if (n_t > (1 << 24)) return fail(VSA_ERR_UNSUPPORTED, "too many tiles");
   r->topk = topk_for(g->sparsity, r->n_video);
+  r->tile_ref.clear();
+  r->n_ref = 0;
+  r->kr = 0;
+  if (g->segment_reference != nullptr) {
+    if (g->token_tags != nullptr) return fail(VSA_ERR_INVALID_ARG, "segment_reference needs segment_len, not tags");
+    if (!(g->reference_keep > 0.0 && g->reference_keep <= 1.0))
+      return fail(VSA_ERR_INVALID_ARG, "reference_keep must lie in (0, 1]");
+    for (size_t s = 0; s < r->segments.size(); ++s) {
+      const int32_t f = g->segment_reference[s];
+      if (f != 0 && f != 1) return fail(VSA_ERR_INVALID_ARG, "segment_reference flags must be 0 or 1");
+      const int64_t nt = (r->segments[s] + r->tile - 1) / r->tile;
+      r->tile_ref.insert(r->tile_ref.end(), static_cast<size_t>(nt), static_cast<uint8_t>(f));
+      if (f) r->n_ref += nt;
+    }
+    r->kr = (r->n_video > 0) ? ref_keep_for(g->reference_keep, r->n_ref) : 0;
+  }
   r->scale = (g->softmax_scale != 0.0f) ? g->softmax_scale
                                         : static_cast<float>(1.0 / std::sqrt(static_cast<double>(g->head_dim)));
   if (!(std::isfinite(r->scale)) || r->scale <= 0.0f) return fail(VSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
@@ -407,6 +437,12 @@ struct vsa_plan_s {
   bool qk_fp8 = false;     // 8-bit Q/K (E4M3 codes, one scale per token and head) for the fine logits
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
+  // reference keep: kr of the n_ref reference tiles kept per video query tile (idx rows hold kr + topk);
+  // the always-kept prefix tiles and the reference tiles (device copies only when n_ref > 0)
+  int32_t kr = 0, n_ref = 0;
+  std::vector<int32_t> exempt_tiles, ref_tiles;
+  int32_t* d_exempt = nullptr;
+  int32_t* d_refs = nullptr;
   std::vector<int32_t> tile_token, tile_valid;
   int32_t* d_tile_token = nullptr;
   int32_t* d_tile_valid = nullptr;
@@ -539,19 +575,23 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
                     const int* gate_nonzero = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const int64_t BH = static_cast<int64_t>(p->B) * p->H;
-  if (p->V > 0 && p->topk > 0) {
-    const size_t row_bytes = static_cast<size_t>(p->V) * 4;
+  // one selection per video query tile over `ncols` candidates (the video tiles, or the listed reference
+  // tiles), written at column `off` of idx rows kr + topk wide
+  auto select = [&](const int32_t* cols, int ncols, int k, int off) -> vsa_status {
+    const size_t row_bytes = static_cast<size_t>(ncols) * 4;
     int rows = static_cast<int>(std::min<size_t>(8, std::max<size_t>(1, (200 * 1024) / row_bytes)));
     const size_t smem = row_bytes * rows;
-    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "too many video tiles for the top-k kernel");
+    if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "too many candidate tiles for the top-k kernel");
     VSA_TRY(allow_smem(vsa::topk_kernel, smem));
     const int64_t nrows = BH * p->V;
     const int64_t blocks = (nrows + rows - 1) / rows;
     if (blocks > 0x7fffffff) return fail(VSA_ERR_UNSUPPORTED, "top-k grid too large");
     vsa::topk_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(S, idx, static_cast<int>(BH), p->n_t, p->P,
-                                                                     p->topk, rows);
-    VSA_TRY(launch_check("topk"));
-  }
+                                                                     k, rows, cols, ncols, p->kr + p->topk, off);
+    return launch_check("topk");
+  };
+  if (p->V > 0 && p->kr > 0) VSA_TRY(select(p->d_refs, p->n_ref, p->kr, 0));
+  if (p->V > 0 && p->topk > 0) VSA_TRY(select(nullptr, p->V, p->topk, p->kr));
   dim3 grid((p->n_t + vsa::kCompRows - 1) / vsa::kCompRows, static_cast<unsigned>(BH));
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
@@ -613,6 +653,9 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.sub_shift = p->r.sh;
   a.P = p->P;
   a.topk = p->topk;
+  a.kr = p->kr;
+  a.n_exempt = p->n_ref > 0 ? static_cast<int>(p->exempt_tiles.size()) : p->P;
+  a.exempt = p->n_ref > 0 ? p->d_exempt : nullptr;
   a.scale_log2 = static_cast<float>(static_cast<double>(p->r.scale) * 1.4426950408889634);
   a.n_items = static_cast<int64_t>(p->B) * p->H * n_rb;
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
@@ -674,7 +717,13 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->d_status = p->d_status;
   q->seq_tiles = p->seq_tiles;
   q->qk_fp8 = p->qk_fp8;
-  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk, q->seq_tiles, q->qk_fp8);
+  q->kr = p->kr;
+  q->n_ref = p->n_ref;
+  q->exempt_tiles = p->exempt_tiles;
+  q->ref_tiles = p->ref_tiles;
+  q->d_exempt = p->d_exempt;
+  q->d_refs = p->d_refs;
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk + q->kr, q->seq_tiles, q->qk_fp8);
   q->owns_device = false;
   return q;
 }
@@ -690,7 +739,8 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   const size_t tokens = static_cast<size_t>(p->B) * static_cast<size_t>(p->r.L);
   h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
   h.fwd = 0;
-  size_t off = align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk, p->seq_tiles, p->qk_fp8).total);
+  size_t off =
+      align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8).total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
     off += 4 * h.chunk_bytes;  // q, k, v, out
@@ -755,10 +805,12 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->seq_len = r.L;
   d->softmax_scale = r.scale;
   d->workspace_bytes =
-      make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.tile, r.n_video, r.topk, g->seq_tiles != 0,
+      make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.tile, r.n_video, r.topk + r.kr, g->seq_tiles != 0,
                   g->qk_fp8 != 0).total;
-  d->selected_pairs = r.n_video * (r.n_prefix + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
+  d->selected_pairs = r.n_video * (r.n_prefix - r.n_ref + r.kr + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
   d->tile_size = r.tile;
+  d->n_ref_tiles = static_cast<int32_t>(r.n_ref);
+  d->ref_topk = r.kr;
 }
 
 }  // namespace
@@ -827,7 +879,10 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   if (r.tile == kTile) build_seq_tables(r, p->mask_tiled, &p->row_token, &p->mask_seq, &p->coord);
   p->seq_tiles = g->seq_tiles != 0;
   p->qk_fp8 = g->qk_fp8 != 0;
-  p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk, p->seq_tiles, p->qk_fp8);
+  p->kr = r.kr;
+  p->n_ref = static_cast<int32_t>(r.n_ref);
+  for (int32_t j = 0; j < p->P && p->n_ref > 0; ++j) (r.tile_ref[j] ? p->ref_tiles : p->exempt_tiles).push_back(j);
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
@@ -836,6 +891,8 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     cudaFree(p->d_mask_seq);
     cudaFree(p->d_mask_tiled);
     cudaFree(p->d_status);
+    cudaFree(p->d_exempt);
+    cudaFree(p->d_refs);
     delete p;
   };
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -848,7 +905,9 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
       cudaMalloc(&p->d_row_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_coord, coord_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_mask_seq, mask_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_mask_tiled, block_mask_bytes) != cudaSuccess ||
-      cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess) {
+      cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess ||
+      (p->n_ref > 0 && (cudaMalloc(&p->d_exempt, std::max<size_t>(4, p->exempt_tiles.size() * 4)) != cudaSuccess ||
+                        cudaMalloc(&p->d_refs, p->ref_tiles.size() * 4) != cudaSuccess))) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
   }
@@ -865,6 +924,10 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     e = cudaMemcpyAsync(p->d_mask_seq, p->mask_seq.data(), p->mask_seq.size() * 8, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !p->mask_tiled.empty())
     e = cudaMemcpyAsync(p->d_mask_tiled, p->mask_tiled.data(), p->mask_tiled.size() * 8, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->exempt_tiles.empty() && p->d_exempt)
+    e = cudaMemcpyAsync(p->d_exempt, p->exempt_tiles.data(), p->exempt_tiles.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->ref_tiles.empty())
+    e = cudaMemcpyAsync(p->d_refs, p->ref_tiles.data(), p->ref_tiles.size() * 4, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 4 * sizeof(int), s);
   if (e != cudaSuccess) {
     cleanup();
@@ -883,8 +946,11 @@ vsa_status vsa_plan_info(vsa_plan p, vsa_plan_dims* out) {
   out->seq_len = p->r.L;
   out->softmax_scale = p->r.scale;
   out->workspace_bytes = p->ws.total;
-  out->selected_pairs = static_cast<int64_t>(p->V) * (p->P + p->topk) + static_cast<int64_t>(p->P) * p->n_t;
+  out->selected_pairs =
+      static_cast<int64_t>(p->V) * (p->P - p->n_ref + p->kr + p->topk) + static_cast<int64_t>(p->P) * p->n_t;
   out->tile_size = p->r.tile;
+  out->n_ref_tiles = p->n_ref;
+  out->ref_topk = p->kr;
   return VSA_OK;
 }
 
@@ -917,6 +983,8 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
     cudaFree(p->d_mask_seq);
     cudaFree(p->d_mask_tiled);
     cudaFree(p->d_status);
+    cudaFree(p->d_exempt);
+    cudaFree(p->d_refs);
   }
   if (prev >= 0) cudaSetDevice(prev);
   delete p;

@@ -118,6 +118,16 @@ typedef struct vsa_geometry {
   int32_t cube_t, cube_h, cube_w; /* video cube shape, product = tile_size; all 0 = the default:
                                      4x4x4 for 64 tokens (the method's), 4x4x8 for 128 (the
                                      pages do not state it: the 64-token cube doubled along w) */
+  const int32_t* segment_reference; /* NULL, or n_segments flags (segments only, not tags): 1 marks a
+                                       reference segment ("FastH3 OmniRef inference", section "The
+                                       Blackwell stack": "reference keep").  Its R tiles are not
+                                       always-kept keys: each video query tile keeps the kr of them
+                                       with the highest pooled scores (ties: lower index),
+                                       kr = max(1, min(ceil(reference_keep * R), R)) in binary64;
+                                       the other prefix tiles stay always kept and prefix query
+                                       tiles stay dense.  idx rows then hold kr + topk entries: the
+                                       kept reference tiles, then the video tiles, each ascending. */
+  double reference_keep;            /* in (0, 1]; read when a segment is a reference segment */
 } vsa_geometry;
 
 typedef struct vsa_plan_s* vsa_plan; /* opaque, library-owned */
@@ -132,8 +142,10 @@ typedef struct vsa_plan_dims {
   float softmax_scale;    /* the scale actually used */
   size_t workspace_bytes; /* device scratch vsa_forward needs */
   int64_t selected_pairs; /* (query tile, key tile) pairs per (b, h):
-                             V * (P + topk) + P * n_tiles */
+                             V * (P - R + kr + topk) + P * n_tiles */
   int32_t tile_size;      /* tokens per tile (64 or 128) */
+  int32_t n_ref_tiles;    /* R: prefix tiles of reference segments */
+  int32_t ref_topk;       /* kr: reference tiles kept per video query tile (0 without any) */
 } vsa_plan_dims;
 
 /* ---- S1: tile plan (host) ------------------------------------------------
@@ -193,7 +205,9 @@ vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf1
 
 /* ---- S4: top-k selection and the compression branch ---------------------
  * idx[b,h,iv,:] = the topk video key tiles with the highest scores[b,h,P+iv,
- * P+j] (ties: lower index first), as global indices in ascending order;
+ * P+j] (ties: lower index first), as global indices in ascending order
+ * (with reference segments: first the kr kept reference tiles, ascending, so a
+ * row holds kr + topk entries);
  * o_c[b,h,i,:] = sum_j softmax_j(scores[b,h,i,:]) * pv[b,h,j,:] over all
  * n_tiles tiles, in binary32.
  * Passage: "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse

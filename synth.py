@@ -52,6 +52,8 @@ class Workload:
     gate_per_channel: bool = False  # gate [B, L, H*D] (one per channel) instead of [B, L, H]
     tile: int = 64  # tokens per attention tile (64, or 128 for the OmniRef-style variant)
     cube: tuple = None  # video cube (t, h, w) of a tile; None = the plan's default for `tile`
+    ref_segments: tuple = None  # per prefix segment: True for a reference segment (reference keep)
+    ref_keep: float = 0.0  # keep ratio of reference tiles
 
     @property
     def seq_len(self) -> int:
@@ -74,6 +76,10 @@ WORKLOADS = {
         Workload("768p_t128_s0.9", 1, 56, 128, (512, 0, 768), (24, 48, 64), 0.9, structured=True, tile=128,
                  description="1344x768-shaped with 128-token tiles (4x4x8 cubes): 56 heads, D=128, text 512 + "
                              "audio 768, video 24x48x64, sparsity 0.9"),
+        Workload("omniref_768p", 1, 56, 128, (512, 6144, 768), (24, 48, 64), 0.9, structured=True, tile=128,
+                 ref_segments=(False, True, False), ref_keep=0.1,
+                 description="OmniRef-shaped: 1344x768 video with 128-token tiles, text 512 + 6144 reference "
+                             "tokens (reference keep 0.1) + audio 768, 56 heads, D=128, sparsity 0.9"),
     ]
 }
 

@@ -46,7 +46,7 @@ def test_exports_every_declared_symbol(vsa):
 
 def _kw(w, **over):
     kw = dict(batch=w.batch, heads=w.heads, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
-              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube)
+              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube, ref_segments=w.ref_segments, ref_keep=w.ref_keep)
     kw.update(over)
     return kw
 
@@ -55,13 +55,16 @@ def _kw(w, **over):
 def test_plan_matches_oracle_geometry(vsa, oracle_mod, name):
     w = synth.workload(name)
     d = vsa.vsa_plan_query(**_kw(w))
-    geo = oracle_mod.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube)
+    geo = oracle_mod.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube, ref_segments=w.ref_segments)
     assert (d["n_tiles"], d["n_prefix_tiles"], d["n_video_tiles"]) == (geo.n_tiles, geo.n_prefix, geo.n_video)
     assert d["topk"] == oracle_mod.topk_count(w.sparsity, geo.n_video)
     assert d["seq_len"] == w.seq_len
     assert d["softmax_scale"] == np.float32(oracle_mod.default_scale(w.head_dim))
     P, V, k, n = geo.n_prefix, geo.n_video, d["topk"], geo.n_tiles
-    assert d["selected_pairs"] == V * (P + k) + P * n
+    R = geo.n_ref
+    kr = oracle_mod.ref_count(w.ref_keep, R) if R else 0
+    assert (d["n_ref_tiles"], d["ref_topk"]) == (R, kr)
+    assert d["selected_pairs"] == V * (P - R + kr + k) + P * n
     if name in ("tiny", "small", "480p"):
         tok, val = vsa.vsa_plan_tables_host(**_kw(w))
         assert np.array_equal(tok, geo.tile_token)
@@ -184,3 +187,22 @@ def test_plan_tile128_matches_oracle_geometry(vsa, oracle_mod, segments, grid, c
     assert np.array_equal(tok, geo.tile_token) and np.array_equal(val, geo.tile_valid)
     d64 = vsa.vsa_plan_query(**dict(kw, tile_size=64, cube=None))
     assert d["workspace_bytes"] > 0 and d64["n_tiles"] >= d["n_tiles"]
+
+
+def test_reference_keep_plan_and_limits(vsa, oracle_mod):
+    """Reference segments: counts as the oracle's, an idx row of kr + topk entries, and the argument checks."""
+    kw = dict(batch=1, heads=4, head_dim=128, segments=(40, 200, 24), grid=(8, 8, 8), sparsity=0.5,
+              ref_segments=(0, 1, 0), ref_keep=0.5)
+    d = vsa.vsa_plan_query(**kw)
+    geo = oracle_mod.geometry(kw["segments"], kw["grid"], ref_segments=kw["ref_segments"])
+    assert (d["n_ref_tiles"], d["ref_topk"], d["topk"]) == (4, 2, 4)
+    assert d["selected_pairs"] == geo.n_video * (6 - 4 + 2 + 4) + 6 * geo.n_tiles
+    plain = vsa.vsa_plan_query(**dict(kw, ref_segments=None))
+    assert d["workspace_bytes"] - plain["workspace_bytes"] >= 0  # idx rows grow by kr entries
+    for bad in (dict(ref_keep=0.0), dict(ref_keep=1.5), dict(ref_segments=(0, 2, 0))):
+        with pytest.raises(vsa.VsaError) as e:
+            vsa.vsa_plan_query(**dict(kw, **bad))
+        assert vsa.STATUS_NAMES[e.value.status] == "VSA_ERR_INVALID_ARG"
+    # no video tiles: no reference selection either
+    d0 = vsa.vsa_plan_query(**dict(kw, grid=(0, 0, 0)))
+    assert d0["ref_topk"] == 0 and d0["n_ref_tiles"] == 4
