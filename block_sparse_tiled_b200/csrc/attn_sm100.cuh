@@ -176,7 +176,7 @@ struct AttnLayout {
   static constexpr int kNumBars = bDonePV + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;          // tmem base, abort flag
   static constexpr int oRing = ((oMisc + 8 + 15) / 16) * 16;  // int ring[kRing]: claimed items, -1 = none left
-  static constexpr int oM = oRing + kRing * 4;               // float m[64] (log2 units)
+  static constexpr int oM = oRing + kRing * 4;               // float -m[64]: negated running max (log2 units)
   static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
   static constexpr int oRed = oDelta + 256;                  // float red[groups][4 quadrants][group columns]
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
@@ -588,7 +588,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int c0 = grp * CG;
     const int bar_vote = 1 + 2 * grp, bar_sync = 2 + 2 * grp;  // named barriers of this group
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    float* m_g = m_s + c0;
+    float* m_g = m_s + c0;   // the group's columns of the running maximum area, which holds -m
+    float* nm_g = m_g;
     float* delta_g = delta_s + c0;
     float* red_g = red_s + grp * 4 * CG;
     const float cl = a.scale_log2;
@@ -675,56 +676,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
         // x = logit * log2(e) - m  (m = 0 before the first block of the item); with 8-bit Q/K the
         // logit is the code product times the key and query scales
+        // (two columns per instruction: fma2/mul2 round each lane as fmaf/fmul do; nm_g holds -m)
         if constexpr (kF8) {
 #pragma unroll
-          for (int j = 0; j < CG; ++j) x[j] *= ks;
+          for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], ks, ks);
           if (n == 0) {
 #pragma unroll
             for (int j = 0; j < CG; j += 4) {
               const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
-              x[j] *= c4.x;
-              x[j + 1] *= c4.y;
-              x[j + 2] *= c4.z;
-              x[j + 3] *= c4.w;
+              mul2(x[j], x[j + 1], x[j], x[j + 1], c4.x, c4.y);
+              mul2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], c4.z, c4.w);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < CG; j += 4) {
               const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
-              const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
-              x[j] = fmaf(x[j], c4.x, -m4.x);
-              x[j + 1] = fmaf(x[j + 1], c4.y, -m4.y);
-              x[j + 2] = fmaf(x[j + 2], c4.z, -m4.z);
-              x[j + 3] = fmaf(x[j + 3], c4.w, -m4.w);
+              const float4 m4 = *reinterpret_cast<const float4*>(nm_g + j);
+              fma2(x[j], x[j + 1], x[j], x[j + 1], c4.x, c4.y, m4.x, m4.y);
+              fma2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], c4.z, c4.w, m4.z, m4.w);
             }
           }
         } else if (n == 0) {
 #pragma unroll
-          for (int j = 0; j < CG; ++j) x[j] *= cl;
+          for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], cl, cl);
         } else {
 #pragma unroll
           for (int j = 0; j < CG; j += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(m_g + j);
-            x[j] = fmaf(x[j], cl, -m4.x);
-            x[j + 1] = fmaf(x[j + 1], cl, -m4.y);
-            x[j + 2] = fmaf(x[j + 2], cl, -m4.z);
-            x[j + 3] = fmaf(x[j + 3], cl, -m4.w);
+            const float4 m4 = *reinterpret_cast<const float4*>(nm_g + j);
+            fma2(x[j], x[j + 1], x[j], x[j + 1], cl, cl, m4.x, m4.y);
+            fma2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], cl, cl, m4.z, m4.w);
           }
         }
-        if (kmask != 0xffffffffu && !((kmask >> lane) & 1u)) {  // not a key: a pad or out-of-tile row
+        if (kmask != 0xffffffffu) {  // the same word in every lane: a uniform branch
+          if (!((kmask >> lane) & 1u)) {  // not a key: a pad or out-of-tile row
 #pragma unroll
-          for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
+            for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
+          }
         }
         bool slow = true;
         if (n > 0) {
-          float t8[CG / 2];
-#pragma unroll
-          for (int j = 0; j < CG / 2; ++j) t8[j] = fmaxf(x[j], x[j + CG / 2]);
-#pragma unroll
-          for (int wdt = CG / 4; wdt > 0; wdt >>= 1)
-#pragma unroll
-            for (int j = 0; j < wdt; ++j) t8[j] = fmaxf(t8[j], t8[j + wdt]);
-          slow = named_bar_or(bar_vote, 128, t8[0] > kRescaleLog2);
+          static_assert(CG == 16, "the vote's maximum is written for 16 columns");
+          const float t = max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
+                               max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15]));
+          slow = named_bar_or(bar_vote, 128, t > kRescaleLog2);
         }
         ROLE_MARK(3);
         if (slow) {
@@ -743,10 +737,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float d;
             if (n == 0) {
               d = (c == -INFINITY) ? 0.0f : c;
-              m_g[tid] = d;
+              nm_g[tid] = -d;
             } else {
               d = fmaxf(c, 0.0f);
-              m_g[tid] += d;
+              nm_g[tid] -= d;  // -(m + d), rounded as m + d would be
             }
             delta_g[tid] = d;
           }
@@ -773,10 +767,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ROLE_MARK(4);
         // probabilities, partial row sums, this group's part of the P^T row (bf16, 128-byte swizzle)
 #pragma unroll
-        for (int j = 0; j < CG; ++j) {
-          x[j] = ex2_approx(x[j]);
-          l[j] += x[j];
-        }
+        for (int j = 0; j < CG; ++j) x[j] = ex2_approx(x[j]);
+#pragma unroll
+        for (int j = 0; j < CG; j += 2) add2(l[j], l[j + 1], l[j], l[j + 1], x[j], x[j + 1]);
         ROLE_MARK(5);
         mbar_wait(&bars[Ly::bPEmpty + pb], (pu & 1) ^ 1, ctl, 14);
         ROLE_MARK(6);
