@@ -279,10 +279,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < 4; ++s) {
       if (s < kSBufs) {
         mbar_init(&bars[Ly::bSFull + s], 1);
-        mbar_init(&bars[Ly::bSEmpty + s], kSoftWarps);
+        mbar_init(&bars[Ly::bSEmpty + s], kSoftWarps * 32);  // every softmax thread arrives
       }
       if (s < Ly::kPBufs) {
-        mbar_init(&bars[Ly::bPFull + s], kSoftWarps);
+        mbar_init(&bars[Ly::bPFull + s], kSoftWarps * 32);
         mbar_init(&bars[Ly::bPEmpty + s], 1);
       }
     }
@@ -671,8 +671,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
         ROLE_MARK(2);
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[Ly::bSEmpty + sb]);
+        mbar_arrive(&bars[Ly::bSEmpty + sb]);  // per thread: no warp-level branch or sync
 
         // x = logit * log2(e) - m  (m = 0 before the first block of the item); with 8-bit Q/K the
         // logit is the code product times the key and query scales
@@ -785,8 +784,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<U128*>(prow + ((c ^ (kl & 7)) << 4)) = w4;
         }
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[Ly::bPFull + pb]);
+        mbar_arrive(&bars[Ly::bPFull + pb]);
       }
 
       // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored):
