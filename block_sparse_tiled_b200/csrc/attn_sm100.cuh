@@ -51,6 +51,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "prep_kernels.cuh"
 #include "ptx.cuh"
@@ -642,14 +643,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int j = 0; j < CG; ++j) l[j] = 0.0f;
 
-      for (int n = 0; n < nb; ++n, ++g) {
+      // one block of the item; the first block (kFirst) takes the exact column maximum and needs no vote
+      auto block = [&](auto first_c, const int n) {
+        constexpr bool kFirst = decltype(first_c)::value;
         const int sb = g % kSBufs;
         const uint32_t su = g / kSBufs;
         const int pb = g % Ly::kPBufs;
         const uint32_t pu = g / Ly::kPBufs;
         ROLE_MARK(7);
         uint32_t kmask;
-        float ks = 1.0f;
+        [[maybe_unused]] float ks = 1.0f;
         if constexpr (kF8) {
           // the next block's key scale (and, every 32 blocks, mask words) are fetched one block ahead,
           // while this block waits and works
@@ -679,7 +682,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if constexpr (kF8) {
 #pragma unroll
           for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], ks, ks);
-          if (n == 0) {
+          if constexpr (kFirst) {
 #pragma unroll
             for (int j = 0; j < CG; j += 4) {
               const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
@@ -695,7 +698,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               fma2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], c4.z, c4.w, m4.z, m4.w);
             }
           }
-        } else if (n == 0) {
+        } else if constexpr (kFirst) {
 #pragma unroll
           for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], cl, cl);
         } else {
@@ -713,7 +716,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         bool slow = true;
-        if (n > 0) {
+        if constexpr (!kFirst) {
           static_assert(CG == 16, "the vote's maximum is written for 16 columns");
           const float t = max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
                                max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15]));
@@ -734,7 +737,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (tid < CG) {
             const float c = fmaxf(fmaxf(red_g[tid], red_g[CG + tid]), fmaxf(red_g[2 * CG + tid], red_g[3 * CG + tid]));
             float d;
-            if (n == 0) {
+            if constexpr (kFirst) {
               d = (c == -INFINITY) ? 0.0f : c;
               nm_g[tid] = -d;
             } else {
@@ -746,7 +749,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           named_bar_sync(bar_sync, 128);
 #pragma unroll
           for (int j = 0; j < CG; ++j) x[j] -= delta_g[j];
-          if (n > 0) {
+          if constexpr (!kFirst) {
 #pragma unroll
             for (int j = 0; j < CG; ++j) l[j] *= ex2_approx(-delta_g[j]);
             // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
@@ -785,7 +788,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[Ly::bPFull + pb]);
+      };
+      if (nb > 0) {
+        block(std::true_type{}, 0);
+        ++g;
       }
+      for (int n = 1; n < nb; ++n, ++g) block(std::false_type{}, n);
 
       // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored):
       // reduce-scatter over the warp's 32 lanes, lane j (j < CG) then holds column c0 + j
