@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ROLE_MARK(3);
         ok = mbar_wait(&bars[Ly::bQFull + qb], (it / Ly::kQBufs) & 1, ctl, 5);
         ROLE_MARK(0);
-        const uint32_t qbase = smem_u32(sm + Ly::oQ + qb * Ly::kQBytes);
+        const uint64_t qd0 = umma_desc_sw128(smem_u32(sm + Ly::oQ + qb * Ly::kQBytes), 16, 1024);
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int kst = g % Ly::kKStages;
           const int sb = g % kSBufs;
@@ -509,12 +509,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sm + Ly::oK + kst * Ly::kKBytes);
+          // descriptors of the block's first K-step; a step moves the start address (bits 0..13, 16-byte
+          // units, no carry: shared memory addresses stay below 256 KB) by a compile-time offset
+          const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oK + kst * Ly::kKBytes), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kQKSteps; ++kk) {
             // 32 bytes of every row per step: 16 bf16 or 32 8-bit elements
-            const uint64_t ad = umma_desc_sw128(kbase + (kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(qbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+            const uint64_t ad = ad0 + static_cast<uint64_t>(((kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32) >> 4);
+            const uint64_t bd = qd0 + static_cast<uint64_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
             if constexpr (kF8)
               umma_ss_f8(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
             else
@@ -557,16 +559,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ROLE_MARK(2);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vbase = smem_u32(sm + Ly::oV + vst * Ly::kKVBytes);
-          const uint32_t pbase = smem_u32(sm + Ly::oP + pb * Ly::kPBytes);
           // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
           const uint32_t lbo_v = (D > 64) ? Ly::kHalfBytes
                                             : static_cast<uint32_t>(Ly::oZ - (Ly::oV + vst * Ly::kKVBytes));
+          const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oV + vst * Ly::kKVBytes), lbo_v, 1024);
+          const uint64_t bd0 = umma_desc_sw128(smem_u32(sm + Ly::oP + pb * Ly::kPBytes), 8192, 1024);
 #pragma unroll
           for (int kk = 0; kk < kPVSteps; ++kk) {
-            const uint64_t ad = umma_desc_sw128(vbase + kk * 2048, lbo_v, 1024);
-            const uint64_t bd = umma_desc_sw128(pbase + kk * 2048, 8192, 1024);
-            umma_ss(tmem + kOCol0 + ob * 64, ad, bd, kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+            // a K-step is 16 keys = 2048 bytes further (start address in 16-byte units)
+            umma_ss(tmem + kOCol0 + ob * 64, ad0 + static_cast<uint64_t>(kk * 128), bd0 + static_cast<uint64_t>(kk * 128),
+                    kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars[Ly::bVEmpty + vst]);
           umma_commit(&bars[Ly::bPEmpty + pb]);
