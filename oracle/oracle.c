@@ -9,12 +9,14 @@
  *
  * Source of the method (the only place the pages state what VSA-H3 computes):
  *   "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse Attention is
- *   not optional here": 64-token (4,4,4) tiles over the post-patchify video
- *   grid, segment-pure prefix tiles, per-head fp32 pooled tile scores,
- *   topk = max(1, min(ceil((1 - sparsity) * n_video_tiles), n_video_tiles)),
- *   prefix keys always selected, prefix queries dense, and a compression
- *   branch softmax(scores) @ pool(v) broadcast over each tile row and scaled
- *   by the gate with no activation.
+ *   not optional here": the latent video grid is cut into 4x4x4 cubes of 64
+ *   tokens and each prefix segment into runs that never cross a segment;
+ *   tiles are scored per head in fp32 from their pooled (mean) Q and K;
+ *   topk = max(1, min(ceil((1 - sparsity) * n_video_tiles), n_video_tiles))
+ *   video key tiles are kept per video query tile, prefix keys are kept for
+ *   all of them and prefix queries see every key; a compression branch
+ *   softmax(scores) @ pool(v) gives one vector per tile that is multiplied by
+ *   the gate (no activation) and added to each row of the tile.
  * Supporting passages:
  *   "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Block-sparse FP4
  *   attention for VSA tiles": per-query-block lists of key blocks, partially
@@ -43,7 +45,7 @@
  *   R12 the per-channel variant: one gate per (batch, token, channel h*D + d), [B, L, H*D].
  *   R16 the 8-bit Q/K variant ("FastH3 OmniRef inference", section "The Blackwell stack" and
  *      "Fallbacks": query/key rounding to 8 bits with bf16 P.V, per-token FP8 Q/K; the
- *      multi-GPU notes of "FastH3 NVFP4 on RTX PRO 6000": one scale per token and head):
+ *      multi-GPU notes of "FastH3 NVFP4 on RTX PRO 6000": a scale for each token of each head):
  *      8 bits = OCP FP8 E4M3 ("E4M3FN": bias 7, no infinities, largest 448); one binary32
  *      scale per (batch, token, head), s = amax / 448 in binary32 where amax is the largest
  *      |x_d| of the token's head row; code_d = E4M3 round-to-nearest-even of the binary32
