@@ -22,7 +22,13 @@
 //     against the current m, and only when some logit exceeds m by more than
 //     kRescaleLog2 (or on the first block of an item) is the exact column
 //     maximum taken across the 128 lanes and O^T, l rescaled.  Any m with no
-//     overflow gives the same softmax, so this is exact up to rounding;
+//     overflow gives the same softmax, so this is exact up to rounding.
+//     Deciding "exceeds" takes a vote of the column group every block, unless
+//     the first block already shows that no later logit can overflow: with
+//     bf16 Q/K a logit is at most |q| max|k| (Cauchy-Schwarz), so when that
+//     bound is within skip_cap - log2(max|v|) of the first block's maximum for
+//     every column, P, l and O^T stay finite without further rescaling and the
+//     group skips the votes for the rest of the item;
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
 // O^T is double-buffered in TMEM, so one item's epilogue (in its own warps)
 // overlaps the next item's blocks.
@@ -125,6 +131,12 @@ struct AttnArgs {
   PartIO io;                 // where gate and out live (one tensor, or sequence parts, possibly on peers)
   const float* q_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each query row (tile order)
   const float* k_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each key row
+  // Overflow bound (bf16 Q/K; NULL: none, every block votes on a rescale): the Euclidean norm of each
+  // query row [B, H, n_rb, 64] in tile-order rows, and per (b, h) the largest key norm and |v| (float
+  // pairs); skip_cap = 124 - ceil(log2(keys of the longest list)).
+  const float* q_norm;
+  const float* kv_max;
+  float skip_cap;
   float scale_log2;  // softmax scale * log2(e)
   int64_t n_items;   // B * H * n_rb
 };
@@ -185,7 +197,8 @@ struct AttnLayout {
   static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
   static constexpr int oQtok = oGate + 256;                  // int qtok[64]: token within its part (epilogue)
   static constexpr int oQpart = oQtok + 256;                 // int qpart[64]: part holding the token
-  static constexpr int oEnd = oQpart + 256;
+  static constexpr int oSkip = oQpart + 256;                 // int skip[groups]: the item needs no votes
+  static constexpr int oEnd = oSkip + 16;
   static size_t bytes(int /*n_t*/) { return 1024 /*alignment slack*/ + oEnd; }
 };
 
@@ -599,6 +612,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // 8-bit Q/K: query scales (times cl) of the group's columns, one buffer per item parity (at a fixed
     // offset from m_g); the group's first warp fills the buffer before the item's first barrier
     constexpr int kQscFromM = (Ly::oQS - Ly::oM) / 4;
+    int* skip_s = reinterpret_cast<int*>(sm + Ly::oSkip);
+    // bf16 Q/K with an overflow bound: lanes 0..15 of the group's first warp hold, per item, the least
+    // first-block maximum m1 of their column for which no later block can overflow:
+    //   cl |q| max|k| + ceil(log2 max|v|)+ - skip_cap   (compared with m1 in log2 units; NaN: never)
+    // Tile-order rows are the query rows of the block; boxes read from sequence order hold a partial
+    // tile's rows at their cube positions, in the same order, so there the tile-order row is the rank
+    // of the position among the valid ones.
+    [[maybe_unused]] float lim = 0.0f;
+    auto item_limit = [&](int w, int r) -> float {
+      const int64_t bhw = w / n_t;
+      float qn;
+      if constexpr (kSeq) {
+        const uint64_t m = __ldg(a.key_mask + (w - bhw * n_t));
+        qn = ((m >> r) & 1ull) ? __ldg(a.q_norm + static_cast<int64_t>(w) * 64 + __popcll(m & ((1ull << r) - 1ull)))
+                               : 0.0f;
+      } else {
+        qn = __ldg(a.q_norm + static_cast<int64_t>(w) * 64 + r);
+      }
+      const float kmax = __ldg(a.kv_max + 2 * bhw), vmax = __ldg(a.kv_max + 2 * bhw + 1);
+      const int ev = max(0, static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 126);
+      return cl * qn * kmax + static_cast<float>(ev) - a.skip_cap;
+    };
     uint32_t g = 0;
     int it = 0;
     ROLE_TIMER_START();
@@ -608,6 +643,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if constexpr (kF8) {
         if (qd == 0 && lane < CG && w >= 0)
           m_g[kQscFromM + (it & 1) * 64 + lane] = __ldg(a.q_scale + static_cast<int64_t>(w) * 64 + c0 + lane) * cl;
+      }
+      if constexpr (!kF8) {
+        if (a.q_norm != nullptr && qd == 0 && lane < CG && w >= 0) lim = item_limit(w, c0 + lane);
       }
       if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
@@ -644,6 +682,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float l[CG];
 #pragma unroll
       for (int j = 0; j < CG; ++j) l[j] = 0.0f;
+      bool skip = false;  // set by the first block: the item's later blocks take no vote
 
       // one block of the item; the first block (kFirst) takes the exact column maximum and needs no vote
       auto block = [&](auto first_c, const int n) {
@@ -719,10 +758,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         bool slow = true;
         if constexpr (!kFirst) {
-          static_assert(CG == 16, "the vote's maximum is written for 16 columns");
-          const float t = max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
-                               max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15]));
-          slow = named_bar_or(bar_vote, 128, t > kRescaleLog2);
+          if (skip) {  // the same in all 128 threads of the group
+            slow = false;
+          } else {
+            static_assert(CG == 16, "the vote's maximum is written for 16 columns");
+            const float t = max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
+                                 max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15]));
+            slow = named_bar_or(bar_vote, 128, t > kRescaleLog2);
+          }
         }
         ROLE_MARK(3);
         if (slow) {
@@ -742,6 +785,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if constexpr (kFirst) {
               d = (c == -INFINITY) ? 0.0f : c;
               nm_g[tid] = -d;
+              if constexpr (!kF8) {
+                if (a.q_norm != nullptr) {  // lanes 0..15 of the group's first warp
+                  const uint32_t ok = __ballot_sync(0xffffu, lim <= d);
+                  if (tid == 0) skip_s[grp] = (ok == 0xffffu) ? 1 : 0;
+                }
+              }
             } else {
               d = fmaxf(c, 0.0f);
               nm_g[tid] -= d;  // -(m + d), rounded as m + d would be
@@ -749,6 +798,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             delta_g[tid] = d;
           }
           named_bar_sync(bar_sync, 128);
+          if constexpr (kFirst && !kF8) skip = (a.q_norm != nullptr) && skip_s[grp] != 0;
 #pragma unroll
           for (int j = 0; j < CG; ++j) x[j] -= delta_g[j];
           if constexpr (!kFirst) {

@@ -50,6 +50,75 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 }
 
 // ---------------------------------------------------------------------------
+// Magnitude statistics of a tile held in shared memory as [3][rows][D] bf16 (Q, K, V; pad rows zero),
+// for the attention's overflow bound (a logit is at most |q| |k| by Cauchy-Schwarz):
+//   q_n[r]   = Euclidean norm of query row r, binary32
+//   kv[0]    = max over the tile's key rows of the Euclidean norm  } atomicMax on the binary32 bits,
+//   kv[1]    = max over the tile's value entries of |v|             } so kv holds the (b, h) maxima
+// Threads [128 t, 128 t + 128) handle tensor t, thread r row r; each row is summed over its 16-byte
+// chunks starting at chunk r (shared-memory banks), the same order wherever this function runs.
+// A NaN or infinity in a row makes its statistic NaN or infinity (the |v| maximum compares magnitude
+// bits, so a NaN is the largest), which the attention reads as "no bound".
+// ---------------------------------------------------------------------------
+template <int D, int kRows>
+__device__ __forceinline__ void tile_stats(const uint16_t* tiles, float* q_n, uint32_t* kv) {
+  constexpr int kChunks = D / 8;
+  const int tsr = threadIdx.x >> 7, r = threadIdx.x & 127;
+  if (r >= kRows) return;  // whole warps (kRows is 64 or 128)
+  const uint4* row = reinterpret_cast<const uint4*>(tiles + (tsr * kRows + r) * D);
+  float ss = 0.0f;
+  uint32_t mag = 0;
+  int c = r % kChunks;
+#pragma unroll 4
+  for (int j = 0; j < kChunks; ++j) {
+    const uint4 u = row[c];
+    c = (c + 1 == kChunks) ? 0 : c + 1;
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if (tsr == 2) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mag = max(mag, max(w[e] & 0x7fffu, (w[e] >> 16) & 0x7fffu));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+        ss = fmaf(lo, lo, ss);
+        ss = fmaf(hi, hi, ss);
+      }
+    }
+  }
+  if (tsr == 0) {
+    q_n[r] = __fsqrt_rn(ss);
+    return;
+  }
+  // non-negative binary32 values (and NaN with the sign bit clear) order like their bits
+  uint32_t bits = (tsr == 1) ? (__float_as_uint(__fsqrt_rn(ss)) & 0x7fffffffu) : (mag << 16);
+  bits = __reduce_max_sync(0xffffffffu, bits);
+  if ((threadIdx.x & 31) == 0) atomicMax(kv + (tsr - 1), bits);
+}
+
+// Magnitude statistics from tile-order copies [B, H, n_t, rows, D] (the step entry point of the
+// attention): one CTA per (tile, head, batch) stages the three tiles and runs tile_stats.
+template <int D, int kRows>
+__global__ void __launch_bounds__(384) tile_stats_kernel(const uint16_t* __restrict__ q_t,
+                                                          const uint16_t* __restrict__ k_t,
+                                                          const uint16_t* __restrict__ v_t, float* __restrict__ q_n,
+                                                          uint32_t* __restrict__ kv, int H, int n_t) {
+  constexpr int kChunks = D / 8;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_raw);
+  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  const int64_t row0 = (bh * n_t + tile) * kRows;
+  const int tsr = threadIdx.x >> 7, tl = threadIdx.x & 127;
+  const uint16_t* src = (tsr == 0) ? q_t : (tsr == 1) ? k_t : v_t;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + row0 * D);
+  uint4* d4 = reinterpret_cast<uint4*>(tiles + tsr * kRows * D);
+  for (int e = tl; e < kRows * kChunks; e += 128) d4[e] = __ldg(s4 + e);
+  __syncthreads();
+  tile_stats<D, kRows>(tiles, q_n + row0, kv + 2 * bh);
+}
+
+// ---------------------------------------------------------------------------
 // S2 (+ S3 pooling): sequence order [B, L, H, D] -> tile order [B, H, n_t, 64*kSub, D]
 // One CTA per (tile, head, batch) moves the tile of Q, K and V (64 rows, or 128
 // for 128-token tiles: kSub = 2) with 16-byte loads/stores (each 256-byte token
@@ -75,7 +144,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     void* __restrict__ q_t, void* __restrict__ k_t, uint16_t* __restrict__ v_t, float* __restrict__ q_s,
     float* __restrict__ k_s, float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
-    int n_t, const PartIO io) {
+    int n_t, const PartIO io, float* __restrict__ q_n, uint32_t* __restrict__ kv) {
   constexpr int kRows = kTile * kSub;                             // rows of one tile
   constexpr int kChunks = D / 8;                                  // 16-byte chunks per row
   constexpr int kIters = kF8 ? kRows / 8 : kRows * kChunks / 128;  // chunks each thread moves per tensor
@@ -164,6 +233,10 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   }
   if (!pool) return;
   __syncthreads();
+  // with pooling, the magnitude statistics of the staged tiles too (bf16 copies only)
+  if constexpr (!kF8) {
+    if (q_n != nullptr) tile_stats<D, kRows>(tiles, q_n + tile_row0, kv + 2 * (static_cast<int64_t>(b) * H + h));
+  }
   const int n = tile_valid[tile];
   float* out = (tsr == 0) ? pq : (tsr == 1) ? pk : pv;
   for (int d = tl; d < D; d += 128) {

@@ -281,6 +281,8 @@ void build_seq_tables(const Resolved& r, const std::vector<uint64_t>& mask_tiled
 // seq_tiles: no tile-order copies (their regions are empty).
 // qk_fp8: q_t and k_t hold 8-bit codes, 128 bytes per row whatever D, and q_s, k_s one float per row.
 // tile: tokens per tile (the copies hold n_t * tile rows per (b, h)).
+// Without qk_fp8, q_n and kv_max hold the attention's overflow-bound statistics: the norm of every
+// query row (tile-order rows) and, per (b, h), the largest key norm and |v| (two floats).
 vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t tile, int64_t V, int64_t topk,
                                  bool seq_tiles,
                                  bool qk_fp8) {
@@ -295,6 +297,8 @@ vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, i
   w.v_t = off; off += align256(tiles);
   w.q_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
   w.k_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
+  w.q_n = off; off += align256(qk_fp8 ? 0 : rows * 4);
+  w.kv_max = off; off += align256(qk_fp8 ? 0 : static_cast<size_t>(B * H * 8));
   w.pq = off; off += align256(pooled);
   w.pk = off; off += align256(pooled);
   w.pv = off; off += align256(pooled);
@@ -454,6 +458,9 @@ struct vsa_plan_s {
   int32_t* d_coord = nullptr;  // [n_t][4]
   uint64_t* d_mask_seq = nullptr;
   uint64_t* d_mask_tiled = nullptr;
+  // vsa_sparse_attn_fwd (bf16 plans): the overflow-bound statistics of its tile-order inputs, query row
+  // norms then the (b, h) maxima
+  float* d_stats = nullptr;
   int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter, [3] gate nonzero
   vsa_workspace_layout ws{};
   // Head-slice plans share the parent's device tables and status word and own nothing on the device.
@@ -517,9 +524,11 @@ vsa_status with_head_dim(int D, F&& f) {
 vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H, 0}; }
 
 // qs/ks: with an 8-bit plan, the per-row scales (qt/kt then receive codes).
+// qn/kv (bf16 plans, with pooling): the overflow-bound statistics of the staged tiles; kv must hold
+// zeros on entry (the kernel raises it with atomicMax).
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
                       float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr, float* qs = nullptr,
-                      float* ks = nullptr) {
+                      float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr) {
   const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
@@ -532,7 +541,7 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   auto launch = [&](auto kernel) -> vsa_status {
     VSA_TRY(allow_smem(kernel, smem));
     kernel<<<grid, 384, smem, s>>>(qq, kk, vv, qt, kt, vo, qs, ks, pq, pk, pv, p->d_tile_token, p->d_tile_valid,
-                                   p->r.L, p->H, p->n_t, pio);
+                                   p->r.L, p->H, p->n_t, pio, qn, kv);
     return VSA_OK;
   };
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
@@ -546,6 +555,35 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
                  : by_tile(vsa::gather_pool_kernel<D, false, false, 1>, vsa::gather_pool_kernel<D, false, false, 2>);
   }));
   return launch_check("gather_pool");
+}
+
+// Plan-owned statistics of the step attention: row norms (256-aligned), then B*H float pairs.
+size_t stats_rows_bytes(const vsa_plan_s* p) {
+  return align256(static_cast<size_t>(p->B) * p->H * p->n_t * p->r.tile * 4);
+}
+size_t stats_bytes(const vsa_plan_s* p) { return stats_rows_bytes(p) + static_cast<size_t>(p->B) * p->H * 8; }
+
+// The overflow-bound statistics of tile-order copies (what the gather computes while pooling); kv is
+// zeroed here.
+vsa_status run_tile_stats(vsa_plan p, const void* qt, const void* kt, const void* vt, float* qn, uint32_t* kv,
+                          cudaStream_t s) {
+  VSA_CUDA_TRY(cudaMemsetAsync(kv, 0, static_cast<size_t>(p->B) * p->H * 8, s));
+  if (p->n_t == 0) return VSA_OK;
+  const size_t smem = static_cast<size_t>(3) * p->r.tile * p->D * 2;
+  dim3 grid(p->n_t, p->H, p->B);
+  const auto* a = static_cast<const uint16_t*>(qt);
+  const auto* b = static_cast<const uint16_t*>(kt);
+  const auto* c = static_cast<const uint16_t*>(vt);
+  auto launch = [&](auto kernel) -> vsa_status {
+    VSA_TRY(allow_smem(kernel, smem));
+    kernel<<<grid, 384, smem, s>>>(a, b, c, qn, kv, p->H, p->n_t);
+    return VSA_OK;
+  };
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    return p->r.sh ? launch(vsa::tile_stats_kernel<D, 128>) : launch(vsa::tile_stats_kernel<D, 64>);
+  }));
+  return launch_check("tile statistics");
 }
 
 vsa_status run_pool(vsa_plan p, const void* qt, const void* kt, const void* vt, float* pq, float* pk, float* pv,
@@ -606,7 +644,7 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
                     const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
                     const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr, const float* qs = nullptr,
-                    const float* ks = nullptr) {
+                    const float* ks = nullptr, const float* qn = nullptr, const uint32_t* kv = nullptr) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
   // the kernel works in 64-row blocks: one per tile, or two per 128-token tile
@@ -648,6 +686,15 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.io = io ? *io : single_io(p);
   a.q_scale = qs;
   a.k_scale = ks;
+  // overflow bound: P <= 2^gap per key, so l <= keys * 2^gap < 2^126 (its reciprocal stays normal) and
+  // |O| <= keys * 2^gap * max|v| < 2^125 when gap <= 124 - ceil(log2 keys) - ceil(log2 max|v|)+
+  if (!p->qk_fp8 && qn != nullptr && kv != nullptr) {
+    int lg = 0;
+    while ((int64_t{1} << lg) < static_cast<int64_t>(p->n_t) * p->r.tile) ++lg;
+    a.q_norm = qn;
+    a.kv_max = reinterpret_cast<const float*>(kv);
+    a.skip_cap = static_cast<float>(124 - lg);
+  }
   a.gate_ld = gate_ld > 0 ? gate_ld : (p->gate_pc ? p->H * p->D : p->H);
   a.n_t = static_cast<int>(n_rb);
   a.sub_shift = p->r.sh;
@@ -765,6 +812,9 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
   auto* qsc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.q_s) : nullptr;
   auto* ksc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.k_s) : nullptr;
+  auto* qn = p->qk_fp8 ? nullptr : reinterpret_cast<float*>(w + p->ws.q_n);
+  auto* kv = p->qk_fp8 ? nullptr : reinterpret_cast<uint32_t*>(w + p->ws.kv_max);
+  if (kv != nullptr) VSA_CUDA_TRY(cudaMemsetAsync(kv, 0, static_cast<size_t>(p->B) * p->H * 8, s));
   // does any gate differ from zero?  (if not, the compression branch is skipped on the device)
   int* gate_nz = p->d_status + 3;
   // sequence parts: the gate is spread over the parts and is not scanned; the branch is kept
@@ -787,11 +837,12 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   // With seq_tiles the attention reads Q/K/V straight from sequence order and the gather only pools;
   // otherwise the gather writes tile-order copies, which the attention reads with better DRAM locality.
   const bool seq = p->seq_tiles;
-  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io, qsc, ksc));
+  VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io, qsc, ksc,
+                     qn, kv));
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
-  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io, qsc, ksc);
+  return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io, qsc, ksc, qn, kv);
 }
 
 // Gate elements per token: H, or H*D for a per-channel gate.
@@ -893,6 +944,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     cudaFree(p->d_status);
     cudaFree(p->d_exempt);
     cudaFree(p->d_refs);
+    cudaFree(p->d_stats);
     delete p;
   };
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -907,7 +959,8 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
       cudaMalloc(&p->d_mask_tiled, block_mask_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess ||
       (p->n_ref > 0 && (cudaMalloc(&p->d_exempt, std::max<size_t>(4, p->exempt_tiles.size() * 4)) != cudaSuccess ||
-                        cudaMalloc(&p->d_refs, p->ref_tiles.size() * 4) != cudaSuccess))) {
+                        cudaMalloc(&p->d_refs, p->ref_tiles.size() * 4) != cudaSuccess)) ||
+      (!p->qk_fp8 && cudaMalloc(&p->d_stats, stats_bytes(p)) != cudaSuccess)) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
   }
@@ -985,6 +1038,7 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
     cudaFree(p->d_status);
     cudaFree(p->d_exempt);
     cudaFree(p->d_refs);
+    cudaFree(p->d_stats);
   }
   if (prev >= 0) cudaSetDevice(prev);
   delete p;
@@ -1030,7 +1084,12 @@ vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* 
   if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q_t, k_t, v_t, o_c, gate, out}));
   if (p->V > 0) VSA_TRY(check_ptrs({idx}));
-  return run_attn(p, q_t, k_t, v_t, idx, o_c, gate, out, static_cast<cudaStream_t>(stream));
+  const auto s = static_cast<cudaStream_t>(stream);
+  // the overflow bound from these inputs' own statistics (the forward takes them from its gather)
+  float* qn = p->d_stats;
+  auto* kv = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p->d_stats) + stats_rows_bytes(p));
+  VSA_TRY(run_tile_stats(p, q_t, k_t, v_t, qn, kv, s));
+  return run_attn(p, q_t, k_t, v_t, idx, o_c, gate, out, s, 0, nullptr, nullptr, nullptr, nullptr, nullptr, qn, kv);
 }
 
 vsa_status vsa_forward(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const vsa_bf16* gate,

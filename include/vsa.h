@@ -228,7 +228,10 @@ vsa_status vsa_topk_select(vsa_plan p, const float* scores_dev, const float* pv_
  * attention for VSA tiles" (block lists, exempt prefix key tile visited
  * first); "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
  * Attention is not optional here" (dense prefix queries; gated compression
- * branch with no activation). */
+ * branch with no activation).
+ * The call first takes the norms of q_t's rows and the largest key norm and
+ * |v| of k_t, v_t (one extra kernel, into a buffer the plan owns, so calls on
+ * one plan must not overlap); the output is bit-identical to vsa_forward's. */
 vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf16* k_t_dev,
                                const vsa_bf16* v_t_dev, const int32_t* idx_dev,
                                const float* o_c_dev, const vsa_bf16* gate_dev,
@@ -339,9 +342,14 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
 /* Byte offsets of the intermediates inside vsa_forward's workspace.  With
  * qk_fp8, q_t and k_t hold E4M3 codes [B, H, n_tiles, 64, 128] (128 bytes per
  * row whatever D; bytes D..127 zero) and q_s, k_s the row scales [B, H,
- * n_tiles, 64] float32 (0 for pad rows); otherwise q_s and k_s are empty. */
+ * n_tiles, 64] float32 (0 for pad rows); otherwise q_s and k_s are empty.
+ * Without qk_fp8, q_n holds the Euclidean norm of every query row [B, H,
+ * n_tiles, tile_size] float32 (tile-order rows, 0 for pad rows) and kv_max,
+ * per (b, h), the largest key-row norm and the largest |v| (two float32); the
+ * attention bounds its logits by them (Cauchy-Schwarz) to skip rescale checks
+ * that cannot fire.  With qk_fp8 both are empty. */
 typedef struct vsa_workspace_layout {
-  size_t q_t, k_t, v_t, q_s, k_s, pq, pk, pv, scores, idx, o_c, total;
+  size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c, total;
 } vsa_workspace_layout;
 vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
 
