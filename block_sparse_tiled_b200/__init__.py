@@ -453,9 +453,9 @@ def device_status(plan, stream=None):
 def workspace_views(plan, workspace):
     """Typed views of vsa_forward's intermediates inside ``workspace`` (no tile-order views for a plan
     with seq_tiles, whose workspace holds none).  With qk_fp8, q_t and k_t are the E4M3 codes
-    [B, H, n_t, tile, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, tile]; without it, q_n
-    holds the query row norms [B, H, n_t, tile] and kv_max the (b, h) maxima of key norm and |v|
-    [B, H, 2] (the attention's overflow bound)."""
+    [B, H, n_t, tile, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, tile].  q_n holds the
+    query row norms [B, H, n_t, tile] (with qk_fp8 of the dequantised rows) and kv_max the (b, h)
+    maxima of key norm and |v| [B, H, 2] (the attention's overflow bound)."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
@@ -482,8 +482,8 @@ def workspace_views(plan, workspace):
         "v_t": tiles("v_t"),
         "q_s": row_scales("q_s"),
         "k_s": row_scales("k_s"),
-        "q_n": None if f8 else view(lay["q_n"], B * H * n_t * T, torch.float32, (B, H, n_t, T)),
-        "kv_max": None if f8 else view(lay["kv_max"], B * H * 2, torch.float32, (B, H, 2)),
+        "q_n": view(lay["q_n"], B * H * n_t * T, torch.float32, (B, H, n_t, T)),
+        "kv_max": view(lay["kv_max"], B * H * 2, torch.float32, (B, H, 2)),
         "pq": view(lay["pq"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pk": view(lay["pk"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),
         "pv": view(lay["pv"], B * H * n_t * D, torch.float32, (B, H, n_t, D)),

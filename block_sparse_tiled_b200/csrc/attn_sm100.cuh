@@ -24,8 +24,8 @@
 //     maximum taken across the 128 lanes and O^T, l rescaled.  Any m with no
 //     overflow gives the same softmax, so this is exact up to rounding.
 //     Deciding "exceeds" takes a vote of the column group every block, unless
-//     the first block already shows that no later logit can overflow: with
-//     bf16 Q/K a logit is at most |q| max|k| (Cauchy-Schwarz), so when that
+//     the first block already shows that no later logit can overflow: a
+//     logit is at most |q| max|k| (Cauchy-Schwarz), so when that
 //     bound is within skip_cap - log2(max|v|) of the first block's maximum for
 //     every column, P, l and O^T stay finite without further rescaling and the
 //     group skips the votes for the rest of the item;
@@ -131,9 +131,10 @@ struct AttnArgs {
   PartIO io;                 // where gate and out live (one tensor, or sequence parts, possibly on peers)
   const float* q_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each query row (tile order)
   const float* k_scale;      // 8-bit Q/K only: [B, H, n_rb, 64] scale of each key row
-  // Overflow bound (bf16 Q/K; NULL: none, every block votes on a rescale): the Euclidean norm of each
-  // query row [B, H, n_rb, 64] in tile-order rows, and per (b, h) the largest key norm and |v| (float
-  // pairs); skip_cap = 124 - ceil(log2(keys of the longest list)).
+  // Overflow bound (NULL: none, every block votes on a rescale): the Euclidean norm of each query row
+  // [B, H, n_rb, 64] in tile-order rows (8-bit Q/K: of the dequantised row, scale times code norm), and
+  // per (b, h) the largest key norm and |v| (float pairs); skip_cap = 124 - ceil(log2(keys of the
+  // longest list)).
   const float* q_norm;
   const float* kv_max;
   float skip_cap;
@@ -613,13 +614,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // offset from m_g); the group's first warp fills the buffer before the item's first barrier
     constexpr int kQscFromM = (Ly::oQS - Ly::oM) / 4;
     int* skip_s = reinterpret_cast<int*>(sm + Ly::oSkip);
-    // bf16 Q/K with an overflow bound: lanes 0..15 of the group's first warp hold, per item, the least
+    // With an overflow bound, lanes 0..15 of the group's first warp hold, per item, the least
     // first-block maximum m1 of their column for which no later block can overflow:
     //   cl |q| max|k| + ceil(log2 max|v|)+ - skip_cap   (compared with m1 in log2 units; NaN: never)
     // Tile-order rows are the query rows of the block; boxes read from sequence order hold a partial
     // tile's rows at their cube positions, in the same order, so there the tile-order row is the rank
     // of the position among the valid ones.
-    [[maybe_unused]] float lim = 0.0f;
+    float lim = 0.0f;
     auto item_limit = [&](int w, int r) -> float {
       const int64_t bhw = w / n_t;
       float qn;
@@ -644,9 +645,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (qd == 0 && lane < CG && w >= 0)
           m_g[kQscFromM + (it & 1) * 64 + lane] = __ldg(a.q_scale + static_cast<int64_t>(w) * 64 + c0 + lane) * cl;
       }
-      if constexpr (!kF8) {
-        if (a.q_norm != nullptr && qd == 0 && lane < CG && w >= 0) lim = item_limit(w, c0 + lane);
-      }
+      if (a.q_norm != nullptr && qd == 0 && lane < CG && w >= 0) lim = item_limit(w, c0 + lane);
       if (named_bar_or(bar_vote, 128, w < 0)) break;  // the group stops together
       const int64_t bh = w / n_t;
       const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
@@ -785,11 +784,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if constexpr (kFirst) {
               d = (c == -INFINITY) ? 0.0f : c;
               nm_g[tid] = -d;
-              if constexpr (!kF8) {
-                if (a.q_norm != nullptr) {  // lanes 0..15 of the group's first warp
-                  const uint32_t ok = __ballot_sync(0xffffu, lim <= d);
-                  if (tid == 0) skip_s[grp] = (ok == 0xffffu) ? 1 : 0;
-                }
+              if (a.q_norm != nullptr) {  // lanes 0..15 of the group's first warp
+                const uint32_t ok = __ballot_sync(0xffffu, lim <= d);
+                if (tid == 0) skip_s[grp] = (ok == 0xffffu) ? 1 : 0;
               }
             } else {
               d = fmaxf(c, 0.0f);
@@ -798,7 +795,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             delta_g[tid] = d;
           }
           named_bar_sync(bar_sync, 128);
-          if constexpr (kFirst && !kF8) skip = (a.q_norm != nullptr) && skip_s[grp] != 0;
+          if constexpr (kFirst) skip = (a.q_norm != nullptr) && skip_s[grp] != 0;
 #pragma unroll
           for (int j = 0; j < CG; ++j) x[j] -= delta_g[j];
           if constexpr (!kFirst) {

@@ -51,7 +51,8 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 
 // ---------------------------------------------------------------------------
 // Magnitude statistics of a tile held in shared memory as [3][rows][D] bf16 (Q, K, V; pad rows zero),
-// for the attention's overflow bound (a logit is at most |q| |k| by Cauchy-Schwarz):
+// for the attention's overflow bound (a logit is at most |q| |k| by Cauchy-Schwarz; kQK = false: the
+// value statistic only, the 8-bit gather takes the Q/K norms from its codes):
 //   q_n[r]   = Euclidean norm of query row r, binary32
 //   kv[0]    = max over the tile's key rows of the Euclidean norm  } atomicMax on the binary32 bits,
 //   kv[1]    = max over the tile's value entries of |v|             } so kv holds the (b, h) maxima
@@ -60,11 +61,12 @@ __device__ __forceinline__ T* part_base(const PartIO& io, int op, T* single, int
 // A NaN or infinity in a row makes its statistic NaN or infinity (the |v| maximum compares magnitude
 // bits, so a NaN is the largest), which the attention reads as "no bound".
 // ---------------------------------------------------------------------------
-template <int D, int kRows>
+template <int D, int kRows, bool kQK = true>
 __device__ __forceinline__ void tile_stats(const uint16_t* tiles, float* q_n, uint32_t* kv) {
   constexpr int kChunks = D / 8;
   const int tsr = threadIdx.x >> 7, r = threadIdx.x & 127;
   if (r >= kRows) return;  // whole warps (kRows is 64 or 128)
+  if (!kQK && tsr < 2) return;
   const uint4* row = reinterpret_cast<const uint4*>(tiles + (tsr * kRows + r) * D);
   float ss = 0.0f;
   uint32_t mag = 0;
@@ -194,6 +196,9 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
   // q_t == NULL: pooling only (the attention then reads sequence order itself)
   const bool write_tiles = (q_t != nullptr);
   const bool codes = kF8 && tsr < 2;
+  // 8-bit keys: this thread's largest row norm, as bits (non-negative binary32 values, and NaN with the
+  // sign bit clear, order like their bits, so a NaN wins)
+  [[maybe_unused]] uint32_t kn_bits = 0;
 #pragma unroll
   for (int u = 0; u < kIters; ++u) {
     int r, c;
@@ -226,17 +231,42 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
       uint8_t* crow = static_cast<uint8_t*>(tsr == 0 ? q_t : k_t) + (tile_row0 + r) * kF8RowBytes;
       *reinterpret_cast<uint2*>(crow + c * 8) = make_uint2(packed[0], packed[1]);  // idle lanes: zero padding
       if (c == 0) (tsr == 0 ? q_s : k_s)[tile_row0 + r] = sc;
+      if (q_n != nullptr) {
+        // the Euclidean norm of the row as the attention sees it: scale times the norm of its codes
+        float css = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+              static_cast<__nv_fp8x2_storage_t>(packed[j >> 1] >> (16 * (j & 1))), __NV_E4M3);
+          const float2 cv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+          css = fmaf(cv.x, cv.x, css);
+          css = fmaf(cv.y, cv.y, css);
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) css += __shfl_xor_sync(0xffffffffu, css, off);
+        const float nrm = sc * __fsqrt_rn(css);
+        if (tsr == 0) {
+          if (c == 0) q_n[tile_row0 + r] = nrm;
+        } else {
+          kn_bits = max(kn_bits, __float_as_uint(nrm) & 0x7fffffffu);
+        }
+      }
     } else if (active) {
       uint16_t* dst = (tsr == 0) ? static_cast<uint16_t*>(q_t) : (tsr == 1) ? static_cast<uint16_t*>(k_t) : v_t;
       reinterpret_cast<uint4*>(dst + tile_row0 * D)[r * kChunks + c] = val[u];
     }
   }
+  if constexpr (kF8) {
+    if (q_n != nullptr && tsr == 1 && write_tiles) {
+      const uint32_t bits = __reduce_max_sync(0xffffffffu, kn_bits);
+      if ((threadIdx.x & 31) == 0) atomicMax(kv + 2 * (static_cast<int64_t>(b) * H + h), bits);
+    }
+  }
   if (!pool) return;
   __syncthreads();
-  // with pooling, the magnitude statistics of the staged tiles too (bf16 copies only)
-  if constexpr (!kF8) {
-    if (q_n != nullptr) tile_stats<D, kRows>(tiles, q_n + tile_row0, kv + 2 * (static_cast<int64_t>(b) * H + h));
-  }
+  // with pooling, the magnitude statistics of the staged tiles too (8-bit Q/K: the value statistic only)
+  if (q_n != nullptr)
+    tile_stats<D, kRows, !kF8>(tiles, q_n + tile_row0, kv + 2 * (static_cast<int64_t>(b) * H + h));
   const int n = tile_valid[tile];
   float* out = (tsr == 0) ? pq : (tsr == 1) ? pk : pv;
   for (int d = tl; d < D; d += 128) {

@@ -281,8 +281,8 @@ void build_seq_tables(const Resolved& r, const std::vector<uint64_t>& mask_tiled
 // seq_tiles: no tile-order copies (their regions are empty).
 // qk_fp8: q_t and k_t hold 8-bit codes, 128 bytes per row whatever D, and q_s, k_s one float per row.
 // tile: tokens per tile (the copies hold n_t * tile rows per (b, h)).
-// Without qk_fp8, q_n and kv_max hold the attention's overflow-bound statistics: the norm of every
-// query row (tile-order rows) and, per (b, h), the largest key norm and |v| (two floats).
+// q_n and kv_max hold the attention's overflow-bound statistics: the norm of every query row (tile-order
+// rows; with qk_fp8 of the dequantised row) and, per (b, h), the largest key norm and |v| (two floats).
 vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t tile, int64_t V, int64_t topk,
                                  bool seq_tiles,
                                  bool qk_fp8) {
@@ -297,8 +297,8 @@ vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, i
   w.v_t = off; off += align256(tiles);
   w.q_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
   w.k_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
-  w.q_n = off; off += align256(qk_fp8 ? 0 : rows * 4);
-  w.kv_max = off; off += align256(qk_fp8 ? 0 : static_cast<size_t>(B * H * 8));
+  w.q_n = off; off += align256(rows * 4);
+  w.kv_max = off; off += align256(static_cast<size_t>(B * H * 8));
   w.pq = off; off += align256(pooled);
   w.pk = off; off += align256(pooled);
   w.pv = off; off += align256(pooled);
@@ -524,8 +524,8 @@ vsa_status with_head_dim(int D, F&& f) {
 vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H, 0}; }
 
 // qs/ks: with an 8-bit plan, the per-row scales (qt/kt then receive codes).
-// qn/kv (bf16 plans, with pooling): the overflow-bound statistics of the staged tiles; kv must hold
-// zeros on entry (the kernel raises it with atomicMax).
+// qn/kv (with pooling): the overflow-bound statistics of the staged tiles (8-bit Q/K: Q/K norms from the
+// codes); kv must hold zeros on entry (the kernel raises it with atomicMax).
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
                       float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr, float* qs = nullptr,
                       float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr) {
@@ -688,7 +688,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.k_scale = ks;
   // overflow bound: P <= 2^gap per key, so l <= keys * 2^gap < 2^126 (its reciprocal stays normal) and
   // |O| <= keys * 2^gap * max|v| < 2^125 when gap <= 124 - ceil(log2 keys) - ceil(log2 max|v|)+
-  if (!p->qk_fp8 && qn != nullptr && kv != nullptr) {
+  if (qn != nullptr && kv != nullptr) {
     int lg = 0;
     while ((int64_t{1} << lg) < static_cast<int64_t>(p->n_t) * p->r.tile) ++lg;
     a.q_norm = qn;
@@ -812,9 +812,9 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   auto* oc = reinterpret_cast<float*>(w + p->ws.o_c);
   auto* qsc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.q_s) : nullptr;
   auto* ksc = p->qk_fp8 ? reinterpret_cast<float*>(w + p->ws.k_s) : nullptr;
-  auto* qn = p->qk_fp8 ? nullptr : reinterpret_cast<float*>(w + p->ws.q_n);
-  auto* kv = p->qk_fp8 ? nullptr : reinterpret_cast<uint32_t*>(w + p->ws.kv_max);
-  if (kv != nullptr) VSA_CUDA_TRY(cudaMemsetAsync(kv, 0, static_cast<size_t>(p->B) * p->H * 8, s));
+  auto* qn = reinterpret_cast<float*>(w + p->ws.q_n);
+  auto* kv = reinterpret_cast<uint32_t*>(w + p->ws.kv_max);
+  VSA_CUDA_TRY(cudaMemsetAsync(kv, 0, static_cast<size_t>(p->B) * p->H * 8, s));
   // does any gate differ from zero?  (if not, the compression branch is skipped on the device)
   int* gate_nz = p->d_status + 3;
   // sequence parts: the gate is spread over the parts and is not scanned; the branch is kept

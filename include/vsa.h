@@ -343,11 +343,12 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
  * qk_fp8, q_t and k_t hold E4M3 codes [B, H, n_tiles, 64, 128] (128 bytes per
  * row whatever D; bytes D..127 zero) and q_s, k_s the row scales [B, H,
  * n_tiles, 64] float32 (0 for pad rows); otherwise q_s and k_s are empty.
- * Without qk_fp8, q_n holds the Euclidean norm of every query row [B, H,
- * n_tiles, tile_size] float32 (tile-order rows, 0 for pad rows) and kv_max,
- * per (b, h), the largest key-row norm and the largest |v| (two float32); the
- * attention bounds its logits by them (Cauchy-Schwarz) to skip rescale checks
- * that cannot fire.  With qk_fp8 both are empty. */
+ * q_n holds the Euclidean norm of every query row [B, H, n_tiles, tile_size]
+ * float32 (tile-order rows, 0 for pad rows; with qk_fp8 the norm of the
+ * dequantised row, scale times code norm) and kv_max, per (b, h), the largest
+ * key-row norm (likewise) and the largest |v| (two float32); the attention
+ * bounds its logits by them (Cauchy-Schwarz) to skip rescale checks that
+ * cannot fire. */
 typedef struct vsa_workspace_layout {
   size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c, total;
 } vsa_workspace_layout;

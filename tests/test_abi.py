@@ -152,15 +152,12 @@ def test_seq_tiles_workspace_and_limits(vsa):
 
 def test_qk_fp8_workspace_and_limits(vsa):
     """8-bit Q/K: q_t/k_t hold one 128-byte code row per tile row (instead of D bf16 values) plus one float32
-    scale per row each, and no overflow-bound statistics (a bf16 plan's query row norms, one float32 per
-    row, and its (b, h) maxima, two float32 per head, 256-byte aligned); it needs tile-order copies (no
-    seq_tiles)."""
+    scale per row each; it needs tile-order copies (no seq_tiles)."""
     kw = dict(batch=1, heads=56, head_dim=128, segments=(512, 0, 768), grid=(24, 48, 64), sparsity=0.9)
     a = vsa.vsa_plan_query(**kw)["workspace_bytes"]
     b = vsa.vsa_plan_query(qk_fp8=True, **kw)["workspace_bytes"]
     rows = 56 * 1172 * 64
-    stats = rows * 4 + 512
-    assert a - b == 2 * rows * 128 * 2 + stats - (2 * rows * 128 + 2 * rows * 4)
+    assert a - b == 2 * rows * 128 * 2 - (2 * rows * 128 + 2 * rows * 4)
     with pytest.raises(vsa.VsaError) as e:
         vsa.vsa_plan_query(qk_fp8=True, seq_tiles=True, **kw)
     assert e.value.status == 3  # VSA_ERR_UNSUPPORTED

@@ -9,6 +9,7 @@ from a kernel over the tile-order inputs (step entry point).
 What is checked here:
   * the statistics: query row norms and the (b, h) maxima against float64 norms of the tile-order
     copies (64- and 128-token tiles, D = 96), and the sequence-order route's equal to the tile route's;
+    with 8-bit Q/K the norms of the dequantised rows;
   * a workload built so that every group skips (the premise is recomputed here in float64) while the
     logits of later blocks exceed the first block's maximum by about 2^95: parity with the oracle;
   * a workload whose bound is too loose to skip (logit jumps of about 2^290): parity with the oracle;
@@ -134,6 +135,28 @@ def test_statistics(vsa, name, over):
         v2 = vsa.workspace_views(plan2, ws2)
         assert torch.equal(v2["q_n"], views["q_n"]) and torch.equal(v2["kv_max"], views["kv_max"])
         plan2.destroy()
+
+
+@pytest.mark.parametrize("tile,D", [(64, 128), (128, 96)])
+def test_statistics_fp8(vsa, oracle_mod, tile, D):
+    """8-bit Q/K: the norms are those of the dequantised rows (scale times the norm of the E4M3 codes),
+    the |v| maximum that of the bf16 values."""
+    w = dataclasses.replace(synth.workload("small"), tile=tile, head_dim=D)
+    x = synth.make_inputs(w, seed=5, device="cuda")
+    plan = vsa.vsa_plan_tiles(batch=w.batch, heads=w.heads, head_dim=D, segments=w.segments, grid=w.grid,
+                              sparsity=w.sparsity, tile_size=tile, qk_fp8=True)
+    ws = vsa.alloc_workspace(plan)
+    vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], workspace=ws)
+    torch.cuda.synchronize()
+    assert vsa.device_status(plan) == (0, 0)
+    views = vsa.workspace_views(plan, ws)
+    deq = {n: oracle_mod.dequant_e4m3(views[n + "_t"].cpu().numpy(), views[n + "_s"].cpu().numpy())
+           for n in ("q", "k")}
+    assert np.allclose(f64(views["q_n"]), np.linalg.norm(deq["q"], axis=-1), rtol=1e-5, atol=0)
+    kv = f64(views["kv_max"])
+    assert np.allclose(kv[..., 0], np.linalg.norm(deq["k"], axis=-1).max(axis=(2, 3)), rtol=1e-5, atol=0)
+    assert np.array_equal(kv[..., 1], np.abs(f64(views["v_t"])).max(axis=(2, 3, 4)))
+    plan.destroy()
 
 
 @pytest.mark.parametrize("tile,seq_tiles", [(64, False), (128, False), (64, True)])
