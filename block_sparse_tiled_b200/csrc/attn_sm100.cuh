@@ -196,9 +196,9 @@ struct AttnLayout {
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
   static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
   static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
-  static constexpr int oQtok = oGate + 256;                  // int qtok[64]: token within its part (epilogue)
-  static constexpr int oQpart = oQtok + 256;                 // int qpart[64]: part holding the token
-  static constexpr int oSkip = oQpart + 256;                 // int skip[groups]: the item needs no votes
+  static constexpr int oDst = oGate + 256;                   // bf16* dst[64]: out row of each query (epilogue)
+  static constexpr int oGsrc = oDst + 512;                   // const bf16* gsrc[64]: its per-channel gate row
+  static constexpr int oSkip = oGsrc + 512;                  // int skip[groups]: the item needs no votes
   static constexpr int oEnd = oSkip + 16;
   static size_t bytes(int /*n_t*/) { return 1024 /*alignment slack*/ + oEnd; }
 };
@@ -263,8 +263,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* lpart_s = reinterpret_cast<float*>(sm + Ly::oLsum);
   float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
   float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
-  int32_t* qtok_s = reinterpret_cast<int32_t*>(sm + Ly::oQtok);
-  int32_t* qpart_s = reinterpret_cast<int32_t*>(sm + Ly::oQpart);
+  uint16_t** dst_s = reinterpret_cast<uint16_t**>(sm + Ly::oDst);
+  const uint16_t** gsrc_s = reinterpret_cast<const uint16_t**>(sm + Ly::oGsrc);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // n_t: 64-row blocks per (b, h); n_sel: tiles (the selection's unit), P and topk count tiles
@@ -888,21 +888,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int h = static_cast<int>(bh - b * a.H);
       const int ob = it & 1;
       if (tid < 64) {
+        // per query row: where its output row starts (NULL: a pad, not stored), its per-token gate or
+        // the start of its per-channel gate row
         const int32_t tok = __ldg(a.tile_token + static_cast<int64_t>(s) * 64 + tid);
-        int64_t lt = -1;
-        int part = 0;
-        if (tok >= 0 && a.io.table != nullptr) {
-          part = static_cast<int>(tok / a.io.Ls);
-          lt = tok - part * a.io.Ls;
-        } else if (tok >= 0) {
-          lt = tok;
+        uint16_t* dst = nullptr;
+        const uint16_t* gsrc = nullptr;
+        float g = 0.0f;
+        if (tok >= 0) {
+          int part = 0;
+          int64_t lt = tok;
+          if (a.io.table != nullptr) {
+            part = static_cast<int>(tok / a.io.Ls);
+            lt = tok - part * a.io.Ls;
+          }
+          const int64_t row = b * a.io.Ls + lt;  // row of the token in its part (or in the one tensor)
+          uint16_t* obase = a.io.table ? static_cast<uint16_t*>(const_cast<void*>(a.io.table[kPartOut * a.io.nparts + part]))
+                                       : a.out;
+          dst = obase + (row * a.io.Htot + a.io.h0 + h) * D;
+          const uint16_t* gb =
+              a.io.table ? static_cast<const uint16_t*>(a.io.table[kPartGate * a.io.nparts + part]) : a.gate;
+          if (a.gate_pc)
+            gsrc = gb + row * a.gate_ld + static_cast<int64_t>(a.io.h0 + h) * D;
+          else if (use_oc)
+            g = bf16_bits_to_f32(__ldg(gb + row * a.gate_ld + a.io.h0 + h));
         }
-        qtok_s[tid] = static_cast<int32_t>(lt);
-        qpart_s[tid] = part;
-        const uint16_t* gb = a.io.table ? static_cast<const uint16_t*>(a.io.table[kPartGate * a.io.nparts + part]) : a.gate;
-        gate_s[tid] = (tok >= 0 && !a.gate_pc && use_oc)
-                          ? bf16_bits_to_f32(__ldg(gb + (b * a.io.Ls + lt) * a.gate_ld + a.io.h0 + h))
-                          : 0.0f;
+        dst_s[tid] = dst;
+        gsrc_s[tid] = gsrc;
+        gate_s[tid] = g;
       }
       const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_sel + i) * D + d) : 0.0f;
       ROLE_MARK(3);
@@ -914,7 +926,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       mbar_wait(&bars[Ly::bOFull + ob], (it >> 1) & 1, ctl, 17);
       ROLE_MARK(1);
-      named_bar_sync(9, 128);  // rl, gate, qtok ready
+      named_bar_sync(9, 128);  // rl, gate, row pointers ready
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         tc_fence_after();
@@ -930,20 +942,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int q = 32 * half + j;
-            const int64_t lt = qtok_s[q];
-            if (lt >= 0) {
-              const int part = qpart_s[q];
-              const int64_t row = b * a.io.Ls + lt;  // row of the token in its part (or in the one tensor)
+            uint16_t* dst = dst_s[q];
+            if (dst != nullptr) {
               float gq = gate_s[q];
-              if (a.gate_pc && use_oc) {
-                const uint16_t* gb =
-                    a.io.table ? static_cast<const uint16_t*>(a.io.table[kPartGate * a.io.nparts + part]) : a.gate;
-                gq = bf16_bits_to_f32(__ldg(gb + row * a.gate_ld + static_cast<int64_t>(a.io.h0 + h) * D + d));
-              }
+              if (a.gate_pc && use_oc) gq = bf16_bits_to_f32(__ldg(gsrc_s[q] + d));
               const float val = fmaf(o[j], rl_s[q], gq * oc);
-              uint16_t* ob = a.io.table ? static_cast<uint16_t*>(const_cast<void*>(a.io.table[kPartOut * a.io.nparts + part]))
-                                        : a.out;
-              ob[(row * a.io.Htot + a.io.h0 + h) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+              dst[d] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
             }
           }
         }
