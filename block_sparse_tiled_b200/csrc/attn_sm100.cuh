@@ -194,12 +194,12 @@ struct AttnLayout {
   static constexpr int oDelta = oM + 256;                    // float delta[64]: m increase of a rescale
   static constexpr int oRed = oDelta + 256;                  // float red[groups][4 quadrants][group columns]
   static constexpr int oLsum = oRed + 1024;                  // float lpart[2 buffers][4 quadrants][64]
-  static constexpr int oRl = oLsum + 2048;                   // float 1 / l[64]   (epilogue)
-  static constexpr int oGate = oRl + 256;                    // float gate[64]   (epilogue)
-  static constexpr int oDst = oGate + 256;                   // bf16* dst[64]: out row of each query (epilogue)
+  static constexpr int oRg = oLsum + 2048;                   // float2 {1 / l, gate}[64]   (epilogue)
+  static constexpr int oDst = oRg + 512;                     // bf16* dst[64]: out row of each query (epilogue)
   static constexpr int oGsrc = oDst + 512;                   // const bf16* gsrc[64]: its per-channel gate row
   static constexpr int oSkip = oGsrc + 512;                  // int skip[groups]: the item needs no votes
-  static constexpr int oEnd = oSkip + 16;
+  static constexpr int oRows = oSkip + 16;                   // uint32 rows[2]: token rows of the item (ballots)
+  static constexpr int oEnd = oRows + 8;
   static size_t bytes(int /*n_t*/) { return 1024 /*alignment slack*/ + oEnd; }
 };
 
@@ -261,10 +261,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* delta_s = reinterpret_cast<float*>(sm + Ly::oDelta);
   float* red_s = reinterpret_cast<float*>(sm + Ly::oRed);
   float* lpart_s = reinterpret_cast<float*>(sm + Ly::oLsum);
-  float* rl_s = reinterpret_cast<float*>(sm + Ly::oRl);
-  float* gate_s = reinterpret_cast<float*>(sm + Ly::oGate);
+  float2* rg_s = reinterpret_cast<float2*>(sm + Ly::oRg);
   uint16_t** dst_s = reinterpret_cast<uint16_t**>(sm + Ly::oDst);
   const uint16_t** gsrc_s = reinterpret_cast<const uint16_t**>(sm + Ly::oGsrc);
+  uint32_t* rows_s = reinterpret_cast<uint32_t*>(sm + Ly::oRows);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // n_t: 64-row blocks per (b, h); n_sel: tiles (the selection's unit), P and topk count tiles
@@ -914,7 +914,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         dst_s[tid] = dst;
         gsrc_s[tid] = gsrc;
-        gate_s[tid] = g;
+        rg_s[tid].y = g;
+        const uint32_t tokens = __ballot_sync(0xffffffffu, tok >= 0);  // tid < 64: two whole warps
+        if (lane == 0) rows_s[tid >> 5] = tokens;
       }
       const float oc = (d < D && use_oc) ? __ldg(a.o_c + (bh * n_sel + i) * D + d) : 0.0f;
       ROLE_MARK(3);
@@ -922,11 +924,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ROLE_MARK(0);
       if (tid < 64) {
         const float* lp = lpart_s + ob * 4 * 64 + tid;
-        rl_s[tid] = rcp_approx((lp[0] + lp[64]) + (lp[128] + lp[192]));
+        rg_s[tid].x = rcp_approx((lp[0] + lp[64]) + (lp[128] + lp[192]));
       }
       mbar_wait(&bars[Ly::bOFull + ob], (it >> 1) & 1, ctl, 17);
       ROLE_MARK(1);
       named_bar_sync(9, 128);  // rl, gate, row pointers ready
+      const bool full = (rows_s[0] & rows_s[1]) == ~0u;  // all 64 query rows are tokens
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         tc_fence_after();
@@ -938,16 +941,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[Ly::bOEmpty + ob]);
         }
+        // out = O^T / l + gate * o_c (per-channel gate: gate[d]); a block of 64 tokens (every block but
+        // a tile's ragged end) stores without a per-row test
+        auto store = [&](int j, uint16_t* dst) {
+          const int q = 32 * half + j;
+          const float2 rg = rg_s[q];
+          const float gq = (a.gate_pc && use_oc) ? bf16_bits_to_f32(__ldg(gsrc_s[q] + d)) : rg.y;
+          dst[d] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(o[j], rg.x, gq * oc)));
+        };
         if (d < D) {
+          if (full) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int q = 32 * half + j;
-            uint16_t* dst = dst_s[q];
-            if (dst != nullptr) {
-              float gq = gate_s[q];
-              if (a.gate_pc && use_oc) gq = bf16_bits_to_f32(__ldg(gsrc_s[q] + d));
-              const float val = fmaf(o[j], rl_s[q], gq * oc);
-              dst[d] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+            for (int j = 0; j < 32; ++j) store(j, dst_s[32 * half + j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              uint16_t* dst = dst_s[32 * half + j];
+              if (dst != nullptr) store(j, dst);
             }
           }
         }
