@@ -281,7 +281,7 @@ def run_vsa(args, w, world, rank, local):
         if record:
             e[0].record(stream)
         vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], v["q_t"], v["k_t"], v["v_t"], v["pq"], v["pk"], v["pv"],
-                             stream=stream)
+                             q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
         if record:
             e[1].record(stream)
         vsa.vsa_pool_and_score(plan, None, None, None, v["pq"], v["pk"], v["pv"], v["scores"], stream=stream)
@@ -291,7 +291,7 @@ def run_vsa(args, w, world, rank, local):
         if record:
             e[3].record(stream)
         vsa.vsa_sparse_attn_fwd(plan, v["q_t"], v["k_t"], v["v_t"], v["idx"], v["o_c"], x["gate"], out,
-                                stream=stream)
+                                q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
         if record:
             e[4].record(stream)
             for n, evt in zip(("t0", "t1", "t2", "t3", "t4"), e):
@@ -362,7 +362,11 @@ def run_vsa(args, w, world, rank, local):
         "traffic": measured_attn_traffic() if w.name == "768p_s0.9" else None,
         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
     }
-    launches = 5 * args.steps
+    # library kernels per timed step: gather+pool, scores, one top-k pass per candidate set (reference
+    # tiles, video tiles), compression, attention
+    nv = dims["n_video_tiles"]
+    topk_passes = int(nv > 0 and dims["ref_topk"] > 0) + int(nv > 0 and dims["topk"] > 0)
+    launches = (4 + topk_passes) * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

@@ -109,10 +109,10 @@ def load_library(path: str = LIB_PATH):
     lib.vsa_plan_tables.argtypes = [P, P, P]
     lib.vsa_plan_workspace.argtypes = [P, ctypes.POINTER(WorkspaceLayout)]
     lib.vsa_plan_destroy.argtypes = [P]
-    lib.vsa_gather_tiles.argtypes = [P] * 11
+    lib.vsa_gather_tiles.argtypes = [P] * 13
     lib.vsa_pool_and_score.argtypes = [P] * 9
     lib.vsa_topk_select.argtypes = [P] * 6
-    lib.vsa_sparse_attn_fwd.argtypes = [P] * 9
+    lib.vsa_sparse_attn_fwd.argtypes = [P] * 11
     lib.vsa_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.vsa_forward_noalloc.argtypes = [P] * 7
     lib.vsa_forward_host_workspace.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
@@ -269,12 +269,13 @@ def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity
     return Plan(h, kw)
 
 
-def vsa_gather_tiles(plan, q, k, v, q_t, k_t, v_t, pq=None, pk=None, pv=None, stream=None):
+def vsa_gather_tiles(plan, q, k, v, q_t, k_t, v_t, pq=None, pk=None, pv=None, q_norm=None, kv_max=None,
+                     stream=None):
     bf, f32 = torch.bfloat16, torch.float32
     _check(load_library().vsa_gather_tiles(
         plan.handle, _ptr(q, bf, "q"), _ptr(k, bf, "k"), _ptr(v, bf, "v"), _ptr(q_t, bf, "q_t"),
         _ptr(k_t, bf, "k_t"), _ptr(v_t, bf, "v_t"), _ptr(pq, f32, "pq"), _ptr(pk, f32, "pk"), _ptr(pv, f32, "pv"),
-        _stream(stream)), "vsa_gather_tiles")
+        _ptr(q_norm, f32, "q_norm"), _ptr(kv_max, f32, "kv_max"), _stream(stream)), "vsa_gather_tiles")
 
 
 def vsa_pool_and_score(plan, q_t, k_t, v_t, pq, pk, pv, scores, stream=None):
@@ -292,12 +293,13 @@ def vsa_topk_select(plan, scores, pv, idx, o_c, stream=None):
         _ptr(o_c, f32, "o_c"), _stream(stream)), "vsa_topk_select")
 
 
-def vsa_sparse_attn_fwd(plan, q_t, k_t, v_t, idx, o_c, gate, out, stream=None):
-    bf = torch.bfloat16
+def vsa_sparse_attn_fwd(plan, q_t, k_t, v_t, idx, o_c, gate, out, q_norm=None, kv_max=None, stream=None):
+    bf, f32 = torch.bfloat16, torch.float32
     _check(load_library().vsa_sparse_attn_fwd(
         plan.handle, _ptr(q_t, bf, "q_t"), _ptr(k_t, bf, "k_t"), _ptr(v_t, bf, "v_t"),
-        _ptr(idx, torch.int32, "idx"), _ptr(o_c, torch.float32, "o_c"), _ptr(gate, bf, "gate"),
-        _ptr(out, bf, "out"), _stream(stream)), "vsa_sparse_attn_fwd")
+        _ptr(idx, torch.int32, "idx"), _ptr(o_c, f32, "o_c"), _ptr(gate, bf, "gate"),
+        _ptr(out, bf, "out"), _ptr(q_norm, f32, "q_norm"), _ptr(kv_max, f32, "kv_max"), _stream(stream)),
+        "vsa_sparse_attn_fwd")
 
 
 def alloc_workspace(plan, device=None) -> torch.Tensor:

@@ -1046,14 +1046,22 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
 }
 
 vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, vsa_bf16* q_t,
-                            vsa_bf16* k_t, vsa_bf16* v_t, float* pq, float* pk, float* pv, void* stream) {
+                            vsa_bf16* k_t, vsa_bf16* v_t, float* pq, float* pk, float* pv, float* q_norm,
+                            float* kv_max, void* stream) {
   VSA_TRY(check_plan(p));
   if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q, k, v, q_t, k_t, v_t}));
   const int npool = (pq != nullptr) + (pk != nullptr) + (pv != nullptr);
   if (npool != 0 && npool != 3) return fail(VSA_ERR_INVALID_ARG, "pq, pk, pv must be all NULL or all set");
   if (npool == 3) VSA_TRY(check_ptrs({pq, pk, pv}));
-  return run_gather(p, q, k, v, q_t, k_t, v_t, pq, pk, pv, static_cast<cudaStream_t>(stream));
+  if ((q_norm == nullptr) != (kv_max == nullptr))
+    return fail(VSA_ERR_INVALID_ARG, "q_norm and kv_max must be both NULL or both set");
+  if (q_norm != nullptr && npool != 3) return fail(VSA_ERR_INVALID_ARG, "the statistics are taken while pooling");
+  if (q_norm != nullptr) VSA_TRY(check_ptrs({q_norm, kv_max}));
+  const auto s = static_cast<cudaStream_t>(stream);
+  auto* kv = reinterpret_cast<uint32_t*>(kv_max);
+  if (kv != nullptr) VSA_CUDA_TRY(cudaMemsetAsync(kv, 0, static_cast<size_t>(p->B) * p->H * 8, s));
+  return run_gather(p, q, k, v, q_t, k_t, v_t, pq, pk, pv, s, nullptr, nullptr, nullptr, q_norm, kv);
 }
 
 vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k_t, const vsa_bf16* v_t, float* pq,
@@ -1079,13 +1087,20 @@ vsa_status vsa_topk_select(vsa_plan p, const float* scores, const float* pv, int
 
 vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k_t, const vsa_bf16* v_t,
                                const int32_t* idx, const float* o_c, const vsa_bf16* gate, vsa_bf16* out,
-                               void* stream) {
+                               const float* q_norm, const float* kv_max, void* stream) {
   VSA_TRY(check_plan(p));
   if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q_t, k_t, v_t, o_c, gate, out}));
   if (p->V > 0) VSA_TRY(check_ptrs({idx}));
   const auto s = static_cast<cudaStream_t>(stream);
-  // the overflow bound from these inputs' own statistics (the forward takes them from its gather)
+  if ((q_norm == nullptr) != (kv_max == nullptr))
+    return fail(VSA_ERR_INVALID_ARG, "q_norm and kv_max must be both NULL or both set");
+  if (q_norm != nullptr) {  // the caller's statistics of these tiles (vsa_gather_tiles with statistics)
+    VSA_TRY(check_ptrs({q_norm, kv_max}));
+    return run_attn(p, q_t, k_t, v_t, idx, o_c, gate, out, s, 0, nullptr, nullptr, nullptr, nullptr, nullptr, q_norm,
+                    reinterpret_cast<const uint32_t*>(kv_max));
+  }
+  // otherwise the overflow bound from these inputs' own statistics, into the plan's buffer
   float* qn = p->d_stats;
   auto* kv = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p->d_stats) + stats_rows_bytes(p));
   VSA_TRY(run_tile_stats(p, q_t, k_t, v_t, qn, kv, s));

@@ -183,12 +183,18 @@ vsa_status vsa_plan_destroy(vsa_plan p);
  * q_t/k_t/v_t[b,h,tile,r,:] = q/k/v[b, token(tile, r), h, :], pad rows zero.
  * If pq, pk and pv are all non-NULL the pooled tiles (S3's first half) are
  * written in the same pass, bit-identical to vsa_pool_and_score's.
+ * If q_norm and kv_max are non-NULL too (both or neither; only with pooling),
+ * the same pass writes the attention's overflow-bound statistics of the
+ * tiles: q_norm [B, H, n_tiles, tile_size] float32, the Euclidean norm of
+ * every query row (0 for pads), and kv_max [B, H, 2] float32, the largest
+ * key-row norm and |v| of each (b, h) -- the values vsa_forward keeps in its
+ * workspace (q_n, kv_max), to be passed on to vsa_sparse_attn_fwd.
  * Passage: "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", section "Model
  * integration" (gather to tile order once; pad rows zero). */
 vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16* k_dev,
                             const vsa_bf16* v_dev, vsa_bf16* q_t_dev, vsa_bf16* k_t_dev,
                             vsa_bf16* v_t_dev, float* pq_dev, float* pk_dev, float* pv_dev,
-                            void* stream);
+                            float* q_norm_dev, float* kv_max_dev, void* stream);
 
 /* ---- S3: pooling and pooled tile scores ----------------------------------
  * pooled[b,h,t,d] = (sum over the tile's valid rows r, in tile order, from
@@ -229,13 +235,18 @@ vsa_status vsa_topk_select(vsa_plan p, const float* scores_dev, const float* pv_
  * first); "Mike0021/FastH3-4step-Preview-VSA", section "Video Sparse
  * Attention is not optional here" (dense prefix queries; gated compression
  * branch with no activation).
- * The call first takes the norms of q_t's rows and the largest key norm and
- * |v| of k_t, v_t (one extra kernel, into a buffer the plan owns, so calls on
- * one plan must not overlap); the output is bit-identical to vsa_forward's. */
+ * The rescale checks of the softmax are bounded with the tiles' magnitude
+ * statistics (see vsa_gather_tiles): pass those of exactly these q_t, k_t,
+ * v_t as q_norm_dev and kv_max_dev (statistics of other tensors void the
+ * bound, and the output may then overflow to infinity), or NULL for both:
+ * the call then takes them itself first (one extra kernel reading the
+ * tiles, into a buffer the plan owns, so such calls on one plan must not
+ * overlap).  Either way the output is bit-identical to vsa_forward's. */
 vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t_dev, const vsa_bf16* k_t_dev,
                                const vsa_bf16* v_t_dev, const int32_t* idx_dev,
                                const float* o_c_dev, const vsa_bf16* gate_dev,
-                               vsa_bf16* out_dev, void* stream);
+                               vsa_bf16* out_dev, const float* q_norm_dev,
+                               const float* kv_max_dev, void* stream);
 
 /* ---- the whole forward ---------------------------------------------------
  * S2..S5 in one call, sequence order in and out.  `workspace_dev` must hold

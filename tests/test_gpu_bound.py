@@ -9,6 +9,7 @@ from a kernel over the tile-order inputs (step entry point).
 What is checked here:
   * the statistics: query row norms and the (b, h) maxima against float64 norms of the tile-order
     copies (64- and 128-token tiles, D = 96), and the sequence-order route's equal to the tile route's;
+    the step route's (passed from the gather to the attention) equal to the fused forward's;
     with 8-bit Q/K the norms of the dequantised rows;
   * a workload built so that every group skips (the premise is recomputed here in float64) while the
     logits of later blocks exceed the first block's maximum by about 2^95: parity with the oracle;
@@ -135,6 +136,42 @@ def test_statistics(vsa, name, over):
         v2 = vsa.workspace_views(plan2, ws2)
         assert torch.equal(v2["q_n"], views["q_n"]) and torch.equal(v2["kv_max"], views["kv_max"])
         plan2.destroy()
+
+
+@pytest.mark.parametrize("tile", [64, 128])
+def test_step_route_with_statistics(vsa, tile):
+    """The step entry points with the gather's statistics passed to the attention: the statistics equal
+    the fused forward's, and the output is bit-identical to the fused forward and to the step route that
+    lets the attention take its own statistics."""
+    w = dataclasses.replace(synth.workload("small"), tile=tile)
+    x = synth.make_inputs(w, seed=6, device="cuda")
+    plan, ws, out = run(vsa, w, x)
+    views = vsa.workspace_views(plan, ws)
+    B, H, D, n_t, V = w.batch, w.heads, w.head_dim, plan.dims["n_tiles"], plan.dims["n_video_tiles"]
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    t = {n: torch.empty(B, H, n_t, tile, D, **bf) for n in ("q_t", "k_t", "v_t")}
+    pq, pk, pv = (torch.empty(B, H, n_t, D, **f32) for _ in range(3))
+    qn = torch.full((B, H, n_t, tile), float("nan"), **f32)
+    kv = torch.full((B, H, 2), float("nan"), **f32)  # the call zeroes it before raising it
+    vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], t["q_t"], t["k_t"], t["v_t"], pq, pk, pv, q_norm=qn, kv_max=kv)
+    S = torch.empty(B, H, n_t, n_t, **f32)
+    vsa.vsa_pool_and_score(plan, None, None, None, pq, pk, pv, S)
+    idx = torch.empty(B, H, max(V, 1), max(plan.dims["topk"], 1), dtype=torch.int32, device="cuda")
+    o_c = torch.empty(B, H, n_t, D, **f32)
+    vsa.vsa_topk_select(plan, S, pv, idx, o_c)
+    out_passed = torch.empty_like(out)
+    vsa.vsa_sparse_attn_fwd(plan, t["q_t"], t["k_t"], t["v_t"], idx, o_c, x["gate"], out_passed, q_norm=qn,
+                            kv_max=kv)
+    out_own = torch.empty_like(out)
+    vsa.vsa_sparse_attn_fwd(plan, t["q_t"], t["k_t"], t["v_t"], idx, o_c, x["gate"], out_own)
+    torch.cuda.synchronize()
+    assert vsa.device_status(plan) == (0, 0)
+    assert torch.equal(qn, views["q_n"]) and torch.equal(kv, views["kv_max"])
+    assert torch.equal(out_passed, out) and torch.equal(out_own, out)
+    with pytest.raises(vsa.VsaError):  # both statistics or neither
+        vsa.vsa_sparse_attn_fwd(plan, t["q_t"], t["k_t"], t["v_t"], idx, o_c, x["gate"], out_own, q_norm=qn)
+    plan.destroy()
 
 
 @pytest.mark.parametrize("tile,D", [(64, 128), (128, 96)])

@@ -206,5 +206,5 @@ def test_fp8_step_entry_points_refuse(vsa):
     assert vsa.STATUS_NAMES[e.value.status] == "VSA_ERR_UNSUPPORTED"
     lib = vsa.load_library()
     p = [ctypes.c_void_p(a.data_ptr()) for a in t]
-    assert lib.vsa_sparse_attn_fwd(plan.handle, *p, p[0], p[0], p[0], p[0], None) == 3
+    assert lib.vsa_sparse_attn_fwd(plan.handle, *p, p[0], p[0], p[0], p[0], None, None, None) == 3
     plan.destroy()
