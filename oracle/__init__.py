@@ -238,6 +238,26 @@ def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=No
     return out
 
 
+def fine_split(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=None) -> np.ndarray:
+    """The fine branch with the pages' prefix split (reading R19): the dense prefix query tiles take
+    their logits from the 8-bit Q/K of ``qk8`` (as fine() with qk8), the video query tiles from the bf16
+    q, k (as fine() without).  Both branches run in full over their own tiles and the rows are merged by
+    the tile each token belongs to; bf16 P.V throughout.  ("FastH3 OmniRef inference", section "Device
+    profiles": the dense prefix query tiles run at 8-bit Q/K with bf16 P.V, the video query tiles on
+    another kernel.)"""
+    B, L, H, _ = np.shape(q)
+    n_t, P = geo.n_tiles, geo.n_prefix
+    sel = np.ones((B, H, n_t), bool) if todo is None else np.asarray(todo, bool)
+    is_prefix = np.zeros((B, H, n_t), bool)
+    is_prefix[:, :, :P] = True
+    pre = fine(q, k, v, geo, idx, topk, scale, todo=sel & is_prefix, qk8=qk8)
+    vid = fine(q, k, v, geo, idx, topk, scale, todo=sel & ~is_prefix)
+    tok_prefix = np.zeros(L, bool)  # tokens of prefix tiles
+    for i in range(P):
+        tok_prefix[geo.tile_token[i, :geo.tile_valid[i]]] = True
+    return np.where(tok_prefix[None, :, None, None], pre, vid)
+
+
 def fine_tiles(q, k, v, geo: Geometry, idx, topk: int, scale: float, items, qk8=None) -> np.ndarray:
     """Fine branch of the listed query tiles only.  items: int64 array of
     (b*H + h)*n_t + i.  Returns [n_items, tile, D] float64 in tile row order
@@ -386,7 +406,8 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
     Selection (pool, scores, top-k) always runs in full; the fine branch and
     the output run for the query tiles flagged in ``todo`` ([B, H, n_t] bool,
     None = all).  qk8: the fine branch's logits use 8-bit Q/K (R16); the
-    selection still reads the bf16 inputs.  tile, cube: the tile size and video
+    selection still reads the bf16 inputs; qk8="prefix": only the dense prefix
+    query tiles do (R19, fine_split).  tile, cube: the tile size and video
     cube shape (64 and 4x4x4 as the method states; 128 per R17).  ref_segments,
     ref_keep: reference segments and their keep ratio (R18)."""
     t0 = time.perf_counter()
@@ -401,6 +422,9 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
     idx = select(S, geo.n_prefix, kc, geo.is_ref, kr)
     o_c = compress(S, pv)
     q8 = (*quant_e4m3(q), *quant_e4m3(k)) if qk8 else None
-    o_f = fine(q, k, v, geo, idx, kc, scale, todo, qk8=q8)
+    if qk8 == "prefix":
+        o_f = fine_split(q, k, v, geo, idx, kc, scale, todo, qk8=q8)
+    else:
+        o_f = fine(q, k, v, geo, idx, kc, scale, todo, qk8=q8)
     out = output(o_f, o_c, gate, geo, todo)
     return ForwardResult(geo, kc, scale, pq, pk, pv, S, idx, o_c, o_f, out, time.perf_counter() - t0)

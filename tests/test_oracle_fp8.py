@@ -227,3 +227,67 @@ def test_fine_q8_within_bound_of_bf16(oracle_mod, sparsity):
         err = np.abs(got[0, :, h] - ref[0, :, h]).max(axis=1)
         assert (err <= bound * (1 + 1e-9)).all()
     assert np.abs(got - ref).max() > 0
+
+
+# ---------------------------------------------------------------------------
+# the pages' prefix split: 8-bit Q/K for the dense prefix query tiles only (R19)
+# ---------------------------------------------------------------------------
+
+
+def _split_case(oracle_mod, name, seed, **over):
+    w = synth.workload(name, **over)
+    x = synth.make_inputs(w, seed=seed)
+    b = {n: synth.as_bits(x[n]) for n in ("q", "k", "v", "gate")}
+    sel = oracle_mod.selection(b["q"], b["k"], b["v"], w.segments, w.grid, w.sparsity)
+    args = (b["q"], b["k"], b["v"], sel["geo"], sel["idx"], sel["topk"], sel["scale"])
+    q8 = (*oracle_mod.quant_e4m3(b["q"]), *oracle_mod.quant_e4m3(b["k"]))
+    return w, sel, args, q8
+
+
+def _prefix_tokens(geo, L):
+    t = np.zeros(L, bool)
+    for i in range(geo.n_prefix):
+        t[geo.tile_token[i, :geo.tile_valid[i]]] = True
+    return t
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(sparsity=0.0)), ("small", dict(heads=2))])
+def test_fine_split_rows_follow_their_branch(oracle_mod, name, over):
+    """Prefix query rows take the 8-bit logits, video query rows the bf16 ones, each over the same key
+    sets: the split equals the all-8-bit branch on every prefix token and the bf16 branch on every video
+    token, and differs from each on the other side (so the rows are not swapped)."""
+    w, sel, args, q8 = _split_case(oracle_mod, name, 4, **over)
+    got = oracle_mod.fine_split(*args, qk8=q8)
+    all8 = oracle_mod.fine(*args, qk8=q8)
+    bf16 = oracle_mod.fine(*args)
+    pre = _prefix_tokens(sel["geo"], w.seq_len)
+    assert pre.any() and (~pre).any()
+    assert np.array_equal(got[:, pre], all8[:, pre])
+    assert np.array_equal(got[:, ~pre], bf16[:, ~pre])
+    assert np.abs(got[:, pre] - bf16[:, pre]).max() > 0
+    assert np.abs(got[:, ~pre] - all8[:, ~pre]).max() > 0
+
+
+def test_fine_split_special_cases(oracle_mod):
+    """No prefix: the split is the bf16 branch; no video: it is the all-8-bit branch."""
+    for segs, grid, same_as_8bit in (((), (8, 8, 8), False), ((100, 30), (0, 0, 0), True)):
+        w = synth.Workload("split", 1, 2, 64, segs, grid, 0.5)
+        x = synth.make_inputs(w, seed=9)
+        b = {n: synth.as_bits(x[n]) for n in ("q", "k", "v")}
+        sel = oracle_mod.selection(b["q"], b["k"], b["v"], w.segments, w.grid, w.sparsity)
+        args = (b["q"], b["k"], b["v"], sel["geo"], sel["idx"], sel["topk"], sel["scale"])
+        q8 = (*oracle_mod.quant_e4m3(b["q"]), *oracle_mod.quant_e4m3(b["k"]))
+        want = oracle_mod.fine(*args, qk8=q8 if same_as_8bit else None)
+        assert np.array_equal(oracle_mod.fine_split(*args, qk8=q8), want)
+
+
+def test_forward_prefix_split_matches_composition(oracle_mod):
+    """forward(qk8="prefix") is the selection, the split fine branch and the gated output."""
+    w, sel, args, q8 = _split_case(oracle_mod, "tiny", 6)
+    x = synth.make_inputs(w, seed=6)
+    b = {n: synth.as_bits(x[n]) for n in ("q", "k", "v", "gate")}
+    ref = oracle_mod.forward(b["q"], b["k"], b["v"], b["gate"], w.segments, w.grid, w.sparsity, qk8="prefix")
+    o_f = oracle_mod.fine_split(*args, qk8=q8)
+    assert np.array_equal(ref.o_f, o_f)
+    assert np.array_equal(ref.idx, sel["idx"])
+    assert np.array_equal(ref.out, oracle_mod.output(o_f, sel["o_c"], b["gate"], sel["geo"]))
