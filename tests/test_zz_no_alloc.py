@@ -3,15 +3,12 @@ device memory (its scratch is a static array inside libvsa).  Checked through
 the C ABI against vsa_forward with a caller workspace, on two calls in a row
 with different inputs, so the second call runs over the first call's leftover
 scratch contents."""
-import numpy as np
 import pytest
 import torch
 
 import synth
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, MEAN_ABS = 2e-2, 2e-3
 
 
 @pytest.fixture(scope="module")
@@ -44,9 +41,8 @@ def test_noalloc_matches_forward_on_two_calls(vsa):
         vsa.vsa_forward_noalloc(plan, x["q"], x["k"], x["v"], x["gate"], out)
         torch.cuda.synchronize()
         assert vsa.device_status(plan) == (0, 0)
-        err = (out.double() - ref.double()).abs().cpu().numpy()
-        assert np.isfinite(err).all()
-        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (seed, err.max(), err.mean())
+        # the same kernels on the same plan: bit-identical, so leftover scratch from the first call would show
+        assert torch.equal(out, ref), seed
     plan.destroy()
 
 
