@@ -85,7 +85,7 @@ class PlanDims(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t)
                 for n in ("q_t", "k_t", "v_t", "q_s", "k_s", "q_n", "kv_max", "pq", "pk", "pv", "scores", "idx", "o_c",
-                          "total")]
+                          "q_c", "k_c", "q_n8", "kv_max8", "total")]
 
 
 _lib = None
@@ -154,6 +154,16 @@ def _ptr(t, dtype=None, name="tensor"):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _qk_mode(qk_fp8) -> int:
+    """qk_fp8: False / True (8-bit Q/K logits for every query tile) / "prefix" (for the dense prefix query
+    tiles only, the pages' split) -> the geometry's 0 / 1 / 2."""
+    if isinstance(qk_fp8, str):
+        if qk_fp8 != "prefix":
+            raise ValueError(f"qk_fp8 must be a bool or 'prefix', got {qk_fp8!r}")
+        return 2
+    return int(bool(qk_fp8))
+
+
 def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=0.0, softmax_scale=0.0,
                   token_tags=None, video_tag=0, tile_size=64, gate_per_channel=False, seq_tiles=False, qk_fp8=False,
                   cube=None, ref_segments=None, ref_keep=0.0):
@@ -182,7 +192,7 @@ def make_geometry(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity=
     g.softmax_scale = float(softmax_scale)
     g.gate_per_channel = int(bool(gate_per_channel))
     g.seq_tiles = int(bool(seq_tiles))
-    g.qk_fp8 = int(bool(qk_fp8))
+    g.qk_fp8 = _qk_mode(qk_fp8)
     g.cube_t, g.cube_h, g.cube_w = (int(c) for c in (cube or (0, 0, 0)))
     if ref_segments is not None:
         flags = (ctypes.c_int32 * max(1, len(ref_segments)))(*[int(f) for f in ref_segments])
@@ -261,7 +271,7 @@ def vsa_plan_tiles(batch, heads, head_dim, segments=(), grid=(0, 0, 0), sparsity
     kw = dict(batch=batch, heads=heads, head_dim=head_dim, segments=tuple(segments), grid=tuple(grid),
               sparsity=sparsity, softmax_scale=softmax_scale, token_tags=token_tags, video_tag=video_tag,
               tile_size=tile_size, gate_per_channel=bool(gate_per_channel), seq_tiles=bool(seq_tiles),
-              qk_fp8=bool(qk_fp8), cube=None if cube is None else tuple(cube),
+              qk_fp8=qk_fp8 if isinstance(qk_fp8, str) else bool(qk_fp8), cube=None if cube is None else tuple(cube),
               ref_segments=None if ref_segments is None else tuple(ref_segments), ref_keep=float(ref_keep))
     g, keep = make_geometry(**kw)
     h = ctypes.c_void_p()
@@ -457,12 +467,15 @@ def workspace_views(plan, workspace):
     with seq_tiles, whose workspace holds none).  With qk_fp8, q_t and k_t are the E4M3 codes
     [B, H, n_t, tile, 128] (uint8) and q_s, k_s their row scales [B, H, n_t, tile].  q_n holds the
     query row norms [B, H, n_t, tile] (with qk_fp8 of the dequantised rows) and kv_max the (b, h)
-    maxima of key norm and |v| [B, H, 2] (the attention's overflow bound)."""
+    maxima of key norm and |v| [B, H, 2] (the attention's overflow bound).  With qk_fp8="prefix" q_t and
+    k_t are the bf16 copies, q_c and k_c the codes, q_s and k_s their scales, and q_n8, kv_max8 the
+    statistics of the dequantised rows."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
     seq = bool(g.get("seq_tiles", False))
-    f8 = bool(g.get("qk_fp8", False))
+    mode = _qk_mode(g.get("qk_fp8", False))
+    f8, split = mode == 1, mode == 2
     T = d["tile_size"]  # rows per tile
 
     def view(off, n, dtype, shape):
@@ -476,9 +489,15 @@ def workspace_views(plan, workspace):
         return view(lay[name], B * H * n_t * T * 128, torch.uint8, (B, H, n_t, T, 128))
 
     def row_scales(name):
-        return view(lay[name], B * H * n_t * T, torch.float32, (B, H, n_t, T)) if f8 else None
+        return view(lay[name], B * H * n_t * T, torch.float32, (B, H, n_t, T)) if (f8 or split) else None
 
+    extra = {} if not split else {
+        "q_c": codes("q_c"), "k_c": codes("k_c"),
+        "q_n8": view(lay["q_n8"], B * H * n_t * T, torch.float32, (B, H, n_t, T)),
+        "kv_max8": view(lay["kv_max8"], B * H * 2, torch.float32, (B, H, 2)),
+    }
     return {
+        **extra,
         "q_t": codes("q_t") if f8 else tiles("q_t"),
         "k_t": codes("k_t") if f8 else tiles("k_t"),
         "v_t": tiles("v_t"),

@@ -139,7 +139,8 @@ struct AttnArgs {
   const float* kv_max;
   float skip_cap;
   float scale_log2;  // softmax scale * log2(e)
-  int64_t n_items;   // B * H * n_rb
+  int s_lo, n_s;     // the launch covers row blocks [s_lo, s_lo + n_s) of every (b, h)
+  int64_t n_items;   // B * H * n_s
 };
 
 // Tensor maps for loading tiles straight from sequence order (q, k, v): a 4-D map over [b, token, head, d]
@@ -376,8 +377,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         more = false;
         return;
       }
-      const int64_t claimed = atomicAdd(a.sched, 1);
-      const int v = (claimed < a.n_items) ? static_cast<int>(claimed) : -1;
+      const int claimed = atomicAdd(a.sched, 1);  // items fit in an int (the plan checks B*H*n_t*64 < 2^31)
+      // claimed -> item (b*H + h)*n_t + s of the launch's row blocks
+      const int v = (claimed < a.n_items) ? (claimed / a.n_s) * n_t + a.s_lo + claimed % a.n_s : -1;
       ring_s[slot] = v;
       mbar_arrive(&bars[Ly::bRFull + slot]);
       ++pub;

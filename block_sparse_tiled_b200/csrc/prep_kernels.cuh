@@ -156,6 +156,8 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
 
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool pool = (pq != nullptr);
+  // without pooling and without a V destination (a second, codes-only pass) V is not read at all
+  const bool skip_v = !pool && v_t == nullptr;
   if (threadIdx.x < kRows) tok_s[threadIdx.x] = tile_token[static_cast<int64_t>(tile) * kRows + threadIdx.x];
   __syncthreads();
 
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
     const bool active = chunk_of(u, &r, &c);
     const int32_t tok = tok_s[r];
     val[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (active && tok >= 0) {
+    if (active && tok >= 0 && !(tsr == 2 && skip_v)) {
       if constexpr (kParts) {  // the token's part, and heads h0 + h of its Htot
         int64_t lt;
         const uint16_t* base = part_base(io, tsr, src, tok, &lt);
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(384) gather_pool_kernel(
           kn_bits = max(kn_bits, __float_as_uint(nrm) & 0x7fffffffu);
         }
       }
-    } else if (active) {
+    } else if (active && !(tsr == 2 && skip_v)) {
       uint16_t* dst = (tsr == 0) ? static_cast<uint16_t*>(q_t) : (tsr == 1) ? static_cast<uint16_t*>(k_t) : v_t;
       reinterpret_cast<uint4*>(dst + tile_row0 * D)[r * kChunks + c] = val[u];
     }
@@ -486,31 +488,15 @@ __global__ void __launch_bounds__(256) gate_any_kernel(const uint16_t* __restric
   if (__syncthreads_or(any) && threadIdx.x == 0) *flag = 1;
 }
 
+// The compression GEMM of one CTA's 128 rows (i0 ..) of one (b, h), given each row's maximum in m_s:
+// W = exp(S - max) is staged 32 columns at a time with its row sums alongside, and every thread
+// accumulates 8 rows x D/16 columns of W . pv; o_c = that / row sum.
 template <int D>
-__global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
-                                                        float* __restrict__ o_c, int n_t,
-                                                        const int* __restrict__ gate_nonzero) {
-  if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
+__device__ __forceinline__ void compress_rows(const float* __restrict__ Sb, const float* __restrict__ PVb,
+                                              float* __restrict__ o_c, int bh, int n_t, int i0, const float* m_s,
+                                              float* l_s, float (*W_s)[kCompRows + 4], float (*PV_s)[D]) {
   constexpr int kCols = D / 16;  // columns per thread (4, 6 or 8)
   static_assert(kCols == 4 || kCols == 6 || kCols == 8, "head_dim 64, 96 or 128");
-  __shared__ float m_s[kCompRows], l_s[kCompRows];
-  __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
-  __shared__ __align__(16) float PV_s[kCompJ][D];
-  const int bh = blockIdx.y, i0 = blockIdx.x * kCompRows;
-  const float* Sb = S + static_cast<int64_t>(bh) * n_t * n_t;
-  const float* PVb = pv + static_cast<int64_t>(bh) * n_t * D;
-
-  {  // row maxima: 2 threads per row
-    const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
-    const int i = i0 + r;
-    float m = -INFINITY;
-    if (i < n_t)
-      for (int j = part; j < n_t; j += 2) m = fmaxf(m, __ldg(Sb + static_cast<int64_t>(i) * n_t + j));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    if (part == 0) m_s[r] = m;
-  }
-  __syncthreads();
-
   // staging map for W: thread -> (row r = t >> 1, 16 consecutive j of the chunk)
   const int wr = threadIdx.x >> 1, wj0 = (threadIdx.x & 1) * 16;
   const int wi = i0 + wr;
@@ -570,6 +556,111 @@ __global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restric
     for (int c = 0; c < kCols; ++c)
       o_c[(static_cast<int64_t>(bh) * n_t + i) * D + out_col(c)] = acc[a][c] * inv;
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
+                                                        float* __restrict__ o_c, int n_t,
+                                                        const int* __restrict__ gate_nonzero) {
+  if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
+  __shared__ float m_s[kCompRows], l_s[kCompRows];
+  __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
+  __shared__ __align__(16) float PV_s[kCompJ][D];
+  const int bh = blockIdx.y, i0 = blockIdx.x * kCompRows;
+  const float* Sb = S + static_cast<int64_t>(bh) * n_t * n_t;
+  const float* PVb = pv + static_cast<int64_t>(bh) * n_t * D;
+
+  {  // row maxima: 2 threads per row
+    const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
+    const int i = i0 + r;
+    float m = -INFINITY;
+    if (i < n_t)
+      for (int j = part; j < n_t; j += 2) m = fmaxf(m, __ldg(Sb + static_cast<int64_t>(i) * n_t + j));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    if (part == 0) m_s[r] = m;
+  }
+  __syncthreads();
+  compress_rows<D>(Sb, PVb, o_c, bh, n_t, i0, m_s, l_s, W_s, PV_s);
+}
+
+// ---------------------------------------------------------------------------
+// S4 in one pass over each score row: top-k of the video columns and the compression branch.
+// A CTA owns 128 rows of one (b, h).  Each warp takes 16 of them in turn and holds a row in registers
+// as order keys (kMaxJ per lane, so n_t <= 32 kMaxJ): the row maximum (the compression's shift) is a
+// warp max of the keys; for a video query row the k-th largest video key T comes from a bitwise search
+// whose per-bit counts are one redux.sync each, and the row's picks (every key > T, then the keys == T
+// lowest index first) are written ascending to idx[row * out_stride + out_off ...].  Then the CTA runs
+// the compression GEMM of its rows (compress_rows), unless every gate is zero.  The selection is the
+// top-k kernel's (same keys, same threshold, same order) and the compression the compression kernel's
+// (same maxima and staging), so both outputs are bit-identical to the two-kernel path.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float order_key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+template <int D, int kMaxJ>
+__global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __restrict__ S,
+                                                               const float* __restrict__ pv, float* __restrict__ o_c,
+                                                               int32_t* __restrict__ idx, int n_t, int P, int k,
+                                                               int out_stride, int out_off,
+                                                               const int* __restrict__ gate_nonzero) {
+  __shared__ float m_s[kCompRows], l_s[kCompRows];
+  __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
+  __shared__ __align__(16) float PV_s[kCompJ][D];
+  const int bh = blockIdx.y, i0 = blockIdx.x * kCompRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int V = n_t - P;
+  const float* Sb = S + static_cast<int64_t>(bh) * n_t * n_t;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int r = warp; r < kCompRows; r += 8) {
+    const int i = i0 + r;
+    if (i >= n_t) break;
+    const float* srow = Sb + static_cast<int64_t>(i) * n_t;
+    uint32_t key[kMaxJ];
+    uint32_t kmax = 0u;
+#pragma unroll
+    for (int jj = 0; jj < kMaxJ; ++jj) {
+      const int j = 32 * jj + lane;
+      key[jj] = (j < n_t) ? order_key(__ldg(srow + j)) : 0u;
+      kmax = max(kmax, key[jj]);
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) m_s[r] = order_key_value(kmax);
+    if (i < P || k <= 0) continue;
+    // candidates: the video columns (every valid key is >= 1, so the threshold never admits a 0 key)
+#pragma unroll
+    for (int jj = 0; jj < kMaxJ; ++jj)
+      if (32 * jj + lane < P) key[jj] = 0u;
+    uint32_t T = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      uint32_t cnt = 0u;
+#pragma unroll
+      for (int jj = 0; jj < kMaxJ; ++jj) cnt += (key[jj] >= cand) ? 1u : 0u;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= static_cast<uint32_t>(k)) T = cand;
+    }
+    uint32_t gt = 0u;
+#pragma unroll
+    for (int jj = 0; jj < kMaxJ; ++jj) gt += (key[jj] > T) ? 1u : 0u;
+    const int need = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));  // ties taken, lowest index first
+    int32_t* out = idx + (static_cast<int64_t>(bh) * V + (i - P)) * out_stride + out_off;
+    int written = 0, eq_seen = 0;
+#pragma unroll
+    for (int jj = 0; jj < kMaxJ; ++jj) {
+      if (32 * jj >= n_t) break;
+      const bool is_gt = key[jj] > T;
+      const bool is_eq = key[jj] == T;
+      const uint32_t eq_ballot = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = is_gt || (is_eq && eq_seen + __popc(eq_ballot & lt_mask) < need);
+      const uint32_t take_ballot = __ballot_sync(0xffffffffu, take);
+      if (take) out[written + __popc(take_ballot & lt_mask)] = 32 * jj + lane;
+      written += __popc(take_ballot);
+      eq_seen += __popc(eq_ballot);
+    }
+  }
+  __syncthreads();
+  if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
+  compress_rows<D>(Sb, pv + static_cast<int64_t>(bh) * n_t * D, o_c, bh, n_t, i0, m_s, l_s, W_s, PV_s);
 }
 
 }  // namespace vsa

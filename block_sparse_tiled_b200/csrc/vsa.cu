@@ -88,7 +88,7 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g->seq_tiles != 0 && g->seq_tiles != 1) return fail(VSA_ERR_INVALID_ARG, "seq_tiles must be 0 or 1");
   if (g->seq_tiles && g->batch > 4)
     return fail(VSA_ERR_UNSUPPORTED, "seq_tiles needs batch <= 4 (one 5-D tensor map per batch)");
-  if (g->qk_fp8 != 0 && g->qk_fp8 != 1) return fail(VSA_ERR_INVALID_ARG, "qk_fp8 must be 0 or 1");
+  if (g->qk_fp8 < 0 || g->qk_fp8 > 2) return fail(VSA_ERR_INVALID_ARG, "qk_fp8 must be 0, 1 or 2");
   if (g->qk_fp8 && g->seq_tiles)
     return fail(VSA_ERR_UNSUPPORTED, "qk_fp8 reads 8-bit tile-order copies: it needs seq_tiles = 0");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
@@ -285,18 +285,19 @@ void build_seq_tables(const Resolved& r, const std::vector<uint64_t>& mask_tiled
 // rows; with qk_fp8 of the dequantised row) and, per (b, h), the largest key norm and |v| (two floats).
 vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t tile, int64_t V, int64_t topk,
                                  bool seq_tiles,
-                                 bool qk_fp8) {
+                                 bool qk_fp8, bool qk_split = false) {
   vsa_workspace_layout w{};
   size_t off = 0;
   const size_t rows = static_cast<size_t>(B * H * n_t * tile);
   const size_t tiles = seq_tiles ? 0 : rows * D * 2;
   const size_t qk_tiles = qk_fp8 ? rows * vsa::kF8RowBytes : tiles;
+  const bool scales = qk_fp8 || qk_split;
   const size_t pooled = static_cast<size_t>(B * H * n_t * D * 4);
   w.q_t = off; off += align256(qk_tiles);
   w.k_t = off; off += align256(qk_tiles);
   w.v_t = off; off += align256(tiles);
-  w.q_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
-  w.k_s = off; off += align256(qk_fp8 ? rows * 4 : 0);
+  w.q_s = off; off += align256(scales ? rows * 4 : 0);
+  w.k_s = off; off += align256(scales ? rows * 4 : 0);
   w.q_n = off; off += align256(rows * 4);
   w.kv_max = off; off += align256(static_cast<size_t>(B * H * 8));
   w.pq = off; off += align256(pooled);
@@ -305,6 +306,11 @@ vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, i
   w.scores = off; off += align256(static_cast<size_t>(B * H * n_t * n_t * 4));
   w.idx = off; off += align256(static_cast<size_t>(B * H * V * topk * 4));
   w.o_c = off; off += align256(pooled);
+  // prefix split: 8-bit codes of Q and K beside the bf16 copies, and their overflow-bound statistics
+  w.q_c = off; off += align256(qk_split ? rows * vsa::kF8RowBytes : 0);
+  w.k_c = off; off += align256(qk_split ? rows * vsa::kF8RowBytes : 0);
+  w.q_n8 = off; off += align256(qk_split ? rows * 4 : 0);
+  w.kv_max8 = off; off += align256(qk_split ? static_cast<size_t>(B * H * 8) : 0);
   w.total = off;
   return w;
 }
@@ -439,6 +445,7 @@ struct vsa_plan_s {
   const void** d_part_table = nullptr;
   bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
   bool qk_fp8 = false;     // 8-bit Q/K (E4M3 codes, one scale per token and head) for the fine logits
+  bool qk_split = false;   // the same for the dense prefix query tiles only; video query tiles keep bf16
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
   // reference keep: kr of the n_ref reference tiles kept per video query tile (idx rows hold kr + topk);
@@ -526,9 +533,12 @@ vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H,
 // qs/ks: with an 8-bit plan, the per-row scales (qt/kt then receive codes).
 // qn/kv (with pooling): the overflow-bound statistics of the staged tiles (8-bit Q/K: Q/K norms from the
 // codes); kv must hold zeros on entry (the kernel raises it with atomicMax).
+// f8: write Q and K as 8-bit codes (qt, kt: 128-byte code rows, qs, ks: row scales); vt NULL without
+// pooling: V is not read.
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
                       float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr, float* qs = nullptr,
-                      float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr) {
+                      float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr, int f8 = -1) {
+  const bool codes = (f8 < 0) ? p->qk_fp8 : (f8 != 0);
   const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
@@ -548,7 +558,7 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
     constexpr int D = decltype(dc)::value;
     const bool parts = pio.table != nullptr;
     auto by_tile = [&](auto k64, auto k128) { return p->r.sh ? launch(k128) : launch(k64); };
-    if (p->qk_fp8)
+    if (codes)
       return parts ? by_tile(vsa::gather_pool_kernel<D, true, true, 1>, vsa::gather_pool_kernel<D, true, true, 2>)
                    : by_tile(vsa::gather_pool_kernel<D, false, true, 1>, vsa::gather_pool_kernel<D, false, true, 2>);
     return parts ? by_tile(vsa::gather_pool_kernel<D, true, false, 1>, vsa::gather_pool_kernel<D, true, false, 2>)
@@ -629,8 +639,30 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
     return launch_check("topk");
   };
   if (p->V > 0 && p->kr > 0) VSA_TRY(select(p->d_refs, p->n_ref, p->kr, 0));
-  if (p->V > 0 && p->topk > 0) VSA_TRY(select(nullptr, p->V, p->topk, p->kr));
   dim3 grid((p->n_t + vsa::kCompRows - 1) / vsa::kCompRows, static_cast<unsigned>(BH));
+  // Up to 40 x 32 tiles: the video top-k and the compression in one pass over each score row (a row's
+  // keys held in registers); longer rows: the top-k kernel, then the compression kernel.
+  const int J = (p->n_t + 31) / 32;
+  const int k = (p->V > 0) ? p->topk : 0;
+  if (J <= 40) {
+    VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+      constexpr int D = decltype(dc)::value;
+      auto launch = [&](auto kernel) {
+        kernel<<<grid, 256, 0, s>>>(S, pv, o_c, idx, p->n_t, p->P, k, p->kr + p->topk, p->kr, gate_nonzero);
+      };
+      if (J <= 8)
+        launch(vsa::select_compress_kernel<D, 8>);
+      else if (J <= 16)
+        launch(vsa::select_compress_kernel<D, 16>);
+      else if (J <= 24)
+        launch(vsa::select_compress_kernel<D, 24>);
+      else
+        launch(vsa::select_compress_kernel<D, 40>);
+      return VSA_OK;
+    }));
+    return launch_check("select_compress");
+  }
+  if (k > 0) VSA_TRY(select(nullptr, p->V, p->topk, p->kr));
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
     vsa::compress_kernel<D><<<grid, 256, 0, s>>>(S, pv, o_c, p->n_t, gate_nonzero);
@@ -644,9 +676,11 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
                     const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
                     const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr, const float* qs = nullptr,
-                    const float* ks = nullptr, const float* qn = nullptr, const uint32_t* kv = nullptr) {
+                    const float* ks = nullptr, const float* qn = nullptr, const uint32_t* kv = nullptr, int f8 = -1,
+                    int s_lo = 0, int n_s = -1) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
+  const bool codes = (f8 < 0) ? p->qk_fp8 : (f8 != 0);  // Q and K as 8-bit codes (8-bit S^T product)
   // the kernel works in 64-row blocks: one per tile, or two per 128-token tile
   const int64_t n_rb = static_cast<int64_t>(p->n_t) << p->r.sh;
   const int64_t rows = static_cast<int64_t>(p->B) * p->H * n_rb * kTile;
@@ -658,7 +692,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     for (int t = 0; t < 3; ++t)
       VSA_TRY(make_seq_maps(&sm.prefix[t], sm.video[t], seq_qkv[t], p->B, p->r.L, p->H, p->D, p->r.L - vid, p->r.T,
                             p->r.Hg, p->r.W));
-  } else if (p->qk_fp8) {
+  } else if (codes) {
     VSA_TRY(make_code_map(&mq, qt, rows));
     VSA_TRY(make_code_map(&mk, kt, rows));
     VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
@@ -667,7 +701,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     VSA_TRY(make_tile_map(&mk, kt, rows, p->D));
     VSA_TRY(make_tile_map(&mv, vt, rows, p->D));
   }
-  if (p->qk_fp8 && (qs == nullptr || ks == nullptr)) return fail(VSA_ERR_INVALID_ARG, "8-bit Q/K needs its scales");
+  if (codes && (qs == nullptr || ks == nullptr)) return fail(VSA_ERR_INVALID_ARG, "8-bit Q/K needs its scales");
   vsa::AttnArgs a{};
   a.idx = idx;
   a.tile_token = seq ? p->d_row_token : p->d_tile_token;  // query row -> token (-1: not stored)
@@ -704,7 +738,13 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.n_exempt = p->n_ref > 0 ? static_cast<int>(p->exempt_tiles.size()) : p->P;
   a.exempt = p->n_ref > 0 ? p->d_exempt : nullptr;
   a.scale_log2 = static_cast<float>(static_cast<double>(p->r.scale) * 1.4426950408889634);
-  a.n_items = static_cast<int64_t>(p->B) * p->H * n_rb;
+  // the row blocks this launch covers: [s_lo, s_lo + n_s) of every (b, h)
+  if (n_s < 0) n_s = static_cast<int>(n_rb) - s_lo;
+  if (s_lo < 0 || n_s < 0 || s_lo + n_s > n_rb) return fail(VSA_ERR_INVALID_ARG, "attention row-block range");
+  if (n_s == 0) return VSA_OK;
+  a.s_lo = s_lo;
+  a.n_s = n_s;
+  a.n_items = static_cast<int64_t>(p->B) * p->H * n_s;
   const int64_t grid = std::min<int64_t>(a.n_items, p->num_sms);
   // the item counter of the persistent schedule starts at zero for every launch
   VSA_CUDA_TRY(cudaMemsetAsync(a.sched, 0, sizeof(int), s));
@@ -717,7 +757,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
     constexpr int D = decltype(dc)::value;
     if (seq) return launch(vsa::vsa_attn_kernel<D, true, false>, vsa::AttnLayout<D>::bytes(p->n_t));
-    if (p->qk_fp8) return launch(vsa::vsa_attn_kernel<D, false, true>, vsa::AttnLayout<D, true>::bytes(p->n_t));
+    if (codes) return launch(vsa::vsa_attn_kernel<D, false, true>, vsa::AttnLayout<D, true>::bytes(p->n_t));
     return launch(vsa::vsa_attn_kernel<D, false, false>, vsa::AttnLayout<D>::bytes(p->n_t));
   }));
   return launch_check("attention");
@@ -764,13 +804,15 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->d_status = p->d_status;
   q->seq_tiles = p->seq_tiles;
   q->qk_fp8 = p->qk_fp8;
+  q->qk_split = p->qk_split;
   q->kr = p->kr;
   q->n_ref = p->n_ref;
   q->exempt_tiles = p->exempt_tiles;
   q->ref_tiles = p->ref_tiles;
   q->d_exempt = p->d_exempt;
   q->d_refs = p->d_refs;
-  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk + q->kr, q->seq_tiles, q->qk_fp8);
+  q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk + q->kr, q->seq_tiles, q->qk_fp8,
+                      q->qk_split);
   q->owns_device = false;
   return q;
 }
@@ -787,7 +829,9 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   h.chunk_bytes = align256(tokens * static_cast<size_t>(hc) * p->D * 2);
   h.fwd = 0;
   size_t off =
-      align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8).total);
+      align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8,
+                           p->qk_split)
+                   .total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
     off += 4 * h.chunk_bytes;  // q, k, v, out
@@ -839,9 +883,32 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   const bool seq = p->seq_tiles;
   VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io, qsc, ksc,
                      qn, kv));
+  // prefix split: a second gather writes the 8-bit codes of Q and K (no pooling, V not read) with their
+  // own overflow-bound statistics; the value maximum comes from the first gather's statistics
+  auto* qc = w + p->ws.q_c;
+  auto* kc = w + p->ws.k_c;
+  auto* qn8 = reinterpret_cast<float*>(w + p->ws.q_n8);
+  auto* kv8 = reinterpret_cast<uint32_t*>(w + p->ws.kv_max8);
+  if (p->qk_split) {
+    auto* qs2 = reinterpret_cast<float*>(w + p->ws.q_s);
+    auto* ks2 = reinterpret_cast<float*>(w + p->ws.k_s);
+    VSA_CUDA_TRY(cudaMemsetAsync(kv8, 0, static_cast<size_t>(p->B) * p->H * 8, s));
+    VSA_TRY(run_gather(p, q, k, v, qc, kc, nullptr, nullptr, nullptr, nullptr, s, io, qs2, ks2, qn8, kv8, 1));
+    VSA_CUDA_TRY(cudaMemcpy2DAsync(kv8 + 1, 8, kv + 1, 8, 4, static_cast<size_t>(p->B) * p->H,
+                                   cudaMemcpyDeviceToDevice, s));
+  }
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
+  if (p->qk_split) {
+    // the dense prefix query row blocks on the 8-bit S^T kernel, then the video ones on the bf16 kernel
+    const int pre = p->P << p->r.sh;
+    VSA_TRY(run_attn(p, qc, kc, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io,
+                     reinterpret_cast<float*>(w + p->ws.q_s), reinterpret_cast<float*>(w + p->ws.k_s), qn8, kv8, 1, 0,
+                     pre));
+    return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io, nullptr, nullptr, qn, kv, 0,
+                    pre);
+  }
   return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io, qsc, ksc, qn, kv);
 }
 
@@ -857,7 +924,8 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->softmax_scale = r.scale;
   d->workspace_bytes =
       make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.tile, r.n_video, r.topk + r.kr, g->seq_tiles != 0,
-                  g->qk_fp8 != 0).total;
+                  g->qk_fp8 == 1, g->qk_fp8 == 2)
+          .total;
   d->selected_pairs = r.n_video * (r.n_prefix - r.n_ref + r.kr + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
   d->tile_size = r.tile;
   d->n_ref_tiles = static_cast<int32_t>(r.n_ref);
@@ -929,11 +997,13 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   build_block_masks(r, p->tile_valid, &p->mask_tiled);
   if (r.tile == kTile) build_seq_tables(r, p->mask_tiled, &p->row_token, &p->mask_seq, &p->coord);
   p->seq_tiles = g->seq_tiles != 0;
-  p->qk_fp8 = g->qk_fp8 != 0;
+  p->qk_fp8 = g->qk_fp8 == 1;
+  p->qk_split = g->qk_fp8 == 2;
   p->kr = r.kr;
   p->n_ref = static_cast<int32_t>(r.n_ref);
   for (int32_t j = 0; j < p->P && p->n_ref > 0; ++j) (r.tile_ref[j] ? p->ref_tiles : p->exempt_tiles).push_back(j);
-  p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8);
+  p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8,
+                      p->qk_split);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);
@@ -960,7 +1030,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
       cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess ||
       (p->n_ref > 0 && (cudaMalloc(&p->d_exempt, std::max<size_t>(4, p->exempt_tiles.size() * 4)) != cudaSuccess ||
                         cudaMalloc(&p->d_refs, p->ref_tiles.size() * 4) != cudaSuccess)) ||
-      (!p->qk_fp8 && cudaMalloc(&p->d_stats, stats_bytes(p)) != cudaSuccess)) {
+      (!p->qk_fp8 && !p->qk_split && cudaMalloc(&p->d_stats, stats_bytes(p)) != cudaSuccess)) {
     cleanup();
     return fail(VSA_ERR_CUDA, "cudaMalloc of the plan tables failed");
   }
@@ -1049,7 +1119,8 @@ vsa_status vsa_gather_tiles(vsa_plan p, const vsa_bf16* q, const vsa_bf16* k, co
                             vsa_bf16* k_t, vsa_bf16* v_t, float* pq, float* pk, float* pv, float* q_norm,
                             float* kv_max, void* stream) {
   VSA_TRY(check_plan(p));
-  if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
+  if (p->qk_fp8 || p->qk_split)
+    return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q, k, v, q_t, k_t, v_t}));
   const int npool = (pq != nullptr) + (pk != nullptr) + (pv != nullptr);
   if (npool != 0 && npool != 3) return fail(VSA_ERR_INVALID_ARG, "pq, pk, pv must be all NULL or all set");
@@ -1070,7 +1141,8 @@ vsa_status vsa_pool_and_score(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* k
   VSA_TRY(check_ptrs({pq, pk, pv, scores}));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q_t != nullptr) {
-    if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
+    if (p->qk_fp8 || p->qk_split)
+    return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
     VSA_TRY(check_ptrs({q_t, k_t, v_t}));
     VSA_TRY(run_pool(p, q_t, k_t, v_t, pq, pk, pv, s));
   }
@@ -1089,7 +1161,8 @@ vsa_status vsa_sparse_attn_fwd(vsa_plan p, const vsa_bf16* q_t, const vsa_bf16* 
                                const int32_t* idx, const float* o_c, const vsa_bf16* gate, vsa_bf16* out,
                                const float* q_norm, const float* kv_max, void* stream) {
   VSA_TRY(check_plan(p));
-  if (p->qk_fp8) return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
+  if (p->qk_fp8 || p->qk_split)
+    return fail(VSA_ERR_UNSUPPORTED, "the step entry points take bf16 tiles: use vsa_forward with qk_fp8");
   VSA_TRY(check_ptrs({q_t, k_t, v_t, o_c, gate, out}));
   if (p->V > 0) VSA_TRY(check_ptrs({idx}));
   const auto s = static_cast<cudaStream_t>(stream);

@@ -104,6 +104,12 @@ typedef struct vsa_geometry {
                                 with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
                                 by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4, 64-token tiles */
   int32_t qk_fp8;            /* 0: the fine branch's logits use the bf16 Q and K;
+                                2: the pages' prefix split: the dense prefix query tiles take the
+                                8-bit logits described under 1, the video query tiles keep bf16
+                                (their FP4 kernel on the pages is not built); needs seq_tiles = 0
+                                and, like 1, only the whole-forward entry points accept it.
+                                Passage: "FastH3 OmniRef inference", section "Device profiles"
+                                (dense prefix query tiles at 8-bit Q/K with bf16 P.V);
                                 1: 8-bit Q/K: each (token, head) row of Q and K is quantised to
                                 OCP FP8 E4M3 codes with one binary32 scale s = amax / 448
                                 (code = E4M3(x / s), round to nearest even, saturating; an
@@ -360,8 +366,13 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
  * key-row norm (likewise) and the largest |v| (two float32); the attention
  * bounds its logits by them (Cauchy-Schwarz) to skip rescale checks that
  * cannot fire. */
+/* With qk_fp8 = 2 (the prefix split) q_t and k_t hold the bf16 copies, q_c and k_c
+ * the E4M3 codes [B, H, n_tiles, 64, 128] with their row scales in q_s, k_s, and
+ * q_n8, kv_max8 the statistics of the dequantised rows (q_c .. kv_max8 are empty
+ * otherwise). */
 typedef struct vsa_workspace_layout {
-  size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c, total;
+  size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c;
+  size_t q_c, k_c, q_n8, kv_max8, total;
 } vsa_workspace_layout;
 vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
 

@@ -162,11 +162,26 @@ def test_qk_fp8_workspace_and_limits(vsa):
         vsa.vsa_plan_query(qk_fp8=True, seq_tiles=True, **kw)
     assert e.value.status == 3  # VSA_ERR_UNSUPPORTED
     g, keep = vsa.make_geometry(**kw)
-    g.qk_fp8 = 2
+    g.qk_fp8 = 3
     import ctypes
 
     d = vsa.PlanDims()
     assert vsa.load_library().vsa_plan_query(ctypes.byref(g), ctypes.byref(d)) == 1  # VSA_ERR_INVALID_ARG
+
+
+def test_qk_prefix_split_workspace(vsa):
+    """The prefix split (qk_fp8 = 2) keeps the bf16 copies and adds 8-bit code rows of Q and K (128 bytes
+    per tile row each), their scales and the dequantised rows' norms and (b, h) maxima."""
+    kw = dict(batch=1, heads=56, head_dim=128, segments=(512, 0, 768), grid=(24, 48, 64), sparsity=0.9)
+    a = vsa.vsa_plan_query(**kw)["workspace_bytes"]
+    c = vsa.vsa_plan_query(qk_fp8="prefix", **kw)["workspace_bytes"]
+    rows = 56 * 1172 * 64
+    assert c - a == 2 * rows * 128 + 2 * rows * 4 + rows * 4 + 512  # codes, scales, norms, maxima (aligned)
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_plan_query(qk_fp8="prefix", seq_tiles=True, **kw)
+    assert e.value.status == 3  # VSA_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        vsa.make_geometry(qk_fp8="video", **kw)
 
 
 @pytest.mark.parametrize("segments,grid,cube", [
