@@ -4,15 +4,27 @@
 
 One step = one whole VSA-H3 forward (gather + pool, pooled scores, top-k +
 compression, block-sparse attention + gated epilogue) over one synthetic
-input already resident in HBM.  The default workload is the 1344x768-shaped
+input already resident in HBM, timed through the public call vsa_forward.
+The per-stage times (and the attention time the roofline uses) come from a
+second pass right after, through the step entry points.  The default workload is the 1344x768-shaped
 one at sparsity 0.9 (56 heads, D=128, 73,728 video + 1,280 prefix tokens).
 
 Metric: effective TFLOP/s counting only the selected (query tile, key tile)
 pairs, 4*T*T*D FLOP each for T-token tiles (T = 64, or 128 for the
 128-token-tile workload), per whole forward; ms per call is reported too.
-Multi-GPU (torchrun): every rank runs its own forward on its own seeded input
-(the forward shards by (batch, head) with no exchange), value = all ranks'
-FLOPs / the slowest rank's time ("scaling": "weak").
+Multi-GPU (torchrun), two modes:
+  --mode ulysses (the default with more than one rank): ONE forward split over
+      the ranks the way sequence parallelism holds it.  Rank r keeps tokens
+      [r*L/N, (r+1)*L/N) of q, k, v, gate and out in its own HBM, maps the other
+      ranks' parts through CUDA IPC, and runs vsa_forward_parts for heads
+      [r*H/N, (r+1)*H/N): the gather kernel's loads and the epilogue's stores
+      carry the two all-to-all exchanges over NVLink (plain peer loads and
+      stores, no library kernel on peer memory).  value = one forward's FLOPs /
+      the slowest rank's time ("scaling": "strong").
+  --mode replicas: every rank runs its own whole forward on its own seeded
+      input (no exchange); value = all ranks' FLOPs / the slowest rank's time
+      ("scaling": "weak").
+With one GPU both modes are the plain forward.
 
 ``--impl reference`` times the CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
@@ -204,7 +216,7 @@ def omp_threads():
     return int(n) if n else (os.cpu_count() or 1)
 
 
-def run_reference(args, w, world, rank):
+def run_reference(args, w, world, rank, mode="replicas"):
     """CPU oracle arm: rank 0 only."""
     if rank != 0:
         return
@@ -220,8 +232,9 @@ def run_reference(args, w, world, rank):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based normal)",
-        "config": config_dict(w),
+        "scaling": "weak" if mode == "replicas" else "strong", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based normal)",
+        "config": config_dict(w, world=world, mode=mode),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -231,7 +244,7 @@ def run_reference(args, w, world, rank):
 # ----------------------------------------------------------------------------- GPU arm
 
 
-def config_dict(w, dims=None):
+def config_dict(w, dims=None, world=1, mode="replicas"):
     import oracle
 
     geo = oracle.geometry(w.segments, w.grid, tile=w.tile, cube=w.cube, ref_segments=w.ref_segments) \
@@ -251,10 +264,52 @@ def config_dict(w, dims=None):
         "selected_tile_pairs": pairs * w.batch * w.heads,
         "selected_tflop_per_call": pairs * w.batch * w.heads * tile_flops(w.head_dim, w.tile) / 1e12,
         "l2": "no flush: Q/K/V/out are %.1f GB per step, > 126 MB L2" % (4 * w.batch * w.seq_len * w.heads * w.head_dim * 2 / 1e9),
+        "parallelism": (f"independent forward per GPU x{world}" if world == 1 or mode == "replicas"
+                        else f"ulysses sequence parallel sp{world} (heads and token parts over {world} GPUs)"),
     }
 
 
-def run_vsa(args, w, world, rank, local):
+def prep_roofline(w, dims, stage_ms, peaks, sm_mhz):
+    """Achieved rates of the selection kernels against their own rooflines: HBM bytes for the gather
+    and for top-k + compression (algorithmic bytes per launch, counted from the tensors each reads and
+    writes), fp32 FMA throughput for the pooled scores (nominal: 128 FMA lanes per SM per clock at the
+    sampled SM clock, no measured fp32 peak exists)."""
+    B, H, D, L = w.batch, w.heads, w.head_dim, w.seq_len
+    n_t, P, k, kr = dims["n_tiles"], dims["n_prefix_tiles"], dims["topk"], dims["ref_topk"]
+    T = dims["tile_size"]
+    V = n_t - P
+    bh = B * H
+    gather_bytes = (3 * B * L * H * D * 2            # q, k, v read (each token once)
+                    + 3 * bh * n_t * T * D * 2         # tile-order copies written (pads included)
+                    + 3 * bh * n_t * D * 4             # pooled tiles written
+                    + bh * n_t * T * 4 + bh * 8)       # query row norms, key/value maxima
+    scores_flop = 2 * bh * n_t * n_t * D
+    scores_bytes = 2 * bh * n_t * D * 4 + bh * n_t * n_t * 4
+    sel_bytes = bh * n_t * n_t * 4 + bh * n_t * D * 4 + bh * V * (k + kr) * 4 + bh * n_t * D * 4
+    compress_flop = 2 * bh * n_t * n_t * D
+    hbm = peaks["hbm_gbs"]
+    fp32_nominal = 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12  # TFLOP/s
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms * 1e-3) / 1e9
+
+    g = gbs(gather_bytes, stage_ms["gather_pool"])
+    t = gbs(sel_bytes, stage_ms["topk_compress"])
+    sc = scores_flop / (stage_ms["scores"] * 1e-3) / 1e12
+    return {
+        "gather_pool": {"bound": "hbm", "bytes": gather_bytes, "achieved_gbs": g, "peak_gbs": hbm, "frac": g / hbm},
+        "scores": {"bound": "alu", "flop": scores_flop, "bytes": scores_bytes, "achieved_tflops": sc,
+                   "peak_tflops_nominal_fp32": fp32_nominal, "frac": sc / fp32_nominal,
+                   "achieved_gbs": gbs(scores_bytes, stage_ms["scores"])},
+        "topk_compress": {"bound": "hbm", "bytes": sel_bytes, "achieved_gbs": t, "peak_gbs": hbm, "frac": t / hbm,
+                          "compress_flop": compress_flop,
+                          "compress_tflops": compress_flop / (stage_ms["topk_compress"] * 1e-3) / 1e12},
+        "peak_note": f"HBM: {peaks['source']} copy bandwidth; fp32: nominal, 148 SMs x 128 FMA/clk at the "
+                     f"sampled median SM clock",
+    }
+
+
+def run_vsa(args, w, world, rank, local, mode="replicas"):
     import torch
 
     import block_sparse_tiled_b200 as vsa
@@ -274,43 +329,24 @@ def run_vsa(args, w, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     flops_call = dims["selected_pairs"] * w.batch * w.heads * tile_flops(w.head_dim, w.tile)
 
-    ev = {n: [] for n in ("t0", "t1", "t2", "t3", "t4")}
-
-    def step(record):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
-        if record:
-            e[0].record(stream)
-        vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], v["q_t"], v["k_t"], v["v_t"], v["pq"], v["pk"], v["pv"],
-                             q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
-        if record:
-            e[1].record(stream)
-        vsa.vsa_pool_and_score(plan, None, None, None, v["pq"], v["pk"], v["pv"], v["scores"], stream=stream)
-        if record:
-            e[2].record(stream)
-        vsa.vsa_topk_select(plan, v["scores"], v["pv"], v["idx"], v["o_c"], stream=stream)
-        if record:
-            e[3].record(stream)
-        vsa.vsa_sparse_attn_fwd(plan, v["q_t"], v["k_t"], v["v_t"], v["idx"], v["o_c"], x["gate"], out,
-                                q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
-        if record:
-            e[4].record(stream)
-            for n, evt in zip(("t0", "t1", "t2", "t3", "t4"), e):
-                ev[n].append(evt)
+    def forward():
+        vsa.vsa_forward(plan, x["q"], x["k"], x["v"], x["gate"], out=out, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
-        step(False)
+        forward()
     torch.cuda.synchronize()
     code, where = vsa.device_status(plan)
     if code != 0:
         raise RuntimeError(f"device status {code} at site {where} during warm-up")
 
+    # ---- the timed region: K whole forwards through the public call, one per step
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record(stream)
         for _ in range(args.steps):
-            step(True)
+            forward()
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -319,14 +355,36 @@ def run_vsa(args, w, world, rank, local):
     code, where = vsa.device_status(plan)
     if code != 0:
         raise RuntimeError(f"device status {code} at site {where} in the timed region")
+    ms_step = elapsed_ms / args.steps
+    value = world * flops_call / (ms_step * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # ---- stage pass, right after: the same forward through the four step entry points (the gather's
+    # overflow-bound statistics passed on to the attention, as vsa_forward does), with an event between
+    # stages; the attention's mean time here is the roofline's kernel time
+    ev = {n: [] for n in ("t0", "t1", "t2", "t3", "t4")}
+    for _ in range(args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e[0].record(stream)
+        vsa.vsa_gather_tiles(plan, x["q"], x["k"], x["v"], v["q_t"], v["k_t"], v["v_t"], v["pq"], v["pk"], v["pv"],
+                             q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
+        e[1].record(stream)
+        vsa.vsa_pool_and_score(plan, None, None, None, v["pq"], v["pk"], v["pv"], v["scores"], stream=stream)
+        e[2].record(stream)
+        vsa.vsa_topk_select(plan, v["scores"], v["pv"], v["idx"], v["o_c"], stream=stream)
+        e[3].record(stream)
+        vsa.vsa_sparse_attn_fwd(plan, v["q_t"], v["k_t"], v["v_t"], v["idx"], v["o_c"], x["gate"], out,
+                                q_norm=v["q_n"], kv_max=v["kv_max"], stream=stream)
+        e[4].record(stream)
+        for n, evt in zip(("t0", "t1", "t2", "t3", "t4"), e):
+            ev[n].append(evt)
+    torch.cuda.synchronize()
 
     def avg(a, b):
         return statistics.mean(x.elapsed_time(y) for x, y in zip(ev[a], ev[b]))
 
     stage_ms = {"gather_pool": avg("t0", "t1"), "scores": avg("t1", "t2"), "topk_compress": avg("t2", "t3"),
                 "attention": avg("t3", "t4")}
-    ms_step = elapsed_ms / args.steps
-    value = world * flops_call / (ms_step * 1e-3) / 1e12
 
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     hx = {}
@@ -352,37 +410,163 @@ def run_vsa(args, w, world, rank, local):
 
     peaks = load_peaks()
     attn_tflops = flops_call / (stage_ms["attention"] * 1e-3) / 1e12
+    sm_mhz = clocks.get("sm_mhz")
+    # clock-normalised: SM cycles per 64-query x 128-key block of the attention (per SM), and per launch
+    blocks = flops_call / (2 * tile_flops(w.head_dim, 64))
+    attn_cycles = stage_ms["attention"] * 1e-3 * sm_mhz * 1e6 if sm_mhz else None
     roofline = {
-        "kernel": "vsa_attn_kernel<128>", "bound": "tensor", "achieved": attn_tflops,
-        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-        "frac": attn_tflops / peaks["bf16_tflops_sustained"],
-        "peak_kind": f"{peaks['source']} sustained dense bf16 (kernel timed inside a seconds-long loop)",
-        "frac_of_burst_peak": attn_tflops / peaks["bf16_tflops"],
+        "kernel": f"vsa_attn_kernel<{w.head_dim}>", "bound": "tensor", "achieved": attn_tflops,
+        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
+        "peak_kind": f"{peaks['source']} burst dense bf16 (cuBLAS)",
+        "frac_of_sustained_peak": attn_tflops / peaks["bf16_tflops_sustained"],
+        "kernel_time": "mean of the attention launches in the stage pass that follows the timed region",
         "algorithmic_flop_per_launch": flops_call,
+        "attn_mcycles_per_launch": attn_cycles / 1e6 if attn_cycles else None,
+        "cycles_per_block_per_sm": attn_cycles * 148 / blocks if attn_cycles else None,
         "traffic": measured_attn_traffic() if w.name == "768p_s0.9" else None,
         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
     }
-    # library kernels per timed step: gather+pool, scores, one top-k pass per candidate set (reference
-    # tiles, video tiles), compression, attention
+    # library kernels per timed step (one vsa_forward): gate check, gather+pool, scores, a top-k pass over
+    # the reference candidates (with reference segments), top-k + compression in one kernel (rows of up to
+    # 1280 tiles; longer rows take a top-k and a compression kernel), attention
     nv = dims["n_video_tiles"]
-    topk_passes = int(nv > 0 and dims["ref_topk"] > 0) + int(nv > 0 and dims["topk"] > 0)
-    launches = (4 + topk_passes) * args.steps
+    fused = (dims["n_tiles"] + 31) // 32 <= 40
+    launches = (5 + int(nv > 0 and dims["ref_topk"] > 0) + int(not fused)) * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak" if mode == "replicas" else "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based normal, structured tile offsets)",
-        "config": dict(config_dict(w, dims), parallelism=f"independent forward per GPU x{world}"),
+        "config": config_dict(w, dims, world=world, mode=mode),
         "stage_ms": stage_ms, "roofline": roofline,
+        "prep_roofline": prep_roofline(w, dims, stage_ms, peaks, sm_mhz),
         "e2e": {"value": world * flops_call / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "head_chunk": vsa.default_head_chunk(w.heads, w.head_dim)},
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, fl, desc = oracle_sample(w, args.cpu_every)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
                                 "sample": desc, "seconds": dt}
+    plan.destroy()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_ulysses(args, w, world, rank, local):
+    """Sequence-parallel forward over `world` ranks (see the module docstring)."""
+    import torch
+    import torch.distributed as dist
+    from torch.multiprocessing.reductions import reduce_tensor
+
+    import block_sparse_tiled_b200 as vsa
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L, H = w.seq_len, w.heads
+    ls, hn, h0 = vsa.ulysses_partition(L, H, world, rank)
+    # every rank draws the same seeded input and keeps its token part of it
+    x = synth.make_inputs(w, seed=0, device=dev)
+    mine = {n: x[n][:, rank * ls:(rank + 1) * ls].contiguous() for n in ("q", "k", "v", "gate")}
+    mine["out"] = torch.empty_like(mine["q"])
+    del x
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    # the other ranks' parts, mapped through CUDA IPC handles exchanged over the process group
+    handles = {n: reduce_tensor(t) for n, t in mine.items()}
+    every = [None] * world
+    dist.all_gather_object(every, handles)
+    parts = {n: [] for n in mine}
+    for r in range(world):
+        for n in mine:
+            if r == rank:
+                parts[n].append(mine[n])
+            else:
+                fn, fargs = every[r][n]
+                parts[n].append(fn(*fargs))
+    plan = vsa.vsa_plan_tiles(batch=w.batch, heads=hn, head_dim=w.head_dim, segments=w.segments, grid=w.grid,
+                              sparsity=w.sparsity, tile_size=w.tile, cube=w.cube, ref_segments=w.ref_segments,
+                              ref_keep=w.ref_keep)
+    dims = plan.dims
+    ws = vsa.alloc_workspace(plan, dev)
+    stream = torch.cuda.current_stream(dev)
+    flops_call = dims["selected_pairs"] * w.batch * H * tile_flops(w.head_dim, w.tile)  # the whole forward
+
+    def step():
+        vsa.vsa_forward_parts(plan, parts["q"], parts["k"], parts["v"], parts["gate"], parts["out"], h0,
+                              workspace=ws, stream=stream)
+
+    barrier(world)  # every part is written before any rank reads it
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    code, where = vsa.device_status(plan)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at site {where} during warm-up")
+    with ClockSampler(local) as clk:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_step = max_over_ranks(start.elapsed_time(stop) / args.steps, world, dev)
+    value = flops_call / (ms_step * 1e-3) / 1e12
+
+    # end to end: every rank copies its token part in from pinned host memory, the ranks meet, run the
+    # forward, meet again (every out part complete) and copy their out part back
+    hx = {n: torch.empty(mine[n].shape, dtype=mine[n].dtype, pin_memory=True) for n in ("q", "k", "v", "gate")}
+    for n in hx:
+        hx[n].copy_(mine[n])
+    hout = torch.empty(mine["out"].shape, dtype=mine["out"].dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize()
+    barrier(world)
+    s0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        for n in hx:
+            mine[n].copy_(hx[n], non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        step()
+        torch.cuda.synchronize()
+        barrier(world)
+        hout.copy_(mine["out"], non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_ms = max_over_ranks((time.perf_counter() - s0) * 1e3 / e2e_steps, world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hout.numel() * hout.element_size()
+    code, where = vsa.device_status(plan)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at site {where}")
+    B, D = w.batch, w.head_dim
+    remote = (world - 1) / world
+    exchange = {"q_k_v_read_from_peers": int(3 * B * L * hn * D * 2 * remote),
+                "gate_read_from_peers": int(B * L * hn * 2 * remote),
+                "out_written_to_peers": int(B * L * hn * D * 2 * remote)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based normal, structured tile offsets)",
+        "config": config_dict(w, dims=None, world=world, mode="ulysses"),
+        "mode": "ulysses", "heads_per_rank": hn, "tokens_per_part": ls,
+        "exchange_bytes_per_rank": exchange,
+        "e2e": {"value": flops_call / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+                "timing": "wall clock per step around each rank's copies, barriers and forward; max over ranks"},
+        # per rank and step: gather+pool, scores, select+compression, attention (no gate check over parts)
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    # release the peer mappings before any rank frees what they map
+    parts = None
+    torch.cuda.synchronize()
+    barrier(world)
     plan.destroy()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -432,6 +616,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["vsa", "reference"], default="vsa")
+    ap.add_argument("--mode", choices=["auto", "ulysses", "replicas"], default="auto",
+                    help="with several ranks: one forward split over them (ulysses, the default) or one whole "
+                         "forward per rank (replicas)")
     ap.add_argument("--workload", default="768p_s0.9")
     ap.add_argument("--sparsity", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -441,6 +628,9 @@ def main():
                     help="side measurement: vsa_forward with tile-order copies against a seq_tiles plan")
     ap.add_argument("--ab-qk-fp8", action="store_true",
                     help="side measurement: vsa_forward with bf16 Q/K logits against 8-bit (E4M3) Q/K")
+    ap.add_argument("--ab-prefix-fp8", action="store_true",
+                    help="side measurement: vsa_forward with bf16 Q/K logits against the prefix split (8-bit Q/K "
+                         "for the dense prefix query tiles only)")
     args = ap.parse_args()
     import synth
 
@@ -453,12 +643,19 @@ def main():
     if args.ab_qk_fp8:
         run_ab(args, w, {"qk_bf16": {}, "qk_fp8": {"qk_fp8": True}})
         return
+    if args.ab_prefix_fp8:
+        run_ab(args, w, {"qk_bf16": {}, "qk_prefix_fp8": {"qk_fp8": "prefix"}})
+        return
     world, rank, local = dist_setup(args)
     try:
+        # auto: one forward split over the ranks (with one rank, the plain forward)
+        mode = "ulysses" if args.mode == "auto" else args.mode
         if args.impl == "reference":
-            run_reference(args, w, world, rank)
+            run_reference(args, w, world, rank, mode)
+        elif mode == "ulysses" and world > 1:
+            run_ulysses(args, w, world, rank, local)
         else:
-            run_vsa(args, w, world, rank, local)
+            run_vsa(args, w, world, rank, local, mode)
     finally:
         if world > 1:
             import torch.distributed as dist
