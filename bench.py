@@ -79,7 +79,8 @@ def measured_attn_traffic():
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
     h = hashlib.sha256()
-    for rel in ("block_sparse_tiled_b200/csrc/attn_sm100.cuh", "block_sparse_tiled_b200/csrc/ptx.cuh"):
+    for rel in ("block_sparse_tiled_b200/csrc/attn_sm100.cuh", "block_sparse_tiled_b200/csrc/attn_pair_sm100.cuh",
+                "block_sparse_tiled_b200/csrc/ptx.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     if vals.get("kernel_source_sha256") != h.hexdigest():
@@ -415,7 +416,9 @@ def run_vsa(args, w, world, rank, local, mode="replicas"):
     blocks = flops_call / (2 * tile_flops(w.head_dim, 64))
     attn_cycles = stage_ms["attention"] * 1e-3 * sm_mhz * 1e6 if sm_mhz else None
     roofline = {
-        "kernel": f"vsa_attn_kernel<{w.head_dim}>", "bound": "tensor", "achieved": attn_tflops,
+        "kernel": f"attention stage: vsa_attn_kernel<{w.head_dim}> (video query row blocks) and "
+                  f"vsa_attn_pair_kernel<{w.head_dim}> (prefix query row blocks, two at a time)",
+        "bound": "tensor", "achieved": attn_tflops,
         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
         "peak_kind": f"{peaks['source']} burst dense bf16 (cuBLAS)",
         "frac_of_sustained_peak": attn_tflops / peaks["bf16_tflops_sustained"],
@@ -621,6 +624,8 @@ def main():
                          "forward per rank (replicas)")
     ap.add_argument("--workload", default="768p_s0.9")
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (a head slice of it, e.g. for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-every", type=int, default=1)
     ap.add_argument("--ref-every", type=int, default=16)
@@ -637,6 +642,8 @@ def main():
     w = synth.workload(args.workload)
     if args.sparsity is not None:
         w = dataclasses.replace(w, sparsity=args.sparsity, name=f"{w.name}@s{args.sparsity}")
+    if args.heads is not None:
+        w = dataclasses.replace(w, heads=args.heads, name=f"{w.name}@h{args.heads}")
     if args.ab_seq_tiles:
         run_ab(args, w, {"tile_order": {}, "seq_tiles": {"seq_tiles": True}})
         return

@@ -9,6 +9,8 @@
 #include <cuda_fp8.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace vsa {
 
 constexpr int kTile = 64;
@@ -537,10 +539,12 @@ __device__ __forceinline__ void compress_rows(const float* __restrict__ Sb, cons
         *reinterpret_cast<float4*>(pvv + 4) = *reinterpret_cast<const float4*>(&PV_s[jj][64 + 4 * tx]);
       else if constexpr (kCols == 6)
         *reinterpret_cast<float2*>(pvv + 4) = *reinterpret_cast<const float2*>(&PV_s[jj][64 + 2 * tx]);
+      // two columns per instruction (each lane rounded as fmaf): the same sums, half the instructions
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) acc[a][c] = fmaf(wv[a], pvv[c], acc[a][c]);
+        for (int c = 0; c < kCols; c += 2)
+          fma2(acc[a][c], acc[a][c + 1], wv[a], wv[a], pvv[c], pvv[c + 1], acc[a][c], acc[a][c + 1]);
     }
     __syncthreads();
   }

@@ -13,9 +13,14 @@
 #include <type_traits>
 #include <vector>
 
+#include "attn_pair_sm100.cuh"
 #include "attn_sm100.cuh"
 #include "prep_kernels.cuh"
 #include "vsa.h"
+
+#ifndef VSA_PAIR_PREFIX
+#define VSA_PAIR_PREFIX 1
+#endif
 
 namespace {
 
@@ -446,6 +451,9 @@ struct vsa_plan_s {
   bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
   bool qk_fp8 = false;     // 8-bit Q/K (E4M3 codes, one scale per token and head) for the fine logits
   bool qk_split = false;   // the same for the dense prefix query tiles only; video query tiles keep bf16
+  // bf16 attention: the dense prefix query row blocks run two at a time on vsa_attn_pair_kernel (built
+  // with VSA_PAIR_PREFIX=0 they stay on vsa_attn_kernel, one at a time)
+  bool pair_prefix = VSA_PAIR_PREFIX != 0;
   Resolved r;
   int32_t n_t = 0, P = 0, V = 0, topk = 0;
   // reference keep: kr of the n_ref reference tiles kept per video query tile (idx rows hold kr + topk);
@@ -742,6 +750,29 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   if (n_s < 0) n_s = static_cast<int>(n_rb) - s_lo;
   if (s_lo < 0 || n_s < 0 || s_lo + n_s > n_rb) return fail(VSA_ERR_INVALID_ARG, "attention row-block range");
   if (n_s == 0) return VSA_OK;
+  // bf16 tile-order attention over every row block: the prefix query row blocks go two at a time (128
+  // queries sharing every key block) to the dense pair kernel, the video ones to vsa_attn_kernel
+  const int pre_rb = p->P << p->r.sh;
+  if (!seq && !codes && p->pair_prefix && s_lo == 0 && n_s == n_rb && pre_rb > 0) {
+    vsa::AttnArgs ap = a;
+    ap.s_lo = pre_rb;
+    ap.n_s = (pre_rb + 1) / 2;
+    ap.n_items = static_cast<int64_t>(p->B) * p->H * ap.n_s;
+    VSA_CUDA_TRY(cudaMemsetAsync(ap.sched, 0, sizeof(int), s));
+    VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+      constexpr int D = decltype(dc)::value;
+      const size_t smem = vsa::PairLayout<D>::bytes();
+      if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
+      VSA_TRY(allow_smem(vsa::vsa_attn_pair_kernel<D>, smem));
+      const int64_t gp = std::min<int64_t>(ap.n_items, p->num_sms);
+      vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, s>>>(mq, mk, mv, ap);
+      return VSA_OK;
+    }));
+    VSA_TRY(launch_check("prefix attention"));
+    s_lo = pre_rb;
+    n_s = static_cast<int>(n_rb) - pre_rb;
+    if (n_s == 0) return VSA_OK;
+  }
   a.s_lo = s_lo;
   a.n_s = n_s;
   a.n_items = static_cast<int64_t>(p->B) * p->H * n_s;
@@ -805,6 +836,7 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->seq_tiles = p->seq_tiles;
   q->qk_fp8 = p->qk_fp8;
   q->qk_split = p->qk_split;
+  q->pair_prefix = p->pair_prefix;
   q->kr = p->kr;
   q->n_ref = p->n_ref;
   q->exempt_tiles = p->exempt_tiles;
