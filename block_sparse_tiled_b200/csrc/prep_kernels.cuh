@@ -562,6 +562,129 @@ __device__ __forceinline__ void compress_rows(const float* __restrict__ Sb, cons
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// The compression GEMM of one CTA's 128 rows on the tensor cores.  Per 64-column chunk the threads stage
+// W = exp(S - max) (its binary32 row sums alongside, as compress_rows takes them) and the chunk's pooled
+// V rows, each value x as two bf16 parts, hi = bf16(x) and lo = bf16(x - hi) (x to 16 mantissa bits);
+// one thread then issues W_hi pv_hi + W_hi pv_lo + W_lo pv_hi (tcgen05.mma kind::f16, M = 128 rows,
+// N = D, K = 16, binary32 accumulation in 128 TMEM columns) -- only the lo * lo term (2^-18 of a
+// product) is left out.  o_c = the accumulator row / its row sum.  Shared memory (64 KB): W_hi, W_lo
+// as [128 rows][64] bf16, K-major with the 128-byte swizzle; pv_hi, pv_lo as [D / 64 halves][64 rows]
+// [64] bf16, d contiguous (MN-major).  The MMAs of a chunk are waited for (bounded) before the next
+// chunk overwrites the staging buffers.
+// ---------------------------------------------------------------------------
+constexpr int kTcJ = 64;
+constexpr int kTcStage = 16384;  // one staging buffer
+constexpr int kTcSmem = 4 * kTcStage + 1024 /*alignment*/ + 64;
+
+__device__ __forceinline__ uint32_t bf16_hi_lo(float x, uint16_t* lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  *lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+  return __bfloat16_as_ushort(h);
+}
+
+template <int D>
+__device__ __forceinline__ void compress_rows_tc(const float* __restrict__ Sb, const float* __restrict__ PVb,
+                                                 float* __restrict__ o_c, int bh, int n_t, int i0,
+                                                 const float* m_s, float* l_s, uint8_t* stage, uint64_t* mbar,
+                                                 uint32_t tmem, const WaitCtl& ctl) {
+  constexpr int kHalves = (D + 63) / 64;
+  constexpr uint32_t kIdesc = umma_idesc_bf16(128, D, 0, 1);
+  uint8_t* a_hi = stage;
+  uint8_t* a_lo = stage + kTcStage;
+  uint8_t* b_hi = stage + 2 * kTcStage;
+  uint8_t* b_lo = stage + 3 * kTcStage;
+  // W staging: thread -> (row wr = t >> 1, 32 consecutive columns of the chunk)
+  const int wr = threadIdx.x >> 1, wh = threadIdx.x & 1;
+  const int wi = i0 + wr;
+  const float wm = m_s[wr];
+  float lsum = 0.0f;
+  int nchunk = 0;
+  for (int j0 = 0; j0 < n_t; j0 += kTcJ, ++nchunk) {
+    if (nchunk > 0) mbar_wait(mbar, (nchunk - 1) & 1, ctl, 60);  // the previous chunk's MMAs are done
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // four 16-byte chunks of 8 columns
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const int j = j0 + 32 * wh + 8 * q + e;
+        float w0 = 0.0f, w1 = 0.0f;
+        if (wi < n_t && j < n_t) w0 = expf(__ldg(Sb + static_cast<int64_t>(wi) * n_t + j) - wm);
+        if (wi < n_t && j + 1 < n_t) w1 = expf(__ldg(Sb + static_cast<int64_t>(wi) * n_t + j + 1) - wm);
+        lsum += w0;
+        lsum += w1;
+        uint16_t l0, l1;
+        const uint32_t h0 = bf16_hi_lo(w0, &l0), h1 = bf16_hi_lo(w1, &l1);
+        hw[e >> 1] = h0 | (h1 << 16);
+        lw[e >> 1] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+      }
+      const int c16 = 4 * wh + q;
+      const int off = wr * 128 + ((c16 ^ (wr & 7)) << 4);
+      *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    // pv staging: 64 rows x D floats as float4 pieces (4 d each), each becoming 8 bytes of hi and of lo
+    for (int e = threadIdx.x; e < kTcJ * (kHalves * 16); e += 256) {
+      const int jr = e / (kHalves * 16), p4 = e - jr * (kHalves * 16);  // row, float4 index (64 d per half)
+      const int d = 4 * p4;
+      const int j = j0 + jr;
+      float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (j < n_t && d < D) v = __ldg(reinterpret_cast<const float4*>(PVb + static_cast<int64_t>(j) * D + d));
+      uint16_t l[4];
+      const uint32_t h0 = bf16_hi_lo(v.x, &l[0]), h1 = bf16_hi_lo(v.y, &l[1]);
+      const uint32_t h2 = bf16_hi_lo(v.z, &l[2]), h3 = bf16_hi_lo(v.w, &l[3]);
+      const int half = d >> 6, c16 = (d & 63) >> 3;
+      const int off = half * (kTcJ * 128) + jr * 128 + ((c16 ^ (jr & 7)) << 4) + (d & 4) * 2;
+      *reinterpret_cast<uint2*>(b_hi + off) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+      *reinterpret_cast<uint2*>(b_lo + off) = make_uint2(static_cast<uint32_t>(l[0]) | (static_cast<uint32_t>(l[1]) << 16),
+                                                         static_cast<uint32_t>(l[2]) | (static_cast<uint32_t>(l[3]) << 16));
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint64_t ah = umma_desc_sw128(smem_u32(a_hi), 16, 1024), al = umma_desc_sw128(smem_u32(a_lo), 16, 1024);
+      const uint64_t bh0 = umma_desc_sw128(smem_u32(b_hi), kTcJ * 128, 1024);
+      const uint64_t bl0 = umma_desc_sw128(smem_u32(b_lo), kTcJ * 128, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kTcJ / 16; ++kk) {
+        const uint64_t ka = static_cast<uint64_t>(kk * 2), kb = static_cast<uint64_t>(kk * 128);  // 32 B, 2 KB
+        umma_ss(tmem, ah + ka, bh0 + kb, kIdesc, (j0 > 0 || kk > 0) ? 1u : 0u);
+        umma_ss(tmem, ah + ka, bl0 + kb, kIdesc, 1u);
+        umma_ss(tmem, al + ka, bh0 + kb, kIdesc, 1u);
+      }
+      umma_commit(mbar);
+    }
+    __syncwarp();
+  }
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  if (wh == 0) l_s[wr] = lsum;
+  // the last chunk's MMAs complete on their own: wait for them (bounded, whatever the abort flag says)
+  // before TMEM is read and freed
+  if (nchunk > 0) mbar_wait_drain(mbar, (nchunk - 1) & 1, ctl, 61);
+  tc_fence_after();
+  __syncthreads();
+  // epilogue: warp w reads TMEM lane quadrant w % 4 (rows 32 (w % 4) ..) and column half w / 4
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = 32 * (warp & 3) + lane, i = i0 + r;
+  constexpr int kHalfD = D / 2;  // 32, 48 or 64 columns
+  const float inv = (i < n_t) ? 1.0f / l_s[r] : 0.0f;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + (warp >> 2) * kHalfD;
+#pragma unroll
+  for (int c0 = 0; c0 < kHalfD; c0 += 16) {
+    float o[16];
+    tmem_ld16(t_lane + c0, o);
+    tmem_wait_ld();
+    if (i < n_t) {
+      float* dst = o_c + (static_cast<int64_t>(bh) * n_t + i) * D + (warp >> 2) * kHalfD + c0;
+#pragma unroll
+      for (int e = 0; e < 16; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restrict__ S, const float* __restrict__ pv,
                                                         float* __restrict__ o_c, int n_t,
@@ -607,13 +730,26 @@ __global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __
                                                                const float* __restrict__ pv, float* __restrict__ o_c,
                                                                int32_t* __restrict__ idx, int n_t, int P, int k,
                                                                int out_stride, int out_off,
-                                                               const int* __restrict__ gate_nonzero) {
+                                                               const int* __restrict__ gate_nonzero,
+                                                               int* __restrict__ status) {
   __shared__ float m_s[kCompRows], l_s[kCompRows];
-  __shared__ __align__(16) float W_s[kCompJ][kCompRows + 4];
-  __shared__ __align__(16) float PV_s[kCompJ][D];
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  extern __shared__ uint8_t dyn_raw[];
+  uint8_t* stage = dyn_raw + ((1024u - (smem_u32(dyn_raw) & 1023u)) & 1023u);  // swizzle atoms: 1 KB aligned
   const int bh = blockIdx.y, i0 = blockIdx.x * kCompRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int V = n_t - P;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_s, 128);
+    tmem_relinquish();
+  }
   const float* Sb = S + static_cast<int64_t>(bh) * n_t * n_t;
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int r = warp; r < kCompRows; r += 8) {
@@ -662,9 +798,22 @@ __global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __
       eq_seen += __popc(eq_ballot);
     }
   }
+  tc_fence_before();
   __syncthreads();
-  if (gate_nonzero != nullptr && *gate_nonzero == 0) return;  // every gate is zero: o_c is never read
-  compress_rows<D>(Sb, pv + static_cast<int64_t>(bh) * n_t * D, o_c, bh, n_t, i0, m_s, l_s, W_s, PV_s);
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  // every gate zero: o_c is never read
+  if (gate_nonzero == nullptr || *gate_nonzero != 0) {
+    const WaitCtl ctl{&abort_s, status, kWaitTimeoutNs};
+    compress_rows_tc<D>(Sb, pv + static_cast<int64_t>(bh) * n_t * D, o_c, bh, n_t, i0, m_s, l_s, stage, &mbar, tmem,
+                        ctl);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
 }
 
 }  // namespace vsa

@@ -489,6 +489,10 @@ struct vsa_plan_s {
     cudaStream_t h2d = nullptr, d2h = nullptr;
     cudaEvent_t ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {}, ev_gate = nullptr, ev_start = nullptr;
   } pipe;
+  // the prefix pair kernel runs on `side`, forked from and joined back to the caller's stream, so that
+  // vsa_attn_kernel starts on the SMs its last items leave idle (created on first use)
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 namespace {
@@ -656,17 +660,15 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
     VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
       constexpr int D = decltype(dc)::value;
       auto launch = [&](auto kernel) {
-        kernel<<<grid, 256, 0, s>>>(S, pv, o_c, idx, p->n_t, p->P, k, p->kr + p->topk, p->kr, gate_nonzero);
+        VSA_TRY(allow_smem(kernel, vsa::kTcSmem));
+        kernel<<<grid, 256, vsa::kTcSmem, s>>>(S, pv, o_c, idx, p->n_t, p->P, k, p->kr + p->topk, p->kr, gate_nonzero,
+                                               p->d_status);
+        return VSA_OK;
       };
-      if (J <= 8)
-        launch(vsa::select_compress_kernel<D, 8>);
-      else if (J <= 16)
-        launch(vsa::select_compress_kernel<D, 16>);
-      else if (J <= 24)
-        launch(vsa::select_compress_kernel<D, 24>);
-      else
-        launch(vsa::select_compress_kernel<D, 40>);
-      return VSA_OK;
+      if (J <= 8) return launch(vsa::select_compress_kernel<D, 8>);
+      if (J <= 16) return launch(vsa::select_compress_kernel<D, 16>);
+      if (J <= 24) return launch(vsa::select_compress_kernel<D, 24>);
+      return launch(vsa::select_compress_kernel<D, 40>);
     }));
     return launch_check("select_compress");
   }
@@ -753,24 +755,40 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   // bf16 tile-order attention over every row block: the prefix query row blocks go two at a time (128
   // queries sharing every key block) to the dense pair kernel, the video ones to vsa_attn_kernel
   const int pre_rb = p->P << p->r.sh;
+  bool joined = true;  // no side-stream work to join back
   if (!seq && !codes && p->pair_prefix && s_lo == 0 && n_s == n_rb && pre_rb > 0) {
     vsa::AttnArgs ap = a;
     ap.s_lo = pre_rb;
     ap.n_s = (pre_rb + 1) / 2;
     ap.n_items = static_cast<int64_t>(p->B) * p->H * ap.n_s;
-    VSA_CUDA_TRY(cudaMemsetAsync(ap.sched, 0, sizeof(int), s));
+    ap.sched = p->d_status + 4;  // its own item counter
+    s_lo = pre_rb;
+    n_s = static_cast<int>(n_rb) - pre_rb;
+    // with video row blocks to run too, the pair kernel goes on the side stream (forked from s)
+    cudaStream_t ps = s;
+    if (n_s > 0) {
+      if (p->side == nullptr) {
+        VSA_CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
+        VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
+        VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
+      }
+      VSA_CUDA_TRY(cudaEventRecord(p->ev_fork, s));
+      VSA_CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
+      ps = p->side;
+      joined = false;
+    }
+    VSA_CUDA_TRY(cudaMemsetAsync(ap.sched, 0, sizeof(int), ps));
     VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
       constexpr int D = decltype(dc)::value;
       const size_t smem = vsa::PairLayout<D>::bytes();
       if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
       VSA_TRY(allow_smem(vsa::vsa_attn_pair_kernel<D>, smem));
       const int64_t gp = std::min<int64_t>(ap.n_items, p->num_sms);
-      vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, s>>>(mq, mk, mv, ap);
+      vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, ps>>>(mq, mk, mv, ap);
       return VSA_OK;
     }));
     VSA_TRY(launch_check("prefix attention"));
-    s_lo = pre_rb;
-    n_s = static_cast<int>(n_rb) - pre_rb;
+    if (!joined) VSA_CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
     if (n_s == 0) return VSA_OK;
   }
   a.s_lo = s_lo;
@@ -791,12 +809,24 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     if (codes) return launch(vsa::vsa_attn_kernel<D, false, true>, vsa::AttnLayout<D, true>::bytes(p->n_t));
     return launch(vsa::vsa_attn_kernel<D, false, false>, vsa::AttnLayout<D>::bytes(p->n_t));
   }));
-  return launch_check("attention");
+  VSA_TRY(launch_check("attention"));
+  if (!joined) VSA_CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));  // the caller's stream sees both kernels
+  return VSA_OK;
 }
 
 // ---------------------------------------------------------------- host pipeline helpers
+void release_side(vsa_plan_s* p) {
+  if (p->side) cudaStreamDestroy(p->side);
+  if (p->ev_fork) cudaEventDestroy(p->ev_fork);
+  if (p->ev_join) cudaEventDestroy(p->ev_join);
+  p->side = nullptr;
+  p->ev_fork = p->ev_join = nullptr;
+}
+
 void release_host_pipe(vsa_plan_s* p) {
   auto& h = p->pipe;
+  for (vsa_plan_s* sub : {h.sub, h.sub_last})
+    if (sub) release_side(sub);
   delete h.sub;
   delete h.sub_last;
   h.sub = h.sub_last = nullptr;
@@ -1059,7 +1089,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
       cudaMalloc(&p->d_row_token, tok_bytes) != cudaSuccess || cudaMalloc(&p->d_coord, coord_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_mask_seq, mask_bytes) != cudaSuccess ||
       cudaMalloc(&p->d_mask_tiled, block_mask_bytes) != cudaSuccess ||
-      cudaMalloc(&p->d_status, 4 * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&p->d_status, 8 * sizeof(int)) != cudaSuccess ||
       (p->n_ref > 0 && (cudaMalloc(&p->d_exempt, std::max<size_t>(4, p->exempt_tiles.size() * 4)) != cudaSuccess ||
                         cudaMalloc(&p->d_refs, p->ref_tiles.size() * 4) != cudaSuccess)) ||
       (!p->qk_fp8 && !p->qk_split && cudaMalloc(&p->d_stats, stats_bytes(p)) != cudaSuccess)) {
@@ -1083,7 +1113,7 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
     e = cudaMemcpyAsync(p->d_exempt, p->exempt_tiles.data(), p->exempt_tiles.size() * 4, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !p->ref_tiles.empty())
     e = cudaMemcpyAsync(p->d_refs, p->ref_tiles.data(), p->ref_tiles.size() * 4, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 4 * sizeof(int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, 8 * sizeof(int), s);
   if (e != cudaSuccess) {
     cleanup();
     return fail(VSA_ERR_CUDA, std::string("plan upload: ") + cudaGetErrorString(e));
@@ -1129,6 +1159,7 @@ vsa_status vsa_plan_destroy(vsa_plan p) {
   cudaSetDevice(p->device);
   cudaDeviceSynchronize();
   release_host_pipe(p);
+  release_side(p);
   cudaFree(p->d_part_table);
   if (p->owns_device) {
     cudaFree(p->d_tile_token);
