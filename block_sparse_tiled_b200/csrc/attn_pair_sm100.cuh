@@ -1,15 +1,20 @@
-// Dense attention of the prefix query tiles, two 64-row blocks (128 queries) per work item, on sm_100a.
+// Attention of query row blocks that share their key list, two 64-row blocks (128 queries) per work
+// item, on sm_100a.
 //
 // A prefix query tile attends to every key tile ("Mike0021/FastH3-4step-Preview-VSA", section "Video
 // Sparse Attention is not optional here": prefix queries attend densely), so any two prefix query row
-// blocks of one head share every key block.  This kernel runs them together in the standard orientation
+// blocks of one head share every key block; and with 128-token tiles ("FastH3 OmniRef inference",
+// section "Device profiles") the two 64-row halves of a video query tile share that tile's key list.
+// This kernel runs such pairs together in the standard orientation
 //     S [128 queries x 128 keys] = Q_pair (M = 128, K-major) * K_blk^T (N = 128, K-major)
 //     O [128 queries x D]       += P (M = 128, read from TMEM) * V_blk (N = D, MN-major)
-// so one tcgen05.mma covers twice the work of the transposed N = 64 form that the video query tiles use
-// (vsa_attn_kernel), and P reaches the tensor core through TMEM: no shared-memory P, no proxy fence.
-// Work item = (b, h, pair j): query row blocks 2j and 2j + 1 of the prefix (the second one absent when
-// the prefix has an odd number of row blocks: its rows are computed from zero-filled or neighbouring
-// rows and never stored).  Key blocks are row blocks (2n, 2n + 1) of the whole sequence, all of them.
+// so one tcgen05.mma covers twice the work of the transposed N = 64 form that the other video query
+// tiles use (vsa_attn_kernel), and P reaches the tensor core through TMEM: no shared-memory P, no proxy
+// fence.  Work item = (b, h, pair j): query row blocks 2j and 2j + 1 of the launch's range [0, r_end)
+// (the second one absent when r_end is odd: its rows are computed from zero-filled or neighbouring rows
+// and never stored).  Key blocks: for a prefix query tile, row blocks (2n, 2n + 1) of the whole
+// sequence, all of them; for a 128-token video query tile, the tiles of its key list (the always-kept
+// prefix tiles, then the kept reference and selected video tiles), one tile per block.
 //
 // The softmax is row-wise: two threads per query row, one per 64-key half of every block, each keeping
 // its half-row's sum in registers.  The running maximum follows the lazy rule of vsa_attn_kernel: a
@@ -70,8 +75,9 @@ struct PairLayout {
   static size_t bytes() { return 1024 /*alignment slack*/ + oEnd; }
 };
 
-// a.n_s: pairs per (b, h); a.s_lo: the number of prefix row blocks (a pair's second block exists when it
-// is below this); the other fields as for vsa_attn_kernel (tile-order inputs, bf16).
+// a.s_lo, a.r_end: the launch's query row blocks [r_lo, r_end) (the prefix row blocks; with 128-token
+// tiles any tile-aligned range); a.n_s: pairs per (b, h); the other fields as for vsa_attn_kernel
+// (tile-order inputs, bf16).
 template <int D>
 __global__ void __launch_bounds__(kPairThreads, 1)
     vsa_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -94,9 +100,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = a.n_t, sh = a.sub_shift, n_sel = n_t >> sh;
-  const int pre_rb = a.s_lo;            // prefix row blocks
-  const int npairs = a.n_s;             // items per (b, h)
-  const int nb = (n_t + 1) / 2;         // key blocks: every row block, two at a time
+  const int r_lo = a.s_lo, r_end = a.r_end;  // query row blocks of the launch: [r_lo, r_end), in pairs
+  const int npairs = a.n_s;                  // items per (b, h)
+  const int P = a.P, V = n_sel - P, E = a.n_exempt, W = a.kr + a.topk;
+  // Key blocks of the item whose first query row block is s0: for a prefix query tile every row block,
+  // two at a time; for a video query tile of 128 tokens (sh = 1; both row blocks are that tile) the E
+  // always-kept and the kr + topk listed tiles, one 128-key block each.
+  auto item_blocks = [&](int s0) -> int { return ((s0 >> sh) < P) ? (n_t + 1) / 2 : E + W; };
+  // first key row block of block n; the block's second half is the next row block (or, past the last
+  // row block, a masked repeat)
+  auto block_row = [&](int64_t bh, int s0, int n) -> int {
+    const int i = s0 >> sh;
+    if (i < P) return 2 * n;
+    const int sel = (n < E) ? (a.exempt ? __ldg(a.exempt + n) : n) : __ldg(a.idx + (bh * V + (i - P)) * W + (n - E));
+    return sel << 1;
+  };
   const WaitCtl ctl{abort_flag, a.status, kWaitTimeoutNs};
 
   // ---------------------------------------------------------------- setup
@@ -195,7 +213,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       w = __shfl_sync(0xffffffffu, w, 0);
       if (w < 0 || !ok) break;
       const int64_t bh = w / npairs;
-      const int s0 = 2 * static_cast<int>(w - bh * npairs);
+      const int s0 = r_lo + 2 * static_cast<int>(w - bh * npairs);
       if (is_k) {
         // the item's 128 query rows: row blocks s0 and s0 + 1 (rows past the tensor read as zeros)
         if (lane == 0) {
@@ -210,9 +228,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         __syncwarp();
       }
+      const int nb = item_blocks(s0);
+      int rows = 0;  // lane j: the first key row block of block 32 * (n / 32) + j
       for (int n = 0; n < nb && ok; ++n, ++g) {
-        const int ka = 2 * n;
-        const int kb = (2 * n + 1 < n_t) ? 2 * n + 1 : ka;  // an odd count repeats its last block, masked
+        if ((n & 31) == 0) rows = (n + lane < nb) ? block_row(bh, s0, n + lane) : 0;
+        const int ka = __shfl_sync(0xffffffffu, rows, n & 31);
+        const int kb = (ka + 1 < n_t) ? ka + 1 : ka;  // past the last row block: a masked repeat
         const int st = g % nstages;
         const uint32_t u = g / nstages;
         if (lane == 0) {
@@ -248,6 +269,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int it = 0;; ++it) {
         const int w = ring_take(it, 46);
         if (w < 0 || !ok) break;
+        const int64_t bh = w / npairs;
+        const int nb = item_blocks(r_lo + 2 * static_cast<int>(w - bh * npairs));
         ok = mbar_wait(&bars[Ly::bQFull], it & 1, ctl, 34);
         const uint64_t qd0 = umma_desc_sw128(smem_u32(sm + Ly::oQ), 16, 1024);
         for (int n = 0; n < nb && ok; ++n, ++g) {
@@ -281,6 +304,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int it = 0;; ++it) {
         const int w = ring_take(it, 47);
         if (w < 0 || !ok) break;
+        const int64_t bh = w / npairs;
+        const int nb = item_blocks(r_lo + 2 * static_cast<int>(w - bh * npairs));
         for (int n = 0; n < nb && ok; ++n, ++g) {
           const int vst = g % Ly::kVStages;
           const int pb = g & 1;
@@ -319,9 +344,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       w = __shfl_sync(0xffffffffu, w, 0);
       if (named_bar_or(1, 256, w < 0)) break;  // the softmax warps stop together
       const int64_t bh = w / npairs;
-      const int s0 = 2 * static_cast<int>(w - bh * npairs);
+      const int s0 = r_lo + 2 * static_cast<int>(w - bh * npairs);
       const int s = s0 + (r >> 6);             // this row's query row block
-      const bool row_ok = s < pre_rb;
+      const bool row_ok = s < r_end;
+      const int nb = item_blocks(s0);
       // overflow bound of this row: cl |q| max|k| + ceil(log2 max|v|)+ - skip_cap (rows not stored: none)
       float lim = -INFINITY;
       if (a.q_norm != nullptr && row_ok) {
@@ -335,10 +361,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
       for (int j = 0; j < 8; ++j) lacc[j] = 0.0f;
       bool skip = false;
+      uint32_t mlo = 0, mhi = 0;  // lane j: the key-mask word of this half of block 32 * (n / 32) + j
       for (int n = 0; n < nb; ++n, ++g) {
         const int sb = g & 1;
-        const int kt = 2 * n + hf;  // key row block of this half
-        const uint64_t kmask = (kt < n_t) ? __ldg(a.key_mask + kt) : 0ull;
+        if ((n & 31) == 0) {
+          uint64_t m = 0ull;
+          if (n + lane < nb) {
+            const int kt = block_row(bh, s0, n + lane) + hf;  // key row block of this half
+            m = (kt < n_t) ? __ldg(a.key_mask + kt) : 0ull;
+          }
+          mlo = static_cast<uint32_t>(m);
+          mhi = static_cast<uint32_t>(m >> 32);
+        }
+        const uint64_t kmask = static_cast<uint64_t>(__shfl_sync(0xffffffffu, mlo, n & 31)) |
+                               (static_cast<uint64_t>(__shfl_sync(0xffffffffu, mhi, n & 31)) << 32);
         const uint32_t s_col = t_lane + kPairS0 + sb * 128 + 64 * hf;
         mbar_wait(&bars[Ly::bSFull + sb], (g >> 1) & 1, ctl, 50);
         tc_fence_after();
@@ -458,11 +494,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       w = __shfl_sync(0xffffffffu, w, 0);
       if (w < 0) break;  // every epilogue warp reads the same ring, so all stop at the same item
       const int64_t bh = w / npairs;
-      const int s0 = 2 * static_cast<int>(w - bh * npairs);
+      const int s0 = r_lo + 2 * static_cast<int>(w - bh * npairs);
       const int s = s0 + (r >> 6);
       const int64_t b = bh / a.H;
       const int h = static_cast<int>(bh - b * a.H);
-      const int32_t tok = (s < pre_rb) ? __ldg(a.tile_token + static_cast<int64_t>(s) * 64 + (r & 63)) : -1;
+      const int32_t tok = (s < r_end) ? __ldg(a.tile_token + static_cast<int64_t>(s) * 64 + (r & 63)) : -1;
       uint16_t* dst = nullptr;
       const uint16_t* gsrc = nullptr;
       float gq = 0.0f;

@@ -140,6 +140,7 @@ struct AttnArgs {
   float skip_cap;
   float scale_log2;  // softmax scale * log2(e)
   int s_lo, n_s;     // the launch covers row blocks [s_lo, s_lo + n_s) of every (b, h)
+  int r_end;         // pair kernel: its pairs cover [s_lo, s_lo + 2 n_s); rows >= r_end are not queries
   int64_t n_items;   // B * H * n_s
 };
 

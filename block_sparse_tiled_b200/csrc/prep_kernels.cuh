@@ -717,9 +717,10 @@ __global__ void __launch_bounds__(256, 2) compress_kernel(const float* __restric
 // warp max of the keys; for a video query row the k-th largest video key T comes from a bitwise search
 // whose per-bit counts are one redux.sync each, and the row's picks (every key > T, then the keys == T
 // lowest index first) are written ascending to idx[row * out_stride + out_off ...].  Then the CTA runs
-// the compression GEMM of its rows (compress_rows), unless every gate is zero.  The selection is the
-// top-k kernel's (same keys, same threshold, same order) and the compression the compression kernel's
-// (same maxima and staging), so both outputs are bit-identical to the two-kernel path.
+// the compression GEMM of its rows on the tensor cores (compress_rows_tc), unless every gate is zero.
+// The selection is the top-k kernel's (same keys, same threshold, same order), so idx is bit-identical
+// to the two-kernel path; o_c takes the same maxima and row sums as the compression kernel and agrees
+// with it to about 2^-16 relative (the binary32 operands enter as bf16 high and low parts).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float order_key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);

@@ -752,18 +752,30 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   if (n_s < 0) n_s = static_cast<int>(n_rb) - s_lo;
   if (s_lo < 0 || n_s < 0 || s_lo + n_s > n_rb) return fail(VSA_ERR_INVALID_ARG, "attention row-block range");
   if (n_s == 0) return VSA_OK;
-  // bf16 tile-order attention over every row block: the prefix query row blocks go two at a time (128
-  // queries sharing every key block) to the dense pair kernel, the video ones to vsa_attn_kernel
+  // bf16 tile-order attention: query row blocks that share their key list go two at a time (128 queries
+  // per key block) to the pair kernel -- the prefix row blocks of a launch over every row block, and with
+  // 128-token tiles every tile of the range (its two row blocks) -- and the other video row blocks to
+  // vsa_attn_kernel
   const int pre_rb = p->P << p->r.sh;
+  int pair_lo = 0, pair_hi = 0;  // row blocks [pair_lo, pair_hi) go in pairs
+  if (!seq && !codes && p->pair_prefix) {
+    if (p->r.sh == 1 && s_lo % 2 == 0 && n_s % 2 == 0) {
+      pair_lo = s_lo;
+      pair_hi = s_lo + n_s;
+    } else if (s_lo == 0 && n_s == n_rb) {
+      pair_hi = pre_rb;
+    }
+  }
   bool joined = true;  // no side-stream work to join back
-  if (!seq && !codes && p->pair_prefix && s_lo == 0 && n_s == n_rb && pre_rb > 0) {
+  if (pair_hi > pair_lo) {
     vsa::AttnArgs ap = a;
-    ap.s_lo = pre_rb;
-    ap.n_s = (pre_rb + 1) / 2;
+    ap.s_lo = pair_lo;
+    ap.r_end = pair_hi;
+    ap.n_s = (pair_hi - pair_lo + 1) / 2;
     ap.n_items = static_cast<int64_t>(p->B) * p->H * ap.n_s;
     ap.sched = p->d_status + 4;  // its own item counter
-    s_lo = pre_rb;
-    n_s = static_cast<int>(n_rb) - pre_rb;
+    n_s = s_lo + n_s - pair_hi;  // what is left: [pair_hi, s_lo + n_s)
+    s_lo = pair_hi;
     // with video row blocks to run too, the pair kernel goes on the side stream (forked from s)
     cudaStream_t ps = s;
     if (n_s > 0) {
@@ -787,7 +799,7 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
       vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, ps>>>(mq, mk, mv, ap);
       return VSA_OK;
     }));
-    VSA_TRY(launch_check("prefix attention"));
+    VSA_TRY(launch_check("pair attention"));
     if (!joined) VSA_CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
     if (n_s == 0) return VSA_OK;
   }
