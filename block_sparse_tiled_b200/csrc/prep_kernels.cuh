@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(384) tile_stats_kernel(const uint16_t* __restr
 constexpr int kF8RowBytes = 128;
 
 template <int D, bool kParts, bool kF8, int kSub>
-__global__ void __launch_bounds__(384) gather_pool_kernel(
+__global__ void __launch_bounds__(384, (kSub == 2 || kF8) ? 2 : 3) gather_pool_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     void* __restrict__ q_t, void* __restrict__ k_t, uint16_t* __restrict__ v_t, float* __restrict__ q_s,
     float* __restrict__ k_s, float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
