@@ -762,7 +762,12 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     if (p->r.sh == 1 && s_lo % 2 == 0 && n_s % 2 == 0) {
       pair_lo = s_lo;
       pair_hi = s_lo + n_s;
-    } else if (s_lo == 0 && n_s == n_rb) {
+    } else if (s_lo == 0 && n_s == n_rb &&
+               static_cast<int64_t>(p->B) * p->H * ((pre_rb + 1) / 2) >= p->num_sms) {
+      // 64-token tiles: the prefix pairs go to the pair kernel only when there are enough of them to fill
+      // the GPU; with a few heads (a head chunk of the host pipeline, a sequence-parallel rank) a handful of
+      // long dense items would hold their SMs while the video launch waits, and vsa_attn_kernel's item
+      // schedule spreads the prefix row blocks among the video ones instead
       pair_hi = pre_rb;
     }
   }

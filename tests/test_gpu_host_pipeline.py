@@ -3,7 +3,11 @@ their own streams overlapping the forward of neighbouring chunks.
 
 Every head's forward is independent of the other heads (pooling, scores,
 top-k, compression and the attention items all work per (b, h)), so the
-chunked result must be bit-identical to vsa_forward on the same inputs.
+chunked result must be bit-identical to vsa_forward on the same inputs --
+except on the prefix query rows of 64-token tiles where a chunk has too few
+heads for the pair kernel and the whole forward enough: those rows run on the
+video attention kernel in the chunks and must agree within the output
+tolerance.
 The cases cover a chunk that divides the heads, one that leaves a remainder
 chunk (a second head-slice plan), one chunk holding every head, the default
 (the smallest chunk with 512-byte copy rows), pageable host memory, a second call reusing the pipeline,
@@ -14,6 +18,7 @@ import pytest
 import torch
 
 import synth
+from conftest import assert_routes_agree
 
 pytestmark = pytest.mark.gpu
 
@@ -25,8 +30,9 @@ def vsa():
     build.build()
     import block_sparse_tiled_b200 as m
 
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
+    m.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(0)
     return m
 
 
@@ -59,12 +65,14 @@ def test_host_pipeline_matches_device_forward(vsa, name, chunk):
     hx = host_copies(x)
     out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], head_chunk=chunk)
     assert not out.is_cuda
-    assert torch.equal(out, ref)
+    hc = chunk or vsa.default_head_chunk(w.heads, w.head_dim)
+    assert_routes_agree(w, out, ref, hc)
     assert vsa.device_status(plan) == (0, 0)
     # a second call reuses the plan's pipeline and staging workspace
+    first = out.clone()
     out.zero_()
     vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"], out=out, head_chunk=chunk)
-    assert torch.equal(out, ref)
+    assert torch.equal(out, first)
     plan.destroy()
 
 
@@ -77,7 +85,7 @@ def test_host_pipeline_1344x768_default_chunks(vsa):
     hx = host_copies(x)
     del x
     out = vsa.vsa_forward_host(plan, hx["q"], hx["k"], hx["v"], hx["gate"])
-    assert torch.equal(out, ref)
+    assert_routes_agree(w, out, ref, vsa.default_head_chunk(w.heads, w.head_dim))
     assert vsa.device_status(plan) == (0, 0)
     plan.destroy()
 

@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import synth
+from conftest import prefix_on_pair_kernel
 
 pytestmark = pytest.mark.gpu
 
@@ -172,6 +173,19 @@ def test_tiny_sparsity0_is_dense_attention(vsa, oracle_mod):
 def test_edge_cases(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
     w = synth.Workload("edge", B, H, D, tuple(segments), tuple(grid), sparsity)
     full_parity(vsa, oracle_mod, w, seed=3)
+
+
+@pytest.mark.parametrize("segments,grid,sparsity,B,H,D", [
+    ((128, 0, 64), (4, 8, 8), 0.5, 2, 40, 128),  # 3 prefix tiles: a full pair and a half pair; 160 pairs
+    ((100, 30), (0, 0, 0), 0.9, 1, 148, 64),     # prefix only: one pair of ragged tiles per head
+    ((70, 0, 5), (5, 6, 7), 0.6, 2, 50, 96),     # ragged prefix and video tiles, head_dim 96
+])
+def test_prefix_pairs_full_parity(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
+    """64-token tiles with enough heads that the prefix query row blocks go to the pair kernel, in full
+    against the oracle (the smaller workloads above leave them to the video kernel)."""
+    w = synth.Workload("pairs", B, H, D, tuple(segments), tuple(grid), sparsity)
+    assert prefix_on_pair_kernel(w)
+    full_parity(vsa, oracle_mod, w, seed=9)
 
 
 def sampled_parity(vsa, oracle_mod, w, heads, video_every, batches=(0,), seq_tiles=False):

@@ -8,7 +8,10 @@ waits on another), each for its head group over all parts.  The assembled
 output is checked against the CPU oracle (selection of each rank's heads bit
 for bit, the output within max-abs 2e-2 and mean-abs 2e-3), and must also
 equal vsa_forward on the whole tensors bit for bit (every head's computation
-is the same; only where its rows are read from and written to differs)."""
+is the same; only where its rows are read from and written to differs) --
+except on the prefix query rows of 64-token tiles when a rank has too few
+heads for the pair kernel and the whole forward enough, where the two agree
+within the output tolerance."""
 import dataclasses
 
 import numpy as np
@@ -16,6 +19,7 @@ import pytest
 import torch
 
 import synth
+from conftest import assert_routes_agree
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +108,7 @@ def test_parts_match_oracle_and_whole_forward(vsa, oracle_mod, name, world, over
     err = np.abs(g - ref)
     assert np.isfinite(g).all()
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
-    assert torch.equal(got, reference(vsa, w, x))
+    assert_routes_agree(w, got, reference(vsa, w, x), w.heads // world)
 
 
 def test_parts_argument_errors(vsa):
