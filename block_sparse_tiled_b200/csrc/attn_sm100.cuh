@@ -30,6 +30,12 @@
 //     every column, P, l and O^T stay finite without further rescaling and the
 //     group skips the votes for the rest of the item;
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
+// Blocks go two at a time through one handshake (a super-block of 256 keys): the
+// S^T issuer fills both 64-column halves of one S^T buffer and signals once, the
+// softmax exponentiates both halves against one m (a super-block that needs the
+// exact maximum takes it over both halves in a first pass over S^T), writes both
+// 128-key halves of one P^T buffer and releases S^T and P^T with one arrival
+// each, and the P.V issuer runs both halves' MMAs on one P^T-full wait.
 // O^T is double-buffered in TMEM, so one item's epilogue (in its own warps)
 // overlaps the next item's blocks.
 // D = 64 uses the same M = 128 PV product with a zero upper half of V^T, and
@@ -105,9 +111,9 @@ constexpr int kAttnThreads = 32 * (kEpiWarp0 + 4);
 // at most 2^23 keys per row, row sums stay below 2^47 and P.V partial sums far
 // below the binary32 range.
 constexpr float kRescaleLog2 = 24.0f;
-constexpr int kSBufs = 2;            // S^T buffers in TMEM (64 columns each)
-constexpr int kOCol0 = 64 * kSBufs;  // O^T double buffer follows (2 x 64 columns)
-constexpr uint32_t kTmemCols = (kOCol0 + 128 <= 256) ? 256 : 512;
+constexpr int kSBufs = 2;             // S^T buffers in TMEM, one per super-block (two 64-column halves)
+constexpr int kOCol0 = 128 * kSBufs;  // O^T double buffer follows (2 x 64 columns)
+constexpr uint32_t kTmemCols = 512;
 
 struct AttnArgs {
   const int32_t* idx;         // [B, H, V, kr + topk]: kept reference tiles, then video tiles (each ascending)
@@ -163,10 +169,11 @@ struct AttnLayout {
   static constexpr int kKVBytes = 128 * 64 * kHalves * 2;                  // 128 keys of V (bf16)
   static constexpr int kKBytes = kF8 ? 128 * 128 : kKVBytes;               // 128 keys of K
   static constexpr int kHalfBytes = 128 * 128;  // one 64-column half of a 128-row block
-  static constexpr int kPBytes = 128 * 64 * 2;  // P^T of one block
+  static constexpr int kPHalfBytes = 128 * 64 * 2;  // P^T of one 128-key block
+  static constexpr int kPBytes = 2 * kPHalfBytes;    // P^T of one super-block (256 keys)
   static constexpr int kQBufs = 1;
   static constexpr int kKStages = kF8 ? 4 : 2;
-  static constexpr int kVStages = 3;
+  static constexpr int kVStages = 2;
   static constexpr int kPBufs = 2;  // P^T buffers in shared memory
   static constexpr int kRing = 8;  // claimed items in flight
   static constexpr int kZeroBytes = (D == 64) ? 16384 : 0;
@@ -500,8 +507,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ============================================================ S^T issuer
+    // Super-block j of an item = its 128-key blocks 2j and 2j + 1 (the second absent at an odd end): both
+    // go into S^T buffer sb (two 64-column halves), which the softmax releases with one arrival.
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0, G = 0;  // 128-key blocks (K stages) and super-blocks (S^T buffers) so far
       int it = 0;
       bool ok = true;
       ROLE_TIMER_START();
@@ -510,38 +519,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
-        const int nb = (list_len(i) + 1) / 2;
+        const int nb = (list_len(i) + 1) / 2, nsb = (nb + 1) / 2;
         const int qb = it % Ly::kQBufs;
         ROLE_MARK(3);
         ok = mbar_wait(&bars[Ly::bQFull + qb], (it / Ly::kQBufs) & 1, ctl, 5);
         ROLE_MARK(0);
         const uint64_t qd0 = umma_desc_sw128(smem_u32(sm + Ly::oQ + qb * Ly::kQBytes), 16, 1024);
-        for (int n = 0; n < nb && ok; ++n, ++g) {
-          const int kst = g % Ly::kKStages;
-          const int sb = g % kSBufs;
+        for (int j = 0; j < nsb && ok; ++j, ++G) {
+          const int sb = G % kSBufs;
           ROLE_MARK(3);
-          ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6);
-          ROLE_MARK(1);
-          ok = ok && mbar_wait(&bars[Ly::bSEmpty + sb], ((g / kSBufs) & 1) ^ 1, ctl, 7);
+          ok = mbar_wait(&bars[Ly::bSEmpty + sb], ((G / kSBufs) & 1) ^ 1, ctl, 7);
           ROLE_MARK(2);
-          if (!ok) break;
-          tc_fence_after();
-          // descriptors of the block's first K-step; a step moves the start address (bits 0..13, 16-byte
-          // units, no carry: shared memory addresses stay below 256 KB) by a compile-time offset
-          const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oK + kst * Ly::kKBytes), 16, 1024);
+          const int nh = min(2, nb - 2 * j);
+          for (int h = 0; h < nh && ok; ++h, ++g) {
+            const int kst = g % Ly::kKStages;
+            ROLE_MARK(3);
+            ok = mbar_wait(&bars[Ly::bKFull + kst], (g / Ly::kKStages) & 1, ctl, 6);
+            ROLE_MARK(1);
+            if (!ok) break;
+            tc_fence_after();
+            // descriptors of the block's first K-step; a step moves the start address (bits 0..13, 16-byte
+            // units, no carry: shared memory addresses stay below 256 KB) by a compile-time offset
+            const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oK + kst * Ly::kKBytes), 16, 1024);
+            const uint32_t dcol = tmem + sb * 128 + h * 64;
 #pragma unroll
-          for (int kk = 0; kk < kQKSteps; ++kk) {
-            // 32 bytes of every row per step: 16 bf16 or 32 8-bit elements
-            const uint64_t ad = ad0 + static_cast<uint64_t>(((kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32) >> 4);
-            const uint64_t bd = qd0 + static_cast<uint64_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
-            if constexpr (kF8)
-              umma_ss_f8(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
-            else
-              umma_ss(tmem + sb * 64, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kQKSteps; ++kk) {
+              // 32 bytes of every row per step: 16 bf16 or 32 8-bit elements
+              const uint64_t ad = ad0 + static_cast<uint64_t>(((kk >> 2) * Ly::kHalfBytes + (kk & 3) * 32) >> 4);
+              const uint64_t bd = qd0 + static_cast<uint64_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
+              if constexpr (kF8)
+                umma_ss_f8(dcol, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+              else
+                umma_ss(dcol, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars[Ly::bKEmpty + kst]);
           }
-          umma_commit(&bars[Ly::bKEmpty + kst]);
+          if (!ok) break;
           umma_commit(&bars[Ly::bSFull + sb]);
-          if (n == nb - 1) umma_commit(&bars[Ly::bQEmpty + qb]);
+          if (j == nsb - 1) umma_commit(&bars[Ly::bQEmpty + qb]);
         }
       }
       ROLE_MARK(3);
@@ -553,7 +568,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == 3) {
     // ============================================================ P.V issuer
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0, G = 0;  // 128-key blocks (V stages) and super-blocks (P^T buffers) so far
       int it = 0;
       bool ok = true;
       ROLE_TIMER_START();
@@ -562,34 +577,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (w < 0 || !ok) break;
         const int64_t bh = w / n_t;
         const int i = static_cast<int>(w - bh * n_t) >> sh;  // the item's tile
-        const int nb = (list_len(i) + 1) / 2;
+        const int nb = (list_len(i) + 1) / 2, nsb = (nb + 1) / 2;
         const int ob = it & 1;
-        for (int n = 0; n < nb && ok; ++n, ++g) {
-          const int vst = g % Ly::kVStages;
-          const int pb = g % Ly::kPBufs;
+        for (int j = 0; j < nsb && ok; ++j, ++G) {
+          const int pb = G % Ly::kPBufs;
           ROLE_MARK(3);
-          ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8);
-          ROLE_MARK(0);
-          ok = ok && mbar_wait(&bars[Ly::bPFull + pb], (g / Ly::kPBufs) & 1, ctl, 9);
+          ok = mbar_wait(&bars[Ly::bPFull + pb], (G / Ly::kPBufs) & 1, ctl, 9);
           ROLE_MARK(1);
-          ok = ok && (n > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
+          ok = ok && (j > 0 || mbar_wait(&bars[Ly::bOEmpty + ob], ((it >> 1) & 1) ^ 1, ctl, 10));
           ROLE_MARK(2);
-          if (!ok) break;
-          tc_fence_after();
-          // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
-          const uint32_t lbo_v = (D > 64) ? Ly::kHalfBytes
-                                            : static_cast<uint32_t>(Ly::oZ - (Ly::oV + vst * Ly::kKVBytes));
-          const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oV + vst * Ly::kKVBytes), lbo_v, 1024);
-          const uint64_t bd0 = umma_desc_sw128(smem_u32(sm + Ly::oP + pb * Ly::kPBytes), 8192, 1024);
+          const int nh = min(2, nb - 2 * j);
+          for (int h = 0; h < nh && ok; ++h, ++g) {
+            const int vst = g % Ly::kVStages;
+            ROLE_MARK(3);
+            ok = mbar_wait(&bars[Ly::bVFull + vst], (g / Ly::kVStages) & 1, ctl, 8);
+            ROLE_MARK(0);
+            if (!ok) break;
+            tc_fence_after();
+            // V^T atoms along M (= d): the other 64-column half, or the zero region for D = 64
+            const uint32_t lbo_v = (D > 64) ? Ly::kHalfBytes
+                                              : static_cast<uint32_t>(Ly::oZ - (Ly::oV + vst * Ly::kKVBytes));
+            const uint64_t ad0 = umma_desc_sw128(smem_u32(sm + Ly::oV + vst * Ly::kKVBytes), lbo_v, 1024);
+            // rows 128 h .. 128 h + 127 of the super-block's P^T (one 128-key block, 16 KB)
+            const uint64_t bd0 =
+                umma_desc_sw128(smem_u32(sm + Ly::oP + pb * Ly::kPBytes + h * Ly::kPHalfBytes), 8192, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kPVSteps; ++kk) {
-            // a K-step is 16 keys = 2048 bytes further (start address in 16-byte units)
-            umma_ss(tmem + kOCol0 + ob * 64, ad0 + static_cast<uint64_t>(kk * 128), bd0 + static_cast<uint64_t>(kk * 128),
-                    kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kPVSteps; ++kk) {
+              // a K-step is 16 keys = 2048 bytes further (start address in 16-byte units)
+              umma_ss(tmem + kOCol0 + ob * 64, ad0 + static_cast<uint64_t>(kk * 128),
+                      bd0 + static_cast<uint64_t>(kk * 128), kIdescPV, (j > 0 || h > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars[Ly::bVEmpty + vst]);
           }
-          umma_commit(&bars[Ly::bVEmpty + vst]);
+          if (!ok) break;
           umma_commit(&bars[Ly::bPEmpty + pb]);
-          if (n == nb - 1) umma_commit(&bars[Ly::bOFull + ob]);
+          if (j == nsb - 1) umma_commit(&bars[Ly::bOFull + ob]);
         }
       }
       ROLE_MARK(3);
@@ -638,7 +660,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int ev = max(0, static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 126);
       return cl * qn * kmax + static_cast<float>(ev) - a.skip_cap;
     };
-    uint32_t g = 0;
+    uint32_t G = 0;  // super-blocks so far (S^T and P^T buffers)
     int it = 0;
     ROLE_TIMER_START();
     for (;; ++it) {
@@ -657,7 +679,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float* qsc_g = m_g + kQscFromM + ob * 64;
       // lane j: the key-mask word of block n0 + j for this warp's TMEM lane quadrant (rows
       // 32*qd .. 32*qd + 31 of the block: tile a for qd < 2, tile b otherwise); with 8-bit Q/K also
-      // that tile's row-scale offset (b, h, tile) * 64 (refilled one block ahead).
+      // that tile's row-scale offset (b, h, tile) * 64.  Refilled every 32 blocks (16 super-blocks).
       uint32_t vcache = 0;
       int kcache = 0;  // B*H*n_t*64 < 2^31 (checked when the plan is made)
       auto refill = [&](int n0) {
@@ -671,113 +693,109 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if constexpr (kF8) kcache = static_cast<int>((bh * n_t + max(kt, 0)) * 64);
         }
       };
-      // 8-bit Q/K: this lane's key row scale of block n (a missing second tile reads tile 0's, masked)
-      auto key_scale = [&](int n) -> float {
-        return __ldg(a.k_scale + __shfl_sync(0xffffffffu, kcache, n & 31) + (kl & 63));
-      };
-      float ks_next = 1.0f;
-      if constexpr (kF8) {
-        refill(0);
-        ks_next = key_scale(0);
-      }
 
       float l[CG];
 #pragma unroll
       for (int j = 0; j < CG; ++j) l[j] = 0.0f;
-      bool skip = false;  // set by the first block: the item's later blocks take no vote
+      bool skip = false;  // set by the first super-block: the item's later ones take no vote
+      const int nsb = (nb + 1) / 2;
 
-      // one block of the item; the first block (kFirst) takes the exact column maximum and needs no vote
-      auto block = [&](auto first_c, const int n) {
+      // Super-block j of the item: its 128-key blocks 2j and 2j + 1 (nh of them), in S^T buffer sb and
+      // P^T buffer pb, with one S^T-full wait, one S^T-empty and one P^T-full arrival for both.  The
+      // first super-block (kFirst) and one whose vote fires take the exact column maximum over both
+      // blocks first (a first pass over S^T), then exponentiate in a second pass, so that both blocks'
+      // probabilities share one m.
+      auto sblock = [&](auto first_c, const int j) {
         constexpr bool kFirst = decltype(first_c)::value;
-        const int sb = g % kSBufs;
-        const uint32_t su = g / kSBufs;
-        const int pb = g % Ly::kPBufs;
-        const uint32_t pu = g / Ly::kPBufs;
+        const int sb = G % kSBufs;
+        const uint32_t su = G / kSBufs;
+        const int pb = G % Ly::kPBufs;
+        const uint32_t pu = G / Ly::kPBufs;
+        const int nh = min(2, nb - 2 * j);
         ROLE_MARK(7);
-        uint32_t kmask;
-        [[maybe_unused]] float ks = 1.0f;
-        if constexpr (kF8) {
-          // the next block's key scale (and, every 32 blocks, mask words) are fetched one block ahead,
-          // while this block waits and works
-          kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
-          ks = ks_next;
-          if (((n + 1) & 31) == 0 && n + 1 < nb) refill(n + 1);
-          if (n + 1 < nb) ks_next = key_scale(n + 1);
-        } else {
-          if ((n & 31) == 0) refill(n);
-          kmask = __shfl_sync(0xffffffffu, vcache, n & 31);
+        if (((2 * j) & 31) == 0) refill(2 * j);
+        uint32_t km[2];
+        [[maybe_unused]] float ks[2] = {1.0f, 1.0f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          km[h] = __shfl_sync(0xffffffffu, vcache, (2 * j + h) & 31);
+          if constexpr (kF8) ks[h] = __ldg(a.k_scale + __shfl_sync(0xffffffffu, kcache, (2 * j + h) & 31) + (kl & 63));
         }
         ROLE_MARK(0);
-
         mbar_wait(&bars[Ly::bSFull + sb], su & 1, ctl, 12);
         ROLE_MARK(1);
         tc_fence_after();
-        float x[CG];
-        tmem_ld16(t_lane + sb * 64 + c0, x);
-        tmem_wait_ld();
-        ROLE_MARK(2);
-        tc_fence_before();
-        mbar_arrive(&bars[Ly::bSEmpty + sb]);  // per thread: no warp-level branch or sync
-
-        // x = logit * log2(e) - m  (m = 0 before the first block of the item); with 8-bit Q/K the
-        // logit is the code product times the key and query scales
-        // (two columns per instruction: fma2/mul2 round each lane as fmaf/fmul do; nm_g holds -m)
-        if constexpr (kF8) {
+        const uint32_t s_col = t_lane + sb * 128 + c0;
+        // x = logit * log2(e) - m (m = 0 before the first super-block: nm_g is not read then); with 8-bit
+        // Q/K the logit is the code product times the key and query scales (two columns per instruction:
+        // fma2/mul2 round each lane as fmaf/fmul do; nm_g holds -m); rows that are not keys get -inf
+        auto load_scaled = [&](auto use_m_c, int h, float* x) {
+          constexpr bool kUseM = decltype(use_m_c)::value;
+          tmem_ld16(s_col + h * 64, x);
+          tmem_wait_ld();
+          if constexpr (kF8) {
 #pragma unroll
-          for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], ks, ks);
-          if constexpr (kFirst) {
+            for (int jj = 0; jj < CG; jj += 2) mul2(x[jj], x[jj + 1], x[jj], x[jj + 1], ks[h], ks[h]);
 #pragma unroll
-            for (int j = 0; j < CG; j += 4) {
-              const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
-              mul2(x[j], x[j + 1], x[j], x[j + 1], c4.x, c4.y);
-              mul2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], c4.z, c4.w);
+            for (int jj = 0; jj < CG; jj += 4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + jj);
+              if constexpr (kUseM) {
+                const float4 m4 = *reinterpret_cast<const float4*>(nm_g + jj);
+                fma2(x[jj], x[jj + 1], x[jj], x[jj + 1], c4.x, c4.y, m4.x, m4.y);
+                fma2(x[jj + 2], x[jj + 3], x[jj + 2], x[jj + 3], c4.z, c4.w, m4.z, m4.w);
+              } else {
+                mul2(x[jj], x[jj + 1], x[jj], x[jj + 1], c4.x, c4.y);
+                mul2(x[jj + 2], x[jj + 3], x[jj + 2], x[jj + 3], c4.z, c4.w);
+              }
+            }
+          } else if constexpr (kUseM) {
+#pragma unroll
+            for (int jj = 0; jj < CG; jj += 4) {
+              const float4 m4 = *reinterpret_cast<const float4*>(nm_g + jj);
+              fma2(x[jj], x[jj + 1], x[jj], x[jj + 1], cl, cl, m4.x, m4.y);
+              fma2(x[jj + 2], x[jj + 3], x[jj + 2], x[jj + 3], cl, cl, m4.z, m4.w);
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < CG; j += 4) {
-              const float4 c4 = *reinterpret_cast<const float4*>(qsc_g + j);
-              const float4 m4 = *reinterpret_cast<const float4*>(nm_g + j);
-              fma2(x[j], x[j + 1], x[j], x[j + 1], c4.x, c4.y, m4.x, m4.y);
-              fma2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], c4.z, c4.w, m4.z, m4.w);
+            for (int jj = 0; jj < CG; jj += 2) mul2(x[jj], x[jj + 1], x[jj], x[jj + 1], cl, cl);
+          }
+          if (km[h] != 0xffffffffu) {  // the same word in every lane: a uniform branch
+            if (!((km[h] >> lane) & 1u)) {  // not a key: a pad or out-of-tile row
+#pragma unroll
+              for (int jj = 0; jj < CG; ++jj) x[jj] = -INFINITY;
             }
           }
-        } else if constexpr (kFirst) {
-#pragma unroll
-          for (int j = 0; j < CG; j += 2) mul2(x[j], x[j + 1], x[j], x[j + 1], cl, cl);
-        } else {
-#pragma unroll
-          for (int j = 0; j < CG; j += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(nm_g + j);
-            fma2(x[j], x[j + 1], x[j], x[j + 1], cl, cl, m4.x, m4.y);
-            fma2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], cl, cl, m4.z, m4.w);
-          }
-        }
-        if (kmask != 0xffffffffu) {  // the same word in every lane: a uniform branch
-          if (!((kmask >> lane) & 1u)) {  // not a key: a pad or out-of-tile row
-#pragma unroll
-            for (int j = 0; j < CG; ++j) x[j] = -INFINITY;
-          }
-        }
-        bool slow = true;
+        };
+        bool slow = kFirst;
         if constexpr (!kFirst) {
-          if (skip) {  // the same in all 128 threads of the group
-            slow = false;
-          } else {
+          if (!skip) {  // the same in all 128 threads of the group
+            // the vote: does any logit of the super-block exceed m by more than kRescaleLog2?
             static_assert(CG == 16, "the vote's maximum is written for 16 columns");
-            const float t = max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
-                                 max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15]));
+            float t = -INFINITY;
+            for (int h = 0; h < nh; ++h) {
+              float x[CG];
+              load_scaled(std::true_type{}, h, x);
+              t = max3(t, max3(max3(max3(x[0], x[1], x[2]), max3(x[3], x[4], x[5]), max3(x[6], x[7], x[8])),
+                               max3(x[9], x[10], x[11]), max3(max3(x[12], x[13], x[14]), x[15], x[15])),
+                       t);
+            }
             slow = named_bar_or(bar_vote, 128, t > kRescaleLog2);
           }
         }
         ROLE_MARK(3);
         if (slow) {
-          // exact column maximum of this block over the group's 128 lanes; raise m by it
+          // exact column maximum of the super-block over the group's 128 lanes (lane c keeps column c's
+          // maximum over this warp's rows of both blocks); raise m by it
           float cm = -INFINITY;
+          for (int h = 0; h < nh; ++h) {
+            float x[CG];
+            load_scaled(std::integral_constant<bool, !kFirst>{}, h, x);
 #pragma unroll
-          for (int j = 0; j < CG; ++j) {
-            float r;
-            asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x[j]));
-            if (j == lane) cm = r;
+            for (int jj = 0; jj < CG; ++jj) {
+              float r;
+              asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x[jj]));
+              if (jj == lane) cm = fmaxf(cm, r);
+            }
           }
           if (lane < CG) red_g[qd * CG + lane] = cm;
           named_bar_sync(bar_sync, 128);
@@ -799,53 +817,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           named_bar_sync(bar_sync, 128);
           if constexpr (kFirst) skip = (a.q_norm != nullptr) && skip_s[grp] != 0;
-#pragma unroll
-          for (int j = 0; j < CG; ++j) x[j] -= delta_g[j];
           if constexpr (!kFirst) {
 #pragma unroll
-            for (int j = 0; j < CG; ++j) l[j] *= ex2_approx(-delta_g[j]);
-            // O^T holds blocks < n of this item: wait for the last P.V, then rescale this group's columns
-            const uint32_t gp = g - 1;
+            for (int jj = 0; jj < CG; ++jj) l[jj] *= ex2_approx(-delta_g[jj]);
+            // O^T holds the super-blocks < j of this item: wait for the last one's P.V, then rescale this
+            // group's columns
+            const uint32_t gp = G - 1;
             mbar_wait(&bars[Ly::bPEmpty + (gp % Ly::kPBufs)], (gp / Ly::kPBufs) & 1, ctl, 13);
             tc_fence_after();
             float o[CG];
             tmem_ld16(t_lane + kOCol0 + ob * 64 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < CG; ++j) o[j] *= ex2_approx(-delta_g[j]);
+            for (int jj = 0; jj < CG; ++jj) o[jj] *= ex2_approx(-delta_g[jj]);
             tmem_st16(t_lane + kOCol0 + ob * 64 + c0, o);
             tmem_wait_st();
             tc_fence_before();
           }
         }
         ROLE_MARK(4);
-        // probabilities, partial row sums, this group's part of the P^T row (bf16, 128-byte swizzle)
-#pragma unroll
-        for (int j = 0; j < CG; ++j) x[j] = ex2_approx(x[j]);
-#pragma unroll
-        for (int j = 0; j < CG; j += 2) add2(l[j], l[j + 1], l[j], l[j + 1], x[j], x[j + 1]);
-        ROLE_MARK(5);
+        // probabilities against the (new) m, partial row sums, this group's part of the P^T rows of both
+        // blocks (bf16, 128-byte swizzle)
         mbar_wait(&bars[Ly::bPEmpty + pb], (pu & 1) ^ 1, ctl, 14);
         ROLE_MARK(6);
-        uint8_t* prow = sm + Ly::oP + pb * Ly::kPBytes + kl * 128;
+        for (int h = 0; h < nh; ++h) {
+          float x[CG];
+          // the first super-block's m is in nm_g now (its slow path always runs)
+          load_scaled(std::true_type{}, h, x);
+          if (h == nh - 1) {
+            tc_fence_before();
+            mbar_arrive(&bars[Ly::bSEmpty + sb]);  // per thread: no warp-level branch or sync
+          }
 #pragma unroll
-        for (int cc = 0; cc < CG / 8; ++cc) {
-          const int c = grp * (CG / 8) + cc;  // 16-byte chunk = queries 8c .. 8c+7
-          U128 w4;
-          w4.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
-          w4.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
-          w4.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
-          w4.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
-          *reinterpret_cast<U128*>(prow + ((c ^ (kl & 7)) << 4)) = w4;
+          for (int jj = 0; jj < CG; ++jj) x[jj] = ex2_approx(x[jj]);
+#pragma unroll
+          for (int jj = 0; jj < CG; jj += 2) add2(l[jj], l[jj + 1], l[jj], l[jj + 1], x[jj], x[jj + 1]);
+          uint8_t* prow = sm + Ly::oP + pb * Ly::kPBytes + h * Ly::kPHalfBytes + kl * 128;
+#pragma unroll
+          for (int cc = 0; cc < CG / 8; ++cc) {
+            const int c = grp * (CG / 8) + cc;  // 16-byte chunk = queries 8c .. 8c+7
+            U128 w4;
+            w4.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+            w4.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+            w4.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+            w4.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+            *reinterpret_cast<U128*>(prow + ((c ^ (kl & 7)) << 4)) = w4;
+          }
         }
+        ROLE_MARK(5);
         fence_proxy_async_smem();
         mbar_arrive(&bars[Ly::bPFull + pb]);
       };
-      if (nb > 0) {
-        block(std::true_type{}, 0);
-        ++g;
+      if (nsb > 0) {
+        sblock(std::true_type{}, 0);
+        ++G;
       }
-      for (int n = 1; n < nb; ++n, ++g) block(std::false_type{}, n);
+      for (int j = 1; j < nsb; ++j, ++G) sblock(std::false_type{}, j);
+
 
       // hand this warp's partial row sums to the epilogue (buffer ob is free once item it-2 is stored):
       // reduce-scatter over the warp's 32 lanes, lane j (j < CG) then holds column c0 + j

@@ -48,11 +48,13 @@ def prefix_token_mask(w):
     return m
 
 
-def assert_routes_agree(w, got, ref, heads_got, heads_ref=None, max_abs=2e-2, mean_abs=2e-3):
+def assert_routes_agree(w, got, ref, heads_got, heads_ref=None, max_abs=4e-2, mean_abs=4e-3):
     """Outputs [B, L, H, D] of two routes over the same inputs: bit-identical where both run the same
     kernels on the same items (always the video query rows; the prefix rows when both routes put them on
-    the same attention kernel), and within the output tolerance on prefix rows that one route runs on the
-    pair kernel and the other on the video kernel."""
+    the same attention kernel).  On prefix rows that one route runs on the pair kernel and the other on the
+    video kernel, each is held to max-abs 2e-2 / mean-abs 2e-3 against the oracle elsewhere, so the two
+    may differ by twice that (dense rows over every key of 1344x768 come within 0.012 of the oracle with
+    either kernel)."""
     import torch
 
     if prefix_on_pair_kernel(w, heads_got) == prefix_on_pair_kernel(w, heads_ref):
