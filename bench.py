@@ -63,6 +63,19 @@ def load_peaks():
     return dict(source="fallback", bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0)
 
 
+def attn_launches(w, heads):
+    """Attention kernels of one bf16 tile-order forward over `heads` heads: with 128-token tiles the pair
+    kernel alone; with 64-token tiles the video kernel, plus the pair kernel for the prefix query row
+    blocks when their pairs, B * heads * ceil(P / 2), fill the SMs (the library's rule)."""
+    import torch
+
+    if w.tile == 128:
+        return 1
+    prefix_tiles = sum((n + 63) // 64 for n in w.segments)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return 1 + int(prefix_tiles > 0 and w.batch * heads * ((prefix_tiles + 1) // 2) >= sms)
+
+
 def measured_attn_traffic():
     """DRAM bytes (read + write) of one attention launch from the committed ncu
     capture, or None when the kernel sources changed since it was taken."""
@@ -416,8 +429,11 @@ def run_vsa(args, w, world, rank, local, mode="replicas"):
     blocks = flops_call / (2 * tile_flops(w.head_dim, 64))
     attn_cycles = stage_ms["attention"] * 1e-3 * sm_mhz * 1e6 if sm_mhz else None
     roofline = {
-        "kernel": f"attention stage: vsa_attn_kernel<{w.head_dim}> (video query row blocks) and "
-                  f"vsa_attn_pair_kernel<{w.head_dim}> (prefix query row blocks, two at a time)",
+        "kernel": (f"attention stage: vsa_attn_pair_kernel<{w.head_dim}> (every 128-token query tile, its two "
+                   f"64-row halves together)" if w.tile == 128 else
+                   f"attention stage: vsa_attn_kernel<{w.head_dim}> (video query row blocks)" +
+                   (f" and vsa_attn_pair_kernel<{w.head_dim}> (prefix query row blocks, two at a time)"
+                    if attn_launches(w, w.heads) == 2 else "")),
         "bound": "tensor", "achieved": attn_tflops,
         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
         "peak_kind": f"{peaks['source']} burst dense bf16 (cuBLAS)",
@@ -431,10 +447,10 @@ def run_vsa(args, w, world, rank, local, mode="replicas"):
     }
     # library kernels per timed step (one vsa_forward): gate check, gather+pool, scores, a top-k pass over
     # the reference candidates (with reference segments), top-k + compression in one kernel (rows of up to
-    # 1280 tiles; longer rows take a top-k and a compression kernel), attention
+    # 1280 tiles; longer rows take a top-k and a compression kernel), attention (one or two kernels)
     nv = dims["n_video_tiles"]
     fused = (dims["n_tiles"] + 31) // 32 <= 40
-    launches = (5 + int(nv > 0 and dims["ref_topk"] > 0) + int(not fused)) * args.steps
+    launches = (4 + int(nv > 0 and dims["ref_topk"] > 0) + int(not fused) + attn_launches(w, w.heads)) * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -563,7 +579,7 @@ def run_ulysses(args, w, world, rank, local):
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
                 "timing": "wall clock per step around each rank's copies, barriers and forward; max over ranks"},
         # per rank and step: gather+pool, scores, select+compression, attention (no gate check over parts)
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (3 + attn_launches(w, hn)) * args.steps,
         "clocks": clk.summary(),
     }
     # release the peer mappings before any rank frees what they map
