@@ -432,7 +432,11 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ S, 
     const uint32_t cand = T | (1u << bit);
     int cnt = 0;
     for (int j = lane; j < ncols; j += 32) cnt += (keys[j] >= cand) ? 1 : 0;
-    if (warp_sum(cnt) >= k) T = cand;
+    const int total = warp_sum(cnt);
+    if (total >= k) {
+      T = cand;
+      if (total == k) break;  // exactly the selection: the lower bits need not be found (the same in every lane)
+    }
   }
   int gt = 0;
   for (int j = lane; j < ncols; j += 32) gt += (keys[j] > T) ? 1 : 0;
@@ -772,13 +776,26 @@ __global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __
 #pragma unroll
     for (int jj = 0; jj < kMaxJ; ++jj)
       if (32 * jj + lane < P) key[jj] = 0u;
+    // T: the largest threshold with at least k keys at or above it, one bit at a time from the top; once
+    // exactly k keys are at or above the candidate they are the selection (no key ties across the
+    // boundary), so the lower bits need not be found.  Four counters keep the count chains short.
+    static_assert(kMaxJ % 4 == 0, "keys per lane in groups of four");
     uint32_t T = 0u;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
-      uint32_t cnt = 0u;
+      uint32_t c0 = 0u, c1 = 0u, c2 = 0u, c3 = 0u;
 #pragma unroll
-      for (int jj = 0; jj < kMaxJ; ++jj) cnt += (key[jj] >= cand) ? 1u : 0u;
-      if (__reduce_add_sync(0xffffffffu, cnt) >= static_cast<uint32_t>(k)) T = cand;
+      for (int jj = 0; jj < kMaxJ; jj += 4) {
+        c0 += (key[jj] >= cand) ? 1u : 0u;
+        c1 += (key[jj + 1] >= cand) ? 1u : 0u;
+        c2 += (key[jj + 2] >= cand) ? 1u : 0u;
+        c3 += (key[jj + 3] >= cand) ? 1u : 0u;
+      }
+      const uint32_t cnt = __reduce_add_sync(0xffffffffu, (c0 + c1) + (c2 + c3));
+      if (cnt >= static_cast<uint32_t>(k)) {
+        T = cand;
+        if (cnt == static_cast<uint32_t>(k)) break;  // the same in every lane
+      }
     }
     uint32_t gt = 0u;
 #pragma unroll

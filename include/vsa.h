@@ -41,9 +41,15 @@
  *    a multiple of 4.  Video tokens follow the prefix in raster (t, h, w)
  *    order, w fastest.  Inside a tile the valid tokens come first, in
  *    sequence (prefix) or raster (cube) order, then zero pads.
- *  - A plan's device status word and the attention kernel's work counter are
+ *  - A plan's device status word and the attention kernels' work counters are
  *    shared by every call made with that plan: calls with one plan must not
  *    overlap on the GPU (use one plan per concurrent stream).
+ *  - The attention may run as two kernels: row blocks that share their key
+ *    list (the dense prefix query tiles, when B * H * ceil(P/2) reaches the
+ *    SM count; every query tile with 128-token tiles) go two at a time to a
+ *    second kernel, on a stream the plan owns that is forked from the
+ *    caller's stream with an event and joined back to it before the call
+ *    returns, so the caller's stream still orders all of a call's work.
  *  - Errors: argument and shape errors are detected on the host and returned
  *    synchronously with nothing launched; a failed launch returns
  *    VSA_ERR_CUDA; device-side failures (a bounded wait that ran out) are
