@@ -20,13 +20,13 @@
 // statistics are per query, i.e. per TMEM column, across lanes:
 //   - the running maximum m[q] is kept lazily: a block is exponentiated
 //     against the current m, and only when some logit exceeds m by more than
-//     kRescaleLog2 (or on the first block of an item) is the exact column
+//     kRescaleLog2 (or on an item's first super-block, below) is the exact column
 //     maximum taken across the 128 lanes and O^T, l rescaled.  Any m with no
 //     overflow gives the same softmax, so this is exact up to rounding.
-//     Deciding "exceeds" takes a vote of the column group every block, unless
-//     the first block already shows that no later logit can overflow: a
+//     Deciding "exceeds" takes a vote of the column group every super-block,
+//     unless the first one already shows that no later logit can overflow: a
 //     logit is at most |q| max|k| (Cauchy-Schwarz), so when that
-//     bound is within skip_cap - log2(max|v|) of the first block's maximum for
+//     bound is within skip_cap - log2(max|v|) of the first maximum for
 //     every column, P, l and O^T stay finite without further rescaling and the
 //     group skips the votes for the rest of the item;
 //   - l[q] is kept as per-lane partial sums and reduced once per item.
