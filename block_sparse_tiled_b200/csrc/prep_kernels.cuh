@@ -370,10 +370,12 @@ __global__ void __launch_bounds__(256, 2) scores_kernel(const float* __restrict_
       *reinterpret_cast<float4*>(av + 4) = *reinterpret_cast<const float4*>(&As[buf][dd][8 * ty + 4]);
       *reinterpret_cast<float4*>(bv) = *reinterpret_cast<const float4*>(&Bs[buf][dd][4 * tx]);
       *reinterpret_cast<float4*>(bv + 4) = *reinterpret_cast<const float4*>(&Bs[buf][dd][64 + 4 * tx]);
+      // two outputs per instruction (fma.rn.f32x2 rounds each lane as fmaf does: the same chains)
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(av[a], bv[c], acc[a][c]);
+        for (int c = 0; c < 8; c += 2)
+          fma2(acc[a][c], acc[a][c + 1], av[a], av[a], bv[c], bv[c + 1], acc[a][c], acc[a][c + 1]);
     }
     if (st + 1 < nsteps) store(buf ^ 1, ra, rb);
     __syncthreads();
