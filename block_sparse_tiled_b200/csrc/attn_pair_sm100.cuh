@@ -77,15 +77,21 @@ struct PairLayout {
 
 // a.s_lo, a.r_end: the launch's query row blocks [r_lo, r_end) (the prefix row blocks; with 128-token
 // tiles any tile-aligned range); a.n_s: pairs per (b, h); the other fields as for vsa_attn_kernel
-// (tile-order inputs, bf16).
-template <int D>
+// (tile-order inputs).  kF8: Q and K are 8-bit E4M3 code rows (128 bytes whatever D) with one scale per
+// row (a.q_scale, a.k_scale); S is then a kind::f8f6f4 product (32 codes per K-step) of the codes, and the
+// softmax multiplies each logit by its key row's scale and its query row's scale (times the softmax
+// scale) before the exponent; P.V stays bf16 ("FastH3 OmniRef inference", section "Device profiles":
+// 8-bit Q/K for the dense prefix query tiles, bf16 P.V).
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(kPairThreads, 1)
     vsa_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using Ly = PairLayout<D>;
-  constexpr int kQKSteps = D / 16;
+  constexpr int kQKSteps = kF8 ? (D + 31) / 32 : D / 16;
+  constexpr int kQKHalves = kF8 ? 1 : Ly::kHalves;                  // 8 KB boxes per 64 rows of Q or K
+  constexpr uint32_t kQKRowsBytes = kQKHalves * 128 * 128;           // bytes of 128 rows of Q or K
   constexpr int kPVSteps = 128 / 16;
-  constexpr uint32_t kIdescS = umma_idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t kIdescS = kF8 ? umma_idesc_e4m3(128, 128) : umma_idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t kIdescPV = umma_idesc_bf16(128, D, 0, 1);
 
   extern __shared__ uint8_t smem_raw[];
@@ -218,10 +224,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // the item's 128 query rows: row blocks s0 and s0 + 1 (rows past the tensor read as zeros)
         if (lane == 0) {
           ok = mbar_wait(&bars[Ly::bQEmpty], (it & 1) ^ 1, ctl, 31);
-          if (ok) mbar_arrive_expect_tx(&bars[Ly::bQFull], Ly::kRowsBytes);
+          if (ok) mbar_arrive_expect_tx(&bars[Ly::bQFull], kQKRowsBytes);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok && lane < 2 * Ly::kHalves) {
+        if (ok && lane < 2 * kQKHalves) {
           const int hh = lane >> 1, second = lane & 1;
           const int row = static_cast<int>((bh * n_t + s0 + second) * 64);
           tma_load_2d(sm + Ly::oQ + hh * 16384 + second * 8192, &tm_q, &bars[Ly::bQFull], hh * 64, row);
@@ -238,11 +244,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t u = g / nstages;
         if (lane == 0) {
           ok = mbar_wait(&bars[b_empty + st], (u & 1) ^ 1, ctl, is_k ? 32 : 33);
-          if (ok) mbar_arrive_expect_tx(&bars[b_full + st], Ly::kRowsBytes);
+          if (ok) mbar_arrive_expect_tx(&bars[b_full + st], is_k ? kQKRowsBytes : Ly::kRowsBytes);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        if (lane < 2 * Ly::kHalves) {
+        if (lane < 2 * (is_k ? kQKHalves : Ly::kHalves)) {
           const int hh = lane >> 1, second = lane & 1;
           const int row = static_cast<int>((bh * n_t + (second ? kb : ka)) * 64);
           tma_load_2d(ring + st * Ly::kRowsBytes + hh * 16384 + second * 8192, tmap, &bars[b_full + st], hh * 64,
@@ -285,7 +291,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           for (int kk = 0; kk < kQKSteps; ++kk) {
             // 16 elements (32 bytes) of every row per step, the next 64-column half every 4 steps
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-            umma_ss(tmem + kPairS0 + sb * 128, qd0 + off, bd0 + off, kIdescS, kk > 0 ? 1u : 0u);
+            if constexpr (kF8)
+              umma_ss_f8(tmem + kPairS0 + sb * 128, qd0 + off, bd0 + off, kIdescS, kk > 0 ? 1u : 0u);
+            else
+              umma_ss(tmem + kPairS0 + sb * 128, qd0 + off, bd0 + off, kIdescS, kk > 0 ? 1u : 0u);
           }
           umma_commit(&bars[Ly::bKEmpty + kst]);
           umma_commit(&bars[Ly::bSFull + sb]);
@@ -356,12 +365,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const int ev = max(0, static_cast<int>((__float_as_uint(vmax) >> 23) & 0xffu) - 126);
         lim = cl * qn * kmax + static_cast<float>(ev) - a.skip_cap;
       }
+      // the factor that turns this row's raw scores into log2 units: cl, or with 8-bit Q/K the row's scale
+      // times cl (each key's scale is applied to its column first)
+      float xs = cl;
+      if constexpr (kF8) xs = row_ok ? __ldg(a.q_scale + (bh * n_t + s) * 64 + (r & 63)) * cl : 0.0f;
       float m = 0.0f;        // running row maximum, log2 units
       float lacc[8];         // partial sums of this half-row
 #pragma unroll
       for (int j = 0; j < 8; ++j) lacc[j] = 0.0f;
       bool skip = false;
       uint32_t mlo = 0, mhi = 0;  // lane j: the key-mask word of this half of block 32 * (n / 32) + j
+      [[maybe_unused]] int kro = 0;  // 8-bit Q/K: lane j, that half's first key-scale index (b, h, block) * 64
       for (int n = 0; n < nb; ++n, ++g) {
         const int sb = g & 1;
         if ((n & 31) == 0) {
@@ -369,17 +383,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (n + lane < nb) {
             const int kt = block_row(bh, s0, n + lane) + hf;  // key row block of this half
             m = (kt < n_t) ? __ldg(a.key_mask + kt) : 0ull;
+            if constexpr (kF8) kro = static_cast<int>((bh * n_t + min(kt, n_t - 1)) * 64);
           }
           mlo = static_cast<uint32_t>(m);
           mhi = static_cast<uint32_t>(m >> 32);
         }
         const uint64_t kmask = static_cast<uint64_t>(__shfl_sync(0xffffffffu, mlo, n & 31)) |
                                (static_cast<uint64_t>(__shfl_sync(0xffffffffu, mhi, n & 31)) << 32);
+        // 8-bit Q/K: scale column j of chunk c by its key's scale (the same addresses in every lane)
+        [[maybe_unused]] const float* ksc = nullptr;
+        if constexpr (kF8) ksc = a.k_scale + __shfl_sync(0xffffffffu, kro, n & 31);
+        auto key_scale = [&](int c, float* x) {
+          if constexpr (kF8) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 k4 = __ldg(reinterpret_cast<const float4*>(ksc + c + j));
+              mul2(x[j], x[j + 1], x[j], x[j + 1], k4.x, k4.y);
+              mul2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], k4.z, k4.w);
+            }
+          }
+        };
         const uint32_t s_col = t_lane + kPairS0 + sb * 128 + 64 * hf;
         mbar_wait(&bars[Ly::bSFull + sb], (g >> 1) & 1, ctl, 50);
         tc_fence_after();
         // the half-row's largest logit (log2 units, less m), read first when this block may rescale:
-        // fl(s * cl - m) is monotone in s, so the largest raw score gives it
+        // fl(s * xs - m) is monotone in s (xs >= 0), so the largest scaled score gives it
         bool slow = (n == 0);
         float t = -INFINITY;
         if (n == 0 || !skip) {
@@ -389,6 +417,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             float x[32];
             tmem_ld32(s_col + c, x);
             tmem_wait_ld();
+            key_scale(c, x);
             if (kmask != ~0ull) {  // the same word in every lane of the warp
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -397,7 +426,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; j += 2) smax = max3(smax, x[j], x[j + 1]);
           }
-          t = (smax == -INFINITY) ? -INFINITY : fmaf(smax, cl, -m);
+          t = (smax == -INFINITY) ? -INFINITY : fmaf(smax, xs, -m);
           if (n > 0) slow = named_bar_or(1, 256, t > kRescaleLog2);
         }
         float d = 0.0f;  // the increase of m in this block
@@ -454,8 +483,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             tc_fence_before();
             mbar_arrive(&bars[Ly::bSEmpty + sb]);
           }
+          key_scale(c, x);
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) fma2(x[j], x[j + 1], x[j], x[j + 1], cl, cl, nm, nm);
+          for (int j = 0; j < 32; j += 2) fma2(x[j], x[j + 1], x[j], x[j + 1], xs, xs, nm, nm);
           if (kmask != ~0ull) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)

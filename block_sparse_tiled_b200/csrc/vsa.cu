@@ -752,17 +752,17 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   if (n_s < 0) n_s = static_cast<int>(n_rb) - s_lo;
   if (s_lo < 0 || n_s < 0 || s_lo + n_s > n_rb) return fail(VSA_ERR_INVALID_ARG, "attention row-block range");
   if (n_s == 0) return VSA_OK;
-  // bf16 tile-order attention: query row blocks that share their key list go two at a time (128 queries
-  // per key block) to the pair kernel -- the prefix row blocks of a launch over every row block, and with
-  // 128-token tiles every tile of the range (its two row blocks) -- and the other video row blocks to
-  // vsa_attn_kernel
+  // tile-order attention (bf16 or 8-bit Q/K): query row blocks that share their key list go two at a time
+  // (128 queries per key block) to the pair kernel -- the prefix row blocks of a launch that covers them,
+  // when their pairs fill the SMs, and with 128-token tiles every tile of the range (its two row blocks)
+  // -- and the other video row blocks to vsa_attn_kernel
   const int pre_rb = p->P << p->r.sh;
   int pair_lo = 0, pair_hi = 0;  // row blocks [pair_lo, pair_hi) go in pairs
-  if (!seq && !codes && p->pair_prefix) {
+  if (!seq && p->pair_prefix) {
     if (p->r.sh == 1 && s_lo % 2 == 0 && n_s % 2 == 0) {
       pair_lo = s_lo;
       pair_hi = s_lo + n_s;
-    } else if (s_lo == 0 && n_s == n_rb &&
+    } else if (s_lo == 0 && n_s >= pre_rb &&
                static_cast<int64_t>(p->B) * p->H * ((pre_rb + 1) / 2) >= p->num_sms) {
       // 64-token tiles: the prefix pairs go to the pair kernel only when there are enough of them to fill
       // the GPU; with a few heads (a head chunk of the host pipeline, a sequence-parallel rank) a handful of
@@ -799,9 +799,14 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
       constexpr int D = decltype(dc)::value;
       const size_t smem = vsa::PairLayout<D>::bytes();
       if (smem > p->max_smem) return fail(VSA_ERR_UNSUPPORTED, "attention shared memory exceeds the device limit");
-      VSA_TRY(allow_smem(vsa::vsa_attn_pair_kernel<D>, smem));
       const int64_t gp = std::min<int64_t>(ap.n_items, p->num_sms);
-      vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, ps>>>(mq, mk, mv, ap);
+      if (codes) {
+        VSA_TRY(allow_smem(vsa::vsa_attn_pair_kernel<D, true>, smem));
+        vsa::vsa_attn_pair_kernel<D, true><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, ps>>>(mq, mk, mv, ap);
+      } else {
+        VSA_TRY(allow_smem(vsa::vsa_attn_pair_kernel<D>, smem));
+        vsa::vsa_attn_pair_kernel<D><<<static_cast<unsigned>(gp), vsa::kPairThreads, smem, ps>>>(mq, mk, mv, ap);
+      }
       return VSA_OK;
     }));
     VSA_TRY(launch_check("pair attention"));

@@ -6,7 +6,9 @@ pad rows); pooled tiles, scores and the selection stay bit-exact (they read
 the bf16 inputs); the output is within the bf16 path's tolerance (max-abs
 2e-2, mean-abs 2e-3) of the float64 oracle whose logits use the dequantised
 8-bit Q and K.  The sequence-part, host-pipeline and 1344x768 routes are
-checked the same way (bit-identical to the device forward, or sampled)."""
+checked the same way (bit-identical to the device forward, or sampled).  The
+8-bit prefix query row blocks run on the pair kernel when their pairs fill the
+SMs, else on the transposed kernel; both are checked in full."""
 import ctypes
 import dataclasses
 
@@ -15,6 +17,7 @@ import pytest
 import torch
 
 import synth
+from conftest import prefix_on_pair_kernel
 
 pytestmark = pytest.mark.gpu
 
@@ -116,6 +119,19 @@ def test_fp8_full_parity(vsa, oracle_mod, name):
 def test_fp8_edge_cases(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
     w = synth.Workload("edge8", B, H, D, tuple(segments), tuple(grid), sparsity)
     full_parity(vsa, oracle_mod, w, seed=3)
+
+
+@pytest.mark.parametrize("segments,grid,sparsity,B,H,D", [
+    ((128, 0, 64), (4, 8, 8), 0.5, 2, 40, 128),  # 3 prefix tiles: a full pair and a half pair; 160 pairs
+    ((100, 30), (0, 0, 0), 0.9, 1, 148, 64),     # prefix only: one pair of ragged tiles per head, D = 64
+    ((70, 0, 5), (5, 6, 7), 0.6, 2, 50, 96),     # ragged prefix and video tiles, head_dim 96
+])
+def test_fp8_prefix_pairs_full_parity(vsa, oracle_mod, segments, grid, sparsity, B, H, D):
+    """Enough heads that the 8-bit prefix query row blocks go to the pair kernel (its kind::f8f6f4 S with
+    the key and query row scales in the softmax), in full against the oracle's 8-bit variant."""
+    w = synth.Workload("pairs8", B, H, D, tuple(segments), tuple(grid), sparsity)
+    assert prefix_on_pair_kernel(w)
+    full_parity(vsa, oracle_mod, w, seed=9)
 
 
 def test_fp8_zero_and_extreme_rows(vsa, oracle_mod):
