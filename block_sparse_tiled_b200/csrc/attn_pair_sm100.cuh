@@ -390,16 +390,26 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         const uint64_t kmask = static_cast<uint64_t>(__shfl_sync(0xffffffffu, mlo, n & 31)) |
                                (static_cast<uint64_t>(__shfl_sync(0xffffffffu, mhi, n & 31)) << 32);
-        // 8-bit Q/K: scale column j of chunk c by its key's scale (the same addresses in every lane)
+        // 8-bit Q/K: scale column j of chunk c by its key's scale (the same addresses in every lane); the
+        // 32 scales of a chunk are loaded before its S columns are waited for, so their latency overlaps
         [[maybe_unused]] const float* ksc = nullptr;
         if constexpr (kF8) ksc = a.k_scale + __shfl_sync(0xffffffffu, kro, n & 31);
-        auto key_scale = [&](int c, float* x) {
+        [[maybe_unused]] float4 k4[4];
+        [[maybe_unused]] int kc = 0;
+        auto load_ks = [&](int c) {  // the chunk's first 16 scales
+          if constexpr (kF8) {
+            kc = c;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) k4[j] = __ldg(reinterpret_cast<const float4*>(ksc + c) + j);
+          }
+        };
+        auto key_scale = [&](float* x) {
           if constexpr (kF8) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 k4 = __ldg(reinterpret_cast<const float4*>(ksc + c + j));
-              mul2(x[j], x[j + 1], x[j], x[j + 1], k4.x, k4.y);
-              mul2(x[j + 2], x[j + 3], x[j + 2], x[j + 3], k4.z, k4.w);
+            for (int j = 0; j < 8; ++j) {
+              const float4 k = j < 4 ? k4[j] : __ldg(reinterpret_cast<const float4*>(ksc + kc) + j);
+              mul2(x[4 * j], x[4 * j + 1], x[4 * j], x[4 * j + 1], k.x, k.y);
+              mul2(x[4 * j + 2], x[4 * j + 3], x[4 * j + 2], x[4 * j + 3], k.z, k.w);
             }
           }
         };
@@ -415,9 +425,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; c += 32) {
             float x[32];
+            load_ks(c);
             tmem_ld32(s_col + c, x);
             tmem_wait_ld();
-            key_scale(c, x);
+            key_scale(x);
             if (kmask != ~0ull) {  // the same word in every lane of the warp
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -477,13 +488,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 32) {
           float x[32];
+          load_ks(c);
           tmem_ld32(s_col + c, x);
           tmem_wait_ld();
           if (c == 32) {  // S^T of this block fully read
             tc_fence_before();
             mbar_arrive(&bars[Ly::bSEmpty + sb]);
           }
-          key_scale(c, x);
+          key_scale(x);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) fma2(x[j], x[j + 1], x[j], x[j + 1], xs, xs, nm, nm);
           if (kmask != ~0ull) {

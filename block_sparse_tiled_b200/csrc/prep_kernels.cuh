@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(384, (kSub == 2 || kF8) ? 2 : 3) gather_pool_k
     void* __restrict__ q_t, void* __restrict__ k_t, uint16_t* __restrict__ v_t, float* __restrict__ q_s,
     float* __restrict__ k_s, float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     const int32_t* __restrict__ tile_token, const int32_t* __restrict__ tile_valid, int64_t L, int H,
-    int n_t, const PartIO io, float* __restrict__ q_n, uint32_t* __restrict__ kv) {
+    int n_t, const PartIO io, float* __restrict__ q_n, uint32_t* __restrict__ kv, int q_tiles) {
   constexpr int kRows = kTile * kSub;                             // rows of one tile
   constexpr int kChunks = D / 8;                                  // 16-byte chunks per row
   constexpr int kIters = kF8 ? kRows / 8 : kRows * kChunks / 128;  // chunks each thread moves per tensor
@@ -158,8 +158,10 @@ __global__ void __launch_bounds__(384, (kSub == 2 || kF8) ? 2 : 3) gather_pool_k
 
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const bool pool = (pq != nullptr);
-  // without pooling and without a V destination (a second, codes-only pass) V is not read at all
+  // without pooling and without a V destination (a second, codes-only pass) V is not read at all, and
+  // there Q only for the first q_tiles tiles (the query tiles that take their logits from the codes)
   const bool skip_v = !pool && v_t == nullptr;
+  const bool skip_q = skip_v && tile >= q_tiles;
   if (threadIdx.x < kRows) tok_s[threadIdx.x] = tile_token[static_cast<int64_t>(tile) * kRows + threadIdx.x];
   __syncthreads();
 
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(384, (kSub == 2 || kF8) ? 2 : 3) gather_pool_k
     const bool active = chunk_of(u, &r, &c);
     const int32_t tok = tok_s[r];
     val[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (active && tok >= 0 && !(tsr == 2 && skip_v)) {
+    if (active && tok >= 0 && !(tsr == 2 && skip_v) && !(tsr == 0 && skip_q)) {
       if constexpr (kParts) {  // the token's part, and heads h0 + h of its Htot
         int64_t lt;
         const uint16_t* base = part_base(io, tsr, src, tok, &lt);
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(384, (kSub == 2 || kF8) ? 2 : 3) gather_pool_k
     int r, c;
     const bool active = chunk_of(u, &r, &c);
     if (active && pool) reinterpret_cast<uint4*>(tiles + tsr * kRows * D)[r * kChunks + c] = val[u];
-    if (!write_tiles) continue;
+    if (!write_tiles || (tsr == 0 && skip_q)) continue;
     if (codes) {
       float f[8];
       const uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};

@@ -476,7 +476,9 @@ struct vsa_plan_s {
   // vsa_sparse_attn_fwd (bf16 plans): the overflow-bound statistics of its tile-order inputs, query row
   // norms then the (b, h) maxima
   float* d_stats = nullptr;
-  int* d_status = nullptr;  // [0] error code, [1] failure site, [2] attention item counter, [3] gate nonzero
+  // [0] error code, [1] failure site, [2] attention item counter, [3] gate nonzero, [4] pair-kernel item
+  // counter, [5] and [6] the two counters of a second attention launch running concurrently
+  int* d_status = nullptr;
   vsa_workspace_layout ws{};
   // Head-slice plans share the parent's device tables and status word and own nothing on the device.
   bool owns_device = true;
@@ -492,7 +494,7 @@ struct vsa_plan_s {
   // the prefix pair kernel runs on `side`, forked from and joined back to the caller's stream, so that
   // vsa_attn_kernel starts on the SMs its last items leave idle (created on first use)
   cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_split = nullptr;
 };
 
 namespace {
@@ -549,11 +551,15 @@ vsa::PartIO single_io(vsa_plan p) { return vsa::PartIO{nullptr, 1, p->r.L, p->H,
 // pooling: V is not read.
 vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, void* qt, void* kt, void* vt, float* pq,
                       float* pk, float* pv, cudaStream_t s, const vsa::PartIO* io = nullptr, float* qs = nullptr,
-                      float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr, int f8 = -1) {
+                      float* ks = nullptr, float* qn = nullptr, uint32_t* kv = nullptr, int f8 = -1,
+                      int q_tiles = -1) {
   const bool codes = (f8 < 0) ? p->qk_fp8 : (f8 != 0);
   const vsa::PartIO pio = io ? *io : single_io(p);
   if (p->n_t == 0) return VSA_OK;
   const bool pool = pq != nullptr;
+  // q_tiles: a codes-only pass (no pooling, no V) writes Q for tiles [0, q_tiles) only
+  if (q_tiles < 0) q_tiles = p->n_t;
+  if (q_tiles < p->n_t && (pool || vt != nullptr)) return fail(VSA_ERR_INVALID_ARG, "partial Q needs a codes-only pass");
   const size_t smem = pool ? static_cast<size_t>(3) * p->r.tile * p->D * 2 : 0;
   dim3 grid(p->n_t, p->H, p->B);
   const auto* qq = static_cast<const uint16_t*>(q);
@@ -563,7 +569,7 @@ vsa_status run_gather(vsa_plan p, const void* q, const void* k, const void* v, v
   auto launch = [&](auto kernel) -> vsa_status {
     VSA_TRY(allow_smem(kernel, smem));
     kernel<<<grid, 384, smem, s>>>(qq, kk, vv, qt, kt, vo, qs, ks, pq, pk, pv, p->d_tile_token, p->d_tile_valid,
-                                   p->r.L, p->H, p->n_t, pio, qn, kv);
+                                   p->r.L, p->H, p->n_t, pio, qn, kv, q_tiles);
     return VSA_OK;
   };
   VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
@@ -683,11 +689,24 @@ vsa_status run_topk(vsa_plan p, const float* S, const float* pv, int32_t* idx, f
 
 // qt/kt/vt: tile-order copies; or, with seq_qkv (q, k, v in sequence order), the kernel reads the
 // tiles itself (needs B <= kSeqMaxBatch).
+// Makes the plan's side stream (and its events) on first use and orders it after the work queued on s.
+vsa_status fork_side(vsa_plan p, cudaStream_t s) {
+  if (p->side == nullptr) {
+    VSA_CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
+    VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
+    VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
+    VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_split, cudaEventDisableTiming));
+  }
+  VSA_CUDA_TRY(cudaEventRecord(p->ev_fork, s));
+  VSA_CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
+  return VSA_OK;
+}
+
 vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, const int32_t* idx, const float* o_c,
                     const void* gate, void* out, cudaStream_t s, int gate_ld = 0, const int* gate_nonzero = nullptr,
                     const void* const* seq_qkv = nullptr, const vsa::PartIO* io = nullptr, const float* qs = nullptr,
                     const float* ks = nullptr, const float* qn = nullptr, const uint32_t* kv = nullptr, int f8 = -1,
-                    int s_lo = 0, int n_s = -1) {
+                    int s_lo = 0, int n_s = -1, bool alt_counters = false) {
   if (p->n_t == 0) return VSA_OK;
   const bool seq = (seq_qkv != nullptr);
   const bool codes = (f8 < 0) ? p->qk_fp8 : (f8 != 0);  // Q and K as 8-bit codes (8-bit S^T product)
@@ -722,7 +741,9 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
   a.gate = static_cast<const uint16_t*>(gate);
   a.out = static_cast<uint16_t*>(out);
   a.status = p->d_status;
-  a.sched = p->d_status + 2;
+  // item counters: [2] (video kernel) and [4] (pair kernel), or [5] and [6] for a launch that runs
+  // concurrently with another run_attn on the same plan
+  a.sched = p->d_status + (alt_counters ? 5 : 2);
   a.L = p->r.L;
   a.H = p->H;
   a.gate_pc = p->gate_pc;
@@ -778,19 +799,13 @@ vsa_status run_attn(vsa_plan p, const void* qt, const void* kt, const void* vt, 
     ap.r_end = pair_hi;
     ap.n_s = (pair_hi - pair_lo + 1) / 2;
     ap.n_items = static_cast<int64_t>(p->B) * p->H * ap.n_s;
-    ap.sched = p->d_status + 4;  // its own item counter
+    ap.sched = p->d_status + (alt_counters ? 6 : 4);  // its own item counter
     n_s = s_lo + n_s - pair_hi;  // what is left: [pair_hi, s_lo + n_s)
     s_lo = pair_hi;
     // with video row blocks to run too, the pair kernel goes on the side stream (forked from s)
     cudaStream_t ps = s;
     if (n_s > 0) {
-      if (p->side == nullptr) {
-        VSA_CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
-        VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
-        VSA_CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
-      }
-      VSA_CUDA_TRY(cudaEventRecord(p->ev_fork, s));
-      VSA_CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
+      VSA_TRY(fork_side(p, s));
       ps = p->side;
       joined = false;
     }
@@ -841,8 +856,9 @@ void release_side(vsa_plan_s* p) {
   if (p->side) cudaStreamDestroy(p->side);
   if (p->ev_fork) cudaEventDestroy(p->ev_fork);
   if (p->ev_join) cudaEventDestroy(p->ev_join);
+  if (p->ev_split) cudaEventDestroy(p->ev_split);
   p->side = nullptr;
-  p->ev_fork = p->ev_join = nullptr;
+  p->ev_fork = p->ev_join = p->ev_split = nullptr;
 }
 
 void release_host_pipe(vsa_plan_s* p) {
@@ -967,8 +983,9 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   const bool seq = p->seq_tiles;
   VSA_TRY(run_gather(p, q, k, v, seq ? nullptr : qt, seq ? nullptr : kt, seq ? nullptr : vt, pq, pk, pv, s, io, qsc, ksc,
                      qn, kv));
-  // prefix split: a second gather writes the 8-bit codes of Q and K (no pooling, V not read) with their
-  // own overflow-bound statistics; the value maximum comes from the first gather's statistics
+  // prefix split: a second gather writes the 8-bit codes of K and of the prefix tiles' Q (no pooling, V
+  // not read) with their own overflow-bound statistics; the value maximum comes from the first gather's
+  // statistics
   auto* qc = w + p->ws.q_c;
   auto* kc = w + p->ws.k_c;
   auto* qn8 = reinterpret_cast<float*>(w + p->ws.q_n8);
@@ -977,7 +994,7 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
     auto* qs2 = reinterpret_cast<float*>(w + p->ws.q_s);
     auto* ks2 = reinterpret_cast<float*>(w + p->ws.k_s);
     VSA_CUDA_TRY(cudaMemsetAsync(kv8, 0, static_cast<size_t>(p->B) * p->H * 8, s));
-    VSA_TRY(run_gather(p, q, k, v, qc, kc, nullptr, nullptr, nullptr, nullptr, s, io, qs2, ks2, qn8, kv8, 1));
+    VSA_TRY(run_gather(p, q, k, v, qc, kc, nullptr, nullptr, nullptr, nullptr, s, io, qs2, ks2, qn8, kv8, 1, p->P));
     VSA_CUDA_TRY(cudaMemcpy2DAsync(kv8 + 1, 8, kv + 1, 8, 4, static_cast<size_t>(p->B) * p->H,
                                    cudaMemcpyDeviceToDevice, s));
   }
@@ -985,13 +1002,22 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
   if (p->qk_split) {
-    // the dense prefix query row blocks on the 8-bit S^T kernel, then the video ones on the bf16 kernel
+    // the dense prefix query row blocks on the 8-bit kernel, the video ones on the bf16 kernel; the two
+    // launches write disjoint output rows and run concurrently: the prefix one on the plan's side stream
+    // (forked from s, with its own item counters), the video one on s, which then waits for the side
     const int pre = p->P << p->r.sh;
-    VSA_TRY(run_attn(p, qc, kc, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io,
+    if (pre == 0)
+      return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io, nullptr, nullptr, qn, kv,
+                      0);
+    VSA_TRY(fork_side(p, s));
+    VSA_TRY(run_attn(p, qc, kc, vt, idx, oc, gate, out, p->side, gate_ld, gate_nz, nullptr, io,
                      reinterpret_cast<float*>(w + p->ws.q_s), reinterpret_cast<float*>(w + p->ws.k_s), qn8, kv8, 1, 0,
+                     pre, true));
+    VSA_CUDA_TRY(cudaEventRecord(p->ev_split, p->side));
+    VSA_TRY(run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io, nullptr, nullptr, qn, kv, 0,
                      pre));
-    return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, nullptr, io, nullptr, nullptr, qn, kv, 0,
-                    pre);
+    VSA_CUDA_TRY(cudaStreamWaitEvent(s, p->ev_split, 0));
+    return VSA_OK;
   }
   return run_attn(p, qt, kt, vt, idx, oc, gate, out, s, gate_ld, gate_nz, seq ? qkv : nullptr, io, qsc, ksc, qn, kv);
 }

@@ -375,7 +375,9 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
 /* With qk_fp8 = 2 (the prefix split) q_t and k_t hold the bf16 copies, q_c and k_c
  * the E4M3 codes [B, H, n_tiles, 64, 128] with their row scales in q_s, k_s, and
  * q_n8, kv_max8 the statistics of the dequantised rows (q_c .. kv_max8 are empty
- * otherwise). */
+ * otherwise).  Only the prefix tiles' query rows are quantised (the video query
+ * tiles keep bf16 logits): the video tiles' part of q_c, q_s and q_n8 is left as
+ * it was. */
 typedef struct vsa_workspace_layout {
   size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c;
   size_t q_c, k_c, q_n8, kv_max8, total;
