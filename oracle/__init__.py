@@ -70,6 +70,13 @@ def _load():
         lib.vsa_oracle_e4m3_round.restype = i32
         lib.vsa_oracle_e4m3_round_array.argtypes = [P, i64, P]
         lib.vsa_oracle_quant_e4m3.argtypes = [P, i64, i32, P, P]
+        lib.vsa_oracle_e2m1_value.argtypes = [i32]
+        lib.vsa_oracle_e2m1_value.restype = f64
+        lib.vsa_oracle_e2m1_round.argtypes = [f32]
+        lib.vsa_oracle_e2m1_round.restype = i32
+        lib.vsa_oracle_e2m1_round_array.argtypes = [P, i64, P]
+        lib.vsa_oracle_quant_fp4.argtypes = [P, i64, i32, P, P]
+        lib.vsa_oracle_smooth_keys.argtypes = [P, i64, i64, i32, i32, P, P]
         lib.vsa_oracle_fine_masked.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, f64,
                                                P]
         lib.vsa_oracle_output.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, i32, P, P, P, P]
@@ -238,20 +245,23 @@ def fine(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=No
     return out
 
 
-def fine_split(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=None) -> np.ndarray:
+def fine_split(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, qk8=None,
+               video_qk=None) -> np.ndarray:
     """The fine branch with the pages' prefix split (reading R19): the dense prefix query tiles take
     their logits from the 8-bit Q/K of ``qk8`` (as fine() with qk8), the video query tiles from the bf16
-    q, k (as fine() without).  Both branches run in full over their own tiles and the rows are merged by
-    the tile each token belongs to; bf16 P.V throughout.  ("FastH3 OmniRef inference", section "Device
-    profiles": the dense prefix query tiles run at 8-bit Q/K with bf16 P.V, the video query tiles on
-    another kernel.)"""
+    q, k (as fine() without), or with ``video_qk`` = (q4, k4) from those bf16 arrays instead (the
+    dequantised FP4 operands of fp4_operands, reading R20).  Both branches run in full over their own
+    tiles and the rows are merged by the tile each token belongs to; bf16 P.V throughout.  ("FastH3
+    OmniRef inference", section "Device profiles": the dense prefix query tiles run at 8-bit Q/K with
+    bf16 P.V, the video query tiles on another kernel.)"""
     B, L, H, _ = np.shape(q)
     n_t, P = geo.n_tiles, geo.n_prefix
     sel = np.ones((B, H, n_t), bool) if todo is None else np.asarray(todo, bool)
     is_prefix = np.zeros((B, H, n_t), bool)
     is_prefix[:, :, :P] = True
     pre = fine(q, k, v, geo, idx, topk, scale, todo=sel & is_prefix, qk8=qk8)
-    vid = fine(q, k, v, geo, idx, topk, scale, todo=sel & ~is_prefix)
+    qv, kv = (q, k) if video_qk is None else video_qk
+    vid = fine(qv, kv, v, geo, idx, topk, scale, todo=sel & ~is_prefix)
     tok_prefix = np.zeros(L, bool)  # tokens of prefix tiles
     for i in range(P):
         tok_prefix[geo.tile_token[i, :geo.tile_valid[i]]] = True
@@ -306,6 +316,68 @@ def quant_e4m3(x_bf16: np.ndarray):
 def dequant_e4m3(code, scale) -> np.ndarray:
     """code * scale in float64 (exact: a 4-bit significand times a binary32 scale)."""
     return e4m3_value(code) * np.asarray(scale, np.float64)[..., None]
+
+
+def e2m1_value(codes) -> np.ndarray:
+    """float64 values of E2M1 codes (low 4 bits of a uint8 array), from the format's definition (R20)."""
+    lib = _load()
+    table = np.array([lib.vsa_oracle_e2m1_value(c) for c in range(16)], np.float64)
+    return table[np.asarray(codes, np.uint8) & 15]
+
+
+def e2m1_round(y) -> np.ndarray:
+    """E2M1 codes of binary32 values: nearest, ties to the even code, saturating at +-6."""
+    y = _c(np.asarray(y, np.float32), np.float32)
+    out = np.empty(y.shape, np.uint8)
+    _load().vsa_oracle_e2m1_round_array(_p(y), y.size, _p(out))
+    return out
+
+
+def quant_fp4(x) -> tuple:
+    """The FP4 block quantiser (R20): x [..., D] binary32 (D a multiple of 16) -> (codes [..., D] uint8,
+    one E2M1 code per element; scales [..., D / 16] uint8, one E4M3 code per 16 elements)."""
+    x = _c(np.asarray(x, np.float32), np.float32)
+    D = x.shape[-1]
+    assert D % 16 == 0
+    code = np.empty(x.shape, np.uint8)
+    scale = np.empty(x.shape[:-1] + (D // 16,), np.uint8)
+    _load().vsa_oracle_quant_fp4(_p(x), x.size // D, D, _p(code), _p(scale))
+    return code, scale
+
+
+def dequant_fp4(code, scale) -> np.ndarray:
+    """code * scale in float64 (exact): each block of 16 elements times its E4M3 scale."""
+    v = e2m1_value(code)
+    sv = np.repeat(e4m3_value(scale), 16, axis=-1)
+    return v * sv
+
+
+def smooth_keys(k_bf16) -> tuple:
+    """Key smoothing (R20): k [B, L, H, D] bf16 bits -> (mu [B, H, D] float32, the per-head key mean,
+    summed in binary64 in token order; k - mu [B, L, H, D] binary32)."""
+    k = _c(k_bf16, np.uint16)
+    B, L, H, D = k.shape
+    mu = np.empty((B, H, D), np.float32)
+    ks = np.empty((B, L, H, D), np.float32)
+    _load().vsa_oracle_smooth_keys(_p(k), B, L, H, D, _p(mu), _p(ks))
+    return mu, ks
+
+
+def bf16_bits_exact(x) -> np.ndarray:
+    """bf16 bits of float64 values that bf16 holds exactly (asserted)."""
+    f = np.asarray(x, np.float64).astype(np.float32)
+    assert (f.astype(np.float64) == np.asarray(x, np.float64)).all()
+    u = f.view(np.uint32)
+    assert not (u & 0xFFFF).any(), "value not representable in bf16"
+    return (u >> 16).astype(np.uint16)
+
+
+def fp4_operands(q_bf16, k_bf16, smooth: bool = True) -> tuple:
+    """(q4, k4): the dequantised FP4 Q and K (R20) as bf16 bits [B, L, H, D]; K smoothed first
+    when ``smooth``.  They replace q, k in the video query tiles' logits."""
+    qf = (_c(q_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32)
+    kf = smooth_keys(k_bf16)[1] if smooth else (_c(k_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32)
+    return tuple(bf16_bits_exact(dequant_fp4(*quant_fp4(t))) for t in (qf, kf))
 
 
 def output_tiles(o_f_tiles, o_c, gate, geo: Geometry, items, H: int) -> np.ndarray:
@@ -399,7 +471,7 @@ class ForwardResult:
 
 
 def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=False, tile=64,
-            cube=None, ref_segments=None, ref_keep=None) -> ForwardResult:
+            cube=None, ref_segments=None, ref_keep=None, fp4=False, k_smooth=True) -> ForwardResult:
     """The whole VSA-H3 forward on bf16-bit arrays q, k, v [B,L,H,D] and gate [B,L,H] (or
     [B,L,H*D], one per channel).
 
@@ -409,7 +481,10 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
     selection still reads the bf16 inputs; qk8="prefix": only the dense prefix
     query tiles do (R19, fine_split).  tile, cube: the tile size and video
     cube shape (64 and 4x4x4 as the method states; 128 per R17).  ref_segments,
-    ref_keep: reference segments and their keep ratio (R18)."""
+    ref_keep: reference segments and their keep ratio (R18).  fp4: the video
+    query tiles' logits use the dequantised FP4 Q and K (R20; K smoothed when
+    k_smooth), the prefix query tiles' follow qk8 (False: bf16, "prefix": 8-bit);
+    fp4 with qk8=True (8-bit video tiles) is refused."""
     t0 = time.perf_counter()
     geo = geometry(segments, grid, tile, cube, ref_segments)
     D = q.shape[-1]
@@ -422,7 +497,11 @@ def forward(q, k, v, gate, segments, grid, sparsity, scale=None, todo=None, qk8=
     idx = select(S, geo.n_prefix, kc, geo.is_ref, kr)
     o_c = compress(S, pv)
     q8 = (*quant_e4m3(q), *quant_e4m3(k)) if qk8 else None
-    if qk8 == "prefix":
+    if fp4:
+        if qk8 not in (False, None, "prefix"):
+            raise ValueError("fp4 video tiles go with bf16 or 8-bit (qk8='prefix') prefix tiles")
+        o_f = fine_split(q, k, v, geo, idx, kc, scale, todo, qk8=q8, video_qk=fp4_operands(q, k, k_smooth))
+    elif qk8 == "prefix":
         o_f = fine_split(q, k, v, geo, idx, kc, scale, todo, qk8=q8)
     else:
         o_f = fine(q, k, v, geo, idx, kc, scale, todo, qk8=q8)

@@ -67,6 +67,28 @@
  *      tiles (0 when R = 0), listed ascending before its topk video tiles.  The other
  *      prefix tiles stay always kept; prefix query tiles (reference ones included) stay
  *      dense; the compression still runs over all tiles.
+ *   R20 FP4 video query tiles ("FastH3 OmniRef inference", sections "Device profiles",
+ *      "Environment" and "Fallbacks": video query tiles on an FP4 kernel, key smoothing
+ *      "subtract the per-head key mean before FP4 quantization"; the emulator fallback
+ *      gives the numerics: FP4 Q/K for video query tiles, per-token 8-bit Q/K for the prefix
+ *      tiles, bf16 P.V, key smoothing; "FastH3 NVFP4 on RTX PRO 6000", model integration
+ *      and "What was tried": activations take a unit global scale and dynamic per-16 block
+ *      scales; the stored format is E2M1 values with one E4M3 scale per 16 values):
+ *      FP4 = OCP E2M1 (bit 3 sign, 2-bit exponent with bias 1, 1-bit mantissa; magnitudes
+ *      0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN).  Rows of D are cut into blocks of
+ *      16 consecutive elements; a block's scale is the E4M3 code e4m3_round(amax / 6)
+ *      (binary32 division, amax the largest |x| of the block) and each element's code is
+ *      e2m1_round(x / value(scale)) (binary32 division; nearest, ties to the even code,
+ *      saturating at 6); a scale of value 0 gives codes +0.  The global scale is 1.
+ *      Key smoothing: mu[b, h, d] = the binary64 sum of k[b, t, h, d] over the L tokens in
+ *      token order, divided by L in binary64, rounded to binary32; the quantised key is
+ *      x = k - mu in binary32.  Queries are not smoothed.  The dequantised values code *
+ *      scale (at most 6 significant bits, magnitudes 2^-10 .. 2688) are bf16 numbers, and
+ *      they replace Q and K in the video query tiles' logits; the prefix query tiles follow
+ *      R16 on the unsmoothed inputs (the split); selection, compression and P.V keep bf16.
+ *      Subtracting mu from every key changes each query row's logits by one constant,
+ *      which the softmax removes: only the rounding changes.  The native kernel's
+ *      quantised P.V ("two-level P") is not defined on the pages and is not modelled.
  *
  * Precision: selection (pool, score, top-k) in IEEE binary32 with the pinned
  * order above; fine attention, compression and the output in binary64.
@@ -163,6 +185,85 @@ void vsa_oracle_quant_e4m3(const uint16_t *x, int64_t N, int D, uint8_t *code, f
             code[r * D + d] = (uint8_t)((amax == 0.0f) ? 0 : vsa_oracle_e4m3_round(q));
         }
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* O1 FP4 (E2M1) codes with one E4M3 scale per 16 values, key          */
+/* smoothing (reading R20)                                             */
+/* ------------------------------------------------------------------ */
+
+/* Value of an E2M1 code: bit 3 sign, bits 2..1 exponent field e (bias 1), bit 0
+ * mantissa m.  e = 0: subnormal, m/2; otherwise (1 + m/2) * 2^(e-1). */
+double vsa_oracle_e2m1_value(int code) {
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* E2M1 code nearest to y; a tie goes to the even code; magnitudes at or above 6 give
+ * +-6 (code 7).  The sign bit is the sign of y (-0 and small negatives give 0x8). */
+int vsa_oracle_e2m1_round(float y) {
+    int sign = signbit(y) ? 8 : 0;
+    double a = fabs((double)y);
+    int lo = 0;
+    double dl, dh;
+    if (a >= 6.0) return sign | 7;
+    while (lo < 7 && vsa_oracle_e2m1_value(lo + 1) <= a) ++lo; /* largest code with value <= a */
+    dl = a - vsa_oracle_e2m1_value(lo);
+    if (dl == 0.0) return sign | lo;
+    dh = vsa_oracle_e2m1_value(lo + 1) - a;
+    if (dl < dh) return sign | lo;
+    if (dh < dl) return sign | (lo + 1);
+    return sign | ((lo & 1) ? lo + 1 : lo);
+}
+
+void vsa_oracle_e2m1_round_array(const float *y, int64_t n, uint8_t *code) {
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n; ++e) code[e] = (uint8_t)vsa_oracle_e2m1_round(y[e]);
+}
+
+/* Block quantisation of rows x [N, D] (binary32; D a multiple of 16): for each block of 16
+ * consecutive elements, amax = max |x|, scale code sc = e4m3_round(amax / 6) (binary32
+ * division), sv = value(sc), code = e2m1_round(x / sv) (binary32 division), or +0 when
+ * sv = 0.  code [N, D], scale [N, D / 16]. */
+void vsa_oracle_quant_fp4(const float *x, int64_t N, int D, uint8_t *code, uint8_t *scale) {
+    const int nb = D / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < N; ++r) {
+        for (int blk = 0; blk < nb; ++blk) {
+            const float *xb = x + r * D + blk * 16;
+            uint8_t *cb = code + r * D + blk * 16;
+            float amax = 0.0f, sv;
+            int sc;
+            for (int j = 0; j < 16; ++j) {
+                float a = fabsf(xb[j]);
+                if (a > amax) amax = a;
+            }
+            sc = vsa_oracle_e4m3_round(amax / 6.0f);
+            sv = (float)vsa_oracle_e4m3_value(sc);
+            scale[r * nb + blk] = (uint8_t)sc;
+            for (int j = 0; j < 16; ++j) cb[j] = (uint8_t)((sv == 0.0f) ? 0 : vsa_oracle_e2m1_round(xb[j] / sv));
+        }
+    }
+}
+
+/* Key smoothing: mu [B, H, D] = (binary64 sum over t of k[b, t, h, d], token order) / L,
+ * rounded to binary32; ks [B, L, H, D] = k - mu in binary32. */
+void vsa_oracle_smooth_keys(const uint16_t *k, int64_t B, int64_t L, int H, int D, float *mu, float *ks) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int d = 0; d < D; ++d) {
+                double sum = 0.0;
+                float m;
+                for (int64_t t = 0; t < L; ++t) sum += (double)bf16_to_float(k[((b * L + t) * H + h) * D + d]);
+                m = (float)(sum / (double)L);
+                mu[(b * H + h) * D + d] = m;
+                for (int64_t t = 0; t < L; ++t) {
+                    int64_t e = ((b * L + t) * H + h) * D + d;
+                    ks[e] = bf16_to_float(k[e]) - m;
+                }
+            }
 }
 
 /* One operand of the fine branch's logits (Q or K), [B, L, H, D]: bf16 bits,
