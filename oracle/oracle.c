@@ -68,12 +68,12 @@
  *      prefix tiles stay always kept; prefix query tiles (reference ones included) stay
  *      dense; the compression still runs over all tiles.
  *   R20 FP4 video query tiles ("FastH3 OmniRef inference", sections "Device profiles",
- *      "Environment" and "Fallbacks": video query tiles on an FP4 kernel, key smoothing
- *      "subtract the per-head key mean before FP4 quantization"; the emulator fallback
- *      gives the numerics: FP4 Q/K for video query tiles, per-token 8-bit Q/K for the prefix
- *      tiles, bf16 P.V, key smoothing; "FastH3 NVFP4 on RTX PRO 6000", model integration
- *      and "What was tried": activations take a unit global scale and dynamic per-16 block
- *      scales; the stored format is E2M1 values with one E4M3 scale per 16 values):
+ *      "Environment" and "Fallbacks": the video query tiles run on an FP4 kernel; key
+ *      smoothing removes each head's mean key before the FP4 rounding; the emulator fallback
+ *      fixes the numerics: FP4 Q and K for the video query tiles, 8-bit per-token Q and K for
+ *      the prefix tiles, bf16 P.V, smoothed K; "FastH3 NVFP4 on RTX PRO 6000", model
+ *      integration and "What was tried": activations carry a global scale of 1 and one scale
+ *      per 16 values computed per call; values are E2M1 with E4M3 block scales):
  *      FP4 = OCP E2M1 (bit 3 sign, 2-bit exponent with bias 1, 1-bit mantissa; magnitudes
  *      0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN).  Rows of D are cut into blocks of
  *      16 consecutive elements; a block's scale is the E4M3 code e4m3_round(amax / 6)

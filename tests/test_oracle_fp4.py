@@ -1,5 +1,5 @@
 """Pins for the oracle's FP4 video-tile variant (reading R20: E2M1 codes with one E4M3 scale per 16
-values and a unit global scale, the per-head key mean subtracted from K before quantisation, the
+values and a global scale of 1, each head's mean key removed from K before the rounding, the
 dequantised Q and K in the video query tiles' logits; the prefix query tiles per the split).
 
 What pins it, independently of the oracle's code:
