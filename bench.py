@@ -652,6 +652,9 @@ def main():
     ap.add_argument("--ab-prefix-fp8", action="store_true",
                     help="side measurement: vsa_forward with bf16 Q/K logits against the prefix split (8-bit Q/K "
                          "for the dense prefix query tiles only)")
+    ap.add_argument("--ab-fp4", action="store_true",
+                    help="side measurement: vsa_forward with bf16 Q/K logits, the prefix split, and the split with "
+                         "FP4 Q and smoothed FP4 K for the video query tiles")
     args = ap.parse_args()
     import synth
 
@@ -668,6 +671,9 @@ def main():
         return
     if args.ab_prefix_fp8:
         run_ab(args, w, {"qk_bf16": {}, "qk_prefix_fp8": {"qk_fp8": "prefix"}})
+        return
+    if args.ab_fp4:
+        run_ab(args, w, {"qk_bf16": {}, "qk_prefix_fp8": {"qk_fp8": "prefix"}, "qk_fp4_video": {"qk_fp8": "fp4"}})
         return
     world, rank, local = dist_setup(args)
     try:

@@ -85,7 +85,7 @@ class PlanDims(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t)
                 for n in ("q_t", "k_t", "v_t", "q_s", "k_s", "q_n", "kv_max", "pq", "pk", "pv", "scores", "idx", "o_c",
-                          "q_c", "k_c", "q_n8", "kv_max8", "total")]
+                          "q_c", "k_c", "q_n8", "kv_max8", "k_sum", "k_mu", "total")]
 
 
 _lib = None
@@ -156,11 +156,13 @@ def _ptr(t, dtype=None, name="tensor"):
 
 def _qk_mode(qk_fp8) -> int:
     """qk_fp8: False / True (8-bit Q/K logits for every query tile) / "prefix" (for the dense prefix query
-    tiles only, the pages' split) -> the geometry's 0 / 1 / 2."""
+    tiles only, the pages' split) / "fp4" (the split, and FP4 Q and smoothed FP4 K for the video query
+    tiles) -> the geometry's 0 / 1 / 2 / 3."""
     if isinstance(qk_fp8, str):
-        if qk_fp8 != "prefix":
-            raise ValueError(f"qk_fp8 must be a bool or 'prefix', got {qk_fp8!r}")
-        return 2
+        modes = {"prefix": 2, "fp4": 3}
+        if qk_fp8 not in modes:
+            raise ValueError(f"qk_fp8 must be a bool, 'prefix' or 'fp4', got {qk_fp8!r}")
+        return modes[qk_fp8]
     return int(bool(qk_fp8))
 
 
@@ -475,7 +477,7 @@ def workspace_views(plan, workspace):
     lay = plan.workspace_layout
     seq = bool(g.get("seq_tiles", False))
     mode = _qk_mode(g.get("qk_fp8", False))
-    f8, split = mode == 1, mode == 2
+    f8, split = mode == 1, mode >= 2
     T = d["tile_size"]  # rows per tile
 
     def view(off, n, dtype, shape):
@@ -496,6 +498,9 @@ def workspace_views(plan, workspace):
         "q_n8": view(lay["q_n8"], B * H * n_t * T, torch.float32, (B, H, n_t, T)),
         "kv_max8": view(lay["kv_max8"], B * H * 2, torch.float32, (B, H, 2)),
     }
+    if mode == 3:
+        extra["k_sum"] = view(lay["k_sum"], B * H * D, torch.float64, (B, H, D))
+        extra["k_mu"] = view(lay["k_mu"], B * H * D, torch.float32, (B, H, D))
     return {
         **extra,
         "q_t": codes("q_t") if f8 else tiles("q_t"),

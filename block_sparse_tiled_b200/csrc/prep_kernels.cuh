@@ -838,4 +838,125 @@ __global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __
   }
 }
 
+// ---------------------------------------------------------------------------
+// FP4 video query tiles: the logits of the video query tiles take Q and K rounded to E2M1 with one
+// E4M3 scale per 16 consecutive values of a row (global scale 1), K first smoothed by its per-head
+// mean; the dense prefix query tiles keep per-token 8-bit Q/K and every P.V stays bf16.  Passages:
+// "FastH3 OmniRef inference", sections "Device profiles" (the video query tiles on the FP4 kernel, the
+// prefix split), "Environment" (each head's mean key removed before the FP4 rounding) and "Fallbacks"
+// (the emulator's numerics: FP4 video query tiles, 8-bit per-token prefix tiles, bf16 P.V, smoothed
+// K); "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", model integration (activations: a global scale of 1,
+// one scale per 16 values computed per call).
+//
+// The dequantised values (an E2M1 value, at most 2 significant bits, times an E4M3 scale, at most 4,
+// between 2^-10 and 2688) are bf16 numbers, so they are written back into the bf16 tile copies and the
+// bf16 attention kernels compute the FP4 logits exactly (products exact, binary32 accumulation).
+// ---------------------------------------------------------------------------
+
+// Column sums of the key copies [B*H, rows, D] (every row, pads are zero) in binary64: block (x, bh)
+// adds rows [x * per_cta, (x + 1) * per_cta) of column d and adds that partial sum atomically.  A sum of
+// bf16 values is exact in binary64 whenever their magnitudes span fewer than 53 - 8 - log2(rows) binary
+// orders (about 28 at 75,008 tokens: data between 2^-20 and 2^8), and then no order of the additions
+// changes it.
+template <int D>
+__global__ void __launch_bounds__(128) key_sum_kernel(const uint16_t* __restrict__ k_t, double* __restrict__ sum,
+                                                      int64_t rows, int per_cta) {
+  const int64_t bh = blockIdx.y;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t r1 = min(r0 + per_cta, rows);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const uint16_t* col = k_t + bh * rows * D + d;
+    double acc = 0.0;
+    for (int64_t r = r0; r < r1; ++r) acc += static_cast<double>(bf16_bits_to_f32(__ldg(col + r * D)));
+    atomicAdd(sum + bh * D + d, acc);
+  }
+}
+
+// mu = the binary64 column sum divided by the token count L in binary64, rounded to binary32.
+__global__ void key_mean_kernel(const double* __restrict__ sum, float* __restrict__ mu, int64_t n, double L) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e < n) mu[e] = __double2float_rn(__ddiv_rn(sum[e], L));
+}
+
+// The dequantised FP4 value of x in a block of scale value sv > 0: the E2M1 magnitude (0, 0.5, 1, 1.5,
+// 2, 3, 4, 6) nearest to |x / sv| (binary32 division), a tie going to the even code -- so the midpoints
+// 0.25, 1.25, 2.5 and 5 round down and 0.75, 1.75 and 3.5 round up -- and 6 above 5; times sv (exact),
+// with the sign of x.
+__device__ __forceinline__ float e2m1_dequant(float x, float sv) {
+  const float a = fabsf(__fdiv_rn(x, sv));
+  float m;
+  if (a <= 0.25f)
+    m = 0.0f;
+  else if (a < 0.75f)
+    m = 0.5f;
+  else if (a <= 1.25f)
+    m = 1.0f;
+  else if (a < 1.75f)
+    m = 1.5f;
+  else if (a <= 2.5f)
+    m = 2.0f;
+  else if (a < 3.5f)
+    m = 3.0f;
+  else if (a <= 5.0f)
+    m = 4.0f;
+  else
+    m = 6.0f;
+  return copysignf(m * sv, x);
+}
+
+// In place over the tile copies [B*H, n_t, rows, D] (bf16): blockIdx.y = 0 rounds the query copy's video
+// tiles (tiles >= P), blockIdx.y = 1 the key copy's every tile after subtracting mu[bh, d] (binary32);
+// valid rows only (pads stay zero).  One thread per block of 16 values of a row: amax = max |x|, scale
+// code E4M3(amax / 6) (binary32 division, nearest even, saturating at 448), then each value becomes its
+// dequantised E2M1 rounding (all zero when the scale is zero).
+template <int D>
+__global__ void __launch_bounds__(256) fp4_round_tiles_kernel(uint16_t* __restrict__ q_t, uint16_t* __restrict__ k_t,
+                                                              const float* __restrict__ mu,
+                                                              const int32_t* __restrict__ tile_valid, int n_t,
+                                                              int rows, int P, int64_t n_rows) {
+  constexpr int kBlocks = D / 16;
+  const bool keys = blockIdx.y == 1;
+  uint16_t* base = keys ? k_t : q_t;
+  const int64_t units = n_rows * kBlocks;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < units;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = e / kBlocks;
+    const int blk = static_cast<int>(e - row * kBlocks);
+    const int r = static_cast<int>(row % rows);
+    const int64_t bt = row / rows;  // (bh, tile)
+    const int tile = static_cast<int>(bt % n_t);
+    if (r >= __ldg(tile_valid + tile) || (!keys && tile < P)) continue;
+    uint4* p = reinterpret_cast<uint4*>(base + row * D + blk * 16);
+    const uint4 w0 = p[0], w1 = p[1];
+    const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float x[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      x[2 * j] = __uint_as_float(w[j] << 16);
+      x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+    if (keys) {
+      const float* m = mu + (bt / n_t) * D + blk * 16;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = __fsub_rn(x[j], __ldg(m + j));
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(x[j]));
+    const __nv_fp8_storage_t sc = __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(sc, __NV_E4M3);
+    const float sv = __half2float(*reinterpret_cast<const __half*>(&hr));
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float a = sv > 0.0f ? e2m1_dequant(x[2 * j], sv) : 0.0f;
+      const float b = sv > 0.0f ? e2m1_dequant(x[2 * j + 1], sv) : 0.0f;
+      // exact: the values are bf16 numbers, so taking the high halves loses nothing
+      o[j] = (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
+    }
+    p[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    p[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 }  // namespace vsa

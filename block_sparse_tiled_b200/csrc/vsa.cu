@@ -93,7 +93,7 @@ vsa_status resolve(const vsa_geometry* g, Resolved* r) {
   if (g->seq_tiles != 0 && g->seq_tiles != 1) return fail(VSA_ERR_INVALID_ARG, "seq_tiles must be 0 or 1");
   if (g->seq_tiles && g->batch > 4)
     return fail(VSA_ERR_UNSUPPORTED, "seq_tiles needs batch <= 4 (one 5-D tensor map per batch)");
-  if (g->qk_fp8 < 0 || g->qk_fp8 > 2) return fail(VSA_ERR_INVALID_ARG, "qk_fp8 must be 0, 1 or 2");
+  if (g->qk_fp8 < 0 || g->qk_fp8 > 3) return fail(VSA_ERR_INVALID_ARG, "qk_fp8 must be 0, 1, 2 or 3");
   if (g->qk_fp8 && g->seq_tiles)
     return fail(VSA_ERR_UNSUPPORTED, "qk_fp8 reads 8-bit tile-order copies: it needs seq_tiles = 0");
   if (g->head_dim != 64 && g->head_dim != 96 && g->head_dim != 128)
@@ -290,7 +290,7 @@ void build_seq_tables(const Resolved& r, const std::vector<uint64_t>& mask_tiled
 // rows; with qk_fp8 of the dequantised row) and, per (b, h), the largest key norm and |v| (two floats).
 vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, int64_t tile, int64_t V, int64_t topk,
                                  bool seq_tiles,
-                                 bool qk_fp8, bool qk_split = false) {
+                                 bool qk_fp8, bool qk_split = false, bool fp4 = false) {
   vsa_workspace_layout w{};
   size_t off = 0;
   const size_t rows = static_cast<size_t>(B * H * n_t * tile);
@@ -316,6 +316,9 @@ vsa_workspace_layout make_layout(int64_t B, int64_t H, int64_t D, int64_t n_t, i
   w.k_c = off; off += align256(qk_split ? rows * vsa::kF8RowBytes : 0);
   w.q_n8 = off; off += align256(qk_split ? rows * 4 : 0);
   w.kv_max8 = off; off += align256(qk_split ? static_cast<size_t>(B * H * 8) : 0);
+  // FP4 video query tiles: the binary64 key column sums and the key means
+  w.k_sum = off; off += align256(fp4 ? static_cast<size_t>(B * H * D * 8) : 0);
+  w.k_mu = off; off += align256(fp4 ? static_cast<size_t>(B * H * D * 4) : 0);
   w.total = off;
   return w;
 }
@@ -451,6 +454,7 @@ struct vsa_plan_s {
   bool seq_tiles = false;  // the attention reads tiles from sequence order (no tile-order copies)
   bool qk_fp8 = false;     // 8-bit Q/K (E4M3 codes, one scale per token and head) for the fine logits
   bool qk_split = false;   // the same for the dense prefix query tiles only; video query tiles keep bf16
+  bool fp4 = false;        // with qk_split: the video query tiles' logits from FP4 Q and smoothed FP4 K
   // bf16 attention: the dense prefix query row blocks run two at a time on vsa_attn_pair_kernel (built
   // with VSA_PAIR_PREFIX=0 they stay on vsa_attn_kernel, one at a time)
   bool pair_prefix = VSA_PAIR_PREFIX != 0;
@@ -612,6 +616,40 @@ vsa_status run_tile_stats(vsa_plan p, const void* qt, const void* kt, const void
     return p->r.sh ? launch(vsa::tile_stats_kernel<D, 128>) : launch(vsa::tile_stats_kernel<D, 64>);
   }));
   return launch_check("tile statistics");
+}
+
+// FP4 video query tiles: the key means of the key copy (binary64 column sums, then / L), the FP4 rounding
+// of the video query tiles of qt and of every key tile of kt (smoothed) in place, and the overflow-bound
+// statistics of the rounded copies.
+vsa_status run_fp4(vsa_plan p, void* qt, void* kt, const void* vt, double* ksum, float* mu, float* qn, uint32_t* kv,
+                   cudaStream_t s) {
+  if (p->n_t == 0) return VSA_OK;
+  const int64_t BH = static_cast<int64_t>(p->B) * p->H;
+  if (BH > 65535) return fail(VSA_ERR_UNSUPPORTED, "FP4 key means: batch * heads must be <= 65535");
+  const int64_t rows = static_cast<int64_t>(p->n_t) * p->r.tile;  // key rows per (b, h)
+  const int per_cta = 512;
+  VSA_CUDA_TRY(cudaMemsetAsync(ksum, 0, static_cast<size_t>(BH) * p->D * sizeof(double), s));
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    const dim3 grid(static_cast<unsigned>((rows + per_cta - 1) / per_cta), static_cast<unsigned>(BH));
+    vsa::key_sum_kernel<D><<<grid, 128, 0, s>>>(static_cast<const uint16_t*>(kt), ksum, rows, per_cta);
+    return VSA_OK;
+  }));
+  VSA_TRY(launch_check("key sums"));
+  const int64_t nm = BH * p->D;
+  vsa::key_mean_kernel<<<static_cast<unsigned>((nm + 255) / 256), 256, 0, s>>>(ksum, mu, nm,
+                                                                               static_cast<double>(p->r.L));
+  VSA_TRY(launch_check("key means"));
+  VSA_TRY(with_head_dim(p->D, [&](auto dc) -> vsa_status {
+    constexpr int D = decltype(dc)::value;
+    const int64_t n_rows = BH * rows;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n_rows * (D / 16) + 255) / 256, 16LL * p->num_sms));
+    vsa::fp4_round_tiles_kernel<D><<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, s>>>(
+        static_cast<uint16_t*>(qt), static_cast<uint16_t*>(kt), mu, p->d_tile_valid, p->n_t, p->r.tile, p->P, n_rows);
+    return VSA_OK;
+  }));
+  VSA_TRY(launch_check("FP4 rounding"));
+  return run_tile_stats(p, qt, kt, vt, qn, kv, s);
 }
 
 vsa_status run_pool(vsa_plan p, const void* qt, const void* kt, const void* vt, float* pq, float* pk, float* pv,
@@ -904,6 +942,7 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->seq_tiles = p->seq_tiles;
   q->qk_fp8 = p->qk_fp8;
   q->qk_split = p->qk_split;
+  q->fp4 = p->fp4;
   q->pair_prefix = p->pair_prefix;
   q->kr = p->kr;
   q->n_ref = p->n_ref;
@@ -912,7 +951,7 @@ vsa_plan_s* make_head_slice_plan(const vsa_plan_s* p, int32_t heads) {
   q->d_exempt = p->d_exempt;
   q->d_refs = p->d_refs;
   q->ws = make_layout(q->B, q->H, q->D, q->n_t, q->r.tile, q->V, q->topk + q->kr, q->seq_tiles, q->qk_fp8,
-                      q->qk_split);
+                      q->qk_split, q->fp4);
   q->owns_device = false;
   return q;
 }
@@ -930,7 +969,7 @@ HostLayout host_layout(const vsa_plan_s* p, int32_t hc) {
   h.fwd = 0;
   size_t off =
       align256(make_layout(p->B, hc, p->D, p->n_t, p->r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8,
-                           p->qk_split)
+                           p->qk_split, p->fp4)
                    .total);
   for (int s = 0; s < 2; ++s) {
     h.slot[s] = off;
@@ -998,6 +1037,10 @@ vsa_status forward_impl(vsa_plan p, const void* q, const void* k, const void* v,
     VSA_CUDA_TRY(cudaMemcpy2DAsync(kv8 + 1, 8, kv + 1, 8, 4, static_cast<size_t>(p->B) * p->H,
                                    cudaMemcpyDeviceToDevice, s));
   }
+  // FP4 video query tiles: the bf16 copies (already pooled) become their FP4 roundings, with new statistics
+  if (p->fp4)
+    VSA_TRY(run_fp4(p, qt, kt, vt, reinterpret_cast<double*>(w + p->ws.k_sum), reinterpret_cast<float*>(w + p->ws.k_mu),
+                    qn, kv, s));
   VSA_TRY(run_scores(p, pq, pk, S, s));
   VSA_TRY(run_topk(p, S, pv, idx, oc, s, gate_nz));
   const void* qkv[3] = {q, k, v};
@@ -1034,7 +1077,7 @@ void fill_dims(const vsa_geometry* g, const Resolved& r, vsa_plan_dims* d) {
   d->softmax_scale = r.scale;
   d->workspace_bytes =
       make_layout(g->batch, g->heads, g->head_dim, d->n_tiles, r.tile, r.n_video, r.topk + r.kr, g->seq_tiles != 0,
-                  g->qk_fp8 == 1, g->qk_fp8 == 2)
+                  g->qk_fp8 == 1, g->qk_fp8 >= 2, g->qk_fp8 == 3)
           .total;
   d->selected_pairs = r.n_video * (r.n_prefix - r.n_ref + r.kr + r.topk) + r.n_prefix * (r.n_prefix + r.n_video);
   d->tile_size = r.tile;
@@ -1108,12 +1151,13 @@ vsa_status vsa_plan_tiles(const vsa_geometry* g, void* stream, vsa_plan* out) {
   if (r.tile == kTile) build_seq_tables(r, p->mask_tiled, &p->row_token, &p->mask_seq, &p->coord);
   p->seq_tiles = g->seq_tiles != 0;
   p->qk_fp8 = g->qk_fp8 == 1;
-  p->qk_split = g->qk_fp8 == 2;
+  p->qk_split = g->qk_fp8 >= 2;  // 3: the split with FP4 video query tiles
+  p->fp4 = g->qk_fp8 == 3;
   p->kr = r.kr;
   p->n_ref = static_cast<int32_t>(r.n_ref);
   for (int32_t j = 0; j < p->P && p->n_ref > 0; ++j) (r.tile_ref[j] ? p->ref_tiles : p->exempt_tiles).push_back(j);
   p->ws = make_layout(p->B, p->H, p->D, p->n_t, r.tile, p->V, p->topk + p->kr, p->seq_tiles, p->qk_fp8,
-                      p->qk_split);
+                      p->qk_split, p->fp4);
   auto cleanup = [p] {
     cudaFree(p->d_tile_token);
     cudaFree(p->d_tile_valid);

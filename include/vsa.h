@@ -110,6 +110,22 @@ typedef struct vsa_geometry {
                                 with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
                                 by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4, 64-token tiles */
   int32_t qk_fp8;            /* 0: the fine branch's logits use the bf16 Q and K;
+                                3: the prefix split of 2, and the video query tiles' logits use
+                                FP4 Q and K: K smoothed first (mu[b, h, d] = the key mean over
+                                the L tokens, a binary64 sum / L rounded to binary32, subtracted
+                                in binary32), then every row of Q and K cut into blocks of 16
+                                values, each block scaled by the E4M3 code of amax / 6 (binary32
+                                division, nearest even, saturating) and each value rounded to
+                                the nearest E2M1 value of x / scale (ties to even, saturating at
+                                6); global scale 1.  The rounded values are bf16 numbers and
+                                run through the bf16 attention.  Needs seq_tiles = 0; only the
+                                whole-forward entry points accept it.  The key mean is exact,
+                                and so independent of the summation order, when the bf16 keys
+                                of a (b, h, d) column span fewer than about 28 binary orders of
+                                magnitude (at L = 75,008).  Passages: "FastH3 OmniRef
+                                inference", sections "Device profiles", "Environment" and
+                                "Fallbacks"; "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", model
+                                integration;
                                 2: the pages' prefix split: the dense prefix query tiles take the
                                 8-bit logits described under 1, the video query tiles keep bf16
                                 (their FP4 kernel on the pages is not built); needs seq_tiles = 0
@@ -377,10 +393,14 @@ vsa_status vsa_forward_noalloc(vsa_plan p, const vsa_bf16* q_dev, const vsa_bf16
  * q_n8, kv_max8 the statistics of the dequantised rows (q_c .. kv_max8 are empty
  * otherwise).  Only the prefix tiles' query rows are quantised (the video query
  * tiles keep bf16 logits): the video tiles' part of q_c, q_s and q_n8 is left as
- * it was. */
+ * it was.  With qk_fp8 = 3 the same, and the video query tiles of q_t and every
+ * valid key row of k_t hold their FP4 roundings (bf16 numbers), k_sum the binary64
+ * key column sums [B, H, D] and k_mu the key means [B, H, D] float32 (k_sum and
+ * k_mu are empty otherwise); q_n and kv_max are the statistics of the rounded
+ * copies. */
 typedef struct vsa_workspace_layout {
   size_t q_t, k_t, v_t, q_s, k_s, q_n, kv_max, pq, pk, pv, scores, idx, o_c;
-  size_t q_c, k_c, q_n8, kv_max8, total;
+  size_t q_c, k_c, q_n8, kv_max8, k_sum, k_mu, total;
 } vsa_workspace_layout;
 vsa_status vsa_plan_workspace(vsa_plan p, vsa_workspace_layout* out);
 

@@ -162,7 +162,7 @@ def test_qk_fp8_workspace_and_limits(vsa):
         vsa.vsa_plan_query(qk_fp8=True, seq_tiles=True, **kw)
     assert e.value.status == 3  # VSA_ERR_UNSUPPORTED
     g, keep = vsa.make_geometry(**kw)
-    g.qk_fp8 = 3
+    g.qk_fp8 = 4
     import ctypes
 
     d = vsa.PlanDims()
@@ -182,6 +182,18 @@ def test_qk_prefix_split_workspace(vsa):
     assert e.value.status == 3  # VSA_ERR_UNSUPPORTED
     with pytest.raises(ValueError):
         vsa.make_geometry(qk_fp8="video", **kw)
+
+
+def test_qk_fp4_workspace(vsa):
+    """FP4 video query tiles (qk_fp8 = 3): the prefix split's workspace plus the binary64 key column sums
+    and the binary32 key means, one per (b, h, d); it needs tile-order copies too."""
+    kw = dict(batch=1, heads=56, head_dim=128, segments=(512, 0, 768), grid=(24, 48, 64), sparsity=0.9)
+    c = vsa.vsa_plan_query(qk_fp8="prefix", **kw)["workspace_bytes"]
+    f = vsa.vsa_plan_query(qk_fp8="fp4", **kw)["workspace_bytes"]
+    assert f - c == 56 * 128 * 8 + 56 * 128 * 4
+    with pytest.raises(vsa.VsaError) as e:
+        vsa.vsa_plan_query(qk_fp8="fp4", seq_tiles=True, **kw)
+    assert e.value.status == 3  # VSA_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("segments,grid,cube", [
