@@ -471,7 +471,9 @@ def workspace_views(plan, workspace):
     query row norms [B, H, n_t, tile] (with qk_fp8 of the dequantised rows) and kv_max the (b, h)
     maxima of key norm and |v| [B, H, 2] (the attention's overflow bound).  With qk_fp8="prefix" q_t and
     k_t are the bf16 copies, q_c and k_c the codes, q_s and k_s their scales, and q_n8, kv_max8 the
-    statistics of the dequantised rows."""
+    statistics of the dequantised rows.  With qk_fp8="fp4" the same, except that q_t's video query tiles
+    and k_t's valid rows hold their FP4 roundings (bf16 numbers; keys after smoothing), k_sum the binary64
+    key column sums [B, H, D] and k_mu the key means [B, H, D]; q_n and kv_max describe the rounded copies."""
     d, g = plan.dims, plan.geometry
     B, H, D, n_t, V, k = g["batch"], g["heads"], g["head_dim"], d["n_tiles"], d["n_video_tiles"], d["topk"]
     lay = plan.workspace_layout
