@@ -128,7 +128,7 @@ typedef struct vsa_geometry {
                                 integration;
                                 2: the pages' prefix split: the dense prefix query tiles take the
                                 8-bit logits described under 1, the video query tiles keep bf16
-                                (their FP4 kernel on the pages is not built); needs seq_tiles = 0
+                                (3 gives them FP4 logits); needs seq_tiles = 0
                                 and, like 1, only the whole-forward entry points accept it.
                                 Passage: "FastH3 OmniRef inference", section "Device profiles"
                                 (dense prefix query tiles at 8-bit Q/K with bf16 P.V);
