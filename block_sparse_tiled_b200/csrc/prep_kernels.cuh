@@ -855,9 +855,11 @@ __global__ void __launch_bounds__(256, 2) select_compress_kernel(const float* __
 
 // Column sums of the key copies [B*H, rows, D] (every row, pads are zero) in binary64: block (x, bh)
 // adds rows [x * per_cta, (x + 1) * per_cta) of column d and adds that partial sum atomically.  A sum of
-// bf16 values is exact in binary64 whenever their magnitudes span fewer than 53 - 8 - log2(rows) binary
-// orders (about 28 at 75,008 tokens: data between 2^-20 and 2^8), and then no order of the additions
-// changes it.
+// bf16 values is exact in binary64 when every value is a multiple of the smallest value's bf16 ulp and
+// the sum of their magnitudes stays below 2^53 such ulps; then no order of the additions changes it.
+// Otherwise (a column holding a value near 1e-16 among values near 1, say) the atomic order can change
+// the last bits of the binary64 sum, which changes the binary32 mean only when the sum lies that close
+// to a binary32 rounding boundary.
 template <int D>
 __global__ void __launch_bounds__(128) key_sum_kernel(const uint16_t* __restrict__ k_t, double* __restrict__ sum,
                                                       int64_t rows, int per_cta) {

@@ -119,10 +119,12 @@ typedef struct vsa_geometry {
                                 the nearest E2M1 value of x / scale (ties to even, saturating at
                                 6); global scale 1.  The rounded values are bf16 numbers and
                                 run through the bf16 attention.  Needs seq_tiles = 0; only the
-                                whole-forward entry points accept it.  The key mean is exact,
-                                and so independent of the summation order, when the bf16 keys
-                                of a (b, h, d) column span fewer than about 28 binary orders of
-                                magnitude (at L = 75,008).  Passages: "FastH3 OmniRef
+                                whole-forward entry points accept it.  The key mean's binary64
+                                sum is computed in parallel: it equals the token-order sum when
+                                that sum is exact (a column's bf16 values within about 2^28 of
+                                one another at L = 75,008), and otherwise may differ in its last
+                                bits, which reaches the binary32 mean only near a rounding
+                                boundary.  Passages: "FastH3 OmniRef
                                 inference", sections "Device profiles", "Environment" and
                                 "Fallbacks"; "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", model
                                 integration;
