@@ -110,6 +110,20 @@ typedef struct vsa_geometry {
                                 with 4-D/5-D TMA boxes: no tile-order copies, a workspace smaller
                                 by 3*B*H*n_tiles*64*D*2 bytes, batch <= 4, 64-token tiles */
   int32_t qk_fp8;            /* 0: the fine branch's logits use the bf16 Q and K;
+                                1: 8-bit Q/K: each (token, head) row of Q and K is quantised to
+                                OCP FP8 E4M3 codes with one binary32 scale s = amax / 448
+                                (code = E4M3(x / s), round to nearest even, saturating; an
+                                all-zero row has s = 0), and the logits are the 8-bit product
+                                times both scales.  Selection, compression and P.V keep bf16.
+                                Every query tile is covered.  Passages: "FastH3 OmniRef
+                                inference", sections "The Blackwell stack" and "Fallbacks"
+                                (8-bit per-token Q/K with bf16 P.V); "FastH3 NVFP4 on RTX PRO
+                                6000 (sm_120)", multi-GPU notes (one FP8 scale per token and
+                                head);
+                                2: the pages' prefix split: the dense prefix query tiles take the
+                                8-bit logits of 1, the video query tiles keep bf16.  Passage:
+                                "FastH3 OmniRef inference", section "Device profiles" (dense
+                                prefix query tiles at 8-bit Q/K with bf16 P.V);
                                 3: the prefix split of 2, and the video query tiles' logits use
                                 FP4 Q and K: K smoothed first (mu[b, h, d] = the key mean over
                                 the L tokens, a binary64 sum / L rounded to binary32, subtracted
@@ -118,33 +132,16 @@ typedef struct vsa_geometry {
                                 division, nearest even, saturating) and each value rounded to
                                 the nearest E2M1 value of x / scale (ties to even, saturating at
                                 6); global scale 1.  The rounded values are bf16 numbers and
-                                run through the bf16 attention.  Needs seq_tiles = 0; only the
-                                whole-forward entry points accept it.  The key mean's binary64
-                                sum is computed in parallel: it equals the token-order sum when
-                                that sum is exact (a column's bf16 values within about 2^28 of
-                                one another at L = 75,008), and otherwise may differ in its last
+                                run through the bf16 attention.  The key mean's binary64 sum is
+                                computed in parallel: it equals the token-order sum when that
+                                sum is exact (a column's bf16 values within about 2^28 of one
+                                another at L = 75,008), and otherwise may differ in its last
                                 bits, which reaches the binary32 mean only near a rounding
-                                boundary.  Passages: "FastH3 OmniRef
-                                inference", sections "Device profiles", "Environment" and
-                                "Fallbacks"; "FastH3 NVFP4 on RTX PRO 6000 (sm_120)", model
-                                integration;
-                                2: the pages' prefix split: the dense prefix query tiles take the
-                                8-bit logits described under 1, the video query tiles keep bf16
-                                (3 gives them FP4 logits); needs seq_tiles = 0
-                                and, like 1, only the whole-forward entry points accept it.
-                                Passage: "FastH3 OmniRef inference", section "Device profiles"
-                                (dense prefix query tiles at 8-bit Q/K with bf16 P.V);
-                                1: 8-bit Q/K: each (token, head) row of Q and K is quantised to
-                                OCP FP8 E4M3 codes with one binary32 scale s = amax / 448
-                                (code = E4M3(x / s), round to nearest even, saturating; an
-                                all-zero row has s = 0), and the logits are the 8-bit product
-                                times both scales.  Selection, compression and P.V keep bf16.
-                                Every query tile is covered.  Needs seq_tiles = 0; only the
-                                whole-forward entry points accept such a plan.  Passages:
-                                "FastH3 OmniRef inference", sections "The Blackwell stack" and
-                                "Fallbacks" (8-bit per-token Q/K with bf16 P.V); "FastH3 NVFP4
-                                on RTX PRO 6000 (sm_120)", multi-GPU notes (one FP8 scale per
-                                token and head). */
+                                boundary.  Passages: "FastH3 OmniRef inference", sections
+                                "Device profiles", "Environment" and "Fallbacks"; "FastH3 NVFP4
+                                on RTX PRO 6000 (sm_120)", model integration.
+                                Modes 1 to 3 need seq_tiles = 0, and only the whole-forward
+                                entry points accept such a plan. */
   int32_t cube_t, cube_h, cube_w; /* video cube shape, product = tile_size; all 0 = the default:
                                      4x4x4 for 64 tokens (the method's), 4x4x8 for 128 (the
                                      pages do not state it: the 64-token cube doubled along w) */
