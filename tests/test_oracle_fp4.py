@@ -292,3 +292,30 @@ def test_forward_fp4_rows_follow_their_branch(oracle_mod, qk8):
     assert np.array_equal(got.out, oracle_mod.output(got.o_f, got.o_c, b["gate"], geo))
     with pytest.raises(ValueError):
         fwd(qk8=True, fp4=True)
+
+
+def test_key_sums_order_free_on_the_480p_keys(oracle_mod):
+    """The GPU adds each key column in 512-row binary64 partial sums over the tile-order copy (pads
+    zero) and combines the partials atomically, in any order.  The structured 480p keys hold residues
+    near 1e-16 (a sample near -2 plus its +2 tile offset), so exactness is not guaranteed a priori; this
+    replays that summation structure on the CPU with three combination orders and finds every binary64
+    column sum equal to the oracle's token-order sum, hence every binary32 mean equal too."""
+    w = synth.workload("480p")
+    kb = synth.as_bits(synth.make_inputs(w, seed=0)["k"])
+    mu, _ = oracle_mod.smooth_keys(kb)
+    geo = oracle_mod.geometry(w.segments, w.grid)
+    tok = geo.tile_token.reshape(-1)
+    f = as_f32(kb)[0]  # [L, H, D]
+    assert (np.abs(f[f != 0]) < 1e-12).any()  # the residues are there
+    rng = np.random.default_rng(0)
+    for h in range(w.heads):
+        rows = np.where(tok[:, None] >= 0, f[np.maximum(tok, 0), h, :], 0.0).astype(np.float64)
+        nb = (rows.shape[0] + 511) // 512
+        part = [np.add.accumulate(rows[i * 512:(i + 1) * 512], axis=0)[-1] for i in range(nb)]
+        token_order = np.add.accumulate(f[:, h, :].astype(np.float64), axis=0)[-1]
+        for order in (range(nb), range(nb - 1, -1, -1), rng.permutation(nb)):
+            s = np.zeros(w.head_dim)
+            for i in order:
+                s = s + part[i]
+            assert np.array_equal(s, token_order), h
+        assert np.array_equal((token_order / w.seq_len).astype(np.float32), mu[0, h])
