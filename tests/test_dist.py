@@ -65,7 +65,10 @@ def test_reference_arm_two_ranks():
     assert d["config"]["workload"] == "tiny"
 
 
-def _ulysses_worker(rank, world, port, q):
+MODES = {"bf16": {}, "prefix": {"qk8": "prefix"}, "fp4": {"qk8": "prefix", "fp4": True}}
+
+
+def _ulysses_worker(rank, world, port, q, mode="bf16"):
     import numpy as np
     import torch.distributed as dist
 
@@ -86,27 +89,31 @@ def _ulysses_worker(rank, world, port, q):
         parts = [None] * world
         dist.all_gather_object(parts, mine)
         heads = {n: np.concatenate([p[n] for p in parts], axis=1)[:, :, h0:h0 + hn] for n in mine}
-        r = oracle.forward(heads["q"], heads["k"], heads["v"], heads["gate"], w.segments, w.grid, w.sparsity)
+        kw = MODES[mode]
+        r = oracle.forward(heads["q"], heads["k"], heads["v"], heads["gate"], w.segments, w.grid, w.sparsity, **kw)
         # head -> seq: every rank gets every head group's output, keeps its token part
         groups = [None] * world
         dist.all_gather_object(groups, (h0, r.out))
         out = np.zeros((w.batch, ls, w.heads, w.head_dim))
         for g0, o in groups:
             out[:, :, g0:g0 + o.shape[2]] = o[:, rank * ls:(rank + 1) * ls]
-        whole = oracle.forward(full["q"], full["k"], full["v"], full["gate"], w.segments, w.grid, w.sparsity)
+        whole = oracle.forward(full["q"], full["k"], full["v"], full["gate"], w.segments, w.grid, w.sparsity, **kw)
         q.put((rank, bool(np.array_equal(out, whole.out[:, rank * ls:(rank + 1) * ls]))))
     finally:
         dist.destroy_process_group()
 
 
-def test_ulysses_decomposition_gloo():
+@pytest.mark.parametrize("mode", list(MODES))
+def test_ulysses_decomposition_gloo(mode):
     """The sequence-parallel decomposition the parts entry point implements (token parts in, head
     groups computed independently, token parts out) reproduces the whole forward: two gloo ranks
-    exchange parts with collectives and run the oracle on their head groups."""
+    exchange parts with collectives and run the oracle on their head groups.  The precision modes need
+    no further exchange either: the 8-bit and FP4 scales are per (token, head) row or block, and the FP4
+    key mean is per head over all tokens, which a rank holds once it has its heads."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ulysses_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_ulysses_worker, args=(r, 2, port, q, mode)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
