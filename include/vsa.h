@@ -11,8 +11,9 @@
  *     topk = max(1, min(ceil((1 - sparsity) * n_video_tiles), n_video_tiles));
  * prefix key tiles are always kept and prefix query tiles attend densely;
  * block-sparse softmax attention runs over the kept tiles; and the
- * compression branch softmax(scores) @ pool(V), broadcast over each tile's
- * rows and scaled by the per-token gate (no activation), is added.
+ * compression term -- the pooled V tiles weighted by the softmax of the
+ * query tile's scores -- is added to each of the tile's rows, times the
+ * per-token gate (no activation).
  *
  * Conventions for every entry point:
  *  - Pointers named *_dev are CUDA device pointers; the caller owns every
@@ -123,7 +124,7 @@ typedef struct vsa_geometry {
                                 2: the pages' prefix split: the dense prefix query tiles take the
                                 8-bit logits of 1, the video query tiles keep bf16.  Passage:
                                 "FastH3 OmniRef inference", section "Device profiles" (dense
-                                prefix query tiles at 8-bit Q/K with bf16 P.V);
+                                prefix query tiles: Q and K rounded to 8 bits, bf16 P.V);
                                 3: the prefix split of 2, and the video query tiles' logits use
                                 FP4 Q and K: K smoothed first (mu[b, h, d] = the key mean over
                                 the L tokens, a binary64 sum / L rounded to binary32, subtracted

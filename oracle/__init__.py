@@ -252,8 +252,8 @@ def fine_split(q, k, v, geo: Geometry, idx, topk: int, scale: float, todo=None, 
     q, k (as fine() without), or with ``video_qk`` = (q4, k4) from those bf16 arrays instead (the
     dequantised FP4 operands of fp4_operands, reading R20).  Both branches run in full over their own
     tiles and the rows are merged by the tile each token belongs to; bf16 P.V throughout.  ("FastH3
-    OmniRef inference", section "Device profiles": the dense prefix query tiles run at 8-bit Q/K with
-    bf16 P.V, the video query tiles on another kernel.)"""
+    OmniRef inference", section "Device profiles": Q and K of the dense prefix query tiles rounded to
+    8 bits with P.V in bf16, the video query tiles on another kernel.)"""
     B, L, H, _ = np.shape(q)
     n_t, P = geo.n_tiles, geo.n_prefix
     sel = np.ones((B, H, n_t), bool) if todo is None else np.asarray(todo, bool)
